@@ -1,0 +1,317 @@
+"""CPU oracle of the HyperQuant tile codec (test infrastructure only).
+
+The oracle is a plain single-threaded C implementation (``hq_oracle.c``) of the codec described
+in "HyperQuant: A Rate-Distortion-Optimal Quantization Pipeline for Large Language and Diffusion
+Models" (gist.science, Technical Summary, "Methodology: The HyperQuant Pipeline").  This module
+builds it with gcc and wraps it with ctypes over numpy arrays.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package.  The product (``post_quantization_tile_b200``) never imports it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+Z, A2, D4, E8 = 0, 1, 2, 3
+LATTICE_DIM = {Z: 1, A2: 2, D4: 4, E8: 8}
+
+ST_CAPACITY = 1 << 3
+ST_NONFINITE = 1 << 4
+ST_CORRUPT = 1 << 5
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle: -O2, binary32 without excess precision, no FMA contraction."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+               "-fexcess-precision=standard", "-Wall", "-Wno-unused-function", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64, u64, i32, f32 = ctypes.c_int64, ctypes.c_uint64, ctypes.c_int, ctypes.c_float
+        L.hqo_philox4x32_10.argtypes = [P, ctypes.c_uint32, ctypes.c_uint32, P]
+        L.hqo_sign_negative.argtypes = [u64, i64]
+        L.hqo_sign_negative.restype = i32
+        L.hqo_f32_to_bf16.argtypes = [f32]
+        L.hqo_f32_to_bf16.restype = ctypes.c_uint16
+        L.hqo_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.hqo_bf16_to_f32.restype = f32
+        L.hqo_rms.argtypes = [P, i32]
+        L.hqo_rms.restype = f32
+        L.hqo_fwht_f32.argtypes = [P, i32]
+        L.hqo_fwht_f64.argtypes = [P, i32]
+        L.hqo_quantize_block.argtypes = [i32, P, P]
+        L.hqo_strip_block.argtypes = [i32, P, P, P]
+        L.hqo_unstrip_block.argtypes = [i32, P, i32, P]
+        L.hqo_dither_d4.argtypes = [u64, i64, i64, i32, P]
+        L.hqo_rice_tile.argtypes = [P, i32, i32, P, i64, P, P]
+        L.hqo_rice_tile.restype = i64
+        L.hqo_parse_tile.argtypes = [P, i64, i32, i32, ctypes.c_uint16, P, P]
+        L.hqo_parse_tile.restype = i32
+        L.hqo_encode.argtypes = [P, i32, i64, i64, i32, i32, f32, u64, i32, i64, P, P, P, P, i64, P, P]
+        L.hqo_encode.restype = ctypes.c_uint32
+        L.hqo_quantize_coeffs.argtypes = [P, i64, i32, i32, i32, i64, u64, P, P, P, P, i64]
+        L.hqo_quantize_coeffs.restype = ctypes.c_uint32
+        L.hqo_parse.argtypes = [P, P, P, i64, i64, i32, i32, P]
+        L.hqo_parse.restype = ctypes.c_uint32
+        L.hqo_decode.argtypes = [P, P, P, P, i64, i64, i32, i32, f32, u64, i32, i64, P]
+        L.hqo_decode.restype = ctypes.c_uint32
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ----------------------------------------------------------------------------------------------
+# primitives
+# ----------------------------------------------------------------------------------------------
+def philox(ctr, key0: int, key1: int) -> np.ndarray:
+    c = np.asarray(ctr, dtype=np.uint32).copy()
+    out = np.zeros(4, dtype=np.uint32)
+    lib().hqo_philox4x32_10(_p(c), ctypes.c_uint32(key0), ctypes.c_uint32(key1), _p(out))
+    return out
+
+
+def signs(seed: int, cols: int) -> np.ndarray:
+    """+1/-1 diagonal for transformed-axis indices 0..cols-1."""
+    L = lib()
+    return np.array([-1 if L.hqo_sign_negative(seed, j) else 1 for j in range(cols)], dtype=np.int8)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    L = lib()
+    flat = np.asarray(x, dtype=np.float32).ravel()
+    return np.array([L.hqo_f32_to_bf16(float(v)) for v in flat], dtype=np.uint16).reshape(np.shape(x))
+
+
+def rms(x: np.ndarray) -> float:
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    return float(lib().hqo_rms(_p(a), a.size))
+
+
+def fwht_f32(x: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(x, dtype=np.float32).copy()
+    lib().hqo_fwht_f32(_p(a), a.size)
+    return a
+
+
+def fwht_f64(x: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(x, dtype=np.float64).copy()
+    lib().hqo_fwht_f64(_p(a), a.size)
+    return a
+
+
+def quantize_blocks(lattice: int, u: np.ndarray) -> np.ndarray:
+    """Nearest lattice point of each row of u[m, d] (integer embedding, see hq_oracle.c)."""
+    d = LATTICE_DIM[lattice]
+    u = np.ascontiguousarray(u, dtype=np.float32).reshape(-1, d)
+    v = np.zeros(u.shape, dtype=np.int32)
+    L = lib()
+    for i in range(u.shape[0]):
+        L.hqo_quantize_block(lattice, _p(u[i]), _p(v[i]))
+    return v
+
+
+def dither_d4(seed: int, bh: int, s: int, blk: int) -> np.ndarray:
+    U = np.zeros(4, dtype=np.float32)
+    lib().hqo_dither_d4(seed, bh, s, blk, _p(U))
+    return U
+
+
+def strip(lattice: int, v: np.ndarray):
+    d = LATTICE_DIM[lattice]
+    v = np.ascontiguousarray(v, dtype=np.int32).reshape(-1, d)
+    sym = np.zeros_like(v)
+    cos = np.zeros(v.shape[0], dtype=np.int32)
+    L = lib()
+    c = ctypes.c_int()
+    for i in range(v.shape[0]):
+        L.hqo_strip_block(lattice, _p(v[i]), _p(sym[i]), ctypes.byref(c))
+        cos[i] = c.value
+    return sym, cos
+
+
+def unstrip(lattice: int, sym: np.ndarray, cos: np.ndarray) -> np.ndarray:
+    d = LATTICE_DIM[lattice]
+    sym = np.ascontiguousarray(sym, dtype=np.int32).reshape(-1, d)
+    v = np.zeros_like(sym)
+    L = lib()
+    for i in range(sym.shape[0]):
+        L.hqo_unstrip_block(lattice, _p(sym[i]), int(cos[i]), _p(v[i]))
+    return v
+
+
+def rice_tile(v: np.ndarray, lattice: int):
+    """Rice-code one tile of integer codes; returns (words, bit length, k, sum q)."""
+    v = np.ascontiguousarray(v, dtype=np.int32)
+    n = v.size
+    cap = (n // 8 + 17 * n) // 32 + 2
+    words = np.zeros(cap, dtype=np.uint32)
+    k, sq = ctypes.c_int(), ctypes.c_int()
+    nbits = lib().hqo_rice_tile(_p(v), n, lattice, _p(words), cap, ctypes.byref(k), ctypes.byref(sq))
+    return words, int(nbits), k.value, sq.value
+
+
+def parse_tile(words: np.ndarray, n: int, lattice: int, meta: int):
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    v = np.zeros(n, dtype=np.int32)
+    bl = ctypes.c_int64()
+    ok = lib().hqo_parse_tile(_p(words), words.size, n, lattice, meta, _p(v), ctypes.byref(bl))
+    return bool(ok), v, int(bl.value)
+
+
+# ----------------------------------------------------------------------------------------------
+# whole-tensor codec
+# ----------------------------------------------------------------------------------------------
+def bound_words(rows: int, cols: int, n: int) -> int:
+    """Worst-case words (k <= 15, sum q <= n per tile), plus one padding word per chunk."""
+    T = rows * (cols // n)
+    C = (cols // n) * ((rows + 31) // 32)
+    return (T * (n // 8 + 15 * n + 2 * n) + 31) // 32 + C + 4
+
+
+@dataclass
+class Code:
+    rows: int
+    cols: int
+    n: int
+    lattice: int
+    beta: float
+    seed: int
+    kv: int
+    kv_S: int
+    scale: np.ndarray       # uint16 [T], bf16 bits
+    meta: np.ndarray        # uint16 [T]
+    chunk_word: np.ndarray  # uint32 [C+1]
+    bits: np.ndarray        # uint32 [total words]
+    status: int
+    v: np.ndarray | None = None   # int32 [T, n]
+    u: np.ndarray | None = None   # float32 [T, n]
+
+    @property
+    def tiles(self) -> int:
+        return self.rows * (self.cols // self.n)
+
+    @property
+    def total_words(self) -> int:
+        return int(self.chunk_word[-1])
+
+    def payload_bits(self) -> int:
+        k = (self.meta & 15).astype(np.int64)
+        sq = (self.meta >> 4).astype(np.int64)
+        cos = self.n // 8 if self.lattice == E8 else 0
+        return int(np.sum(cos + self.n * k + self.n + sq))
+
+
+def encode(x: np.ndarray, n: int, lattice: int, beta: float, seed: int, kv: bool = False, kv_S: int = 0,
+           want_codes: bool = False) -> Code:
+    """x: 2-D numpy array, dtype uint16 (bf16 bits) or float32."""
+    assert x.ndim == 2
+    if x.dtype == np.uint16:
+        dtype = 0
+    elif x.dtype == np.float32:
+        dtype = 1
+    else:
+        raise TypeError("x must be uint16 (bf16 bits) or float32")
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    T = rows * (cols // n)
+    C = (cols // n) * ((rows + 31) // 32)
+    cap = bound_words(rows, cols, n)
+    scale = np.zeros(T, dtype=np.uint16)
+    meta = np.zeros(T, dtype=np.uint16)
+    cw = np.zeros(C + 1, dtype=np.uint32)
+    bits = np.zeros(cap, dtype=np.uint32)
+    v = np.zeros((T, n), dtype=np.int32) if want_codes else None
+    u = np.zeros((T, n), dtype=np.float32) if want_codes else None
+    st = lib().hqo_encode(_p(x), dtype, rows, cols, n, lattice, ctypes.c_float(beta), seed, int(kv), kv_S,
+                          _p(scale), _p(meta), _p(cw), _p(bits), cap,
+                          _p(v) if v is not None else None, _p(u) if u is not None else None)
+    if st & 2:
+        raise ValueError("oracle rejected the arguments")
+    return Code(rows, cols, n, lattice, float(np.float32(beta)), seed, int(kv), kv_S, scale, meta, cw,
+                bits[: int(cw[-1])].copy(), int(st), v, u)
+
+
+def quantize_coeffs(u: np.ndarray, n: int, lattice: int, seed: int = 0, kv: bool = False, kv_S: int = 0):
+    """u: float32 [tiles, n] normalised coefficients.  Returns (v, meta, chunk_word, bits, status)."""
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    tiles = u.shape[0]
+    C = (tiles + 31) // 32
+    cap = bound_words(tiles, n, n)
+    v = np.zeros((tiles, n), dtype=np.int32)
+    meta = np.zeros(tiles, dtype=np.uint16)
+    cw = np.zeros(C + 1, dtype=np.uint32)
+    bits = np.zeros(cap, dtype=np.uint32)
+    st = lib().hqo_quantize_coeffs(_p(u), tiles, n, lattice, int(kv), kv_S, seed, _p(v), _p(meta), _p(cw),
+                                   _p(bits), cap)
+    if st & 2:
+        raise ValueError("oracle rejected the arguments")
+    return v, meta, cw, bits[: int(cw[-1])].copy(), int(st)
+
+
+def parse(code: Code) -> tuple[np.ndarray, int]:
+    v = np.zeros((code.tiles, code.n), dtype=np.int32)
+    bits = np.ascontiguousarray(code.bits, dtype=np.uint32)
+    if bits.size == 0:
+        bits = np.zeros(1, dtype=np.uint32)
+    st = lib().hqo_parse(_p(code.meta), _p(code.chunk_word), _p(bits), code.rows, code.cols, code.n,
+                         code.lattice, _p(v))
+    return v, int(st)
+
+
+def decode(code: Code) -> tuple[np.ndarray, int]:
+    """Reconstruction in float64 [rows, cols] and status bits."""
+    out = np.zeros((code.rows, code.cols), dtype=np.float64)
+    bits = np.ascontiguousarray(code.bits, dtype=np.uint32)
+    if bits.size == 0:
+        bits = np.zeros(1, dtype=np.uint32)
+    st = lib().hqo_decode(_p(code.scale), _p(code.meta), _p(code.chunk_word), _p(bits), code.rows, code.cols,
+                          code.n, code.lattice, ctypes.c_float(code.beta), code.seed, code.kv, code.kv_S, _p(out))
+    return out, int(st)
+
+
+def payload_bps(code: Code) -> float:
+    return code.payload_bits() / float(code.rows * code.cols)
+
+
+def total_bps(code: Code) -> float:
+    C = code.chunk_word.size - 1
+    nbytes = 4 * code.total_words + 2 * code.tiles + 2 * code.tiles + 4 * (C + 1)
+    return 8.0 * nbytes / float(code.rows * code.cols)
+
+
+def calibrate_step(x: np.ndarray, n: int, lattice: int, target_bps: float, seed: int = 0, kv: bool = False,
+                   kv_S: int = 0, iters: int = 40) -> float:
+    """Bisection on log(beta) so the oracle's payload rate on x hits target_bps."""
+    lo, hi = np.log(2.0 ** -8), np.log(2.0 ** 6)
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        b = float(np.float32(np.exp(mid)))
+        r = payload_bps(encode(x, n, lattice, b, seed, kv, kv_S))
+        if r > target_bps:
+            lo = mid
+        else:
+            hi = mid
+    return float(np.float32(np.exp(0.5 * (lo + hi))))

@@ -1,0 +1,761 @@
+/*
+ * hq_oracle.c -- plain, slow, single-threaded CPU oracle of the HyperQuant tile codec.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark may load this file's library.  The product (the CUDA library and its Python
+ * binding) never links, imports or calls it, and the two share no code, header or table.
+ *
+ * Source of the method: "HyperQuant: A Rate-Distortion-Optimal Quantization Pipeline for Large
+ * Language and Diffusion Models" (Domb, Sackstein, Solberg), as summarised on gist.science
+ * (English "Technical Summary", section "Methodology: The HyperQuant Pipeline"):
+ *   1. per-tile Randomized Hadamard Transform RHT_n(x) = H_n D x, D a random sign diagonal;
+ *   2. nearest-point quantization to E8, D4, A2 or Z, mapped to an integer embedding;
+ *   3. lossless bit-stripping of lattice-parity-fixed bits, then Rice coding;
+ *   4. for the KV cache, subtractive dither U ~ Uniform(V(Lambda)) added before quantization
+ *      and subtracted after.
+ * The pages fix only this shape.  Every constant, order, tie rule and bit layout below is a
+ * reading of them; each is listed with its reason in the repository's design notes.
+ *
+ * Arithmetic.  The encode chain (RMS, scale, sign flip, FWHT, normalisation, lattice decision)
+ * runs in IEEE binary32 with round-to-nearest-even, no fused multiply-add (built with
+ * -ffp-contract=off), correctly rounded division and square root.  It decides integer codes, so
+ * it uses the same precision the device kernels use.  Decode (reconstruction) runs in binary64.
+ *
+ * Parity pins (all in tests/, marked "not gpu"):
+ *   philox           : curand's host Philox4x32-10 generator (a library run);
+ *   bf16 rounding    : torch's float32 -> bfloat16 conversion;
+ *   fwht             : scipy's Sylvester Hadamard matrix product, orthogonality, exact inverse;
+ *   rms              : numpy float64 RMS within binary32 rounding;
+ *   lattice decoders : brute-force search over neighbouring lattice points, textbook normalised
+ *                      second moments (Conway & Sloane, SPLAG, Table 2.3);
+ *   rice / layout    : round trip, length formula, sum(q) <= n;
+ *   codec            : inputs built on lattice points decode exactly; dithered KV inner
+ *                      products are unbiased over seeds (Appendix A claim).
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#if !defined(FLT_EVAL_METHOD) || FLT_EVAL_METHOD != 0
+#error "the oracle needs binary32 evaluation without excess precision"
+#endif
+
+#define HQO_Z 0
+#define HQO_A2 1
+#define HQO_D4 2
+#define HQO_E8 3
+
+/* status bits: bit (1 << code), codes as documented for the library's status word */
+#define HQO_ST_CAPACITY (1u << 3)
+#define HQO_ST_NONFINITE (1u << 4)
+#define HQO_ST_CORRUPT (1u << 5)
+
+#define HQO_MAXN 256
+
+/* ------------------------------------------------------------------------------------------ */
+/* Philox4x32-10, from Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2,  */
+/* 3" (SC'11): ten rounds of two 32x32->64 multiplies with the published multipliers, the key  */
+/* bumped by the published Weyl constants between rounds.                                      */
+/* ------------------------------------------------------------------------------------------ */
+void hqo_philox4x32_10(const uint32_t ctr[4], uint32_t key0, uint32_t key1, uint32_t out[4])
+{
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key0, k1 = key1;
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * (uint64_t)x0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * (uint64_t)x2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        uint32_t y0 = hi1 ^ x1 ^ k0;
+        uint32_t y1 = lo1;
+        uint32_t y2 = hi0 ^ x3 ^ k1;
+        uint32_t y3 = lo0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* Sign of the random diagonal D for transformed-axis index J (global column for weights, head
+ * dimension index for KV).  Reading: D depends only on the seed and J, so one diagonal serves
+ * every row / token and (R w).(R x) = w.x holds across rows.  One Philox block covers 128 J. */
+int hqo_sign_negative(uint64_t seed, int64_t J)
+{
+    uint32_t ctr[4] = {(uint32_t)((uint64_t)J >> 7), 0u, 0u, 0u};
+    uint32_t w[4];
+    hqo_philox4x32_10(ctr, (uint32_t)seed, (uint32_t)(seed >> 32), w);
+    return (int)((w[(J & 127) >> 5] >> (J & 31)) & 1u);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* bfloat16 helpers                                                                            */
+/* ------------------------------------------------------------------------------------------ */
+float hqo_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* round to nearest, ties to even; NaN stays NaN */
+uint16_t hqo_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return (uint16_t)((u >> 16) | 0x40u);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+static float f32_from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* c_n = 1/sqrt(n) in binary32: exact for n = 64 and 256, RN(2^-3.5) for n = 128 */
+static float inv_sqrt_n(int n)
+{
+    if (n == 64) return 0.125f;
+    if (n == 128) return f32_from_bits(0x3DB504F3u);
+    return 0.0625f;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Per-tile RMS: q_i = x_i * x_i, summed by the ascending pairwise tree (h = 1, 2, ..., n/2;   */
+/* q[i] += q[i+h] for i = 0 mod 2h), s = sqrt(q[0] * (1/n)).  "per-tile scaling" (Methodology  */
+/* step 2), RMS statistic as the workload description fixes it.                                */
+/* ------------------------------------------------------------------------------------------ */
+float hqo_rms(const float* x, int n)
+{
+    float q[HQO_MAXN];
+    for (int i = 0; i < n; ++i) q[i] = x[i] * x[i];
+    for (int h = 1; h < n; h *= 2)
+        for (int i = 0; i < n; i += 2 * h) q[i] = q[i] + q[i + h];
+    float ms = q[0] * (1.0f / (float)n);
+    return sqrtf(ms);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Fast Walsh-Hadamard transform, Sylvester (natural) order, unnormalised, butterflies in      */
+/* descending stride order h = n/2, n/4, ..., 1.  (Methodology step 1: H_n.)                   */
+/* ------------------------------------------------------------------------------------------ */
+void hqo_fwht_f32(float* x, int n)
+{
+    for (int h = n / 2; h >= 1; h /= 2)
+        for (int i = 0; i < n; ++i)
+            if ((i & h) == 0) {
+                float a = x[i], b = x[i + h];
+                x[i] = a + b;
+                x[i + h] = a - b;
+            }
+}
+
+void hqo_fwht_f64(double* x, int n)
+{
+    for (int h = n / 2; h >= 1; h /= 2)
+        for (int i = 0; i < n; ++i)
+            if ((i & h) == 0) {
+                double a = x[i], b = x[i + h];
+                x[i] = a + b;
+                x[i + h] = a - b;
+            }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Lattice nearest point (Methodology step 2).  Closest-point rules after Conway & Sloane,     */
+/* "Fast quantizing and decoding algorithms for lattice quantizers and codes" (IEEE T-IT 1982).*/
+/* Shared pieces:                                                                              */
+/*   a = rint(u) (ties to even), e = a - u (exact in binary32, and never -0);                  */
+/*   "toward u" for a coordinate is +1 when e < 0, else -1;                                     */
+/*   argmax / argmin of |e| compare max(|e|, 2^-63) and break ties to the lowest index.        */
+/* ------------------------------------------------------------------------------------------ */
+static const float TINY = 1.0842021724855044e-19f; /* 2^-63 */
+
+static float clamp_tiny(float v) { return v < TINY ? TINY : v; }
+
+static int argmax_abs(const float* e, int d)
+{
+    int j = 0;
+    float best = clamp_tiny(fabsf(e[0]));
+    for (int i = 1; i < d; ++i) {
+        float v = clamp_tiny(fabsf(e[i]));
+        if (v > best) { best = v; j = i; }
+    }
+    return j;
+}
+
+static int argmin_abs(const float* e, int d)
+{
+    int j = 0;
+    float best = clamp_tiny(fabsf(e[0]));
+    for (int i = 1; i < d; ++i) {
+        float v = clamp_tiny(fabsf(e[i]));
+        if (v < best) { best = v; j = i; }
+    }
+    return j;
+}
+
+/* Z: the integer nearest to u */
+static void q_z(const float* u, int32_t* v) { v[0] = (int32_t)rintf(u[0]); }
+
+/* D4 = { v in Z^4 : sum v even }.  Round each coordinate; if the sum is odd, move the
+ * coordinate with the largest rounding error one step toward u. */
+void hqo_q_d4(const float* u, int32_t* v)
+{
+    float e[4];
+    int32_t a[4];
+    int sum = 0;
+    for (int i = 0; i < 4; ++i) {
+        float r = rintf(u[i]);
+        e[i] = r - u[i];
+        a[i] = (int32_t)r;
+        sum += a[i];
+    }
+    if (sum & 1) {
+        int j = argmax_abs(e, 4);
+        a[j] += (e[j] < 0.0f) ? 1 : -1;
+    }
+    for (int i = 0; i < 4; ++i) v[i] = a[i];
+}
+
+/* E8 = D8 u (D8 + 1/2), min norm sqrt(2).  Output in doubled coordinates v = 2p (all v_i of
+ * one parity, sum v = 0 mod 4).
+ *   Coset A (D8): a = rint(u); if sum a is odd, move the coordinate with max |e| toward u.
+ *   Coset B (D8 + 1/2): b_i = a_i + 1/2 if e_i < 0 else a_i - 1/2 (nearest half-integer);
+ *     if sum (b_i - 1/2) is odd, move the coordinate farthest from its half-integer, i.e.
+ *     the one with min |e|, to its other half-integer neighbour.
+ *   Choice: |u - A|^2 - |u - B|^2 = sum_i (|e_i| - 1/4) + [A fixed](1 - 2 max|e|)
+ *           - [B fixed](2 min|e|)  (exact algebra, from |u_i - b_i| = 1/2 - |e_i|).
+ *   It is evaluated in binary32 as D = ((S - 2) + cA) - cB with S = pairwise sum of |e_i|;
+ *   B is taken only when D > 0 (ties go to A). */
+void hqo_q_e8(const float* u, int32_t* v)
+{
+    float e[8], ae[8];
+    int32_t a[8];
+    int sumA = 0, nonneg = 0;
+    for (int i = 0; i < 8; ++i) {
+        float r = rintf(u[i]);
+        e[i] = r - u[i];
+        ae[i] = fabsf(e[i]);
+        a[i] = (int32_t)r;
+        sumA += a[i];
+        if (!(e[i] < 0.0f)) nonneg += 1;
+    }
+    int parA = sumA & 1;
+    int parB = (sumA - nonneg) & 1; /* sum of (b_i - 1/2) = sum a_i - #{e_i >= 0} */
+    float S = ((ae[0] + ae[1]) + (ae[2] + ae[3])) + ((ae[4] + ae[5]) + (ae[6] + ae[7]));
+    int jA = argmax_abs(e, 8);
+    int mB = argmin_abs(e, 8);
+    float emax = clamp_tiny(ae[jA]);
+    float emin = clamp_tiny(ae[mB]);
+    float cA = parA ? (1.0f - 2.0f * emax) : 0.0f;
+    float cB = parB ? (2.0f * emin) : 0.0f;
+    float D = ((S - 2.0f) + cA) - cB;
+    if (!(D > 0.0f)) {
+        /* coset A: v = 2a */
+        if (parA) a[jA] += (e[jA] < 0.0f) ? 1 : -1;
+        for (int i = 0; i < 8; ++i) v[i] = 2 * a[i];
+    } else {
+        /* coset B: v = 2b, odd integers */
+        for (int i = 0; i < 8; ++i) v[i] = 2 * a[i] + ((e[i] < 0.0f) ? 1 : -1);
+        if (parB) {
+            int m = mB;
+            int toward = (e[m] < 0.0f) ? 1 : -1;
+            v[m] -= 2 * toward; /* the other neighbouring half-integer */
+        }
+    }
+}
+
+/* A2, minimum distance 1: points (P/2, Q*sqrt(3)/2) with P = Q mod 2.  Work in (P, Q) =
+ * (2 u0, u1 * K), K = RN(2/sqrt 3).  The lattice is the union of the even and the odd
+ * rectangular cosets of 2Z x 2Z; per coordinate X, h = X/2, a = rint(h), e = a - h.  Squared
+ * distances in (P, Q) units weigh dQ three times; |even|^2 - |odd|^2 is proportional to
+ * |eP| + 3|eQ| - 1, so the even point is taken when RN(|eP| + RN(3|eQ|)) <= 1. */
+static const float A2_K = 1.15470053837925153f; /* RN(2/sqrt(3)) */
+
+void hqo_q_a2(const float* u, int32_t* v)
+{
+    float P = 2.0f * u[0];
+    float Q = u[1] * A2_K;
+    float hP = P * 0.5f, hQ = Q * 0.5f;
+    float rP = rintf(hP), rQ = rintf(hQ);
+    float eP = rP - hP, eQ = rQ - hQ;
+    int32_t aP = (int32_t)rP, aQ = (int32_t)rQ;
+    float E = fabsf(eP) + 3.0f * fabsf(eQ);
+    if (E <= 1.0f) {
+        v[0] = 2 * aP;
+        v[1] = 2 * aQ;
+    } else {
+        v[0] = 2 * aP + ((eP < 0.0f) ? 1 : -1);
+        v[1] = 2 * aQ + ((eQ < 0.0f) ? 1 : -1);
+    }
+}
+
+static int lattice_dim(int lattice)
+{
+    switch (lattice) {
+    case HQO_Z: return 1;
+    case HQO_A2: return 2;
+    case HQO_D4: return 4;
+    default: return 8;
+    }
+}
+
+static void quantize_block(int lattice, const float* u, int32_t* v)
+{
+    switch (lattice) {
+    case HQO_Z: q_z(u, v); break;
+    case HQO_A2: hqo_q_a2(u, v); break;
+    case HQO_D4: hqo_q_d4(u, v); break;
+    default: hqo_q_e8(u, v); break;
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Bit-stripping (Methodology step 3): drop the bits the lattice's parity checks fix.          */
+/*   E8 : c = v0 & 1 (coset bit, sent raw); w = (v - c)/2 in D8; p = (w0+..+w6) & 1;          */
+/*        symbols w0..w6, (w7 - p)/2.                                                          */
+/*   D4 : p = (v0+v1+v2) & 1; symbols v0, v1, v2, (v3 - p)/2.                                  */
+/*   A2 : symbols P, (Q - (P & 1))/2.                                                          */
+/*   Z  : the symbol is v.                                                                     */
+/* Every lattice yields one symbol per coordinate.                                             */
+/* ------------------------------------------------------------------------------------------ */
+static void strip_block(int lattice, const int32_t* v, int32_t* sym, int* coset)
+{
+    *coset = 0;
+    if (lattice == HQO_Z) {
+        sym[0] = v[0];
+    } else if (lattice == HQO_A2) {
+        sym[0] = v[0];
+        sym[1] = (v[1] - (v[0] & 1)) >> 1;
+    } else if (lattice == HQO_D4) {
+        int p = (v[0] + v[1] + v[2]) & 1;
+        sym[0] = v[0]; sym[1] = v[1]; sym[2] = v[2];
+        sym[3] = (v[3] - p) >> 1;
+    } else {
+        int c = v[0] & 1;
+        int32_t w[8];
+        for (int i = 0; i < 8; ++i) w[i] = (v[i] - c) >> 1;
+        int p = (w[0] + w[1] + w[2] + w[3] + w[4] + w[5] + w[6]) & 1;
+        for (int i = 0; i < 7; ++i) sym[i] = w[i];
+        sym[7] = (w[7] - p) >> 1;
+        *coset = c;
+    }
+}
+
+static void unstrip_block(int lattice, const int32_t* sym, int coset, int32_t* v)
+{
+    if (lattice == HQO_Z) {
+        v[0] = sym[0];
+    } else if (lattice == HQO_A2) {
+        v[0] = sym[0];
+        v[1] = 2 * sym[1] + (sym[0] & 1);
+    } else if (lattice == HQO_D4) {
+        int p = (sym[0] + sym[1] + sym[2]) & 1;
+        v[0] = sym[0]; v[1] = sym[1]; v[2] = sym[2];
+        v[3] = 2 * sym[3] + p;
+    } else {
+        int p = (sym[0] + sym[1] + sym[2] + sym[3] + sym[4] + sym[5] + sym[6]) & 1;
+        int32_t w[8];
+        for (int i = 0; i < 7; ++i) w[i] = sym[i];
+        w[7] = 2 * sym[7] + p;
+        for (int i = 0; i < 8; ++i) v[i] = 2 * w[i] + coset;
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Rice coding (Methodology step 3).  zz = 2m (m >= 0) or -2m-1 (m < 0); the tile parameter   */
+/* k = min{k >= 0 : sum zz < n 2^(k+1)}, capped at 15 -- "k from the mean index": k is the     */
+/* smallest k with mean(zz) < 2^(k+1), the rational form of the mean-based Rice parameter that  */
+/* is optimal for geometric sources (it codes Gaussian-like symbols within ~0.06 bit of their  */
+/* entropy, where k = ceil(log2 mean) loses ~0.3 bit).  q = zz >> k, r = zz & (2^k - 1).  Below */
+/* the cap, sum zz < n 2^(k+1) gives sum q < 2n.                                               */
+/* Tile bit string (bits LSB-first in little-endian 32-bit words):                             */
+/*   [E8 only: n/8 coset bits, block order]                                                    */
+/*   [for each symbol i in coefficient order: q_i zeros, a one, then r_i in k bits LSB-first]  */
+/* Length L = (E8 ? n/8 : 0) + n k + n + sum q.                                                */
+/* ------------------------------------------------------------------------------------------ */
+static uint32_t zigzag(int32_t m) { return m >= 0 ? (uint32_t)m * 2u : (uint32_t)(-(int64_t)m) * 2u - 1u; }
+static int32_t unzigzag(uint32_t z) { return (z & 1u) ? -(int32_t)((z + 1u) >> 1) : (int32_t)(z >> 1); }
+
+static int rice_k(uint64_t A, int n)
+{
+    int k = 0;
+    while (k < 15 && !(A < ((uint64_t)n << (k + 1)))) ++k;
+    return k;
+}
+
+typedef struct {
+    uint32_t* words;
+    int64_t cap_words;
+    int64_t bitpos; /* absolute bit position in words[] */
+    int overflow;
+} bitw_t;
+
+static void put_bit(bitw_t* w, int bit)
+{
+    int64_t wi = w->bitpos >> 5;
+    if (wi >= w->cap_words) {
+        w->overflow = 1;
+    } else if (bit) {
+        w->words[wi] |= 1u << (w->bitpos & 31);
+    }
+    w->bitpos += 1;
+}
+
+static void put_bits(bitw_t* w, uint32_t value, int nbits)
+{
+    for (int b = 0; b < nbits; ++b) put_bit(w, (int)((value >> b) & 1u));
+}
+
+typedef struct {
+    const uint32_t* words;
+    int64_t nwords;
+    int64_t bitpos;
+    int bad;
+} bitr_t;
+
+static int get_bit(bitr_t* r)
+{
+    int64_t wi = r->bitpos >> 5;
+    if (wi < 0 || wi >= r->nwords) {
+        r->bad = 1;
+        r->bitpos += 1;
+        return 0;
+    }
+    int b = (int)((r->words[wi] >> (r->bitpos & 31)) & 1u);
+    r->bitpos += 1;
+    return b;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* KV dither (Methodology step 4): U uniform on the Voronoi cell of D4.  Philox block with    */
+/* key = seed and counter (s_lo, b*H + h, 0x80000000 | block, s_hi) gives four words w_i;     */
+/* r_i = 2 (w_i >> 8) 2^-24 is uniform on [0,2)^4, a union of D4 fundamental domains since     */
+/* 2Z^4 is a sublattice of D4; U = r - Q_D4(r) is then uniform on V(D4).                       */
+/* ------------------------------------------------------------------------------------------ */
+void hqo_dither_d4(uint64_t seed, int64_t bh, int64_t s, int blk, float U[4])
+{
+    uint32_t ctr[4] = {(uint32_t)(uint64_t)s, (uint32_t)(uint64_t)bh, 0x80000000u | (uint32_t)blk,
+                       (uint32_t)((uint64_t)s >> 32)};
+    uint32_t w[4];
+    hqo_philox4x32_10(ctr, (uint32_t)seed, (uint32_t)(seed >> 32), w);
+    float r[4];
+    for (int i = 0; i < 4; ++i) r[i] = 2.0f * ((float)(w[i] >> 8) * 5.9604644775390625e-08f);
+    int32_t q[4];
+    hqo_q_d4(r, q);
+    for (int i = 0; i < 4; ++i) U[i] = r[i] - (float)q[i];
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Tile geometry.  W[rows, cols] row-major, tile (r, jt) = W[r, jt n : (jt+1) n].  Tile index  */
+/* t = jt * rows + r.  Chunk (jt, rb) holds rows [32 rb, min(32 rb + 32, rows)) of tile column */
+/* jt; chunk index c = jt * RB + rb with RB = ceil(rows / 32).  Chunks start on 32-bit word    */
+/* boundaries; chunk_word[c] is the word offset of chunk c, chunk_word[C] the total.          */
+/* ------------------------------------------------------------------------------------------ */
+
+/* One tile from lattice-unit coefficients u (already normalised, before dither) to symbols.
+ * kv: add the D4 dither of row (bh, s) first.  Returns codes v (integer embedding). */
+static void quantize_tile(const float* u_in, int n, int lattice, int kv, uint64_t seed, int64_t bh,
+                          int64_t s, int32_t* v)
+{
+    int d = lattice_dim(lattice);
+    float z[HQO_MAXN];
+    for (int i = 0; i < n; ++i) z[i] = u_in[i];
+    if (kv) {
+        for (int b = 0; b < n / 4; ++b) {
+            float U[4];
+            hqo_dither_d4(seed, bh, s, b, U);
+            for (int i = 0; i < 4; ++i) z[4 * b + i] = z[4 * b + i] + U[i];
+        }
+    }
+    for (int b = 0; b < n / d; ++b) quantize_block(lattice, z + b * d, v + b * d);
+}
+
+/* Rice-code one tile's codes into the bit writer; returns k and sum q. */
+static void rice_tile(const int32_t* v, int n, int lattice, bitw_t* w, int* k_out, int* sumq_out)
+{
+    int d = lattice_dim(lattice);
+    int32_t sym[HQO_MAXN];
+    int cos[HQO_MAXN / 8];
+    for (int b = 0; b < n / d; ++b) {
+        int c;
+        strip_block(lattice, v + b * d, sym + b * d, &c);
+        if (lattice == HQO_E8) cos[b] = c;
+    }
+    uint64_t A = 0;
+    for (int i = 0; i < n; ++i) A += zigzag(sym[i]);
+    int k = rice_k(A, n);
+    int sumq = 0;
+    if (lattice == HQO_E8)
+        for (int b = 0; b < n / 8; ++b) put_bit(w, cos[b]);
+    for (int i = 0; i < n; ++i) {
+        uint32_t z = zigzag(sym[i]);
+        uint32_t q = z >> k;
+        uint32_t r = z & ((1u << k) - 1u);
+        for (uint32_t j = 0; j < q; ++j) put_bit(w, 0);
+        put_bit(w, 1);
+        put_bits(w, r, k);
+        sumq += (int)q;
+    }
+    *k_out = k;
+    *sumq_out = sumq;
+}
+
+/* Row (b*H + h, s) of a KV tensor [B, H, S, D] flattened to rows = B*H*S. */
+static void kv_row(int64_t r, int64_t S, int64_t* bh, int64_t* s)
+{
+    if (S <= 0) { *bh = 0; *s = r; return; }
+    *bh = r / S;
+    *s = r % S;
+}
+
+static int valid_common(int n, int lattice)
+{
+    return (n == 64 || n == 128 || n == 256) && lattice >= 0 && lattice <= 3;
+}
+
+/* the KV dither is defined for D4 only (its Voronoi cell) */
+static int valid_kv(int kv, int lattice) { return !kv || lattice == HQO_D4; }
+
+/*
+ * Full encode.
+ *   x       : [rows, cols] bf16 (dtype 0) or fp32 (dtype 1), row-major
+ *   beta    : step (lattice units per normalised coefficient), > 0
+ *   kv      : 1 = KV path (D4 dither), kv_S = S of the [B,H,S,D] layout (rows = B*H*S)
+ *   outputs : scale[T] (bf16 bits of the per-tile RMS), meta[T] = k | (sum q << 4),
+ *             chunk_word[C+1], bits[cap_words]; optional v_out[T*n] (integer codes) and
+ *             u_out[T*n] (normalised coefficients before dither)
+ * Returns a bitmask of status bits (0 = ok).
+ */
+uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n, int lattice, float beta,
+                    uint64_t seed, int kv, int64_t kv_S, uint16_t* scale, uint16_t* meta,
+                    uint32_t* chunk_word, uint32_t* bits, int64_t cap_words, int32_t* v_out,
+                    float* u_out)
+{
+    if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || rows <= 0 || cols <= 0 || cols % n) return 1u << 1;
+    uint32_t status = 0;
+    const int64_t NT = cols / n, RB = (rows + 31) / 32;
+    const float cn = inv_sqrt_n(n);
+    memset(bits, 0, (size_t)cap_words * 4);
+    bitw_t w = {bits, cap_words, 0, 0};
+    int64_t c = 0;
+    for (int64_t jt = 0; jt < NT; ++jt) {
+        for (int64_t rb = 0; rb < RB; ++rb, ++c) {
+            chunk_word[c] = (uint32_t)(w.bitpos >> 5);
+            int64_t r_end = (rb + 1) * 32 < rows ? (rb + 1) * 32 : rows;
+            for (int64_t r = rb * 32; r < r_end; ++r) {
+                int64_t t = jt * rows + r;
+                float xt[HQO_MAXN], u[HQO_MAXN];
+                int finite = 1;
+                for (int j = 0; j < n; ++j) {
+                    int64_t idx = r * cols + jt * n + j;
+                    xt[j] = dtype == 0 ? hqo_bf16_to_f32(((const uint16_t*)x)[idx]) : ((const float*)x)[idx];
+                    if (!isfinite(xt[j])) finite = 0;
+                }
+                float s = finite ? hqo_rms(xt, n) : 0.0f;
+                uint16_t sh = hqo_f32_to_bf16(s);
+                float shf = hqo_bf16_to_f32(sh);
+                if (!finite || !isfinite(shf)) {
+                    status |= HQO_ST_NONFINITE;
+                    sh = 0;
+                    shf = 0.0f;
+                } else if (shf < 1.2621774483536189e-29f /* 2^-96 */) {
+                    sh = 0;
+                    shf = 0.0f;
+                }
+                if (shf == 0.0f) {
+                    for (int j = 0; j < n; ++j) u[j] = 0.0f;
+                } else {
+                    for (int j = 0; j < n; ++j)
+                        if (hqo_sign_negative(seed, jt * n + j)) xt[j] = -xt[j];
+                    hqo_fwht_f32(xt, n);
+                    float tden = shf * beta;
+                    float rinv = 1.0f / tden;
+                    float g = cn * rinv;
+                    for (int j = 0; j < n; ++j) u[j] = xt[j] * g;
+                }
+                int64_t bh = 0, sidx = r;
+                if (kv) kv_row(r, kv_S, &bh, &sidx);
+                int32_t v[HQO_MAXN];
+                quantize_tile(u, n, lattice, kv, seed, bh, sidx, v);
+                int k, sumq;
+                rice_tile(v, n, lattice, &w, &k, &sumq);
+                scale[t] = sh;
+                meta[t] = (uint16_t)(k | (sumq << 4));
+                if (v_out) memcpy(v_out + t * n, v, sizeof(int32_t) * (size_t)n);
+                if (u_out) memcpy(u_out + t * n, u, sizeof(float) * (size_t)n);
+            }
+            w.bitpos = (w.bitpos + 31) & ~(int64_t)31; /* chunk ends on a word boundary */
+        }
+    }
+    chunk_word[c] = (uint32_t)(w.bitpos >> 5);
+    if (w.overflow) status |= HQO_ST_CAPACITY;
+    return status;
+}
+
+/*
+ * Quantize caller-given normalised coefficients u[tiles, n] (lattice units): lattice + strip +
+ * Rice + chunk layout with rows = tiles and one tile column.  For kv, the dither of row
+ * (t / kv_S, t % kv_S) is added first.  Outputs as for hqo_encode (no scale).
+ */
+uint32_t hqo_quantize_coeffs(const float* u, int64_t tiles, int n, int lattice, int kv, int64_t kv_S,
+                             uint64_t seed, int32_t* v_out, uint16_t* meta, uint32_t* chunk_word,
+                             uint32_t* bits, int64_t cap_words)
+{
+    if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || tiles <= 0) return 1u << 1;
+    memset(bits, 0, (size_t)cap_words * 4);
+    bitw_t w = {bits, cap_words, 0, 0};
+    int64_t RB = (tiles + 31) / 32;
+    for (int64_t c = 0; c < RB; ++c) {
+        chunk_word[c] = (uint32_t)(w.bitpos >> 5);
+        int64_t t_end = (c + 1) * 32 < tiles ? (c + 1) * 32 : tiles;
+        for (int64_t t = c * 32; t < t_end; ++t) {
+            int64_t bh = 0, sidx = t;
+            if (kv) kv_row(t, kv_S, &bh, &sidx);
+            int32_t v[HQO_MAXN];
+            quantize_tile(u + t * n, n, lattice, kv, seed, bh, sidx, v);
+            int k, sumq;
+            rice_tile(v, n, lattice, &w, &k, &sumq);
+            meta[t] = (uint16_t)(k | (sumq << 4));
+            if (v_out) memcpy(v_out + t * n, v, sizeof(int32_t) * (size_t)n);
+        }
+        w.bitpos = (w.bitpos + 31) & ~(int64_t)31;
+    }
+    chunk_word[RB] = (uint32_t)(w.bitpos >> 5);
+    return w.overflow ? HQO_ST_CAPACITY : 0u;
+}
+
+/* Parse one tile's bit string back to integer codes; checks k and sum q against meta. */
+static int parse_tile(bitr_t* rd, int n, int lattice, uint16_t meta, int32_t* v)
+{
+    int d = lattice_dim(lattice);
+    int k = meta & 15, sumq_meta = meta >> 4;
+    int cos[HQO_MAXN / 8];
+    if (lattice == HQO_E8)
+        for (int b = 0; b < n / 8; ++b) cos[b] = get_bit(rd);
+    int32_t sym[HQO_MAXN];
+    int sumq = 0;
+    for (int i = 0; i < n; ++i) {
+        uint32_t q = 0;
+        while (!get_bit(rd)) {
+            ++q;
+            if (rd->bad || q > (uint32_t)(16 * n)) return 0;
+        }
+        uint32_t r = 0;
+        for (int b = 0; b < k; ++b) r |= (uint32_t)get_bit(rd) << b;
+        sumq += (int)q;
+        if (sumq > 16 * n) return 0;
+        sym[i] = unzigzag((q << k) | r);
+    }
+    if (rd->bad || sumq != sumq_meta) return 0;
+    for (int b = 0; b < n / d; ++b) unstrip_block(lattice, sym + b * d, lattice == HQO_E8 ? cos[b] : 0, v + b * d);
+    return 1;
+}
+
+/* Parse the chunked stream to codes; tiles laid out as in hqo_encode.  Returns status bits. */
+uint32_t hqo_parse(const uint16_t* meta, const uint32_t* chunk_word, const uint32_t* bits, int64_t rows,
+                   int64_t cols, int n, int lattice, int32_t* v_out)
+{
+    if (!valid_common(n, lattice) || rows <= 0 || cols % n) return 1u << 1;
+    const int64_t NT = cols / n, RB = (rows + 31) / 32;
+    const int64_t nwords = chunk_word[NT * RB];
+    uint32_t status = 0;
+    int64_t c = 0;
+    for (int64_t jt = 0; jt < NT; ++jt)
+        for (int64_t rb = 0; rb < RB; ++rb, ++c) {
+            bitr_t rd = {bits, nwords, (int64_t)chunk_word[c] * 32, 0};
+            int64_t r_end = (rb + 1) * 32 < rows ? (rb + 1) * 32 : rows;
+            for (int64_t r = rb * 32; r < r_end; ++r) {
+                int64_t t = jt * rows + r;
+                if (!parse_tile(&rd, n, lattice, meta[t], v_out + t * n)) {
+                    status |= HQO_ST_CORRUPT;
+                    memset(v_out + t * n, 0, sizeof(int32_t) * (size_t)n);
+                }
+            }
+            if (((rd.bitpos + 31) >> 5) != (int64_t)chunk_word[c + 1]) status |= HQO_ST_CORRUPT;
+        }
+    return status;
+}
+
+/*
+ * Reconstruct one tile (binary64) from its integer codes: lattice point p (u units) from the
+ * codes, minus the dither for KV, then x_hat = D H_n p * (s_hat * beta * c_n).
+ *   E8: p = v / 2;  D4, Z: p = v;  A2: p = (P/2, Q sqrt(3)/2).
+ * H_n H_n = n I and u = (H D x) c_n / (s_hat beta) give x = D H u (s_hat beta) c_n.
+ */
+static void reconstruct_tile(const int32_t* v, int n, int lattice, int kv, uint64_t seed, int64_t bh,
+                             int64_t s, uint16_t sh, float beta, int64_t col0, double* out)
+{
+    double p[HQO_MAXN];
+    for (int i = 0; i < n; ++i) {
+        if (lattice == HQO_E8) p[i] = 0.5 * (double)v[i];
+        else if (lattice == HQO_A2) p[i] = (i & 1) ? (double)v[i] * (sqrt(3.0) / 2.0) : 0.5 * (double)v[i];
+        else p[i] = (double)v[i];
+    }
+    if (kv) {
+        for (int b = 0; b < n / 4; ++b) {
+            float U[4];
+            hqo_dither_d4(seed, bh, s, b, U);
+            for (int i = 0; i < 4; ++i) p[4 * b + i] -= (double)U[i];
+        }
+    }
+    hqo_fwht_f64(p, n);
+    double h = (double)hqo_bf16_to_f32(sh) * (double)beta / sqrt((double)n);
+    for (int j = 0; j < n; ++j) {
+        double val = p[j] * h;
+        out[j] = hqo_sign_negative(seed, col0 + j) ? -val : val;
+    }
+}
+
+/* Full decode to binary64 out[rows, cols].  Returns status bits. */
+uint32_t hqo_decode(const uint16_t* scale, const uint16_t* meta, const uint32_t* chunk_word, const uint32_t* bits,
+                    int64_t rows, int64_t cols, int n, int lattice, float beta, uint64_t seed, int kv,
+                    int64_t kv_S, double* out)
+{
+    if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || rows <= 0 || cols % n) return 1u << 1;
+    const int64_t NT = cols / n;
+    int32_t* v = (int32_t*)malloc(sizeof(int32_t) * (size_t)(rows * cols));
+    if (!v) return 1u << 1;
+    uint32_t status = hqo_parse(meta, chunk_word, bits, rows, cols, n, lattice, v);
+    for (int64_t jt = 0; jt < NT; ++jt)
+        for (int64_t r = 0; r < rows; ++r) {
+            int64_t t = jt * rows + r;
+            int64_t bh = 0, sidx = r;
+            if (kv) kv_row(r, kv_S, &bh, &sidx);
+            double tile[HQO_MAXN];
+            reconstruct_tile(v + t * n, n, lattice, kv, seed, bh, sidx, scale[t], beta, jt * n, tile);
+            memcpy(out + r * cols + jt * n, tile, sizeof(double) * (size_t)n);
+        }
+    free(v);
+    return status;
+}
+
+/* Small helpers exposed for the pins. */
+void hqo_quantize_block(int lattice, const float* u, int32_t* v) { quantize_block(lattice, u, v); }
+
+void hqo_strip_block(int lattice, const int32_t* v, int32_t* sym, int* coset) { strip_block(lattice, v, sym, coset); }
+
+void hqo_unstrip_block(int lattice, const int32_t* sym, int coset, int32_t* v) { unstrip_block(lattice, sym, coset, v); }
+
+/* Rice-code a tile of integer codes into words[] (no chunk padding); returns bit length. */
+int64_t hqo_rice_tile(const int32_t* v, int n, int lattice, uint32_t* words, int64_t cap_words, int* k, int* sumq)
+{
+    memset(words, 0, (size_t)cap_words * 4);
+    bitw_t w = {words, cap_words, 0, 0};
+    rice_tile(v, n, lattice, &w, k, sumq);
+    return w.overflow ? -1 : w.bitpos;
+}
+
+int hqo_parse_tile(const uint32_t* words, int64_t nwords, int n, int lattice, uint16_t meta, int32_t* v, int64_t* bitlen)
+{
+    bitr_t rd = {words, nwords, 0, 0};
+    int ok = parse_tile(&rd, n, lattice, meta, v);
+    *bitlen = rd.bitpos;
+    return ok;
+}
