@@ -375,10 +375,15 @@ static void unstrip_block(int lattice, const int32_t* sym, int coset, int32_t* v
 /* is optimal for geometric sources (it codes Gaussian-like symbols within ~0.06 bit of their  */
 /* entropy, where k = ceil(log2 mean) loses ~0.3 bit).  q = zz >> k, r = zz & (2^k - 1).  Below */
 /* the cap, sum zz < n 2^(k+1) gives sum q < 2n.                                               */
-/* Tile bit string (bits LSB-first in little-endian 32-bit words):                             */
-/*   [E8 only: n/8 coset bits, block order]                                                    */
-/*   [for each symbol i in coefficient order: q_i zeros, a one, then r_i in k bits LSB-first]  */
-/* Length L = (E8 ? n/8 : 0) + n k + n + sum q.                                                */
+/* Tile bit string.  Bit position p of a chunk lives in 32-bit word p >> 5 at bit p & 31.      */
+/* A symbol's Rice code is, in reading order: q zeros, a one, then r in k bits, most           */
+/* significant first.  The tile holds                                                          */
+/*   [E8 only: n/8 coset bits, block b at offset b]                                            */
+/*   [symbols 0 .. n/2-1, read forward (increasing position) from offset n/8 (E8) or 0]        */
+/*   [symbols n-1 down to n/2, read backward (decreasing position) from the tile's last bit]   */
+/* The second half is written from the tile's end so that each half can be decoded on its own */
+/* knowing only the tile length L = (E8 ? n/8 : 0) + n (k + 1) + sum q, which k and sum q       */
+/* (stored per tile) give; the two halves meet exactly.                                        */
 /* ------------------------------------------------------------------------------------------ */
 static uint32_t zigzag(int32_t m) { return m >= 0 ? (uint32_t)m * 2u : (uint32_t)(-(int64_t)m) * 2u - 1u; }
 static int32_t unzigzag(uint32_t z) { return (z & 1u) ? -(int32_t)((z + 1u) >> 1) : (int32_t)(z >> 1); }
@@ -393,44 +398,59 @@ static int rice_k(uint64_t A, int n)
 typedef struct {
     uint32_t* words;
     int64_t cap_words;
-    int64_t bitpos; /* absolute bit position in words[] */
+    int64_t bitpos; /* absolute bit position in words[] where the next tile starts */
     int overflow;
 } bitw_t;
 
-static void put_bit(bitw_t* w, int bit)
+static void set_bit(bitw_t* w, int64_t pos, int bit)
 {
-    int64_t wi = w->bitpos >> 5;
+    int64_t wi = pos >> 5;
     if (wi >= w->cap_words) {
         w->overflow = 1;
     } else if (bit) {
-        w->words[wi] |= 1u << (w->bitpos & 31);
+        w->words[wi] |= 1u << (pos & 31);
     }
-    w->bitpos += 1;
 }
 
-static void put_bits(bitw_t* w, uint32_t value, int nbits)
+/* writes one Rice code at *pos, moving by step (+1 forward, -1 backward) */
+static void put_code(bitw_t* w, int64_t* pos, int step, uint32_t q, uint32_t r, int k)
 {
-    for (int b = 0; b < nbits; ++b) put_bit(w, (int)((value >> b) & 1u));
+    for (uint32_t j = 0; j < q; ++j) { set_bit(w, *pos, 0); *pos += step; }
+    set_bit(w, *pos, 1);
+    *pos += step;
+    for (int b = k - 1; b >= 0; --b) { set_bit(w, *pos, (int)((r >> b) & 1u)); *pos += step; }
 }
 
 typedef struct {
     const uint32_t* words;
     int64_t nwords;
-    int64_t bitpos;
     int bad;
 } bitr_t;
 
-static int get_bit(bitr_t* r)
+static int get_bit(bitr_t* r, int64_t pos)
 {
-    int64_t wi = r->bitpos >> 5;
-    if (wi < 0 || wi >= r->nwords) {
+    int64_t wi = pos >> 5;
+    if (pos < 0 || wi >= r->nwords) {
         r->bad = 1;
-        r->bitpos += 1;
         return 0;
     }
-    int b = (int)((r->words[wi] >> (r->bitpos & 31)) & 1u);
-    r->bitpos += 1;
-    return b;
+    return (int)((r->words[wi] >> (pos & 31)) & 1u);
+}
+
+/* reads one Rice code at *pos moving by step; returns 0 on a run longer than limit */
+static int get_code(bitr_t* rd, int64_t* pos, int step, int k, uint32_t limit, uint32_t* q_out, uint32_t* r_out)
+{
+    uint32_t q = 0;
+    while (!get_bit(rd, *pos)) {
+        *pos += step;
+        if (rd->bad || ++q > limit) return 0;
+    }
+    *pos += step;
+    uint32_t r = 0;
+    for (int b = 0; b < k; ++b) { r = (r << 1) | (uint32_t)get_bit(rd, *pos); *pos += step; }
+    *q_out = q;
+    *r_out = r;
+    return !rd->bad;
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -477,7 +497,7 @@ static void quantize_tile(const float* u_in, int n, int lattice, int kv, uint64_
     for (int b = 0; b < n / d; ++b) quantize_block(lattice, z + b * d, v + b * d);
 }
 
-/* Rice-code one tile's codes into the bit writer; returns k and sum q. */
+/* Rice-code one tile's codes into the bit writer at w->bitpos; returns k and sum q. */
 static void rice_tile(const int32_t* v, int n, int lattice, bitw_t* w, int* k_out, int* sumq_out)
 {
     int d = lattice_dim(lattice);
@@ -491,18 +511,25 @@ static void rice_tile(const int32_t* v, int n, int lattice, bitw_t* w, int* k_ou
     uint64_t A = 0;
     for (int i = 0; i < n; ++i) A += zigzag(sym[i]);
     int k = rice_k(A, n);
+    uint32_t q[HQO_MAXN], r[HQO_MAXN];
     int sumq = 0;
-    if (lattice == HQO_E8)
-        for (int b = 0; b < n / 8; ++b) put_bit(w, cos[b]);
     for (int i = 0; i < n; ++i) {
         uint32_t z = zigzag(sym[i]);
-        uint32_t q = z >> k;
-        uint32_t r = z & ((1u << k) - 1u);
-        for (uint32_t j = 0; j < q; ++j) put_bit(w, 0);
-        put_bit(w, 1);
-        put_bits(w, r, k);
-        sumq += (int)q;
+        q[i] = z >> k;
+        r[i] = z & ((1u << k) - 1u);
+        sumq += (int)q[i];
     }
+    int cosb = lattice == HQO_E8 ? n / 8 : 0;
+    int64_t start = w->bitpos;
+    int64_t L = cosb + (int64_t)n * (k + 1) + sumq;
+    for (int b = 0; b < cosb; ++b) set_bit(w, start + b, cos[b]);
+    int64_t pos = start + cosb;                 /* first half, forward */
+    for (int i = 0; i < n / 2; ++i) put_code(w, &pos, +1, q[i], r[i], k);
+    int64_t mid = pos;
+    pos = start + L - 1;                        /* second half, backward from the last bit */
+    for (int i = n - 1; i >= n / 2; --i) put_code(w, &pos, -1, q[i], r[i], k);
+    if (pos != mid - 1) w->overflow = 1;        /* the halves must meet exactly */
+    w->bitpos = start + L;
     *k_out = k;
     *sumq_out = sumq;
 }
@@ -631,31 +658,36 @@ uint32_t hqo_quantize_coeffs(const float* u, int64_t tiles, int n, int lattice, 
     return w.overflow ? HQO_ST_CAPACITY : 0u;
 }
 
-/* Parse one tile's bit string back to integer codes; checks k and sum q against meta. */
-static int parse_tile(bitr_t* rd, int n, int lattice, uint16_t meta, int32_t* v)
+/* Parse one tile starting at bit `start` back to integer codes, using k and sum q from meta:
+ * the first half forward from the start, the second half backward from start + L - 1.  The
+ * halves must meet exactly and sum q must agree.  Returns the tile length, or -1. */
+static int64_t parse_tile(bitr_t* rd, int64_t start, int n, int lattice, uint16_t meta, int32_t* v)
 {
     int d = lattice_dim(lattice);
     int k = meta & 15, sumq_meta = meta >> 4;
+    int cosb = lattice == HQO_E8 ? n / 8 : 0;
+    int64_t L = cosb + (int64_t)n * (k + 1) + sumq_meta;
     int cos[HQO_MAXN / 8];
-    if (lattice == HQO_E8)
-        for (int b = 0; b < n / 8; ++b) cos[b] = get_bit(rd);
+    for (int b = 0; b < cosb; ++b) cos[b] = get_bit(rd, start + b);
     int32_t sym[HQO_MAXN];
+    uint32_t q, r;
     int sumq = 0;
-    for (int i = 0; i < n; ++i) {
-        uint32_t q = 0;
-        while (!get_bit(rd)) {
-            ++q;
-            if (rd->bad || q > (uint32_t)(16 * n)) return 0;
-        }
-        uint32_t r = 0;
-        for (int b = 0; b < k; ++b) r |= (uint32_t)get_bit(rd) << b;
+    int64_t pos = start + cosb;
+    for (int i = 0; i < n / 2; ++i) {
+        if (!get_code(rd, &pos, +1, k, (uint32_t)sumq_meta, &q, &r)) return -1;
         sumq += (int)q;
-        if (sumq > 16 * n) return 0;
         sym[i] = unzigzag((q << k) | r);
     }
-    if (rd->bad || sumq != sumq_meta) return 0;
+    int64_t mid = pos;
+    pos = start + L - 1;
+    for (int i = n - 1; i >= n / 2; --i) {
+        if (!get_code(rd, &pos, -1, k, (uint32_t)sumq_meta, &q, &r)) return -1;
+        sumq += (int)q;
+        sym[i] = unzigzag((q << k) | r);
+    }
+    if (rd->bad || sumq != sumq_meta || pos != mid - 1) return -1;
     for (int b = 0; b < n / d; ++b) unstrip_block(lattice, sym + b * d, lattice == HQO_E8 ? cos[b] : 0, v + b * d);
-    return 1;
+    return L;
 }
 
 /* Parse the chunked stream to codes; tiles laid out as in hqo_encode.  Returns status bits. */
@@ -667,18 +699,24 @@ uint32_t hqo_parse(const uint16_t* meta, const uint32_t* chunk_word, const uint3
     const int64_t nwords = chunk_word[NT * RB];
     uint32_t status = 0;
     int64_t c = 0;
+    bitr_t rd = {bits, nwords, 0};
     for (int64_t jt = 0; jt < NT; ++jt)
         for (int64_t rb = 0; rb < RB; ++rb, ++c) {
-            bitr_t rd = {bits, nwords, (int64_t)chunk_word[c] * 32, 0};
+            int64_t pos = (int64_t)chunk_word[c] * 32;
             int64_t r_end = (rb + 1) * 32 < rows ? (rb + 1) * 32 : rows;
             for (int64_t r = rb * 32; r < r_end; ++r) {
                 int64_t t = jt * rows + r;
-                if (!parse_tile(&rd, n, lattice, meta[t], v_out + t * n)) {
+                rd.bad = 0;
+                int64_t L = parse_tile(&rd, pos, n, lattice, meta[t], v_out + t * n);
+                if (L < 0) {
                     status |= HQO_ST_CORRUPT;
                     memset(v_out + t * n, 0, sizeof(int32_t) * (size_t)n);
+                    int k = meta[t] & 15;
+                    L = (lattice == HQO_E8 ? n / 8 : 0) + (int64_t)n * (k + 1) + (meta[t] >> 4);
                 }
+                pos += L;
             }
-            if (((rd.bitpos + 31) >> 5) != (int64_t)chunk_word[c + 1]) status |= HQO_ST_CORRUPT;
+            if (((pos + 31) >> 5) != (int64_t)chunk_word[c + 1]) status |= HQO_ST_CORRUPT;
         }
     return status;
 }
@@ -754,8 +792,8 @@ int64_t hqo_rice_tile(const int32_t* v, int n, int lattice, uint32_t* words, int
 
 int hqo_parse_tile(const uint32_t* words, int64_t nwords, int n, int lattice, uint16_t meta, int32_t* v, int64_t* bitlen)
 {
-    bitr_t rd = {words, nwords, 0, 0};
-    int ok = parse_tile(&rd, n, lattice, meta, v);
-    *bitlen = rd.bitpos;
-    return ok;
+    bitr_t rd = {words, nwords, 0};
+    int64_t L = parse_tile(&rd, 0, n, lattice, meta, v);
+    *bitlen = L;
+    return L >= 0;
 }

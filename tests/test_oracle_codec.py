@@ -47,10 +47,17 @@ def test_rice_round_trip_and_length(lattice, n):
 
 
 def test_rice_rejects_inconsistent_meta():
+    # a Rice parameter that disagrees with the stream makes the two halves miss each other; a
+    # sum q off by one only moves the meeting point of the halves (the format carries no
+    # checksum) but must still parse within the tile's bounds
     v = _random_codes(oracle.E8, 128, 7, 3.0)
     words, nbits, k, sumq = oracle.rice_tile(v, oracle.E8)
-    ok, _, _ = oracle.parse_tile(words, 128, oracle.E8, k | ((sumq + 1) << 4))
-    assert not ok
+    for bad in [(k + 1) | (sumq << 4), (k - 1) | (sumq << 4)]:
+        ok, _, _ = oracle.parse_tile(words, 128, oracle.E8, bad)
+        assert not ok
+    for bad in [k | ((sumq - 1) << 4), k | ((sumq + 1) << 4)]:
+        ok, back, blen = oracle.parse_tile(words, 128, oracle.E8, bad)
+        assert not ok or blen == nbits + ((bad >> 4) - sumq)
 
 
 def _reconstruct_numpy(code, v):
