@@ -1,0 +1,313 @@
+"""Benchmark: HyperQuant tile codec on B200, LLaMA-7B-shaped linear weights at 4 bps.
+
+Workload: a 4096x4096 and an 11008x4096 bf16 weight (Student-t(5), std 0.02, 1% of input channels
+x20), RHT tile 128, E8 lattice, step calibrated per matrix to 4.00 payload bits per scalar.
+One step = encode + decode of both matrices.  Inputs and codes rotate over three replicas so no
+launch reads data another launch left in the 126 MB L2 (each replica's bf16 input alone is
+124 MB): step k encodes replica k % 3 and decodes the codes of replica (k + 1) % 3, written
+two steps earlier.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  value = bf16 GB/s through encode + decode (bf16 input bytes of
+the batch / step time), summed over ranks; ranks are independent replicas (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "encode/decode GB/s (bf16 in) at 4 bps, % of HBM roofline; bps & MSE vs oracle"
+SHAPES = [(4096, 4096), (11008, 4096)]
+TILE, BPS, SEED = 128, 4.0, 1
+REPLICAS = 3
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def make_inputs():
+    from post_quantization_tile_b200 import workloads as W
+    return [W.llama_weight(r, c, seed=SEED + i) for i, (r, c) in enumerate(SHAPES)]
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle arm (bounded sample)
+# ------------------------------------------------------------------------------------------------
+def oracle_sample(inputs, rows_per_matrix: int, steps: int):
+    import oracle
+    t_total, elems = 0.0, 0
+    for _ in range(steps):
+        for x in inputs:
+            xs = np.ascontiguousarray(x[:rows_per_matrix])
+            t0 = time.perf_counter()
+            code = oracle.encode(xs, TILE, oracle.E8, 0.28, SEED)
+            oracle.decode(code)
+            t_total += time.perf_counter() - t0
+            elems += xs.size
+    gbs = elems * 2 / t_total / 1e9
+    return gbs, t_total, elems
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inputs = make_inputs()
+    rows = 64
+    oracle_sample(inputs, rows, max(1, args.warmup // 3))
+    gbs, secs, elems = oracle_sample(inputs, rows, args.steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "llama7b_linear_4096x4096+11008x4096_bf16_E8_n128_4bps",
+                   "sample": f"first {rows} rows of each matrix per step"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} rows x 4096 of each matrix per step, {args.steps} steps"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import post_quantization_tile_b200 as hq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    host = make_inputs()
+    xs = [[torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).to(dev) for h in host] for _ in range(REPLICAS)]
+    bf16_bytes = sum(r * c * 2 for r, c in SHAPES)
+
+    # step per matrix for 4.00 bps payload (count-only encodes, setup)
+    steps_beta = [hq.calibrate_step(xs[0][i], TILE, hq.E8, BPS, seed=SEED) for i in range(len(SHAPES))]
+    codes = [[hq.encode(xs[r][i], TILE, hq.E8, steps_beta[i], seed=SEED) for i in range(len(SHAPES))]
+             for r in range(REPLICAS)]
+    outs = [torch.empty(r, c, dtype=torch.bfloat16, device=dev) for r, c in SHAPES]
+    import ctypes
+    prm = hq.params(TILE, hq.E8, 0.3)
+    ws = hq.Workspace(max(hq.lib().hq_workspace_bytes(r, c, ctypes.byref(prm)) for r, c in SHAPES), device=dev)
+    torch.cuda.synchronize()
+    payload_bps = [codes[0][i].payload_bps() for i in range(len(SHAPES))]
+    total_bps = [codes[0][i].total_bps() for i in range(len(SHAPES))]
+    code_bytes = [4 * codes[0][i].total_words() + 4 * codes[0][i].scale.numel() +
+                  4 * codes[0][i].chunk_word.numel() for i in range(len(SHAPES))]
+
+    # MSE vs bf16 input for the quality fields (untimed)
+    mse = []
+    for i in range(len(SHAPES)):
+        y = hq.decode(codes[0][i], dtype=torch.float32, ws=ws)
+        xf = xs[0][i].float()
+        mse.append(float(((y - xf) ** 2).mean().item() / (xf ** 2).mean().item()))
+
+    enc_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps * len(SHAPES))]
+    dec_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps * len(SHAPES))]
+
+    def step(k, record=None):
+        r = k % REPLICAS
+        rd = (k + 1) % REPLICAS
+        for i in range(len(SHAPES)):
+            if record is not None:
+                enc_ev[record * len(SHAPES) + i][0].record(stream)
+            hq.encode(xs[r][i], TILE, hq.E8, steps_beta[i], seed=SEED, out=codes[r][i], ws=ws)
+            if record is not None:
+                enc_ev[record * len(SHAPES) + i][1].record(stream)
+        for i in range(len(SHAPES)):
+            if record is not None:
+                dec_ev[record * len(SHAPES) + i][0].record(stream)
+            hq.decode(codes[rd][i], out=outs[i], ws=ws)
+            if record is not None:
+                dec_ev[record * len(SHAPES) + i][1].record(stream)
+
+    for k in range(max(3, args.warmup)):
+        step(k)
+    st, _ = hq.status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for k in range(args.steps):
+            step(args.warmup + k, record=k)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    enc_ms = [statistics.mean(enc_ev[k * len(SHAPES) + i][0].elapsed_time(enc_ev[k * len(SHAPES) + i][1])
+                              for k in range(args.steps)) for i in range(len(SHAPES))]
+    dec_ms = [statistics.mean(dec_ev[k * len(SHAPES) + i][0].elapsed_time(dec_ev[k * len(SHAPES) + i][1])
+                              for k in range(args.steps)) for i in range(len(SHAPES))]
+
+    # e2e through the public API with host buffers: pinned H2D of the inputs, encode, decode,
+    # D2H of the reconstruction, every step
+    pinned_in = [torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).pin_memory() for h in host]
+    pinned_out = [torch.empty(r, c, dtype=torch.bfloat16).pin_memory() for r, c in SHAPES]
+    e2e_steps = max(2, min(args.steps, 5))
+    for k in range(e2e_steps + 1):
+        if k == 1:
+            torch.cuda.synchronize()
+            e0 = time.perf_counter()
+            c0 = torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+        for i in range(len(SHAPES)):
+            xs[0][i].copy_(pinned_in[i], non_blocking=True)
+            hq.encode(xs[0][i], TILE, hq.E8, steps_beta[i], seed=SEED, out=codes[0][i], ws=ws)
+            hq.decode(codes[0][i], out=outs[i], ws=ws)
+            pinned_out[i].copy_(outs[i], non_blocking=True)
+    c1 = torch.cuda.Event(enable_timing=True)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = c0.elapsed_time(c1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    st, _ = hq.status(ws)
+
+    peak, peak_kind = load_peaks()
+    # dominant kernel: the larger of encode / decode of the 11008x4096 matrix
+    i_big = 1
+    enc_bytes = SHAPES[i_big][0] * SHAPES[i_big][1] * 2 + code_bytes[i_big]
+    dec_bytes = code_bytes[i_big] + SHAPES[i_big][0] * SHAPES[i_big][1] * 2
+    if enc_ms[i_big] >= dec_ms[i_big]:
+        kname, kms, kbytes = "encode", enc_ms[i_big], enc_bytes
+    else:
+        kname, kms, kbytes = "decode", dec_ms[i_big], dec_bytes
+    achieved = kbytes / (kms * 1e-3) / 1e9
+    value = world * bf16_bytes / (ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 96
+        gbs, secs, elems = oracle_sample(host, rows, 2)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"encode+decode of the first {rows} rows of each matrix, 2 passes ({elems} scalars, {secs:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "llama7b_linear_4096x4096+11008x4096_bf16_E8_n128_4bps",
+                       "shapes": SHAPES, "tile": TILE, "lattice": "E8", "target_bps": BPS,
+                       "step": steps_beta, "payload_bps": payload_bps, "total_bps": total_bps, "nmse": mse,
+                       "l2": "inputs and codes rotate over 3 replicas (124 MB bf16 each), no L2 reuse across launches",
+                       "parallelism": f"replicas{world}"},
+            "encode_gbs": [SHAPES[i][0] * SHAPES[i][1] * 2 / (enc_ms[i] * 1e-3) / 1e9 for i in range(len(SHAPES))],
+            "decode_gbs": [SHAPES[i][0] * SHAPES[i][1] * 2 / (dec_ms[i] * 1e-3) / 1e9 for i in range(len(SHAPES))],
+            "encode_ms": enc_ms, "decode_ms": dec_ms,
+            "roofline": {"bound": "hbm", "kernel": f"{kname} 11008x4096", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * bf16_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": bf16_bytes, "d2h_bytes_per_step": bf16_bytes},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk.summary(),
+            "status": st,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

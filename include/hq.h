@@ -1,0 +1,192 @@
+/*
+ * hq.h -- C ABI of the HyperQuant tile codec for NVIDIA B200 (sm_100a).
+ *
+ * The codec is the data-parallel path of "HyperQuant: A Rate-Distortion-Optimal Quantization
+ * Pipeline for Large Language and Diffusion Models" (Domb, Sackstein, Solberg; summarised on
+ * gist.science, Technical Summary, "Methodology: The HyperQuant Pipeline"):
+ *   step 1  per-tile Randomized Hadamard Transform  RHT_n(x) = H_n D x,
+ *   step 2  nearest-point quantization to the E8, D4, A2 or Z lattice (integer embedding),
+ *   step 3  lossless bit-stripping and per-tile Rice coding of the lattice indices,
+ *   step 4  subtractive dither U ~ Uniform(V(Lambda)) on the KV path, so inner products stay
+ *           unbiased per vector.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument named as a device pointer must point to memory of the current CUDA
+ *     device; the library never allocates, frees or keeps global state, and never synchronises
+ *     except in hq_status_read.  All work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and the call returns at once.
+ *   - The synchronous return value reports argument errors (HQ_ERR_ARG, HQ_ERR_UNSUPPORTED) and
+ *     launch failures (HQ_ERR_CUDA).  Errors found by the kernels (non-finite input, too small
+ *     an output, a corrupt stream, a bounded wait that ran out) are written to a status word in
+ *     the caller's workspace `ws` and read with hq_status_read.
+ *   - The workspace is caller-owned device memory of at least hq_workspace_bytes(...) bytes,
+ *     256-byte aligned.  Calls that share a workspace must not overlap on the GPU.
+ *   - Tiles.  A weight W[rows, cols] is row-major; tile (r, jt) is W[r, jt*n : (jt+1)*n], along
+ *     the input-channel axis.  Tile index t = jt*rows + r.  Chunk (jt, rb) holds the tiles of
+ *     rows [32 rb, min(32 rb + 32, rows)) of tile column jt; chunk index c = jt*RB + rb with
+ *     RB = ceil(rows / 32).  Each chunk starts on a 32-bit word; chunk_word[c] is its word
+ *     offset in `bits`, chunk_word[C] the total number of words.
+ *   - A KV tensor [B, H, S, D] (contiguous) is coded as rows = B*H*S, cols = n = D: one tile per
+ *     head vector, the random signs shared by every head and token (per-layer seed), the dither
+ *     fresh per (b, h, s) and D4 block.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HQ_FORMAT_VERSION 1
+
+/* Lattices of Methodology step 2. */
+typedef enum { HQ_Z = 0, HQ_A2 = 1, HQ_D4 = 2, HQ_E8 = 3 } hq_lattice_t;
+
+/* Element types of the dense side (input of encode, output of decode). */
+typedef enum { HQ_BF16 = 0, HQ_F32 = 1 } hq_dtype_t;
+
+typedef enum {
+    HQ_OK = 0,
+    HQ_ERR_ARG = 1,          /* bad argument (null pointer, size, alignment, range)          */
+    HQ_ERR_UNSUPPORTED = 2,  /* valid but not provided (e.g. KV dither on a lattice != D4)  */
+    HQ_ERR_CAPACITY = 3,     /* device: `bits` too small; detail = words needed              */
+    HQ_ERR_NONFINITE = 4,    /* device: a tile held NaN/Inf (coded as zeros); detail = count */
+    HQ_ERR_CORRUPT = 5,      /* device: stream inconsistent with meta / chunk_word            */
+    HQ_ERR_TIMEOUT = 6,      /* device: a bounded wait on another block ran out               */
+    HQ_ERR_RANGE = 7,        /* value outside a representable range                          */
+    HQ_ERR_CUDA = 8          /* a CUDA runtime call failed                                    */
+} hq_status_t;
+
+/*
+ * Codec parameters.
+ *   tile    n in {64, 128, 256}, the RHT tile length (Methodology step 1, "e.g. 128").
+ *   lattice one of hq_lattice_t (Methodology step 2).
+ *   step    beta > 0: lattice units per normalised coefficient.  A tile with RMS s is coded as
+ *           u = H_n D x / (sqrt(n) * bf16(s) * beta).  Allowed range [2^-8, 2^6]; the range
+ *           keeps every code below 2^15 in magnitude and every Rice parameter below 10.
+ *           0 selects hq_step_for_rate(lattice, tile, bps).
+ *   bps     target payload bits per scalar, used only when step == 0.
+ *   seed    64-bit seed of the sign diagonal D (and of the KV dither).
+ */
+typedef struct {
+    int32_t tile;
+    int32_t lattice;
+    float step;
+    float bps;
+    uint64_t seed;
+} hq_params_t;
+
+/*
+ * An encoded tensor.  The caller owns the four device arrays and the struct; encode fills them
+ * and the scalar fields, decode reads them.
+ *   rows, cols  dense shape (KV: rows = B*H*S, cols = D)
+ *   kv_S        S of the KV layout (dither counter); 0 for weights
+ *   p           parameters with the step resolved (never 0 after encode)
+ *   kv          1 for the KV path (dithered D4), else 0
+ *   version     HQ_FORMAT_VERSION
+ *   scale       [T] bf16 bit patterns of the per-tile RMS (0 = all-zero tile)
+ *   meta        [T] k | (sum q << 4): the tile's Rice parameter and unary total
+ *   chunk_word  [C + 1] word offset of each chunk, [C] = total words
+ *   bits        [cap_words] the bitstream; cap_words >= hq_encode_bound_words(...) always
+ *               suffices, a smaller buffer yields HQ_ERR_CAPACITY with the needed size
+ */
+typedef struct {
+    int64_t rows, cols;
+    int64_t kv_S;
+    hq_params_t p;
+    int32_t kv;
+    int32_t version;
+    uint16_t* scale;
+    uint16_t* meta;
+    uint32_t* chunk_word;
+    uint32_t* bits;
+    int64_t cap_words;
+} hq_code_t;
+
+/* Number of tiles T and chunks C of a rows x cols tensor with tile length n; -1 if invalid. */
+int64_t hq_num_tiles(int64_t rows, int64_t cols, int32_t tile);
+int64_t hq_num_chunks(int64_t rows, int64_t cols, int32_t tile);
+
+/* Worst-case bitstream words for any finite input (a multiple of 4); -1 if invalid. */
+int64_t hq_encode_bound_words(int64_t rows, int64_t cols, const hq_params_t* p);
+
+/* Workspace bytes needed by any call on a rows x cols tensor with these parameters. */
+size_t hq_workspace_bytes(int64_t rows, int64_t cols, const hq_params_t* p);
+
+/*
+ * Step for a target payload rate from the high-resolution approximation of an entropy-coded
+ * lattice quantizer on Gaussian coefficients (RHT output, Methodology step 1 "approximately
+ * Gaussian"): beta = 2^(h - R) / V^(1/d) with h = log2(sqrt(2 pi e)) and V, d the cell volume
+ * and dimension of the lattice.  A starting point; hq_encode_count gives the realised rate for
+ * an exact search ("within ~0.01 bps of any target", Methodology step 3).
+ */
+float hq_step_for_rate(int32_t lattice, int32_t tile, float bps);
+
+/*
+ * Encode a weight (Methodology steps 1-3).
+ *   x      device, [rows, cols] row-major, dtype elements, 16-byte aligned base, cols % tile == 0
+ *   out    host struct: scale/meta/chunk_word/bits/cap_words set by the caller, the rest filled
+ *   ws     device workspace (hq_workspace_bytes), ws_bytes its size
+ * Device errors: HQ_ERR_NONFINITE (tile coded as zeros), HQ_ERR_CAPACITY, HQ_ERR_TIMEOUT.
+ */
+hq_status_t hq_encode(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                      hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Decode a weight: y[rows, cols] (device, dtype, 16-byte aligned) = D H_n p * (bf16(s) beta /
+ * sqrt(n)) per tile, p the lattice point; bf16 output is the binary32 value rounded to nearest
+ * even.  Device errors: HQ_ERR_CORRUPT (tile written as zeros).
+ */
+hq_status_t hq_decode(const hq_code_t* code, void* y, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Encode a KV tensor kv[B, H, S, D] (device, contiguous) with D == p->tile and the dithered D4
+ * lattice (Methodology step 4): for each D4 block the dither U, uniform on the Voronoi cell of
+ * D4, is added before quantization.  Other lattices return HQ_ERR_UNSUPPORTED.
+ */
+hq_status_t hq_kv_encode(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D,
+                         const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Decode a KV tensor: the dither is regenerated and subtracted before the inverse transform. */
+hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/*
+ * Lattice quantization, bit-stripping and Rice coding of caller-given normalised coefficients
+ * (Methodology steps 2-3, and step 4's dither when kv = 1): u[tiles, tile] fp32 device array in
+ * lattice units, one tile per row, chunks of 32 consecutive rows.  v_out (device, optional,
+ * int32 [tiles, tile]) receives the integer codes: Z and D4 the point itself, E8 twice the point,
+ * A2 (P, Q) with the point at (P/2, Q sqrt(3)/2).  For kv, row t is token (t / kv_S, t % kv_S).
+ * out->scale may be NULL.  This entry point checks codes and bitstreams bit for bit.
+ */
+hq_status_t hq_quantize_coeffs(const float* u, int64_t tiles, const hq_params_t* p, int32_t kv, int64_t kv_S,
+                               int32_t* v_out, hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Count-only encode: writes the total payload bits of encoding x (no bitstream) to
+ * *bits_out (device uint64).  Used to search the step for an exact rate.
+ */
+hq_status_t hq_encode_count(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                            int32_t kv, int64_t kv_S, uint64_t* bits_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then read the status word of `ws`: returns HQ_OK or the most severe
+ * device error (TIMEOUT, CORRUPT, CAPACITY, NONFINITE in that order) and, if detail is not NULL,
+ * its detail value (capacity: words needed; non-finite: tiles affected).
+ */
+hq_status_t hq_status_read(const void* ws, void* stream, int64_t* detail);
+
+/* Static description of a status code. */
+const char* hq_status_str(hq_status_t s);
+
+/* HQ_FORMAT_VERSION of the built library. */
+int32_t hq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

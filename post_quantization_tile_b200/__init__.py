@@ -1,1 +1,319 @@
-"""HyperQuant tile codec for NVIDIA B200 (sm_100a): Python binding over the C-ABI library."""
+"""HyperQuant tile codec for NVIDIA B200 (sm_100a): Python binding over the C-ABI library.
+
+Every step of the codec runs in the CUDA kernels of ``libhq.so`` (built in-tree by
+``post_quantization_tile_b200.build``).  This module only marshals torch device tensors, the
+current CUDA stream and the parameter structs into the C calls declared in ``include/hq.h``.
+There is no CPU fallback: without the library or a CUDA device every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+Z, A2, D4, E8 = 0, 1, 2, 3
+LATTICES = {"Z": Z, "A2": A2, "D4": D4, "E8": E8}
+BF16, F32 = 0, 1
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "capacity", 4: "non-finite input",
+          5: "corrupt stream", 6: "timeout", 7: "range", 8: "CUDA error"}
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhq.so")
+
+
+class HQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)} (status {code})")
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("tile", ctypes.c_int32), ("lattice", ctypes.c_int32), ("step", ctypes.c_float),
+                ("bps", ctypes.c_float), ("seed", ctypes.c_uint64)]
+
+
+class CodeStruct(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("kv_S", ctypes.c_int64), ("p", Params),
+                ("kv", ctypes.c_int32), ("version", ctypes.c_int32), ("scale", ctypes.c_void_p),
+                ("meta", ctypes.c_void_p), ("chunk_word", ctypes.c_void_p), ("bits", ctypes.c_void_p),
+                ("cap_words", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libhq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m post_quantization_tile_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+        L.hq_num_tiles.argtypes = [i64, i64, i32]
+        L.hq_num_tiles.restype = i64
+        L.hq_num_chunks.argtypes = [i64, i64, i32]
+        L.hq_num_chunks.restype = i64
+        L.hq_encode_bound_words.argtypes = [i64, i64, ctypes.POINTER(Params)]
+        L.hq_encode_bound_words.restype = i64
+        L.hq_workspace_bytes.argtypes = [i64, i64, ctypes.POINTER(Params)]
+        L.hq_workspace_bytes.restype = ctypes.c_size_t
+        L.hq_step_for_rate.argtypes = [i32, i32, ctypes.c_float]
+        L.hq_step_for_rate.restype = ctypes.c_float
+        L.hq_encode.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), ctypes.POINTER(CodeStruct), P,
+                                ctypes.c_size_t, P]
+        L.hq_decode.argtypes = [ctypes.POINTER(CodeStruct), P, i32, P, ctypes.c_size_t, P]
+        L.hq_kv_encode.argtypes = [P, i32, i64, i64, i64, i64, ctypes.POINTER(Params), ctypes.POINTER(CodeStruct), P,
+                                   ctypes.c_size_t, P]
+        L.hq_kv_decode.argtypes = [ctypes.POINTER(CodeStruct), P, i32, P, ctypes.c_size_t, P]
+        L.hq_quantize_coeffs.argtypes = [P, i64, ctypes.POINTER(Params), i32, i64, P, ctypes.POINTER(CodeStruct), P,
+                                         ctypes.c_size_t, P]
+        L.hq_encode_count.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, P, P, ctypes.c_size_t, P]
+        L.hq_status_read.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
+        L.hq_status_str.argtypes = [i32]
+        L.hq_status_str.restype = ctypes.c_char_p
+        L.hq_version.restype = i32
+        for f in ["hq_encode", "hq_decode", "hq_kv_encode", "hq_kv_decode", "hq_quantize_coeffs", "hq_encode_count",
+                  "hq_status_read"]:
+            getattr(L, f).restype = i32
+        _lib = L
+    return _lib
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise HQError(code, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError("dense tensors must be bfloat16 or float32")
+
+
+def _require_cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def params(tile: int = 128, lattice: int | str = E8, step: float = 0.0, bps: float = 4.0, seed: int = 0) -> Params:
+    if isinstance(lattice, str):
+        lattice = LATTICES[lattice]
+    return Params(int(tile), int(lattice), float(step), float(bps), int(seed) & ((1 << 64) - 1))
+
+
+class Workspace:
+    """Device scratch for one call at a time (status word, work counter, look-back states)."""
+
+    def __init__(self, nbytes: int, device=None):
+        self.nbytes = max(256, (int(nbytes) + 255) // 256 * 256)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device or "cuda")
+
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int) -> Workspace:
+    dev = torch.cuda.current_device()
+    ws = _ws_cache.get(dev)
+    if ws is None or ws.nbytes < nbytes:
+        ws = Workspace(max(nbytes, 1 << 20), device=f"cuda:{dev}")
+        _ws_cache[dev] = ws
+    return ws
+
+
+@dataclass
+class Code:
+    """An encoded tensor: device arrays plus the header the decoder needs."""
+    rows: int
+    cols: int
+    p: Params
+    kv: int
+    kv_S: int
+    scale: torch.Tensor       # uint16 view of bf16 per-tile RMS  [T]   (stored as int16)
+    meta: torch.Tensor        # [T]  k | (sum q << 4)              (stored as int16)
+    chunk_word: torch.Tensor  # [C+1] word offsets                 (stored as int32)
+    bits: torch.Tensor        # [cap] bitstream words              (stored as int32)
+
+    def struct(self) -> CodeStruct:
+        return CodeStruct(self.rows, self.cols, self.kv_S, self.p, self.kv, lib().hq_version(),
+                          self.scale.data_ptr(), self.meta.data_ptr(), self.chunk_word.data_ptr(),
+                          self.bits.data_ptr(), self.bits.numel())
+
+    @property
+    def step(self) -> float:
+        return float(self.p.step)
+
+    def total_words(self) -> int:
+        return int(self.chunk_word[-1].item()) & 0xFFFFFFFF
+
+    def payload_bits(self) -> int:
+        m = self.meta.to(torch.int64) & 0xFFFF
+        k = m & 15
+        sq = m >> 4
+        cos = self.p.tile // 8 if self.p.lattice == E8 else 0
+        return int((cos + self.p.tile * (k + 1) + sq).sum().item())
+
+    def payload_bps(self) -> float:
+        return self.payload_bits() / float(self.rows * self.cols)
+
+    def total_bps(self) -> float:
+        C = self.chunk_word.numel() - 1
+        T = self.scale.numel()
+        return 8.0 * (4 * self.total_words() + 4 * T + 4 * (C + 1)) / float(self.rows * self.cols)
+
+
+def alloc_code(rows: int, cols: int, p: Params, device=None, cap_words: int | None = None) -> Code:
+    L = lib()
+    T = L.hq_num_tiles(rows, cols, p.tile)
+    C = L.hq_num_chunks(rows, cols, p.tile)
+    if T < 0:
+        raise HQError(1, "alloc_code")
+    bound = L.hq_encode_bound_words(rows, cols, ctypes.byref(p))
+    cap = bound if cap_words is None else int(cap_words)
+    dev = device or "cuda"
+    return Code(rows, cols, p, 0, 0,
+                torch.zeros(T, dtype=torch.int16, device=dev), torch.zeros(T, dtype=torch.int16, device=dev),
+                torch.zeros(C + 1, dtype=torch.int32, device=dev), torch.zeros(cap, dtype=torch.int32, device=dev))
+
+
+def _fill(code: Code, cs: CodeStruct):
+    code.rows, code.cols, code.kv_S, code.kv = cs.rows, cs.cols, cs.kv_S, cs.kv
+    code.p = Params(cs.p.tile, cs.p.lattice, cs.p.step, cs.p.bps, cs.p.seed)
+
+
+def encode(x: torch.Tensor, tile: int = 128, lattice: int | str = E8, step: float = 0.0, bps: float = 4.0,
+           seed: int = 0, out: Code | None = None, ws: Workspace | None = None) -> Code:
+    """Encode a 2-D bf16/fp32 CUDA tensor (Methodology steps 1-3)."""
+    _require_cuda(x, "x")
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows, cols]")
+    p = params(tile, lattice, step, bps, seed)
+    rows, cols = x.shape
+    code = out if out is not None else alloc_code(rows, cols, p, device=x.device)
+    L = lib()
+    need = L.hq_workspace_bytes(rows, cols, ctypes.byref(p))
+    w = ws or workspace(need)
+    cs = code.struct()
+    _check(L.hq_encode(_ptr(x), _dtype_code(x), rows, cols, ctypes.byref(p), ctypes.byref(cs), w.ptr(), w.nbytes,
+                       _stream()), "hq_encode")
+    _fill(code, cs)
+    code.ws = w
+    return code
+
+
+def decode(code: Code, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None,
+           ws: Workspace | None = None) -> torch.Tensor:
+    """Decode to a [rows, cols] CUDA tensor (bf16 = binary32 result rounded to nearest even)."""
+    y = out if out is not None else torch.empty(code.rows, code.cols, dtype=dtype, device=code.bits.device)
+    _require_cuda(y, "out")
+    L = lib()
+    w = ws or workspace(4096)
+    cs = code.struct()
+    fn = L.hq_kv_decode if code.kv else L.hq_decode
+    _check(fn(ctypes.byref(cs), _ptr(y), _dtype_code(y), w.ptr(), w.nbytes, _stream()), "hq_decode")
+    code.ws = w
+    return y
+
+
+def kv_encode(kv: torch.Tensor, step: float = 0.0, bps: float = 4.0, seed: int = 0, lattice: int | str = D4,
+              out: Code | None = None, ws: Workspace | None = None) -> Code:
+    """Encode a KV tensor [B, H, S, D] with the dithered D4 lattice (Methodology step 4)."""
+    _require_cuda(kv, "kv")
+    if kv.dim() != 4:
+        raise ValueError("kv must be [B, H, S, D]")
+    B, H, S, D = kv.shape
+    p = params(D, lattice, step, bps, seed)
+    rows = B * H * S
+    code = out if out is not None else alloc_code(rows, D, p, device=kv.device)
+    L = lib()
+    w = ws or workspace(L.hq_workspace_bytes(rows, D, ctypes.byref(p)))
+    cs = code.struct()
+    _check(L.hq_kv_encode(_ptr(kv), _dtype_code(kv), B, H, S, D, ctypes.byref(p), ctypes.byref(cs), w.ptr(), w.nbytes,
+                          _stream()), "hq_kv_encode")
+    _fill(code, cs)
+    code.ws = w
+    return code
+
+
+def kv_decode(code: Code, shape, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None,
+              ws: Workspace | None = None) -> torch.Tensor:
+    y = decode(code, dtype=dtype, out=out, ws=ws)
+    return y.view(*shape)
+
+
+def quantize_coeffs(u: torch.Tensor, tile: int, lattice: int | str, seed: int = 0, kv: bool = False, kv_S: int = 0,
+                    ws: Workspace | None = None):
+    """Lattice + strip + Rice on normalised fp32 coefficients u[tiles, tile]; returns (codes, Code)."""
+    _require_cuda(u, "u")
+    if u.dtype != torch.float32 or u.dim() != 2 or u.shape[1] != tile:
+        raise ValueError("u must be float32 [tiles, tile]")
+    p = params(tile, lattice, 1.0, 0.0, seed)
+    tiles = u.shape[0]
+    code = alloc_code(tiles, tile, p, device=u.device)
+    v = torch.empty(tiles, tile, dtype=torch.int32, device=u.device)
+    L = lib()
+    w = ws or workspace(L.hq_workspace_bytes(tiles, tile, ctypes.byref(p)))
+    cs = code.struct()
+    _check(L.hq_quantize_coeffs(_ptr(u), tiles, ctypes.byref(p), int(kv), int(kv_S), _ptr(v), ctypes.byref(cs),
+                                w.ptr(), w.nbytes, _stream()), "hq_quantize_coeffs")
+    _fill(code, cs)
+    code.ws = w
+    return v, code
+
+
+def encode_count(x: torch.Tensor, tile: int, lattice: int | str, step: float, seed: int = 0, kv: bool = False,
+                 kv_S: int = 0, ws: Workspace | None = None) -> torch.Tensor:
+    """Total payload bits of encoding x at this step, as a device int64 scalar (no bitstream)."""
+    _require_cuda(x, "x")
+    rows, cols = (x.shape[0] * x.shape[1] * x.shape[2], x.shape[3]) if x.dim() == 4 else x.shape
+    p = params(tile, lattice, step, 0.0, seed)
+    L = lib()
+    w = ws or workspace(L.hq_workspace_bytes(rows, cols, ctypes.byref(p)))
+    outb = torch.zeros(1, dtype=torch.int64, device=x.device)
+    _check(L.hq_encode_count(_ptr(x), _dtype_code(x), rows, cols, ctypes.byref(p), int(kv), int(kv_S), _ptr(outb),
+                             w.ptr(), w.nbytes, _stream()), "hq_encode_count")
+    return outb
+
+
+def calibrate_step(x: torch.Tensor, tile: int, lattice: int | str, target_bps: float, seed: int = 0,
+                   kv: bool = False, kv_S: int = 0, iters: int = 24) -> float:
+    """Bisection on log(step) with count-only encodes so the payload rate hits target_bps
+    ("within ~0.01 bps of any target", Methodology step 3)."""
+    import math
+    n = x.numel()
+    lo, hi = math.log(2.0 ** -8), math.log(2.0 ** 6)
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        b = float(torch.tensor(math.exp(mid), dtype=torch.float32))
+        r = encode_count(x, tile, lattice, b, seed, kv, kv_S).item() / n
+        if r > target_bps:
+            lo = mid
+        else:
+            hi = mid
+    return float(torch.tensor(math.exp(0.5 * (lo + hi)), dtype=torch.float32))
+
+
+def status(ws: Workspace) -> tuple[int, int]:
+    """Synchronise the current stream and read the device status word: (code, detail)."""
+    d = ctypes.c_int64(0)
+    code = lib().hq_status_read(ws.ptr(), _stream(), ctypes.byref(d))
+    return int(code), int(d.value)

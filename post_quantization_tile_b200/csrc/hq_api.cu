@@ -1,0 +1,370 @@
+// hq_api.cu -- C ABI of the HyperQuant tile codec (declarations and contracts in include/hq.h):
+// argument checks, TMA tensor maps, workspace set-up and kernel launches.  No allocation, no
+// synchronisation except in hq_status_read.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/hq.h"
+#include "hq_common.cuh"
+#include "hq_decode.cuh"
+#include "hq_encode.cuh"
+#include "hq_launch.h"
+
+namespace hq {
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 1;
+    return n;
+}
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D map over a row-major [rows, cols] tensor; box = [box_rows][128 bytes], 128-byte swizzle,
+// out-of-range rows read as zero
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int es, int box_rows)
+{
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const CUtensorMapDataType dt = es == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * (cuuint64_t)es};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool valid_tile(int32_t n) { return n == 64 || n == 128 || n == 256; }
+
+struct Geometry {
+    int64_t T, C, RB, items, IB;
+    int TI;
+};
+
+bool geometry(int64_t rows, int64_t cols, int32_t n, Geometry& g)
+{
+    if (!valid_tile(n) || rows < 1 || cols < n || cols % n) return false;
+    if (rows > (int64_t)1 << 31 || cols > (int64_t)1 << 31) return false;
+    const int64_t NT = cols / n;
+    g.TI = kThreads / tpt_for(n);
+    g.RB = (rows + kChunkTiles - 1) / kChunkTiles;
+    g.C = NT * g.RB;
+    g.T = NT * rows;
+    g.IB = (rows + g.TI - 1) / g.TI;
+    g.items = NT * g.IB;
+    return true;
+}
+
+int64_t bound_words(int64_t rows, int64_t cols, int32_t n)
+{
+    Geometry g;
+    if (!geometry(rows, cols, n, g)) return -1;
+    const int64_t lmax = n / 8 + 16 * (int64_t)n + 2 * (int64_t)n;
+    const int64_t words = (g.T * lmax + 31) / 32 + g.C + 8;
+    return (words + 3) & ~(int64_t)3;
+}
+
+size_t ws_bytes_for(int64_t rows, int64_t cols, int32_t n)
+{
+    Geometry g;
+    if (!geometry(rows, cols, n, g)) return 0;
+    return sizeof(WsHeader) + (size_t)g.items * 8u;
+}
+
+bool resolve_params(const hq_params_t* p, hq_params_t& out)
+{
+    if (!p || !valid_tile(p->tile) || p->lattice < HQ_Z || p->lattice > HQ_E8) return false;
+    out = *p;
+    if (out.step == 0.0f) {
+        if (!(p->bps >= 1.0f && p->bps <= 8.0f)) return false;
+        out.step = hq_step_for_rate(p->lattice, p->tile, p->bps);
+    }
+    return out.step >= 0.00390625f && out.step <= 64.0f && std::isfinite(out.step);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hq_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
+
+cudaError_t run_encode(int lattice, int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m,
+                       cudaStream_t st)
+{
+    switch (lattice) {
+    case HQ_Z: return launch_encode_z(n, kv, src, count, a, m, st);
+    case HQ_A2: return launch_encode_a2(n, kv, src, count, a, m, st);
+    case HQ_D4: return launch_encode_d4(n, kv, src, count, a, m, st);
+    default: return launch_encode_e8(n, kv, src, count, a, m, st);
+    }
+}
+
+cudaError_t run_decode(int lattice, int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st)
+{
+    switch (lattice) {
+    case HQ_Z: return launch_decode_z(n, kv, dst, a, m, st);
+    case HQ_A2: return launch_decode_a2(n, kv, dst, a, m, st);
+    case HQ_D4: return launch_decode_d4(n, kv, dst, a, m, st);
+    default: return launch_decode_e8(n, kv, dst, a, m, st);
+    }
+}
+
+// common body of the encode entry points (src 0/1 dense input, src 2 coefficients)
+hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, const hq_params_t* p, int32_t kv,
+                          int64_t kv_S, int32_t* v_out, hq_code_t* out, unsigned long long* count_out, void* ws,
+                          size_t ws_bytes, void* stream)
+{
+    hq_params_t prm;
+    if (!resolve_params(p, prm)) return HQ_ERR_ARG;
+    Geometry g;
+    if (!geometry(rows, cols, prm.tile, g)) return HQ_ERR_ARG;
+    if (kv && prm.lattice != HQ_D4) return HQ_ERR_UNSUPPORTED;
+    if (kv && cols != prm.tile) return HQ_ERR_ARG;
+    if (src == 1 && prm.tile == 256) return HQ_ERR_UNSUPPORTED;
+    if (src == 2 && cols != prm.tile) return HQ_ERR_ARG;
+    if (!x || !aligned16(x) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
+    if (ws_bytes < ws_bytes_for(rows, cols, prm.tile)) return HQ_ERR_ARG;
+    const bool count = count_out != nullptr;
+    if (!count) {
+        if (!out || !out->meta || !out->chunk_word || !out->bits || out->cap_words < 1) return HQ_ERR_ARG;
+        if (src != 2 && !out->scale) return HQ_ERR_ARG;
+    }
+    if (bound_words(rows, cols, prm.tile) >= ((int64_t)1 << 32)) return HQ_ERR_RANGE;
+
+    const int es = src == 0 ? 2 : 4;
+    CUtensorMap map;
+    if (!make_map(&map, x, rows, cols, es, g.TI)) return HQ_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t clear = count ? sizeof(WsHeader) : sizeof(WsHeader) + (size_t)g.items * 8u;
+    cudaError_t e = cudaMemsetAsync(ws, 0, clear, st);
+    if (e != cudaSuccess) return HQ_ERR_CUDA;
+
+    EncodeArgs a{};
+    a.rows = rows;
+    a.cols = cols;
+    a.beta = prm.step;
+    a.seed = prm.seed;
+    a.kv_S = kv ? kv_S : 0;
+    a.items = g.items;
+    a.IB = g.IB;
+    a.RB = g.RB;
+    a.C = g.C;
+    if (!count) {
+        a.scale = out->scale;
+        a.meta = out->meta;
+        a.chunk_word = out->chunk_word;
+        a.bits = out->bits;
+        a.cap_words = out->cap_words;
+    }
+    a.v_out = v_out;
+    a.ws = static_cast<WsHeader*>(ws);
+    a.states = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + sizeof(WsHeader));
+    e = run_encode(prm.lattice, prm.tile, kv != 0, src, count, a, map, st);
+    if (e != cudaSuccess) return HQ_ERR_CUDA;
+    if (count) {
+        e = cudaMemcpyAsync(count_out, &a.ws->count_bits, sizeof(unsigned long long), cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return HQ_ERR_CUDA;
+    } else {
+        out->rows = rows;
+        out->cols = cols;
+        out->kv_S = kv ? kv_S : 0;
+        out->p = prm;
+        out->kv = kv ? 1 : 0;
+        out->version = HQ_FORMAT_VERSION;
+    }
+    return HQ_OK;
+}
+
+hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int32_t kv, void* ws, size_t ws_bytes,
+                          void* stream)
+{
+    if (!code || !y || !aligned16(y) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
+    if (code->version != HQ_FORMAT_VERSION || code->kv != kv) return HQ_ERR_ARG;
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    const hq_params_t& prm = code->p;
+    if (!valid_tile(prm.tile) || prm.lattice < HQ_Z || prm.lattice > HQ_E8) return HQ_ERR_ARG;
+    if (!(prm.step >= 0.00390625f && prm.step <= 64.0f)) return HQ_ERR_ARG;
+    if (kv && prm.lattice != HQ_D4) return HQ_ERR_UNSUPPORTED;
+    Geometry g;
+    if (!geometry(code->rows, code->cols, prm.tile, g)) return HQ_ERR_ARG;
+    if (!code->scale || !code->meta || !code->chunk_word || !code->bits || !aligned16(code->bits)) return HQ_ERR_ARG;
+    if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
+    const int es = dtype == HQ_BF16 ? 2 : 4;
+    CUtensorMap map;
+    if (!make_map(&map, y, code->rows, code->cols, es, g.TI)) return HQ_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
+    DecodeArgs a{};
+    a.rows = code->rows;
+    a.cols = code->cols;
+    a.beta = prm.step;
+    a.seed = prm.seed;
+    a.kv_S = code->kv_S;
+    a.items = g.items;
+    a.IB = g.IB;
+    a.RB = g.RB;
+    a.C = g.C;
+    a.scale = code->scale;
+    a.meta = code->meta;
+    a.chunk_word = code->chunk_word;
+    a.bits = code->bits;
+    a.cap_words = code->cap_words;
+    a.ws = static_cast<WsHeader*>(ws);
+    return cuda_status(run_decode(prm.lattice, prm.tile, kv != 0, es == 2 ? 0 : 1, a, map, st));
+}
+
+}  // namespace
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" {
+
+int64_t hq_num_tiles(int64_t rows, int64_t cols, int32_t tile)
+{
+    Geometry g;
+    return geometry(rows, cols, tile, g) ? g.T : -1;
+}
+
+int64_t hq_num_chunks(int64_t rows, int64_t cols, int32_t tile)
+{
+    Geometry g;
+    return geometry(rows, cols, tile, g) ? g.C : -1;
+}
+
+int64_t hq_encode_bound_words(int64_t rows, int64_t cols, const hq_params_t* p)
+{
+    if (!p) return -1;
+    return bound_words(rows, cols, p->tile);
+}
+
+size_t hq_workspace_bytes(int64_t rows, int64_t cols, const hq_params_t* p)
+{
+    if (!p) return 0;
+    const size_t b = ws_bytes_for(rows, cols, p->tile);
+    return (b + 255u) & ~(size_t)255u;
+}
+
+float hq_step_for_rate(int32_t lattice, int32_t tile, float bps)
+{
+    (void)tile;
+    // differential entropy of N(0,1) in bits and the cell volume / dimension of each lattice
+    const double h = 0.5 * std::log2(2.0 * 3.14159265358979323846 * 2.71828182845904523536);
+    double logV = 0.0;
+    int d = 1;
+    switch (lattice) {
+    case HQ_A2: logV = std::log2(std::sqrt(3.0) / 2.0); d = 2; break;
+    case HQ_D4: logV = 1.0; d = 4; break;
+    case HQ_E8: logV = 0.0; d = 8; break;
+    default: break;
+    }
+    return (float)std::exp2(h - (double)bps - logV / d);
+}
+
+hq_status_t hq_encode(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                      hq_code_t* out, void* ws, size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, 0, 0, nullptr, out, nullptr, ws, ws_bytes, stream);
+}
+
+hq_status_t hq_decode(const hq_code_t* code, void* y, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream)
+{
+    return decode_common(code, y, dtype, 0, ws, ws_bytes, stream);
+}
+
+hq_status_t hq_kv_encode(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D,
+                         const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (B < 1 || H < 1 || S < 1 || !p || D != p->tile) return HQ_ERR_ARG;
+    if (B * H > ((int64_t)1 << 32)) return HQ_ERR_ARG;
+    return encode_common(kv, dtype == HQ_BF16 ? 0 : 1, B * H * S, D, p, 1, S, nullptr, out, nullptr, ws, ws_bytes,
+                         stream);
+}
+
+hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream)
+{
+    return decode_common(code, kv, dtype, 1, ws, ws_bytes, stream);
+}
+
+hq_status_t hq_quantize_coeffs(const float* u, int64_t tiles, const hq_params_t* p, int32_t kv, int64_t kv_S,
+                               int32_t* v_out, hq_code_t* out, void* ws, size_t ws_bytes, void* stream)
+{
+    if (!p) return HQ_ERR_ARG;
+    hq_params_t q = *p;
+    if (q.step == 0.0f) q.step = 1.0f;  // unused on this path (coefficients are already normalised)
+    return encode_common(u, 2, tiles, p->tile, &q, kv, kv ? (kv_S > 0 ? kv_S : tiles) : 0, v_out, out, nullptr, ws,
+                         ws_bytes, stream);
+}
+
+hq_status_t hq_encode_count(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                            int32_t kv, int64_t kv_S, uint64_t* bits_out, void* ws, size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (!bits_out) return HQ_ERR_ARG;
+    return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, kv, kv ? kv_S : 0, nullptr, nullptr,
+                         reinterpret_cast<unsigned long long*>(bits_out), ws, ws_bytes, stream);
+}
+
+hq_status_t hq_status_read(const void* ws, void* stream, int64_t* detail)
+{
+    if (!ws) return HQ_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
+    WsHeader h;
+    if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return HQ_ERR_CUDA;
+    const hq_status_t order[] = {HQ_ERR_TIMEOUT, HQ_ERR_CORRUPT, HQ_ERR_CAPACITY, HQ_ERR_RANGE, HQ_ERR_NONFINITE};
+    for (hq_status_t s : order) {
+        if (h.status & (1u << s)) {
+            if (detail) *detail = s == HQ_ERR_CAPACITY ? (int64_t)h.needed : (s == HQ_ERR_NONFINITE ? (int64_t)h.nonfinite : 0);
+            return s;
+        }
+    }
+    if (detail) *detail = (int64_t)h.needed;
+    return HQ_OK;
+}
+
+const char* hq_status_str(hq_status_t s)
+{
+    switch (s) {
+    case HQ_OK: return "ok";
+    case HQ_ERR_ARG: return "invalid argument";
+    case HQ_ERR_UNSUPPORTED: return "unsupported combination";
+    case HQ_ERR_CAPACITY: return "bitstream buffer too small";
+    case HQ_ERR_NONFINITE: return "non-finite input (tile coded as zeros)";
+    case HQ_ERR_CORRUPT: return "corrupt code stream";
+    case HQ_ERR_TIMEOUT: return "bounded wait ran out";
+    case HQ_ERR_RANGE: return "value out of range";
+    case HQ_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+int32_t hq_version(void) { return HQ_FORMAT_VERSION; }
+
+}  // extern "C"

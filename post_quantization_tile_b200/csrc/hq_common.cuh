@@ -1,0 +1,317 @@
+// hq_common.cuh -- device helpers shared by the encode and decode kernels of the HyperQuant
+// tile codec: tile geometry, Philox4x32-10, TMA / mbarrier wrappers, bit writer and reader.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hq.h"
+
+namespace hq {
+
+// ------------------------------------------------------------------------------------------------
+// Kernel configuration
+// ------------------------------------------------------------------------------------------------
+constexpr int kThreads = 128;          // threads per block
+constexpr int kChunkTiles = 32;        // tiles per chunk (one warp scan)
+constexpr int kStages = 2;             // input pipeline depth
+constexpr uint32_t kSpinLimit = 1u << 22;  // bounded waits: polls before giving up
+
+// status word bits (1 << hq_status_t)
+constexpr uint32_t kStCapacity = 1u << HQ_ERR_CAPACITY;
+constexpr uint32_t kStNonfinite = 1u << HQ_ERR_NONFINITE;
+constexpr uint32_t kStCorrupt = 1u << HQ_ERR_CORRUPT;
+constexpr uint32_t kStTimeout = 1u << HQ_ERR_TIMEOUT;
+constexpr uint32_t kStRange = 1u << HQ_ERR_RANGE;
+
+// Workspace layout (bytes): [0] status u32, [4] nonfinite tiles u32, [8] words needed u64,
+// [16] work counter u32, [24] count-only total u64, [64 ..] look-back states u64 per item.
+struct WsHeader {
+    uint32_t status;
+    uint32_t nonfinite;
+    unsigned long long needed;
+    uint32_t counter;
+    uint32_t pad0;
+    unsigned long long count_bits;
+    uint32_t pad1[8];
+};
+static_assert(sizeof(WsHeader) == 64, "workspace header");
+
+// threads per tile: one thread holds n/TPT coefficients in registers
+__host__ __device__ constexpr int tpt_for(int n) { return n == 256 ? 2 : 1; }
+
+// ------------------------------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11): published multipliers and Weyl key increments.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1)
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint32_t lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    }
+    return c;
+}
+
+// ------------------------------------------------------------------------------------------------
+// bf16 / fp32 bit helpers
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// binary32 -> bfloat16 bits, round to nearest even (finite inputs)
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f)
+{
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 f2sub(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// ------------------------------------------------------------------------------------------------
+// shared-memory, mbarrier and TMA wrappers
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// bounded wait on an mbarrier phase; returns false when the limit ran out
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (i > 64) __nanosleep(64);
+    }
+    return false;
+}
+
+// 2-D tiled TMA load of one box into shared memory, completing on `bar`
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 2-D tiled TMA store of one box from shared memory (bulk group)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// wait until every committed bulk store has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// wait until every committed bulk store has completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// make generic-proxy shared-memory writes visible to the async (TMA) proxy
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16)
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// address of byte `off` of row r inside a swizzled TMA box ([rows][128 B], 128-byte swizzle)
+__device__ __forceinline__ uint32_t swz(int r, int chunk16) { return (uint32_t)(r * 128 + ((chunk16 ^ (r & 7)) << 4)); }
+
+// ------------------------------------------------------------------------------------------------
+// Bit writer.  Codes are appended in reading order into an MSB-first accumulator; full 32-bit
+// reading-order words are ORed into the shared-memory stream.  Forward segments read with
+// increasing bit position (stored word = bit-reversed reading word), backward segments with
+// decreasing position (stored word = reading word).  The accumulator starts with the phantom
+// bits that precede the segment inside its first word, so every emitted word is one stored word.
+// ------------------------------------------------------------------------------------------------
+template <bool FWD>
+struct BitWriter {
+    unsigned long long acc;  // valid bits are the low `nb` bits, earliest read bit highest
+    int nb;
+    int wi;                  // stored word index of the next emitted word
+    uint32_t* stg;
+
+    __device__ __forceinline__ void begin(uint32_t* s, int start_or_end_bit)
+    {
+        stg = s;
+        acc = 0ull;
+        if (FWD) {
+            wi = start_or_end_bit >> 5;
+            nb = start_or_end_bit & 31;
+        } else {
+            wi = start_or_end_bit >> 5;
+            nb = 31 - (start_or_end_bit & 31);
+        }
+    }
+    __device__ __forceinline__ void emit(uint32_t rw)
+    {
+        const uint32_t w = FWD ? __brev(rw) : rw;
+        if (w) atomicOr(stg + wi, w);
+        wi += FWD ? 1 : -1;
+    }
+    // append `len` (<= 32) bits: the low `len` bits of `code`, most significant first
+    __device__ __forceinline__ void put(uint32_t code, int len)
+    {
+        acc = (acc << len) | code;
+        nb += len;
+        if (nb >= 32) {
+            emit((uint32_t)(acc >> (nb - 32)));
+            nb -= 32;
+        }
+    }
+    __device__ __forceinline__ void zeros(uint32_t count)
+    {
+        while (count > 31) {
+            put(0u, 31);
+            count -= 31;
+        }
+        if (count) put(0u, (int)count);
+    }
+    __device__ __forceinline__ void finish()
+    {
+        if (nb > 0) emit((uint32_t)(acc << (32 - nb)));
+    }
+};
+
+// ------------------------------------------------------------------------------------------------
+// Bit reader over a shared-memory stream, mirror of BitWriter: MSB-aligned 64-bit window.
+// ------------------------------------------------------------------------------------------------
+template <bool FWD>
+struct BitReader {
+    unsigned long long W;  // top `avail` bits valid, next bit at bit 63
+    int avail;
+    int wi;
+    int lim;  // last readable word index; reads are clamped to [0, lim]
+    const uint32_t* src;
+
+    __device__ __forceinline__ uint32_t load()
+    {
+        const uint32_t w = src[min(max(wi, 0), lim)];
+        wi += FWD ? 1 : -1;
+        return FWD ? __brev(w) : w;
+    }
+    __device__ __forceinline__ void begin(const uint32_t* s, int start_or_end_bit)
+    {
+        src = s;
+        wi = start_or_end_bit >> 5;
+        const int skip = FWD ? (start_or_end_bit & 31) : (31 - (start_or_end_bit & 31));
+        const uint32_t w0 = load();
+        const uint32_t w1 = load();
+        W = (((unsigned long long)w0 << 32) | w1) << skip;
+        avail = 64 - skip;
+    }
+    __device__ __forceinline__ void refill()
+    {
+        if (avail <= 32) {
+            W |= (unsigned long long)load() << (32 - avail);
+            avail += 32;
+        }
+    }
+    __device__ __forceinline__ void skip(int len)
+    {
+        W = (len >= 64) ? 0ull : (W << len);
+        avail -= len;
+    }
+    // one Rice code: q zeros, a one, r (k bits MSB-first); returns q << k | r.  `ok` is cleared
+    // when the unary run exceeds `limit` (a corrupt stream).
+    __device__ __forceinline__ uint32_t code(int k, uint32_t limit, bool& ok)
+    {
+        refill();
+        uint32_t q = 0;
+        uint32_t hi = (uint32_t)(W >> 32);
+        while (hi == 0u) {  // long unary runs: 32 zeros at a time
+            q += 32;
+            skip(32);
+            refill();
+            hi = (uint32_t)(W >> 32);
+            if (q > limit) {
+                ok = false;
+                return 0u;
+            }
+        }
+        const int z = __clz(hi);
+        q += (uint32_t)z;
+        skip(z + 1);
+        if (avail < k + 1) refill();
+        const uint32_t r = k ? (uint32_t)(W >> (64 - k)) : 0u;
+        skip(k);
+        return (q << k) | r;
+    }
+};
+
+// ------------------------------------------------------------------------------------------------
+// misc
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t zigzag(int32_t m) { return ((uint32_t)m << 1) ^ (uint32_t)(m >> 31); }
+__device__ __forceinline__ int32_t unzigzag(uint32_t z) { return (int32_t)(z >> 1) ^ -(int32_t)(z & 1u); }
+
+// Rice parameter: the smallest k >= 0 with sum zz < n 2^(k+1), capped at 15
+__device__ __forceinline__ int rice_k(uint32_t A, int log2n)
+{
+    const uint32_t m = A >> (log2n + 1);
+    const int k = 32 - __clz(m);
+    return k > 15 ? 15 : k;
+}
+
+__device__ __forceinline__ void status_set(WsHeader* ws, uint32_t bits) { atomicOr(&ws->status, bits); }
+
+}  // namespace hq

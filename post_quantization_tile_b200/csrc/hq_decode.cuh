@@ -1,0 +1,369 @@
+// hq_decode.cuh -- decode kernel of the HyperQuant tile codec (inverse of Methodology steps 1-4).
+//
+// A block decodes one item (TI rows of one tile column = TI/32 chunks) at a time.  The item's
+// words are independent of every other item thanks to the stored chunk offsets, so items are
+// assigned statically.  Thread 0 bulk-copies the item's 16-byte-aligned word range into shared
+// memory (two-stage ring); every thread parses its tile's Rice codes -- the first half forward
+// from the tile start, the second half backward from the tile end, so two threads can share a
+// 256-tile -- rebuilds the integer lattice codes, applies the inverse transform D H_n p and the
+// scale, and writes its row into a swizzled staging box that one TMA store sends to HBM.
+#pragma once
+#include "hq_common.cuh"
+#include "hq_lattice.cuh"
+
+namespace hq {
+
+struct DecodeArgs {
+    int64_t rows, cols;
+    float beta;
+    uint64_t seed;
+    int64_t kv_S;
+    int64_t items, IB, RB, C;
+    const uint16_t* scale;
+    const uint16_t* meta;
+    const uint32_t* chunk_word;
+    const uint32_t* bits;
+    int64_t cap_words;
+    WsHeader* ws;
+};
+
+template <int N, int DST>  // DST: 0 bf16, 1 fp32
+struct DecGeom {
+    static constexpr int TPT = tpt_for(N);
+    static constexpr int V = N / TPT;
+    static constexpr int H = V / 2;
+    static constexpr int TI = kThreads / TPT;
+    static constexpr int CH = TI / kChunkTiles;
+    static constexpr int ES = DST == 0 ? 2 : 4;
+    static constexpr int ROWB = N * ES;
+    static constexpr int NB = ROWB / 128;
+    static constexpr int OUT = NB * TI * 128;
+    static constexpr int LMAX = N / 8 + 16 * N + 2 * N;
+    static constexpr int GUARD = 4;  // words before and after the copied range
+    static constexpr int IN_WORDS = (TI * ((LMAX + 31) / 32) + CH + 8 + 2 * GUARD + 3) / 4 * 4;  // 16-byte stages
+    static constexpr int MASKS = DST == 0 ? N / 2 : N;
+    static constexpr int LOG2N = N == 64 ? 6 : (N == 128 ? 7 : 8);
+};
+
+template <int N, int DST>
+struct DecSmem {
+    using G = DecGeom<N, DST>;
+    alignas(1024) unsigned char out[G::OUT];
+    alignas(16) uint32_t in[kStages][G::IN_WORDS];
+    alignas(16) uint32_t mask[G::MASKS];
+    uint32_t Ls[G::TI];
+    uint32_t rowoff[G::TI];
+    uint32_t chunkbase[kStages][G::CH + 1];  // chunk start word relative to the copied range
+    int64_t item_ring[kStages];
+    int32_t ok_ring[kStages];
+    int64_t mask_jt;
+    alignas(8) uint64_t bar[kStages];
+};
+
+template <int N, int DST>
+__device__ __forceinline__ void build_masks_out(uint32_t* mask, int64_t jt, uint64_t seed)
+{
+    using G = DecGeom<N, DST>;
+    for (int w = threadIdx.x; w < G::MASKS; w += kThreads) {
+        const int per = DST == 0 ? 2 : 1;
+        uint32_t m = 0;
+#pragma unroll
+        for (int e = 0; e < per; ++e) {
+            const int64_t J = jt * N + (int64_t)w * per + e;
+            const uint4 ph = philox4x32_10(make_uint4((uint32_t)((uint64_t)J >> 7), 0u, 0u, 0u), (uint32_t)seed,
+                                           (uint32_t)(seed >> 32));
+            const int wsel = (int)((J & 127) >> 5);
+            const uint32_t word = wsel == 0 ? ph.x : (wsel == 1 ? ph.y : (wsel == 2 ? ph.z : ph.w));
+            m |= ((word >> (J & 31)) & 1u) << (DST == 0 ? (e ? 31 : 15) : 31);
+        }
+        mask[w] = m;
+    }
+}
+
+// Producer: copy the words of item `it` into stage s.  Returns false (stage unusable) when the
+// chunk offsets are inconsistent with the buffer.
+template <int N, int DST>
+__device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs& a, int s, int64_t it)
+{
+    using G = DecGeom<N, DST>;
+    sm.item_ring[s] = it;
+    sm.ok_ring[s] = 0;
+    if (it >= a.items) return;
+    const int64_t jt = it / a.IB, ib = it % a.IB;
+    const int64_t r0 = ib * G::TI;
+    const int rows_valid = (int)min((int64_t)G::TI, a.rows - r0);
+    const int nch = (rows_valid + kChunkTiles - 1) / kChunkTiles;
+    const int64_t c0 = jt * a.RB + ib * G::CH;
+    const int64_t w0 = a.chunk_word[c0];
+    const int64_t w1 = a.chunk_word[c0 + nch];
+    const int64_t lo = w0 & ~(int64_t)3;
+    const int64_t hi = (w1 + 3) & ~(int64_t)3;
+    const bool good = w1 >= w0 && hi <= a.cap_words && (hi - lo) <= (int64_t)(G::IN_WORDS - 2 * G::GUARD);
+    for (int ch = 0; ch <= nch; ++ch) sm.chunkbase[s][ch] = (uint32_t)(a.chunk_word[c0 + ch] - lo + G::GUARD);
+    if (!good) status_set(a.ws, kStCorrupt);
+    const uint32_t bytes = (uint32_t)((hi - lo) * 4);
+    if (good && bytes) {
+        sm.ok_ring[s] = 1;
+        mbar_arrive_expect_tx(&sm.bar[s], bytes);
+        bulk_load_1d(sm.in[s] + G::GUARD, a.bits + lo, bytes, &sm.bar[s]);
+    } else {
+        sm.ok_ring[s] = good ? 1 : 0;
+        mbar_arrive(&sm.bar[s]);  // complete the phase without data
+    }
+}
+
+template <int N, int LAT, bool KV, int DST>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap)
+{
+    using G = DecGeom<N, DST>;
+    using SM = DecSmem<N, DST>;
+    constexpr int TPT = G::TPT, V = G::V, H = G::H, TI = G::TI, D = Lat<LAT>::d;
+    constexpr int COSB = LAT == HQ_E8 ? N / 8 : 0;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // TMA boxes with 128-byte swizzle need 1024-byte aligned shared memory: align by hand
+    SM& sm = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int row_l = tid / TPT;
+    const int tau = tid % TPT;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+        fence_mbar_init();
+        sm.mask_jt = -1;
+        for (int s = 0; s < kStages; ++s) issue_item<N, DST>(sm, a, s, (int64_t)blockIdx.x + (int64_t)s * gridDim.x);
+    }
+    __syncthreads();
+
+    for (int iter = 0;; ++iter) {
+        const int s = iter % kStages;
+        const uint32_t parity = (uint32_t)((iter / kStages) & 1);
+        const int64_t item = sm.item_ring[s];
+        if (item >= a.items) break;
+        const int64_t jt = item / a.IB, ib = item % a.IB;
+        const int64_t r0 = ib * TI;
+        const int rows_valid = (int)min((int64_t)TI, a.rows - r0);
+        const bool valid = row_l < rows_valid;
+        const bool stage_ok = sm.ok_ring[s] != 0;
+
+        if (sm.mask_jt != jt) {
+            build_masks_out<N, DST>(sm.mask, jt, a.seed);
+            __syncthreads();
+            if (tid == 0) sm.mask_jt = jt;
+        }
+
+        // tile lengths from meta -> bit offsets within the chunks
+        const int64_t t = jt * a.rows + r0 + row_l;
+        uint32_t L = 0, mt = 0;
+        if (valid) {
+            mt = a.meta[t];
+            L = (uint32_t)COSB + (uint32_t)N * ((mt & 15u) + 1u) + (mt >> 4);
+        }
+        // per-chunk scan of the tile lengths (warp 0; rows of a chunk may span two warps)
+        uint32_t* Ls = sm.Ls;
+        if (tau == 0) Ls[row_l] = L;
+        __syncthreads();
+        if (warp == 0) {
+#pragma unroll
+            for (int ch = 0; ch < G::CH; ++ch) {
+                const uint32_t v = Ls[ch * 32 + lane];
+                uint32_t incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                sm.rowoff[ch * 32 + lane] = incl - v;
+            }
+        }
+        if (!mbar_wait(&sm.bar[s], parity)) status_set(a.ws, kStTimeout);
+        __syncthreads();
+
+        // ---------------- parse ----------------
+        int32_t sym[V];
+        uint32_t cosbits = 0;
+        bool ok = valid && stage_ok;
+        uint32_t sq_part = 0, sq_want = 0;
+        const uint16_t sbits = valid ? a.scale[t] : (uint16_t)0;
+        if (ok) {
+            const int k = (int)(mt & 15u);
+            const uint32_t sq_meta = mt >> 4;
+            const int ch = row_l / kChunkTiles;
+            const int tile0 = (int)(sm.chunkbase[s][ch] * 32u + sm.rowoff[row_l]);
+            const uint32_t* in = sm.in[s];
+            if constexpr (LAT == HQ_E8) {
+                const int cpos = tile0 + tau * (V / 8);
+                const int cw = min(max(cpos >> 5, 0), G::IN_WORDS - 2);
+                const unsigned long long two = ((unsigned long long)in[cw + 1] << 32) | in[cw];
+                cosbits = (uint32_t)(two >> (cpos & 31)) & ((V / 8) >= 32 ? 0xffffffffu : ((1u << (V / 8)) - 1u));
+            }
+            uint32_t sq = 0;
+            if (tau == 0) {
+                BitReader<true> br;
+                br.lim = G::IN_WORDS - 1;
+                br.begin(in, tile0 + COSB);
+                constexpr int CNT = TPT == 1 ? N / 2 : V;
+#pragma unroll
+                for (int i = 0; i < CNT; ++i) {
+                    const uint32_t z = br.code(k, sq_meta, ok);
+                    sq += z >> k;
+                    sym[i] = unzigzag(z);
+                }
+            }
+            if (TPT == 1 || tau == 1) {
+                BitReader<false> br;
+                br.lim = G::IN_WORDS - 1;
+                br.begin(in, tile0 + (int)L - 1);
+                constexpr int FIRST = TPT == 1 ? N / 2 : 0;
+#pragma unroll
+                for (int i = V - 1; i >= FIRST; --i) {
+                    const uint32_t z = br.code(k, sq_meta, ok);
+                    sq += z >> k;
+                    sym[i] = unzigzag(z);
+                }
+            }
+            sq_part = sq;
+            sq_want = sq_meta;
+        } else {
+#pragma unroll
+            for (int i = 0; i < V; ++i) sym[i] = 0;
+        }
+        if constexpr (TPT == 2) sq_part += __shfl_xor_sync(0xffffffffu, sq_part, 1);
+        if (ok && sq_part != sq_want) ok = false;
+        if constexpr (TPT == 2) {
+            const int other = __shfl_xor_sync(0xffffffffu, (int)ok, 1);
+            ok = ok && other;
+        }
+        if (valid && stage_ok && !ok) status_set(a.ws, kStCorrupt);
+
+        // ---------------- codes -> lattice point (float pairs) ----------------
+        float2 P[H];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int b = 0; b < H / D; ++b) {
+                const int pos = half * H + b * D;
+                int32_t v[D];
+                unstrip_block<LAT>(sym + pos, (cosbits >> (pos / 8)) & 1u, v);
+#pragma unroll
+                for (int i = 0; i < D; ++i) {
+                    float f = __int_as_float(v[i] + __float_as_int(kMagic)) - kMagic;  // exact, |v| < 2^22
+                    if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
+                    if (!ok) f = 0.0f;
+                    if (half) P[b * D + i].y = f;
+                    else P[b * D + i].x = f;
+                }
+            }
+        }
+        if constexpr (KV) {
+            const int64_t r = r0 + row_l;
+            const uint64_t Sv = (uint64_t)a.kv_S;
+            const uint64_t sidx = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+            const uint32_t bh = Sv ? (uint32_t)((uint64_t)r / Sv) : 0u;
+#pragma unroll
+            for (int b = 0; b < H / 4; ++b) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float U[4];
+                    const uint32_t blk = (uint32_t)(tau * (V / 4) + half * (H / 4) + b);
+                    dither_d4(a.seed, bh, sidx, blk, U);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (half) P[4 * b + i].y = __fadd_rn(P[4 * b + i].y, -U[i]);
+                        else P[4 * b + i].x = __fadd_rn(P[4 * b + i].x, -U[i]);
+                    }
+                }
+            }
+        }
+
+        // ---------------- inverse transform: H_n p, exact for integer points ----------------
+        // in-thread strides (H within pairs, then H/2 .. 1); with two threads per tile the
+        // stride n/2 butterfly between the pair comes last
+#pragma unroll
+        for (int m = 0; m < H; ++m) P[m] = make_float2(__fadd_rn(P[m].x, P[m].y), __fadd_rn(P[m].x, -P[m].y));
+#pragma unroll
+        for (int h = H / 2; h >= 1; h /= 2)
+#pragma unroll
+            for (int m = 0; m < H; ++m)
+                if ((m & h) == 0) {
+                    const float2 x = P[m], y = P[m + h];
+                    P[m] = f2add(x, y);
+                    P[m + h] = f2sub(x, y);
+                }
+        if constexpr (TPT == 2) {
+#pragma unroll
+            for (int m = 0; m < H; ++m) {
+                const float ox = __shfl_xor_sync(0xffffffffu, P[m].x, 1);
+                const float oy = __shfl_xor_sync(0xffffffffu, P[m].y, 1);
+                // tau 0 holds a (positions < n/2), tau 1 holds b: a + b -> tau 0, a - b -> tau 1
+                P[m] = tau ? make_float2(__fadd_rn(ox, -P[m].x), __fadd_rn(oy, -P[m].y))
+                           : make_float2(__fadd_rn(P[m].x, ox), __fadd_rn(P[m].y, oy));
+            }
+        }
+
+        // ---------------- scale, sign, store into the staging box ----------------
+        const float sh = __uint_as_float((uint32_t)sbits << 16);
+        const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
+        float ht = __fmul_rn(__fmul_rn(sh, a.beta), cn);
+        if constexpr (LAT == HQ_E8) ht = __fmul_rn(ht, 0.5f);
+        const float2 h2 = make_float2(ht, ht);
+#pragma unroll
+        for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], h2);
+
+        if (tid == 0) bulk_wait_read0();  // previous item's store has read the staging box
+        __syncthreads();
+        // thread-local position pos -> row element e = tau*V + pos
+        if constexpr (DST == 0) {
+            // bf16: 8 elements per 16-byte chunk; chunk c holds elements 8c .. 8c+7
+#pragma unroll
+            for (int c = 0; c < H / 8; ++c) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int e0 = tau * V + half * H + 8 * c;  // first element of the chunk
+                    uint32_t w[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float lo = half ? P[8 * c + 2 * q].y : P[8 * c + 2 * q].x;
+                        const float hi = half ? P[8 * c + 2 * q + 1].y : P[8 * c + 2 * q + 1].x;
+                        const uint32_t bits = (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+                        w[q] = bits ^ sm.mask[e0 / 2 + q];
+                    }
+                    const int cg = e0 / 8;
+                    *reinterpret_cast<uint4*>(sm.out + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < H / 4; ++c) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int e0 = tau * V + half * H + 4 * c;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float f = half ? P[4 * c + q].y : P[4 * c + q].x;
+                        w[q] = __float_as_uint(f) ^ sm.mask[e0 + q];
+                    }
+                    const int cg = e0 / 4;
+                    *reinterpret_cast<uint4*>(sm.out + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int b = 0; b < G::NB; ++b)
+                tma_store_2d(&tmap, (int)(jt * N + b * (128 / G::ES)), (int)r0, sm.out + b * TI * 128);
+            bulk_commit();
+            // refill this input stage with the item kStages ahead
+            issue_item<N, DST>(sm, a, s, item + (int64_t)kStages * gridDim.x);
+        }
+    }
+    if (tid == 0) bulk_wait0();
+}
+
+}  // namespace hq

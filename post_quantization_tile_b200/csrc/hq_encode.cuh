@@ -1,0 +1,553 @@
+// hq_encode.cuh -- encode kernel of the HyperQuant tile codec (Methodology steps 1-4).
+//
+// One block of 128 threads works on an "item": TI consecutive rows of one tile column, i.e.
+// TI tiles = TI/32 chunks.  Threads own whole tiles in registers (two threads per tile when
+// n = 256), so the RMS, the sign flip, the Walsh-Hadamard butterflies, the lattice decision and
+// the Rice parameter need no cross-thread traffic.  Tiles arrive through 2-D TMA boxes with
+// 128-byte swizzle (conflict-free row reads) in a two-stage ring; items are claimed from a
+// global counter so that the single-pass chunk-offset scan (decoupled look-back over items) only
+// ever waits on blocks that are already running.
+#pragma once
+#include "hq_common.cuh"
+#include "hq_lattice.cuh"
+
+namespace hq {
+
+struct EncodeArgs {
+    int64_t rows, cols;
+    float beta;
+    uint64_t seed;
+    int64_t kv_S;
+    int64_t items;   // number of items
+    int64_t IB;      // items per tile column
+    int64_t RB;      // chunks per tile column
+    int64_t C;       // chunks
+    uint16_t* scale;
+    uint16_t* meta;
+    uint32_t* chunk_word;
+    uint32_t* bits;
+    int64_t cap_words;
+    int32_t* v_out;
+    WsHeader* ws;
+    unsigned long long* states;
+};
+
+// SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
+template <int N, int SRC>
+struct EncGeom {
+    static constexpr int TPT = tpt_for(N);
+    static constexpr int V = N / TPT;      // coefficients per thread
+    static constexpr int H = V / 2;        // float2 pairs per thread: P[m] = (c[m], c[m + H])
+    static constexpr int TI = kThreads / TPT;  // tiles (rows) per item
+    static constexpr int ES = SRC == 0 ? 2 : 4;
+    static constexpr int ROWB = N * ES;    // bytes per tile row
+    static constexpr int NB = ROWB / 128;  // 128-byte boxes per row
+    static constexpr int STAGE = NB * TI * 128;
+    static constexpr int CH = TI / kChunkTiles;  // chunks per item
+    // worst-case tile bits: n/8 coset + n (k + 1) with k <= 15 + sum q < 2n
+    static constexpr int LMAX = N / 8 + 16 * N + 2 * N;
+    static constexpr int STG_WORDS = TI * ((LMAX + 31) / 32) + CH + 8;
+    static constexpr int LOG2N = N == 64 ? 6 : (N == 128 ? 7 : 8);
+    static constexpr int MASKS = SRC == 0 ? N / 2 : N;  // sign-mask words per tile column
+};
+
+template <int N, int SRC>
+struct EncSmem {
+    using G = EncGeom<N, SRC>;
+    alignas(1024) unsigned char stage[kStages][G::STAGE];
+    uint32_t stg[G::STG_WORDS];
+    alignas(16) uint32_t mask[G::MASKS];
+    uint32_t Ls[G::TI];
+    uint32_t rowoff[G::TI];
+    uint32_t chunkoff[G::CH + 1];
+    int64_t item_ring[kStages];
+    int64_t mask_jt;
+    uint32_t item_words;
+    uint32_t base;
+    uint32_t flags;
+    alignas(8) uint64_t bar[kStages];
+};
+
+// ------------------------------------------------------------------------------------------------
+// sign masks of tile column jt: D_jj = -1 where bit (J & 31) of Philox(seed, (J >> 7, 0, 0, 0))
+// word (J & 127) >> 5 is set (J = jt n + j, the transformed-axis index).
+// bf16 rows: one word per element pair (bits 15 / 31); fp32 rows: one word per element.
+// ------------------------------------------------------------------------------------------------
+template <int N, int SRC>
+__device__ __forceinline__ void build_masks(uint32_t* mask, int64_t jt, uint64_t seed)
+{
+    using G = EncGeom<N, SRC>;
+    for (int w = threadIdx.x; w < G::MASKS; w += kThreads) {
+        const int per = SRC == 0 ? 2 : 1;
+        uint32_t m = 0;
+#pragma unroll
+        for (int e = 0; e < per; ++e) {
+            const int64_t J = jt * N + (int64_t)w * per + e;
+            const uint4 ph = philox4x32_10(make_uint4((uint32_t)((uint64_t)J >> 7), 0u, 0u, 0u), (uint32_t)seed,
+                                           (uint32_t)(seed >> 32));
+            const int wsel = (int)((J & 127) >> 5);
+            const uint32_t word = wsel == 0 ? ph.x : (wsel == 1 ? ph.y : (wsel == 2 ? ph.z : ph.w));
+            const uint32_t bit = (word >> (J & 31)) & 1u;
+            m |= bit << (SRC == 0 ? (e ? 31 : 15) : 31);
+        }
+        mask[w] = m;
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// load a thread's coefficients from the swizzled stage into float2 pairs
+// TPT == 1: P[m] = (x_m, x_{m+H});  TPT == 2: the first butterfly (stride n/2) is taken here,
+// thread tau computes y_{tau n/2 + i} = x_i +- x_{i + n/2} and P[m] = (y'_m, y'_{m+H}).
+// Also returns the thread's share of the RMS sum (ascending pairwise tree over its raw x).
+// ------------------------------------------------------------------------------------------------
+template <int N, int SRC>
+__device__ __forceinline__ void load_row(const unsigned char* stage, const uint32_t* mask, int row, int tau,
+                                         float2 (&P)[EncGeom<N, SRC>::H], float& sumsq)
+{
+    using G = EncGeom<N, SRC>;
+    constexpr int H = G::H;
+    // element e of the row -> (box, 16-byte chunk, offset)
+    auto chunk_ptr = [&](int c) -> const uint4* {
+        const int b = c >> 3;
+        return reinterpret_cast<const uint4*>(stage + b * (G::TI * 128) + swz(row, c & 7));
+    };
+    if constexpr (SRC == 0) {
+        // bf16: chunk c = elements 8c .. 8c+7
+        if constexpr (G::TPT == 1) {
+            float2 Q[H];
+#pragma unroll
+            for (int c = 0; c < H / 8; ++c) {
+                const uint4 A = *chunk_ptr(c);
+                const uint4 B = *chunk_ptr(c + H / 8);
+                const uint4 MA = *reinterpret_cast<const uint4*>(mask + 4 * c);
+                const uint4 MB = *reinterpret_cast<const uint4*>(mask + 4 * (c + H / 8));
+                const uint32_t a[4] = {A.x ^ MA.x, A.y ^ MA.y, A.z ^ MA.z, A.w ^ MA.w};
+                const uint32_t b[4] = {B.x ^ MB.x, B.y ^ MB.y, B.z ^ MB.z, B.w ^ MB.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    P[8 * c + 2 * q] = make_float2(bf16lo_to_f32(a[q]), bf16lo_to_f32(b[q]));
+                    P[8 * c + 2 * q + 1] = make_float2(bf16hi_to_f32(a[q]), bf16hi_to_f32(b[q]));
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < H; ++m) Q[m] = f2mul(P[m], P[m]);
+#pragma unroll
+            for (int h = 1; h < H; h *= 2)
+#pragma unroll
+                for (int m = 0; m < H; m += 2 * h) Q[m] = f2add(Q[m], Q[m + h]);
+            sumsq = __fadd_rn(Q[0].x, Q[0].y);
+        } else {
+            // N = 256, V = 128, H = 64: quarter k (0..3) of the row = elements 64k .. 64k+63
+            float2 Q[H];
+            const float2 sgn = tau ? make_float2(-1.0f, -1.0f) : make_float2(1.0f, 1.0f);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 X[4];
+                uint32_t x[4][4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    X[k] = *chunk_ptr(c + 8 * k);
+                    const uint4 M = *reinterpret_cast<const uint4*>(mask + 4 * (c + 8 * k));
+                    x[k][0] = X[k].x ^ M.x; x[k][1] = X[k].y ^ M.y; x[k][2] = X[k].z ^ M.z; x[k][3] = X[k].w ^ M.w;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int m = 8 * c + 2 * q + hh;
+                        const float2 lo = hh ? make_float2(bf16hi_to_f32(x[0][q]), bf16hi_to_f32(x[1][q]))
+                                             : make_float2(bf16lo_to_f32(x[0][q]), bf16lo_to_f32(x[1][q]));
+                        const float2 hi = hh ? make_float2(bf16hi_to_f32(x[2][q]), bf16hi_to_f32(x[3][q]))
+                                             : make_float2(bf16lo_to_f32(x[2][q]), bf16lo_to_f32(x[3][q]));
+                        // this thread's half of the RMS: tau 0 sums x[0..128), tau 1 x[128..256)
+                        Q[m] = tau ? f2mul(hi, hi) : f2mul(lo, lo);
+                        // first butterfly, stride n/2: tau 0 keeps sums, tau 1 differences
+                        P[m] = __ffma2_rn(hi, sgn, lo);
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 1; h < H; h *= 2)
+#pragma unroll
+                for (int m = 0; m < H; m += 2 * h) Q[m] = f2add(Q[m], Q[m + h]);
+            sumsq = __fadd_rn(Q[0].x, Q[0].y);
+        }
+    } else {
+        // fp32: chunk c = elements 4c .. 4c+3  (TPT == 1 only: N <= 128 for fp32 weights)
+        static_assert(SRC == 2 || G::TPT == 1 || true, "");
+        if constexpr (G::TPT == 1) {
+            float2 Q[H];
+#pragma unroll
+            for (int c = 0; c < H / 4; ++c) {
+                uint4 A = *chunk_ptr(c);
+                uint4 B = *chunk_ptr(c + H / 4);
+                if constexpr (SRC == 1) {
+                    const uint4 MA = *reinterpret_cast<const uint4*>(mask + 4 * c);
+                    const uint4 MB = *reinterpret_cast<const uint4*>(mask + 4 * (c + H / 4));
+                    A.x ^= MA.x; A.y ^= MA.y; A.z ^= MA.z; A.w ^= MA.w;
+                    B.x ^= MB.x; B.y ^= MB.y; B.z ^= MB.z; B.w ^= MB.w;
+                }
+                P[4 * c + 0] = make_float2(__uint_as_float(A.x), __uint_as_float(B.x));
+                P[4 * c + 1] = make_float2(__uint_as_float(A.y), __uint_as_float(B.y));
+                P[4 * c + 2] = make_float2(__uint_as_float(A.z), __uint_as_float(B.z));
+                P[4 * c + 3] = make_float2(__uint_as_float(A.w), __uint_as_float(B.w));
+            }
+            if constexpr (SRC == 1) {
+#pragma unroll
+                for (int m = 0; m < H; ++m) Q[m] = f2mul(P[m], P[m]);
+#pragma unroll
+                for (int h = 1; h < H; h *= 2)
+#pragma unroll
+                    for (int m = 0; m < H; m += 2 * h) Q[m] = f2add(Q[m], Q[m + h]);
+                sumsq = __fadd_rn(Q[0].x, Q[0].y);
+            } else {
+                sumsq = 0.0f;
+            }
+        } else {
+            // coefficients with n = 256: thread tau holds positions tau*128 + [0, 128)
+#pragma unroll
+            for (int c = 0; c < H / 4; ++c) {
+                const uint4 A = *chunk_ptr(tau * 32 + c);
+                const uint4 B = *chunk_ptr(tau * 32 + c + H / 4);
+                P[4 * c + 0] = make_float2(__uint_as_float(A.x), __uint_as_float(B.x));
+                P[4 * c + 1] = make_float2(__uint_as_float(A.y), __uint_as_float(B.y));
+                P[4 * c + 2] = make_float2(__uint_as_float(A.z), __uint_as_float(B.z));
+                P[4 * c + 3] = make_float2(__uint_as_float(A.w), __uint_as_float(B.w));
+            }
+            sumsq = 0.0f;
+        }
+    }
+}
+
+// in-thread Walsh-Hadamard butterflies on P[m] = (c_m, c_{m+H}), descending strides:
+// H (within each pair), then H/2, ..., 1 (between pairs)
+template <int H>
+__device__ __forceinline__ void fwht_pairs(float2 (&P)[H])
+{
+#pragma unroll
+    for (int m = 0; m < H; ++m) P[m] = make_float2(__fadd_rn(P[m].x, P[m].y), __fadd_rn(P[m].x, -P[m].y));
+#pragma unroll
+    for (int h = H / 2; h >= 1; h /= 2)
+#pragma unroll
+        for (int m = 0; m < H; ++m)
+            if ((m & h) == 0) {
+                const float2 a = P[m], b = P[m + h];
+                P[m] = f2add(a, b);
+                P[m + h] = f2sub(a, b);
+            }
+}
+
+template <int N, int LAT, bool KV, int SRC, bool COUNT>
+__global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a, const __grid_constant__ CUtensorMap tmap)
+{
+    using G = EncGeom<N, SRC>;
+    using SM = EncSmem<N, SRC>;
+    constexpr int TPT = G::TPT, V = G::V, H = G::H, TI = G::TI, D = Lat<LAT>::d;
+    constexpr int COSB = LAT == HQ_E8 ? N / 8 : 0;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // TMA boxes with 128-byte swizzle need 1024-byte aligned shared memory: align by hand
+    SM& sm = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int row_l = tid / TPT;   // row within the item
+    const int tau = tid % TPT;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+        fence_mbar_init();
+        sm.mask_jt = -1;
+        // claim and launch the first kStages items
+        for (int s = 0; s < kStages; ++s) {
+            const int64_t it = (int64_t)atomicAdd(&a.ws->counter, 1u);
+            sm.item_ring[s] = it;
+            if (it < a.items) {
+                const int64_t jt = it / a.IB, ib = it % a.IB;
+                mbar_arrive_expect_tx(&sm.bar[s], G::STAGE);
+#pragma unroll
+                for (int b = 0; b < G::NB; ++b)
+                    tma_load_2d(sm.stage[s] + b * TI * 128, &tmap, (int)(jt * (G::ROWB / G::ES) + b * (128 / G::ES)),
+                                (int)(ib * TI), &sm.bar[s]);
+            }
+        }
+    }
+    __syncthreads();
+
+    for (int iter = 0;; ++iter) {
+        const int s = iter % kStages;
+        const uint32_t parity = (uint32_t)((iter / kStages) & 1);
+        const int64_t item = sm.item_ring[s];
+        if (item >= a.items) break;
+        const int64_t jt = item / a.IB, ib = item % a.IB;
+        const int64_t r0 = ib * TI;
+        const int rows_valid = (int)min((int64_t)TI, a.rows - r0);
+        const bool valid = row_l < rows_valid;
+
+        if constexpr (SRC != 2) {
+            if (sm.mask_jt != jt) {  // block-uniform
+                build_masks<N, SRC>(sm.mask, jt, a.seed);
+                __syncthreads();
+                if (tid == 0) sm.mask_jt = jt;
+            }
+        }
+        if (!mbar_wait(&sm.bar[s], parity)) status_set(a.ws, kStTimeout);
+
+        float2 P[H];
+        float sumsq;
+        load_row<N, SRC>(sm.stage[s], sm.mask, row_l, tau, P, sumsq);
+        __syncthreads();  // stage s consumed; mask table free
+        if (tid == 0) {
+            const int64_t nxt = (int64_t)atomicAdd(&a.ws->counter, 1u);
+            sm.item_ring[s] = nxt;
+            if (nxt < a.items) {
+                const int64_t njt = nxt / a.IB, nib = nxt % a.IB;
+                mbar_arrive_expect_tx(&sm.bar[s], G::STAGE);
+#pragma unroll
+                for (int b = 0; b < G::NB; ++b)
+                    tma_load_2d(sm.stage[s] + b * TI * 128, &tmap,
+                                (int)(njt * (G::ROWB / G::ES) + b * (128 / G::ES)), (int)(nib * TI), &sm.bar[s]);
+            }
+        }
+
+        // ---------------- per-tile scale, RHT, normalisation ----------------
+        uint16_t sbits = 0;
+        bool zero_tile = false;
+        if constexpr (SRC != 2) {
+            if constexpr (TPT == 2) {
+                const float other = __shfl_xor_sync(0xffffffffu, sumsq, 1);
+                sumsq = tau ? __fadd_rn(other, sumsq) : __fadd_rn(sumsq, other);  // first half + second half
+            }
+            const float s_rms = __fsqrt_rn(__fmul_rn(sumsq, 1.0f / (float)N));
+            sbits = f32_to_bf16_bits(s_rms);
+            const float sh = __uint_as_float((uint32_t)sbits << 16);
+            const bool finite = isfinite(sh);
+            if (!finite && valid && tau == 0) {
+                status_set(a.ws, kStNonfinite);
+                atomicAdd(&a.ws->nonfinite, 1u);
+            }
+            zero_tile = !finite || sh < 1.2621774483536189e-29f;  // 2^-96
+            if (zero_tile) sbits = 0;
+            fwht_pairs<H>(P);
+            const float t = __fmul_rn(sh, a.beta);
+            const float rinv = __frcp_rn(t);
+            const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
+            const float g = zero_tile ? 0.0f : __fmul_rn(cn, rinv);
+            const float2 g2 = make_float2(g, g);
+#pragma unroll
+            for (int m = 0; m < H; ++m) P[m] = zero_tile ? make_float2(0.0f, 0.0f) : f2mul(P[m], g2);
+        }
+
+        // ---------------- dither (KV) ----------------
+        if constexpr (KV) {
+            const int64_t r = r0 + row_l;
+            const uint64_t Sv = (uint64_t)a.kv_S;
+            const uint64_t sidx = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+            const uint32_t bh = Sv ? (uint32_t)((uint64_t)r / Sv) : 0u;
+#pragma unroll
+            for (int b = 0; b < H / 4; ++b) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float U[4];
+                    const uint32_t blk = (uint32_t)(tau * (V / 4) + half * (H / 4) + b);
+                    dither_d4(a.seed, bh, sidx, blk, U);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (half) P[4 * b + i].y = __fadd_rn(P[4 * b + i].y, U[i]);
+                        else P[4 * b + i].x = __fadd_rn(P[4 * b + i].x, U[i]);
+                    }
+                }
+            }
+        }
+
+        // ---------------- lattice + strip ----------------
+        int32_t sym[V];
+        uint32_t cosbits = 0;  // coset bit of local block lb at bit lb (E8)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int b = 0; b < H / D; ++b) {
+                float u[D];
+#pragma unroll
+                for (int i = 0; i < D; ++i) u[i] = half ? P[b * D + i].y : P[b * D + i].x;
+                int32_t v[D];
+                quantize_block<LAT>(u, v);
+                const int pos = half * H + b * D;
+                if constexpr (SRC == 2) {
+                    if (valid && a.v_out) {
+                        int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V + pos;
+#pragma unroll
+                        for (int i = 0; i < D; ++i) vo[i] = v[i];
+                    }
+                }
+                const uint32_t c = strip_block<LAT>(v, sym + pos);
+                if constexpr (LAT == HQ_E8) cosbits |= c << (pos / 8);
+            }
+        }
+
+        // ---------------- Rice parameter and tile length ----------------
+        uint32_t A = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) A += zigzag(sym[i]);
+        if constexpr (TPT == 2) A += __shfl_xor_sync(0xffffffffu, A, 1);
+        const int k = rice_k(A, G::LOG2N);
+        uint32_t sq = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) sq += zigzag(sym[i]) >> k;
+        uint32_t sq_tile = sq;
+        if constexpr (TPT == 2) sq_tile += __shfl_xor_sync(0xffffffffu, sq, 1);
+        const uint32_t L = (uint32_t)COSB + (uint32_t)N * (uint32_t)(k + 1) + sq_tile;
+        // the staging stream holds at most LMAX bits per tile; longer tiles (only reachable with
+        // caller-given coefficients of huge magnitude) are reported and left out
+        const bool fits_tile = L <= (uint32_t)G::LMAX;
+        if (!fits_tile && valid && tau == 0) status_set(a.ws, kStRange);
+        const bool emit = valid && fits_tile;
+        if (tau == 0) sm.Ls[row_l] = emit ? L : 0u;
+        __syncthreads();
+
+        // ---------------- chunk layout of the item (warp 0) ----------------
+        if (warp == 0) {
+            uint32_t acc_words = 0;
+#pragma unroll
+            for (int ch = 0; ch < G::CH; ++ch) {
+                const uint32_t v = sm.Ls[ch * 32 + lane];
+                uint32_t incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                sm.rowoff[ch * 32 + lane] = incl - v;
+                const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+                if (lane == 0) sm.chunkoff[ch] = acc_words;
+                acc_words += (tot + 31) >> 5;
+            }
+            if (lane == 0) {
+                sm.chunkoff[G::CH] = acc_words;
+                sm.item_words = acc_words;
+                if constexpr (COUNT) {
+                    uint32_t bits = 0;
+                    for (int i = 0; i < TI; ++i) bits += sm.Ls[i];
+                    atomicAdd(&a.ws->count_bits, (unsigned long long)bits);
+                } else {
+                    const unsigned long long st = ((item == 0 ? 2ull : 1ull) << 32) | acc_words;
+                    st_relaxed_u64(a.states + item, st);
+                }
+            }
+        }
+        __syncthreads();
+        if constexpr (COUNT) continue;
+
+        const uint32_t item_words = sm.item_words;
+        for (uint32_t w = tid; w < item_words + 2; w += kThreads) sm.stg[w] = 0u;
+        __syncthreads();
+
+        // ---------------- Rice bits into the staging stream ----------------
+        if (emit) {
+            const int ch = row_l / kChunkTiles;
+            const int tile0 = (int)(sm.chunkoff[ch] * 32u + sm.rowoff[row_l]);  // tile start bit
+            if constexpr (LAT == HQ_E8) {
+                const int cpos = tile0 + tau * (V / 8);
+                const uint32_t lo = cosbits << (cpos & 31);
+                const uint32_t hi = (cpos & 31) ? (cosbits >> (32 - (cpos & 31))) : 0u;
+                if (lo) atomicOr(&sm.stg[cpos >> 5], lo);
+                if (hi) atomicOr(&sm.stg[(cpos >> 5) + 1], hi);
+            }
+            const uint32_t km = (1u << k) - 1u;
+            const uint32_t one = 1u << k;
+            if (tau == 0) {
+                BitWriter<true> bw;
+                bw.begin(sm.stg, tile0 + COSB);
+                constexpr int CNT = TPT == 1 ? N / 2 : V;
+#pragma unroll
+                for (int i = 0; i < CNT; ++i) {
+                    const uint32_t z = zigzag(sym[i]);
+                    const uint32_t q = z >> k;
+                    if (q > 31 - k) {
+                        bw.zeros(q);
+                        bw.put(one | (z & km), k + 1);
+                    } else {
+                        bw.put(one | (z & km), (int)q + k + 1);
+                    }
+                }
+                bw.finish();
+            }
+            if (TPT == 1 || tau == 1) {
+                BitWriter<false> bw;
+                bw.begin(sm.stg, tile0 + (int)L - 1);
+                constexpr int FIRST = TPT == 1 ? N / 2 : 0;
+#pragma unroll
+                for (int i = V - 1; i >= FIRST; --i) {
+                    const uint32_t z = zigzag(sym[i]);
+                    const uint32_t q = z >> k;
+                    if (q > 31 - k) {
+                        bw.zeros(q);
+                        bw.put(one | (z & km), k + 1);
+                    } else {
+                        bw.put(one | (z & km), (int)q + k + 1);
+                    }
+                }
+                bw.finish();
+            }
+        }
+
+        // ---------------- look-back for the item's word offset (warp 0) ----------------
+        if (warp == 0) {
+            uint32_t excl = 0;
+            if (item > 0) {
+                int64_t j = item - 1;
+                uint32_t spins = 0;
+                while (true) {
+                    const int64_t idx = j - lane;
+                    const unsigned long long st = idx >= 0 ? ld_relaxed_u64(a.states + idx) : (2ull << 32);
+                    const uint32_t flag = (uint32_t)(st >> 32);
+                    const uint32_t pmask = __ballot_sync(0xffffffffu, flag == 2u);
+                    const uint32_t xmask = __ballot_sync(0xffffffffu, flag == 0u);
+                    const int firstP = pmask ? __ffs(pmask) - 1 : 32;
+                    const uint32_t need = firstP >= 31 ? 0xffffffffu : ((2u << firstP) - 1u);
+                    if (xmask & need) {
+                        if (++spins > kSpinLimit) {
+                            if (lane == 0) status_set(a.ws, kStTimeout);
+                            break;
+                        }
+                        __nanosleep(32);
+                        continue;
+                    }
+                    uint32_t val = lane <= firstP ? (uint32_t)st : 0u;
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
+                    excl += val;
+                    if (firstP < 32) break;
+                    j -= 32;
+                }
+            }
+            if (lane == 0) {
+                if (item > 0) st_relaxed_u64(a.states + item, (2ull << 32) | (unsigned long long)(excl + item_words));
+                sm.base = excl;
+            }
+        }
+        __syncthreads();
+
+        // ---------------- store: bits, chunk offsets, scale, meta ----------------
+        const uint32_t base = sm.base;
+        const bool fits = (int64_t)base + (int64_t)item_words <= a.cap_words;
+        if (fits) {
+            for (uint32_t w = tid; w < item_words; w += kThreads) a.bits[base + w] = sm.stg[w];
+        } else if (tid == 0) {
+            status_set(a.ws, kStCapacity);
+        }
+        const int nch = (rows_valid + kChunkTiles - 1) / kChunkTiles;
+        const int64_t c0 = jt * a.RB + ib * G::CH;
+        if (tid < nch) a.chunk_word[c0 + tid] = base + sm.chunkoff[tid];
+        if (item == a.items - 1 && tid == 0) {
+            a.chunk_word[a.C] = base + item_words;
+            atomicMax(&a.ws->needed, (unsigned long long)(base + item_words));
+        }
+        if (valid && tau == 0) {
+            const int64_t t = jt * a.rows + r0 + row_l;
+            if (a.scale) a.scale[t] = sbits;
+            a.meta[t] = (uint16_t)((uint32_t)k | (sq_tile << 4));
+        }
+    }
+}
+
+}  // namespace hq

@@ -1,0 +1,65 @@
+"""The C-ABI library loads and exports every entry point include/hq.h declares (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hq.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hq_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def libhq():
+    from post_quantization_tile_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ["hq_encode", "hq_decode", "hq_kv_encode", "hq_kv_decode", "hq_quantize_coeffs", "hq_status_read"]:
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(libhq):
+    missing = [f for f in declared_functions() if not hasattr(libhq, f)]
+    assert not missing, missing
+
+
+def test_host_only_entry_points(libhq):
+    import post_quantization_tile_b200 as hq
+    L = hq.lib()
+    p = hq.params(128, hq.E8, 0.3)
+    assert L.hq_num_tiles(4096, 4096, 128) == 4096 * 32
+    assert L.hq_num_chunks(4096, 4096, 128) == 32 * 128
+    assert L.hq_num_chunks(70, 256, 64) == 4 * 3
+    assert L.hq_num_tiles(10, 100, 64) == -1
+    b = L.hq_encode_bound_words(4096, 4096, ctypes.byref(p))
+    assert b % 4 == 0 and b >= 4096 * 32 * (16 * 128 + 2 * 128) // 32
+    assert L.hq_workspace_bytes(4096, 4096, ctypes.byref(p)) % 256 == 0
+    assert L.hq_version() == 1
+    assert L.hq_status_str(3) == b"bitstream buffer too small"
+    # high-resolution step: E8 at 4 bps ~ 2^(2.047 - 4)
+    assert abs(L.hq_step_for_rate(hq.E8, 128, 4.0) - 2 ** (0.5 * __import__("math").log2(2 * 3.141592653589793 * 2.718281828459045) - 4)) < 1e-6
+
+
+def test_calls_reject_bad_arguments_without_a_gpu(libhq):
+    import post_quantization_tile_b200 as hq
+    L = hq.lib()
+    p = hq.params(100, hq.E8, 0.3)          # invalid tile
+    cs = hq.CodeStruct()
+    assert L.hq_encode(None, 0, 64, 128, ctypes.byref(p), ctypes.byref(cs), None, 0, None) == 1
+    p = hq.params(128, hq.E8, 1e-4)         # step below 2^-8
+    assert L.hq_encode(ctypes.c_void_p(16), 0, 64, 128, ctypes.byref(p), ctypes.byref(cs), ctypes.c_void_p(256),
+                       1 << 20, None) == 1
+    p = hq.params(128, hq.E8, 0.3)
+    assert L.hq_kv_encode(ctypes.c_void_p(16), 0, 1, 1, 8, 128, ctypes.byref(p), ctypes.byref(cs), ctypes.c_void_p(256),
+                          1 << 20, None) == 2   # dither is defined for D4 only
