@@ -90,27 +90,38 @@ def run_reference(args):
 # GPU arm
 # ------------------------------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples (every 100 ms) kept for the timed window."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index),
-                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
         return self
 
+    def mark(self, start: bool):
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.25)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -119,19 +130,28 @@ class ClockSampler:
             self.f.close()
 
     def summary(self):
+        import datetime
         try:
-            rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+            rows = [[c.strip() for c in r.split(",")] for r in open(self.path).read().strip().splitlines() if r.strip()]
         except Exception:
             return None
-        if not rows:
+        samples = []
+        for r in rows:
+            try:
+                t = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                samples.append((t, float(r[2]), float(r[3]), r[6:10]))
+            except Exception:
+                continue
+        if not samples or self.t0 is None:
             return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        win = [s for s in samples if self.t0 - 0.1 <= s[0] <= self.t1 + 0.1]
+        if not win:  # window shorter than the sampling period: nearest sample after the start
+            after = [s for s in samples if s[0] >= self.t0]
+            win = after[:1] or samples[-1:]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]
-                          and "Not" not in r[5 + i]})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for s in win for i in range(4) if i < len(s[3]) and s[3][i] == "Active"})
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": max(s[2] for s in win),
+                "reasons": reasons, "samples": len(win)}
 
 
 def run_gpu(args):
@@ -205,11 +225,14 @@ def run_gpu(args):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        time.sleep(1.0)  # let the sampler start before the timed region
+        clk.mark(True)
         t0.record(stream)
         for k in range(args.steps):
             step(args.warmup + k, record=k)
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.mark(False)
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1) / args.steps
@@ -295,15 +318,48 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+def run_profile(args):
+    """One kernel on a 16384x4096 bf16 weight (134 MB, larger than L2), fixed step, three
+    launches after one set-up encode: a short, self-contained command for ncu captures."""
+    import torch
+
+    import post_quantization_tile_b200 as hq
+    from post_quantization_tile_b200 import workloads as W
+    x = torch.from_numpy(W.llama_weight(16384, 4096, seed=9).view(np.int16)).view(torch.bfloat16).cuda()
+    beta = 0.29
+    code = hq.encode(x, TILE, hq.E8, beta, seed=SEED)
+    y = torch.empty_like(x)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    torch.cuda.synchronize()
+    for i in range(3):
+        ev[i].record()
+        if args.profile == "encode":
+            hq.encode(x, TILE, hq.E8, beta, seed=SEED, out=code, ws=code.ws)
+        elif args.profile == "decode":
+            hq.decode(code, out=y, ws=code.ws)
+        else:
+            hq.encode_count(x, TILE, hq.E8, beta, seed=SEED, ws=code.ws)
+    ev[3].record()
+    torch.cuda.synchronize()
+    st, _ = hq.status(code.ws)
+    ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(2)] + [ev[2].elapsed_time(ev[3])]
+    print(json.dumps({"profile": args.profile, "ms": ms, "status": st, "words": code.total_words()}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", choices=["encode", "decode", "count"], default=None)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

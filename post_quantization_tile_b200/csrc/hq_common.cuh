@@ -178,34 +178,38 @@ __device__ __forceinline__ uint32_t swz(int r, int chunk16) { return (uint32_t)(
 
 // ------------------------------------------------------------------------------------------------
 // Bit writer.  Codes are appended in reading order into an MSB-first accumulator; full 32-bit
-// reading-order words are ORed into the shared-memory stream.  Forward segments read with
-// increasing bit position (stored word = bit-reversed reading word), backward segments with
-// decreasing position (stored word = reading word).  The accumulator starts with the phantom
-// bits that precede the segment inside its first word, so every emitted word is one stored word.
+// reading-order words go to the shared-memory stream.  Forward segments read with increasing
+// bit position (stored word = bit-reversed reading word), backward segments with decreasing
+// position (stored word = reading word).  The accumulator starts with the phantom bits that
+// precede the segment inside its first word, so every emitted word is one stored word.  The
+// first and the last word of a segment may be shared with a neighbouring segment and are ORed
+// atomically; the words in between belong to this segment alone.
 // ------------------------------------------------------------------------------------------------
 template <bool FWD>
 struct BitWriter {
     unsigned long long acc;  // valid bits are the low `nb` bits, earliest read bit highest
     int nb;
     int wi;                  // stored word index of the next emitted word
+    bool first;
     uint32_t* stg;
 
     __device__ __forceinline__ void begin(uint32_t* s, int start_or_end_bit)
     {
         stg = s;
         acc = 0ull;
-        if (FWD) {
-            wi = start_or_end_bit >> 5;
-            nb = start_or_end_bit & 31;
-        } else {
-            wi = start_or_end_bit >> 5;
-            nb = 31 - (start_or_end_bit & 31);
-        }
+        wi = start_or_end_bit >> 5;
+        nb = FWD ? (start_or_end_bit & 31) : (31 - (start_or_end_bit & 31));
+        first = true;
     }
     __device__ __forceinline__ void emit(uint32_t rw)
     {
         const uint32_t w = FWD ? __brev(rw) : rw;
-        if (w) atomicOr(stg + wi, w);
+        if (first) {
+            atomicOr(stg + wi, w);
+            first = false;
+        } else {
+            stg[wi] = w;
+        }
         wi += FWD ? 1 : -1;
     }
     // append `len` (<= 32) bits: the low `len` bits of `code`, most significant first
@@ -218,19 +222,52 @@ struct BitWriter {
             nb -= 32;
         }
     }
-    __device__ __forceinline__ void zeros(uint32_t count)
-    {
-        while (count > 31) {
-            put(0u, 31);
-            count -= 31;
-        }
-        if (count) put(0u, (int)count);
-    }
     __device__ __forceinline__ void finish()
     {
-        if (nb > 0) emit((uint32_t)(acc << (32 - nb)));
+        if (nb > 0) atomicOr(stg + wi, FWD ? __brev((uint32_t)(acc << (32 - nb))) : (uint32_t)(acc << (32 - nb)));
     }
 };
+
+// one Rice code of arbitrary length (long unary runs): the rare path, kept out of line
+template <bool FWD>
+__device__ __forceinline__ void put_long_code(BitWriter<FWD>& bw, uint32_t q, uint32_t code, int k)
+{
+    while (q > 31) {
+        bw.put(0u, 31);
+        q -= 31;
+    }
+    if (q) bw.put(0u, (int)q);
+    bw.put(code, k + 1);
+}
+
+// Rice codes of four zig-zag values (reading order z0, z1, z2, z3): one append when their
+// codes fit in 32 bits together, else one append per code
+template <bool FWD>
+__device__ __forceinline__ void put4(BitWriter<FWD>& bw, uint32_t z0, uint32_t z1, uint32_t z2, uint32_t z3, int k,
+                                     uint32_t km, uint32_t one)
+{
+    const uint32_t q0 = z0 >> k, q1 = z1 >> k, q2 = z2 >> k, q3 = z3 >> k;
+    const uint32_t c0 = (z0 & km) | one, c1 = (z1 & km) | one, c2 = (z2 & km) | one, c3 = (z3 & km) | one;
+    const uint32_t k1 = (uint32_t)k + 1u;
+    const uint32_t l0 = q0 + k1, l1 = q1 + k1, l2 = q2 + k1, l3 = q3 + k1;
+    const uint32_t L = l0 + l1 + l2 + l3;
+    if (L <= 32u) {
+        // codes are (k+1)-bit values with the zero runs implied by the shifts
+        unsigned long long c = c0;
+        c = (c << l1) | c1;
+        c = (c << l2) | c2;
+        c = (c << l3) | c3;
+        bw.put((uint32_t)c, (int)L);
+    } else {
+        const uint32_t cs[4] = {c0, c1, c2, c3};
+        const uint32_t qs[4] = {q0, q1, q2, q3};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (qs[j] + k1 <= 32u) bw.put(cs[j], (int)(qs[j] + k1));
+            else put_long_code<FWD>(bw, qs[j], cs[j], k);
+        }
+    }
+}
 
 // ------------------------------------------------------------------------------------------------
 // Bit reader over a shared-memory stream, mirror of BitWriter: MSB-aligned 64-bit window.
@@ -249,9 +286,10 @@ struct BitReader {
         wi += FWD ? 1 : -1;
         return FWD ? __brev(w) : w;
     }
-    __device__ __forceinline__ void begin(const uint32_t* s, int start_or_end_bit)
+    __device__ __forceinline__ void begin(const uint32_t* s, int start_or_end_bit, int last_word)
     {
         src = s;
+        lim = last_word;
         wi = start_or_end_bit >> 5;
         const int skip = FWD ? (start_or_end_bit & 31) : (31 - (start_or_end_bit & 31));
         const uint32_t w0 = load();
@@ -266,37 +304,51 @@ struct BitReader {
             avail += 32;
         }
     }
-    __device__ __forceinline__ void skip(int len)
-    {
-        W = (len >= 64) ? 0ull : (W << len);
-        avail -= len;
-    }
-    // one Rice code: q zeros, a one, r (k bits MSB-first); returns q << k | r.  `ok` is cleared
-    // when the unary run exceeds `limit` (a corrupt stream).
-    __device__ __forceinline__ uint32_t code(int k, uint32_t limit, bool& ok)
-    {
-        refill();
-        uint32_t q = 0;
-        uint32_t hi = (uint32_t)(W >> 32);
-        while (hi == 0u) {  // long unary runs: 32 zeros at a time
-            q += 32;
-            skip(32);
-            refill();
-            hi = (uint32_t)(W >> 32);
-            if (q > limit) {
-                ok = false;
-                return 0u;
-            }
-        }
-        const int z = __clz(hi);
-        q += (uint32_t)z;
-        skip(z + 1);
-        if (avail < k + 1) refill();
-        const uint32_t r = k ? (uint32_t)(W >> (64 - k)) : 0u;
-        skip(k);
-        return (q << k) | r;
-    }
 };
+
+// unary runs of 32 or more zeros: the rare path, kept out of line.  Returns the run length
+// beyond the first 32-bit head; clears ok past `limit`.
+template <bool FWD>
+__device__ __forceinline__ uint32_t long_run(BitReader<FWD>& br, uint32_t limit, bool& ok)
+{
+    uint32_t q = 0;
+    uint32_t hi = (uint32_t)(br.W >> 32);
+    while (hi == 0u) {
+        q += 32;
+        br.W <<= 32;
+        br.avail -= 32;
+        br.refill();
+        hi = (uint32_t)(br.W >> 32);
+        if (q > limit) {
+            ok = false;
+            return q;
+        }
+    }
+    return q;
+}
+
+// one Rice code: q zeros, a one, r (k bits MSB-first); returns the zig-zag value q << k | r
+template <bool FWD>
+__device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t limit, bool& ok)
+{
+    br.refill();
+    uint32_t hi = (uint32_t)(br.W >> 32);
+    uint32_t q = 0;
+    if (hi == 0u) {
+        q = long_run<FWD>(br, limit, ok);
+        hi = (uint32_t)(br.W >> 32);
+        if (!ok) return 0u;
+    }
+    const int z = __clz(hi);
+    q += (uint32_t)z;
+    br.W <<= (z + 1);
+    br.avail -= z + 1;
+    if (br.avail < k) br.refill();
+    const uint32_t r = k ? (uint32_t)(br.W >> (64 - k)) : 0u;
+    br.W <<= k;
+    br.avail -= k;
+    return (q << k) | r;
+}
 
 // ------------------------------------------------------------------------------------------------
 // misc

@@ -9,6 +9,7 @@
 // scale, and writes its row into a swizzled staging box that one TMA store sends to HBM.
 #pragma once
 #include "hq_common.cuh"
+#include "hq_encode.cuh"
 #include "hq_lattice.cuh"
 
 namespace hq {
@@ -38,9 +39,13 @@ struct DecGeom {
     static constexpr int ROWB = N * ES;
     static constexpr int NB = ROWB / 128;
     static constexpr int OUT = NB * TI * 128;
-    static constexpr int LMAX = N / 8 + 16 * N + 2 * N;
+    static constexpr int ZZ = V * 2 * kThreads;  // zig-zag scratch, aliases the output box
+    static constexpr int BUF = OUT > ZZ ? OUT : ZZ;
+    // streams written by the encoder have k <= 9 (step range); the buffer takes k <= 11 and
+    // larger items are reported as corrupt
+    static constexpr int LMAX = N / 8 + 12 * N + 2 * N;
     static constexpr int GUARD = 4;  // words before and after the copied range
-    static constexpr int IN_WORDS = (TI * ((LMAX + 31) / 32) + CH + 8 + 2 * GUARD + 3) / 4 * 4;  // 16-byte stages
+    static constexpr int IN_WORDS = (TI * ((LMAX + 31) / 32) + CH + 8 + 2 * GUARD + 3) / 4 * 4;
     static constexpr int MASKS = DST == 0 ? N / 2 : N;
     static constexpr int LOG2N = N == 64 ? 6 : (N == 128 ? 7 : 8);
 };
@@ -48,16 +53,16 @@ struct DecGeom {
 template <int N, int DST>
 struct DecSmem {
     using G = DecGeom<N, DST>;
-    alignas(1024) unsigned char out[G::OUT];
-    alignas(16) uint32_t in[kStages][G::IN_WORDS];
+    alignas(1024) unsigned char buf[G::BUF];   // zig-zag scratch, then the output TMA box
+    alignas(16) uint32_t in[G::IN_WORDS];      // the item's words (one stage)
     alignas(16) uint32_t mask[G::MASKS];
     uint32_t Ls[G::TI];
     uint32_t rowoff[G::TI];
-    uint32_t chunkbase[kStages][G::CH + 1];  // chunk start word relative to the copied range
-    int64_t item_ring[kStages];
-    int32_t ok_ring[kStages];
+    uint32_t chunkbase[G::CH + 1];  // chunk start word relative to the copied range
+    int64_t item_cur;
+    int32_t ok_cur;
     int64_t mask_jt;
-    alignas(8) uint64_t bar[kStages];
+    alignas(8) uint64_t bar;
 };
 
 template <int N, int DST>
@@ -80,14 +85,14 @@ __device__ __forceinline__ void build_masks_out(uint32_t* mask, int64_t jt, uint
     }
 }
 
-// Producer: copy the words of item `it` into stage s.  Returns false (stage unusable) when the
-// chunk offsets are inconsistent with the buffer.
+// Producer (one thread): copy the words of item `it` into the input stage.  An item whose
+// chunk offsets are inconsistent with the buffers is flagged and decoded as zeros.
 template <int N, int DST>
-__device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs& a, int s, int64_t it)
+__device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs& a, int64_t it)
 {
     using G = DecGeom<N, DST>;
-    sm.item_ring[s] = it;
-    sm.ok_ring[s] = 0;
+    sm.item_cur = it;
+    sm.ok_cur = 0;
     if (it >= a.items) return;
     const int64_t jt = it / a.IB, ib = it % a.IB;
     const int64_t r0 = ib * G::TI;
@@ -99,21 +104,21 @@ __device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs
     const int64_t lo = w0 & ~(int64_t)3;
     const int64_t hi = (w1 + 3) & ~(int64_t)3;
     const bool good = w1 >= w0 && hi <= a.cap_words && (hi - lo) <= (int64_t)(G::IN_WORDS - 2 * G::GUARD);
-    for (int ch = 0; ch <= nch; ++ch) sm.chunkbase[s][ch] = (uint32_t)(a.chunk_word[c0 + ch] - lo + G::GUARD);
+    for (int ch = 0; ch <= nch; ++ch) sm.chunkbase[ch] = (uint32_t)(a.chunk_word[c0 + ch] - lo + G::GUARD);
     if (!good) status_set(a.ws, kStCorrupt);
     const uint32_t bytes = (uint32_t)((hi - lo) * 4);
     if (good && bytes) {
-        sm.ok_ring[s] = 1;
-        mbar_arrive_expect_tx(&sm.bar[s], bytes);
-        bulk_load_1d(sm.in[s] + G::GUARD, a.bits + lo, bytes, &sm.bar[s]);
+        sm.ok_cur = 1;
+        mbar_arrive_expect_tx(&sm.bar, bytes);
+        bulk_load_1d(sm.in + G::GUARD, a.bits + lo, bytes, &sm.bar);
     } else {
-        sm.ok_ring[s] = good ? 1 : 0;
-        mbar_arrive(&sm.bar[s]);  // complete the phase without data
+        sm.ok_cur = good ? 1 : 0;
+        mbar_arrive(&sm.bar);  // complete the phase without data
     }
 }
 
 template <int N, int LAT, bool KV, int DST>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap)
+__global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap)
 {
     using G = DecGeom<N, DST>;
     using SM = DecSmem<N, DST>;
@@ -129,23 +134,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
     const int tau = tid % TPT;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+        mbar_init(&sm.bar, 1);
         fence_mbar_init();
         sm.mask_jt = -1;
-        for (int s = 0; s < kStages; ++s) issue_item<N, DST>(sm, a, s, (int64_t)blockIdx.x + (int64_t)s * gridDim.x);
+        issue_item<N, DST>(sm, a, (int64_t)blockIdx.x);
     }
     __syncthreads();
 
     for (int iter = 0;; ++iter) {
-        const int s = iter % kStages;
-        const uint32_t parity = (uint32_t)((iter / kStages) & 1);
-        const int64_t item = sm.item_ring[s];
+        const int64_t item = sm.item_cur;
         if (item >= a.items) break;
         const int64_t jt = item / a.IB, ib = item % a.IB;
         const int64_t r0 = ib * TI;
         const int rows_valid = (int)min((int64_t)TI, a.rows - r0);
         const bool valid = row_l < rows_valid;
-        const bool stage_ok = sm.ok_ring[s] != 0;
+        const bool stage_ok = sm.ok_cur != 0;
 
         if (sm.mask_jt != jt) {
             build_masks_out<N, DST>(sm.mask, jt, a.seed);
@@ -153,21 +156,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
             if (tid == 0) sm.mask_jt = jt;
         }
 
-        // tile lengths from meta -> bit offsets within the chunks
+        // tile lengths from meta -> bit offsets within the chunks (warp 0 scans each chunk)
         const int64_t t = jt * a.rows + r0 + row_l;
         uint32_t L = 0, mt = 0;
         if (valid) {
             mt = a.meta[t];
             L = (uint32_t)COSB + (uint32_t)N * ((mt & 15u) + 1u) + (mt >> 4);
         }
-        // per-chunk scan of the tile lengths (warp 0; rows of a chunk may span two warps)
-        uint32_t* Ls = sm.Ls;
-        if (tau == 0) Ls[row_l] = L;
+        const uint16_t sbits = valid ? a.scale[t] : (uint16_t)0;
+        if (tau == 0) sm.Ls[row_l] = L;
+        if (tid == 0) bulk_wait_read0();  // the previous output box has left shared memory
         __syncthreads();
         if (warp == 0) {
 #pragma unroll
             for (int ch = 0; ch < G::CH; ++ch) {
-                const uint32_t v = Ls[ch * 32 + lane];
+                const uint32_t v = sm.Ls[ch * 32 + lane];
                 uint32_t incl = v;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -177,21 +180,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
                 sm.rowoff[ch * 32 + lane] = incl - v;
             }
         }
-        if (!mbar_wait(&sm.bar[s], parity)) status_set(a.ws, kStTimeout);
+        if (!mbar_wait(&sm.bar, (uint32_t)(iter & 1))) status_set(a.ws, kStTimeout);
         __syncthreads();
 
-        // ---------------- parse ----------------
-        int32_t sym[V];
+        // ---------------- parse: Rice codes -> zig-zag scratch ----------------
         uint32_t cosbits = 0;
         bool ok = valid && stage_ok;
         uint32_t sq_part = 0, sq_want = 0;
-        const uint16_t sbits = valid ? a.scale[t] : (uint16_t)0;
+        const int k = (int)(mt & 15u);
         if (ok) {
-            const int k = (int)(mt & 15u);
             const uint32_t sq_meta = mt >> 4;
+            sq_want = sq_meta;
             const int ch = row_l / kChunkTiles;
-            const int tile0 = (int)(sm.chunkbase[s][ch] * 32u + sm.rowoff[row_l]);
-            const uint32_t* in = sm.in[s];
+            const int tile0 = (int)(sm.chunkbase[ch] * 32u + sm.rowoff[row_l]);
+            const uint32_t* in = sm.in;
             if constexpr (LAT == HQ_E8) {
                 const int cpos = tile0 + tau * (V / 8);
                 const int cw = min(max(cpos >> 5, 0), G::IN_WORDS - 2);
@@ -201,33 +203,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
             uint32_t sq = 0;
             if (tau == 0) {
                 BitReader<true> br;
-                br.lim = G::IN_WORDS - 1;
-                br.begin(in, tile0 + COSB);
-                constexpr int CNT = TPT == 1 ? N / 2 : V;
+                br.begin(in, tile0 + COSB, G::IN_WORDS - 1);
+                constexpr int G8 = (TPT == 1 ? N / 2 : V) / 8;
+#pragma unroll 1
+                for (int g = 0; g < G8; ++g) {
+                    uint32_t z[8];
 #pragma unroll
-                for (int i = 0; i < CNT; ++i) {
-                    const uint32_t z = br.code(k, sq_meta, ok);
-                    sq += z >> k;
-                    sym[i] = unzigzag(z);
+                    for (int j = 0; j < 8; ++j) {
+                        z[j] = get_code<true>(br, k, sq_meta, ok);
+                        sq += z[j] >> k;
+                    }
+                    *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
+                                                          z[4] | (z[5] << 16), z[6] | (z[7] << 16));
                 }
             }
             if (TPT == 1 || tau == 1) {
                 BitReader<false> br;
-                br.lim = G::IN_WORDS - 1;
-                br.begin(in, tile0 + (int)L - 1);
-                constexpr int FIRST = TPT == 1 ? N / 2 : 0;
+                br.begin(in, tile0 + (int)L - 1, G::IN_WORDS - 1);
+                constexpr int G0 = (TPT == 1 ? N / 2 : 0) / 8;
+#pragma unroll 1
+                for (int g = V / 8 - 1; g >= G0; --g) {
+                    uint32_t z[8];
 #pragma unroll
-                for (int i = V - 1; i >= FIRST; --i) {
-                    const uint32_t z = br.code(k, sq_meta, ok);
-                    sq += z >> k;
-                    sym[i] = unzigzag(z);
+                    for (int j = 7; j >= 0; --j) {
+                        z[j] = get_code<false>(br, k, sq_meta, ok);
+                        sq += z[j] >> k;
+                    }
+                    *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
+                                                          z[4] | (z[5] << 16), z[6] | (z[7] << 16));
                 }
             }
             sq_part = sq;
-            sq_want = sq_meta;
-        } else {
-#pragma unroll
-            for (int i = 0; i < V; ++i) sym[i] = 0;
         }
         if constexpr (TPT == 2) sq_part += __shfl_xor_sync(0xffffffffu, sq_part, 1);
         if (ok && sq_part != sq_want) ok = false;
@@ -236,23 +242,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
             ok = ok && other;
         }
         if (valid && stage_ok && !ok) status_set(a.ws, kStCorrupt);
+        __syncthreads();  // the input stage is consumed: fetch the next item's words
+        if (tid == 0) issue_item<N, DST>(sm, a, item + (int64_t)gridDim.x);
 
         // ---------------- codes -> lattice point (float pairs) ----------------
         float2 P[H];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
 #pragma unroll
-            for (int b = 0; b < H / D; ++b) {
-                const int pos = half * H + b * D;
-                int32_t v[D];
-                unstrip_block<LAT>(sym + pos, (cosbits >> (pos / 8)) & 1u, v);
+            for (int g8 = 0; g8 < H / 8; ++g8) {
+                const uint4 w = *zz_slot(sm.buf, half * (H / 8) + g8, tid);
+                const uint32_t zw[4] = {w.x, w.y, w.z, w.w};
+                int32_t sym[8];
 #pragma unroll
-                for (int i = 0; i < D; ++i) {
-                    float f = __int_as_float(v[i] + __float_as_int(kMagic)) - kMagic;  // exact, |v| < 2^22
-                    if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
-                    if (!ok) f = 0.0f;
-                    if (half) P[b * D + i].y = f;
-                    else P[b * D + i].x = f;
+                for (int j = 0; j < 8; ++j) sym[j] = ok ? unzigzag((zw[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) : 0;
+#pragma unroll
+                for (int b = 0; b < 8 / D; ++b) {
+                    const int pos = half * H + g8 * 8 + b * D;
+                    int32_t v[D];
+                    unstrip_block<LAT>(sym + b * D, (cosbits >> (pos / 8)) & 1u, v);
+#pragma unroll
+                    for (int i = 0; i < D; ++i) {
+                        float f = __int_as_float(v[i] + __float_as_int(kMagic)) - kMagic;  // exact, |v| < 2^22
+                        if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
+                        if (half) P[g8 * 8 + b * D + i].y = f;
+                        else P[g8 * 8 + b * D + i].x = f;
+                    }
                 }
             }
         }
@@ -275,6 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
                     }
                 }
             }
+        }
+        if (!ok) {
+#pragma unroll
+            for (int m = 0; m < H; ++m) P[m] = make_float2(0.0f, 0.0f);
         }
 
         // ---------------- inverse transform: H_n p, exact for integer points ----------------
@@ -311,9 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
 #pragma unroll
         for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], h2);
 
-        if (tid == 0) bulk_wait_read0();  // previous item's store has read the staging box
-        __syncthreads();
-        // thread-local position pos -> row element e = tau*V + pos
+        __syncthreads();  // every thread has read its scratch: the box may be overwritten
         if constexpr (DST == 0) {
             // bf16: 8 elements per 16-byte chunk; chunk c holds elements 8c .. 8c+7
 #pragma unroll
@@ -330,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
                         w[q] = bits ^ sm.mask[e0 / 2 + q];
                     }
                     const int cg = e0 / 8;
-                    *reinterpret_cast<uint4*>(sm.out + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
+                    *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
@@ -347,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
                         w[q] = __float_as_uint(f) ^ sm.mask[e0 + q];
                     }
                     const int cg = e0 / 4;
-                    *reinterpret_cast<uint4*>(sm.out + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
+                    *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
@@ -357,10 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeArgs a,
         if (tid == 0) {
 #pragma unroll
             for (int b = 0; b < G::NB; ++b)
-                tma_store_2d(&tmap, (int)(jt * N + b * (128 / G::ES)), (int)r0, sm.out + b * TI * 128);
+                tma_store_2d(&tmap, (int)(jt * N + b * (128 / G::ES)), (int)r0, sm.buf + b * TI * 128);
             bulk_commit();
-            // refill this input stage with the item kStages ahead
-            issue_item<N, DST>(sm, a, s, item + (int64_t)kStages * gridDim.x);
         }
     }
     if (tid == 0) bulk_wait0();

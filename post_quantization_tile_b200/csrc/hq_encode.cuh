@@ -43,9 +43,13 @@ struct EncGeom {
     static constexpr int ROWB = N * ES;    // bytes per tile row
     static constexpr int NB = ROWB / 128;  // 128-byte boxes per row
     static constexpr int STAGE = NB * TI * 128;
+    static constexpr int ZZ = V * 2 * kThreads;  // zig-zag symbol scratch (uint16), aliases the stage
+    static constexpr int BUF = STAGE > ZZ ? STAGE : ZZ;
     static constexpr int CH = TI / kChunkTiles;  // chunks per item
-    // worst-case tile bits: n/8 coset + n (k + 1) with k <= 15 + sum q < 2n
-    static constexpr int LMAX = N / 8 + 16 * N + 2 * N;
+    // staging bound per tile: n/8 coset bits + n (k + 1) + sum q with k <= 11 and sum q < 2n.
+    // The step range keeps k <= 9; longer tiles are reported (HQ_ERR_RANGE) and left out.
+    static constexpr int KMAX = 11;
+    static constexpr int LMAX = N / 8 + (KMAX + 1) * N + 2 * N;
     static constexpr int STG_WORDS = TI * ((LMAX + 31) / 32) + CH + 8;
     static constexpr int LOG2N = N == 64 ? 6 : (N == 128 ? 7 : 8);
     static constexpr int MASKS = SRC == 0 ? N / 2 : N;  // sign-mask words per tile column
@@ -54,19 +58,24 @@ struct EncGeom {
 template <int N, int SRC>
 struct EncSmem {
     using G = EncGeom<N, SRC>;
-    alignas(1024) unsigned char stage[kStages][G::STAGE];
+    alignas(1024) unsigned char buf[G::BUF];  // TMA stage, then the zig-zag scratch
     uint32_t stg[G::STG_WORDS];
     alignas(16) uint32_t mask[G::MASKS];
     uint32_t Ls[G::TI];
     uint32_t rowoff[G::TI];
     uint32_t chunkoff[G::CH + 1];
-    int64_t item_ring[kStages];
+    int64_t item_cur;
     int64_t mask_jt;
     uint32_t item_words;
     uint32_t base;
-    uint32_t flags;
-    alignas(8) uint64_t bar[kStages];
+    alignas(8) uint64_t bar;
 };
+
+// zig-zag scratch: symbols 8g .. 8g+7 of thread t at byte (g * kThreads + t) * 16
+__device__ __forceinline__ uint4* zz_slot(unsigned char* buf, int g, int tid)
+{
+    return reinterpret_cast<uint4*>(buf + ((size_t)g * kThreads + tid) * 16);
+}
 
 // ------------------------------------------------------------------------------------------------
 // sign masks of tile column jt: D_jj = -1 where bit (J & 31) of Philox(seed, (J >> 7, 0, 0, 0))
@@ -237,8 +246,20 @@ __device__ __forceinline__ void fwht_pairs(float2 (&P)[H])
             }
 }
 
+template <int N, int SRC>
+__device__ __forceinline__ void issue_tma(EncSmem<N, SRC>& sm, const CUtensorMap* tmap, const EncodeArgs& a, int64_t it)
+{
+    using G = EncGeom<N, SRC>;
+    if (it >= a.items) return;
+    const int64_t jt = it / a.IB, ib = it % a.IB;
+    mbar_arrive_expect_tx(&sm.bar, G::STAGE);
+#pragma unroll
+    for (int b = 0; b < G::NB; ++b)
+        tma_load_2d(sm.buf + b * G::TI * 128, tmap, (int)(jt * N + b * (128 / G::ES)), (int)(ib * G::TI), &sm.bar);
+}
+
 template <int N, int LAT, bool KV, int SRC, bool COUNT>
-__global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a, const __grid_constant__ CUtensorMap tmap)
+__global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a, const __grid_constant__ CUtensorMap tmap)
 {
     using G = EncGeom<N, SRC>;
     using SM = EncSmem<N, SRC>;
@@ -254,29 +275,17 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
     const int tau = tid % TPT;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+        mbar_init(&sm.bar, 1);
         fence_mbar_init();
         sm.mask_jt = -1;
-        // claim and launch the first kStages items
-        for (int s = 0; s < kStages; ++s) {
-            const int64_t it = (int64_t)atomicAdd(&a.ws->counter, 1u);
-            sm.item_ring[s] = it;
-            if (it < a.items) {
-                const int64_t jt = it / a.IB, ib = it % a.IB;
-                mbar_arrive_expect_tx(&sm.bar[s], G::STAGE);
-#pragma unroll
-                for (int b = 0; b < G::NB; ++b)
-                    tma_load_2d(sm.stage[s] + b * TI * 128, &tmap, (int)(jt * (G::ROWB / G::ES) + b * (128 / G::ES)),
-                                (int)(ib * TI), &sm.bar[s]);
-            }
-        }
+        const int64_t it = (int64_t)atomicAdd(&a.ws->counter, 1u);
+        sm.item_cur = it;
+        issue_tma<N, SRC>(sm, &tmap, a, it);
     }
     __syncthreads();
 
     for (int iter = 0;; ++iter) {
-        const int s = iter % kStages;
-        const uint32_t parity = (uint32_t)((iter / kStages) & 1);
-        const int64_t item = sm.item_ring[s];
+        const int64_t item = sm.item_cur;
         if (item >= a.items) break;
         const int64_t jt = item / a.IB, ib = item % a.IB;
         const int64_t r0 = ib * TI;
@@ -290,28 +299,17 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
                 if (tid == 0) sm.mask_jt = jt;
             }
         }
-        if (!mbar_wait(&sm.bar[s], parity)) status_set(a.ws, kStTimeout);
+        if (!mbar_wait(&sm.bar, (uint32_t)(iter & 1))) status_set(a.ws, kStTimeout);
 
         float2 P[H];
         float sumsq;
-        load_row<N, SRC>(sm.stage[s], sm.mask, row_l, tau, P, sumsq);
-        __syncthreads();  // stage s consumed; mask table free
-        if (tid == 0) {
-            const int64_t nxt = (int64_t)atomicAdd(&a.ws->counter, 1u);
-            sm.item_ring[s] = nxt;
-            if (nxt < a.items) {
-                const int64_t njt = nxt / a.IB, nib = nxt % a.IB;
-                mbar_arrive_expect_tx(&sm.bar[s], G::STAGE);
-#pragma unroll
-                for (int b = 0; b < G::NB; ++b)
-                    tma_load_2d(sm.stage[s] + b * TI * 128, &tmap,
-                                (int)(njt * (G::ROWB / G::ES) + b * (128 / G::ES)), (int)(nib * TI), &sm.bar[s]);
-            }
-        }
+        load_row<N, SRC>(sm.buf, sm.mask, row_l, tau, P, sumsq);
+        unsigned int next_claim = 0;
+        if (tid == 0) next_claim = atomicAdd(&a.ws->counter, 1u);  // used once the stage is free
+        __syncthreads();  // [A] the stage is consumed: sm.buf becomes the zig-zag scratch
 
         // ---------------- per-tile scale, RHT, normalisation ----------------
         uint16_t sbits = 0;
-        bool zero_tile = false;
         if constexpr (SRC != 2) {
             if constexpr (TPT == 2) {
                 const float other = __shfl_xor_sync(0xffffffffu, sumsq, 1);
@@ -325,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
                 status_set(a.ws, kStNonfinite);
                 atomicAdd(&a.ws->nonfinite, 1u);
             }
-            zero_tile = !finite || sh < 1.2621774483536189e-29f;  // 2^-96
+            const bool zero_tile = !finite || sh < 1.2621774483536189e-29f;  // 2^-96
             if (zero_tile) sbits = 0;
             fwht_pairs<H>(P);
             const float t = __fmul_rn(sh, a.beta);
@@ -359,50 +357,68 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
             }
         }
 
-        // ---------------- lattice + strip ----------------
-        int32_t sym[V];
+        // ---------------- lattice + strip -> zig-zag scratch ----------------
+        uint32_t A = 0, zor = 0;
         uint32_t cosbits = 0;  // coset bit of local block lb at bit lb (E8)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
 #pragma unroll
-            for (int b = 0; b < H / D; ++b) {
-                float u[D];
+            for (int g8 = 0; g8 < H / 8; ++g8) {
+                int32_t sym[8];
 #pragma unroll
-                for (int i = 0; i < D; ++i) u[i] = half ? P[b * D + i].y : P[b * D + i].x;
-                int32_t v[D];
-                quantize_block<LAT>(u, v);
-                const int pos = half * H + b * D;
-                if constexpr (SRC == 2) {
-                    if (valid && a.v_out) {
-                        int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V + pos;
+                for (int b = 0; b < 8 / D; ++b) {
+                    const int pos = half * H + g8 * 8 + b * D;
+                    float u[D];
 #pragma unroll
-                        for (int i = 0; i < D; ++i) vo[i] = v[i];
+                    for (int i = 0; i < D; ++i) u[i] = half ? P[g8 * 8 + b * D + i].y : P[g8 * 8 + b * D + i].x;
+                    int32_t v[D];
+                    quantize_block<LAT>(u, v);
+                    if constexpr (SRC == 2) {
+                        if (valid && a.v_out) {
+                            int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V + pos;
+#pragma unroll
+                            for (int i = 0; i < D; ++i) vo[i] = v[i];
+                        }
                     }
+                    const uint32_t c = strip_block<LAT>(v, sym + b * D);
+                    if constexpr (LAT == HQ_E8) cosbits |= c << (pos / 8);
                 }
-                const uint32_t c = strip_block<LAT>(v, sym + pos);
-                if constexpr (LAT == HQ_E8) cosbits |= c << (pos / 8);
+                uint32_t z[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    z[i] = zigzag(sym[i]);
+                    A += z[i];
+                    if constexpr (SRC == 2) zor |= z[i];
+                }
+                *zz_slot(sm.buf, half * (H / 8) + g8, tid) =
+                    make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16), z[4] | (z[5] << 16), z[6] | (z[7] << 16));
             }
         }
 
         // ---------------- Rice parameter and tile length ----------------
-        uint32_t A = 0;
-#pragma unroll
-        for (int i = 0; i < V; ++i) A += zigzag(sym[i]);
         if constexpr (TPT == 2) A += __shfl_xor_sync(0xffffffffu, A, 1);
         const int k = rice_k(A, G::LOG2N);
         uint32_t sq = 0;
-#pragma unroll
-        for (int i = 0; i < V; ++i) sq += zigzag(sym[i]) >> k;
+#pragma unroll 4
+        for (int g = 0; g < V / 8; ++g) {
+            const uint4 w = *zz_slot(sm.buf, g, tid);
+            sq += ((w.x & 0xFFFFu) >> k) + ((w.x >> 16) >> k) + ((w.y & 0xFFFFu) >> k) + ((w.y >> 16) >> k) +
+                  ((w.z & 0xFFFFu) >> k) + ((w.z >> 16) >> k) + ((w.w & 0xFFFFu) >> k) + ((w.w >> 16) >> k);
+        }
         uint32_t sq_tile = sq;
         if constexpr (TPT == 2) sq_tile += __shfl_xor_sync(0xffffffffu, sq, 1);
         const uint32_t L = (uint32_t)COSB + (uint32_t)N * (uint32_t)(k + 1) + sq_tile;
         // the staging stream holds at most LMAX bits per tile; longer tiles (only reachable with
         // caller-given coefficients of huge magnitude) are reported and left out
-        const bool fits_tile = L <= (uint32_t)G::LMAX;
+        bool fits_tile = L <= (uint32_t)G::LMAX && k <= G::KMAX;
+        if constexpr (SRC == 2) {
+            if constexpr (TPT == 2) zor |= __shfl_xor_sync(0xffffffffu, zor, 1);
+            fits_tile = fits_tile && zor <= 0xFFFFu;
+        }
         if (!fits_tile && valid && tau == 0) status_set(a.ws, kStRange);
         const bool emit = valid && fits_tile;
         if (tau == 0) sm.Ls[row_l] = emit ? L : 0u;
-        __syncthreads();
+        __syncthreads();  // [B]
 
         // ---------------- chunk layout of the item (warp 0) ----------------
         if (warp == 0) {
@@ -421,12 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
                 if (lane == 0) sm.chunkoff[ch] = acc_words;
                 acc_words += (tot + 31) >> 5;
             }
+            uint32_t bits = 0;
+            if constexpr (COUNT) {
+#pragma unroll
+                for (int ch = 0; ch < G::CH; ++ch) bits += sm.Ls[ch * 32 + lane];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) bits += __shfl_xor_sync(0xffffffffu, bits, o);
+            }
             if (lane == 0) {
                 sm.chunkoff[G::CH] = acc_words;
                 sm.item_words = acc_words;
                 if constexpr (COUNT) {
-                    uint32_t bits = 0;
-                    for (int i = 0; i < TI; ++i) bits += sm.Ls[i];
                     atomicAdd(&a.ws->count_bits, (unsigned long long)bits);
                 } else {
                     const unsigned long long st = ((item == 0 ? 2ull : 1ull) << 32) | acc_words;
@@ -434,12 +455,19 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
                 }
             }
         }
-        __syncthreads();
-        if constexpr (COUNT) continue;
+        __syncthreads();  // [C]
+        if constexpr (COUNT) {
+            if (tid == 0) {
+                sm.item_cur = next_claim;
+                issue_tma<N, SRC>(sm, &tmap, a, next_claim);
+            }
+            __syncthreads();
+            continue;
+        }
 
         const uint32_t item_words = sm.item_words;
         for (uint32_t w = tid; w < item_words + 2; w += kThreads) sm.stg[w] = 0u;
-        __syncthreads();
+        __syncthreads();  // [D]
 
         // ---------------- Rice bits into the staging stream ----------------
         if (emit) {
@@ -455,39 +483,36 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
             const uint32_t km = (1u << k) - 1u;
             const uint32_t one = 1u << k;
             if (tau == 0) {
+                // first half, forward from the tile start
                 BitWriter<true> bw;
                 bw.begin(sm.stg, tile0 + COSB);
-                constexpr int CNT = TPT == 1 ? N / 2 : V;
-#pragma unroll
-                for (int i = 0; i < CNT; ++i) {
-                    const uint32_t z = zigzag(sym[i]);
-                    const uint32_t q = z >> k;
-                    if (q > 31 - k) {
-                        bw.zeros(q);
-                        bw.put(one | (z & km), k + 1);
-                    } else {
-                        bw.put(one | (z & km), (int)q + k + 1);
-                    }
+                constexpr int G8 = (TPT == 1 ? N / 2 : V) / 8;
+#pragma unroll 1
+                for (int g = 0; g < G8; ++g) {
+                    const uint4 w = *zz_slot(sm.buf, g, tid);
+                    put4<true>(bw, w.x & 0xFFFFu, w.x >> 16, w.y & 0xFFFFu, w.y >> 16, k, km, one);
+                    put4<true>(bw, w.z & 0xFFFFu, w.z >> 16, w.w & 0xFFFFu, w.w >> 16, k, km, one);
                 }
                 bw.finish();
             }
             if (TPT == 1 || tau == 1) {
+                // second half, backward from the tile's last bit (symbols in decreasing order)
                 BitWriter<false> bw;
                 bw.begin(sm.stg, tile0 + (int)L - 1);
-                constexpr int FIRST = TPT == 1 ? N / 2 : 0;
-#pragma unroll
-                for (int i = V - 1; i >= FIRST; --i) {
-                    const uint32_t z = zigzag(sym[i]);
-                    const uint32_t q = z >> k;
-                    if (q > 31 - k) {
-                        bw.zeros(q);
-                        bw.put(one | (z & km), k + 1);
-                    } else {
-                        bw.put(one | (z & km), (int)q + k + 1);
-                    }
+                constexpr int G0 = (TPT == 1 ? N / 2 : 0) / 8;
+#pragma unroll 1
+                for (int g = V / 8 - 1; g >= G0; --g) {
+                    const uint4 w = *zz_slot(sm.buf, g, tid);
+                    put4<false>(bw, w.w >> 16, w.w & 0xFFFFu, w.z >> 16, w.z & 0xFFFFu, k, km, one);
+                    put4<false>(bw, w.y >> 16, w.y & 0xFFFFu, w.x >> 16, w.x & 0xFFFFu, k, km, one);
                 }
                 bw.finish();
             }
+        }
+        __syncthreads();  // [E] scratch free: load the next item
+        if (tid == 0) {
+            sm.item_cur = next_claim;
+            issue_tma<N, SRC>(sm, &tmap, a, next_claim);
         }
 
         // ---------------- look-back for the item's word offset (warp 0) ----------------
@@ -525,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(const EncodeArgs a,
                 sm.base = excl;
             }
         }
-        __syncthreads();
+        __syncthreads();  // [F]
 
         // ---------------- store: bits, chunk offsets, scale, meta ----------------
         const uint32_t base = sm.base;
