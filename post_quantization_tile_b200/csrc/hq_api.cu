@@ -110,6 +110,21 @@ bool resolve_params(const hq_params_t* p, hq_params_t& out)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Make the device that owns `p` current for this library's CUDA runtime, so that launches and
+// tensor maps follow the caller's data (callers switch devices in their own runtime).
+bool use_device_of(const void* p)
+{
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return false;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return false;
+    return cur == attr.device || cudaSetDevice(attr.device) == cudaSuccess;
+}
+
 hq_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
 
 cudaError_t run_encode(int lattice, int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m,
@@ -155,6 +170,7 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
     }
     if (bound_words(rows, cols, prm.tile) >= ((int64_t)1 << 32)) return HQ_ERR_RANGE;
 
+    if (!use_device_of(x)) return HQ_ERR_ARG;
     const int es = src == 0 ? 2 : 4;
     CUtensorMap map;
     if (!make_map(&map, x, rows, cols, es, g.TI)) return HQ_ERR_CUDA;
@@ -213,6 +229,7 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
     if (!geometry(code->rows, code->cols, prm.tile, g)) return HQ_ERR_ARG;
     if (!code->scale || !code->meta || !code->chunk_word || !code->bits || !aligned16(code->bits)) return HQ_ERR_ARG;
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
+    if (!use_device_of(y)) return HQ_ERR_ARG;
     const int es = dtype == HQ_BF16 ? 2 : 4;
     CUtensorMap map;
     if (!make_map(&map, y, code->rows, code->cols, es, g.TI)) return HQ_ERR_CUDA;
@@ -334,6 +351,7 @@ hq_status_t hq_encode_count(const void* x, hq_dtype_t dtype, int64_t rows, int64
 hq_status_t hq_status_read(const void* ws, void* stream, int64_t* detail)
 {
     if (!ws) return HQ_ERR_ARG;
+    if (!use_device_of(ws)) return HQ_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
     WsHeader h;
