@@ -12,8 +12,9 @@
  *
  * Conventions shared by every entry point
  *   - Every pointer argument named as a device pointer must point to memory of the current CUDA
- *     device; the library never allocates, frees or keeps global state, and never synchronises
- *     except in hq_status_read.  All work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *     device; the library never allocates or frees memory and keeps no state between calls
+ *     besides cached driver entry points and the fixed scratch array of hq_encode_noalloc; it
+ *     never synchronises except in hq_status_read.  All work is enqueued on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and the call returns at once.
  *   - The synchronous return value reports argument errors (HQ_ERR_ARG, HQ_ERR_UNSUPPORTED) and
  *     launch failures (HQ_ERR_CUDA).  Errors found by the kernels (non-finite input, too small
@@ -184,6 +185,31 @@ const char* hq_status_str(hq_status_t s);
 
 /* HQ_FORMAT_VERSION of the built library. */
 int32_t hq_version(void);
+
+/*
+ * Allocation-free weight encode.  The method has no counterpart for this entry point; it exists
+ * for callers that must not allocate GPU memory at encode time -- an inference engine that
+ * owns its memory pool and forbids further allocations while it serves, code running between
+ * two synchronisation points where cudaMalloc / cudaFree would stall every stream of the
+ * device, or a host language runtime without a device allocator.  Such a caller passes only the
+ * input and the output arrays (out->scale, meta, chunk_word, bits as for hq_encode).
+ *
+ * The encoder's scratch (status word, work counter, one look-back slot per block of 128 tiles)
+ * is a fixed array of HQ_NOALLOC_SCRATCH_BYTES compiled into the library, present on every GPU
+ * that loads it until the process exits.  It covers tensors with
+ *     64 + 8 * (cols / tile) * ceil(rows / (tile == 256 ? 64 : 128)) <= HQ_NOALLOC_SCRATCH_BYTES
+ * (e.g. 8192 x 28672 at tile 256, 16384 x 8192 at tile 128); larger tensors get HQ_ERR_RANGE
+ * and nothing is enqueued.  The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress) for that device; make that first call before capturing the stream
+ * into a graph.  All calls share the one array and each call clears it on `stream` before its
+ * kernel runs, so calls whose work overlaps on the GPU (different streams without ordering)
+ * race and must not be issued.  Device errors (capacity, non-finite input, timeout) are copied
+ * as the status bit word (1 << hq_status_t) to *status_out (device uint32) when it is not
+ * NULL.  No allocation, no synchronisation.
+ */
+#define HQ_NOALLOC_SCRATCH_BYTES (128 * 1024)
+hq_status_t hq_encode_noalloc(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                              hq_code_t* out, uint32_t* status_out, void* stream);
 
 #ifdef __cplusplus
 }
