@@ -172,9 +172,9 @@ void hqo_fwht_f64(double* x, int n)
 /* Shared pieces:                                                                              */
 /*   a = rint(u) (ties to even), e = a - u (exact in binary32, and never -0);                  */
 /*   "toward u" for a coordinate is +1 when e < 0, else -1;                                     */
-/*   argmax / argmin of |e| compare max(|e|, 2^-63) and break ties to the lowest index.        */
+/*   argmax / argmin of |e| compare max(|e|, 2^-31) and break ties to the lowest index.        */
 /* ------------------------------------------------------------------------------------------ */
-static const float TINY = 1.0842021724855044e-19f; /* 2^-63 */
+static const float TINY = 4.6566128730773926e-10f; /* 2^-31 */
 
 static float clamp_tiny(float v) { return v < TINY ? TINY : v; }
 

@@ -75,7 +75,8 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f)
 }
 
 __device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 f2sub(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+// a - b as a fused multiply-add with an exact product: one rounding, like the subtraction
+__device__ __forceinline__ float2 f2sub(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
 __device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // ------------------------------------------------------------------------------------------------
@@ -327,27 +328,42 @@ __device__ __forceinline__ uint32_t long_run(BitReader<FWD>& br, uint32_t limit,
     return q;
 }
 
-// one Rice code: q zeros, a one, r (k bits MSB-first); returns the zig-zag value q << k | r
+// one Rice code: q zeros, a one, r (k bits MSB-first); returns the zig-zag value q << k | r and
+// adds q to sq.  The caller keeps at least 33 valid bits in the window before a pair of codes;
+// a code that is longer than the bits at hand takes the slow path (refill, long runs).
 template <bool FWD>
-__device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t limit, bool& ok)
+__device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t pow2k, uint32_t limit, bool& ok,
+                                             uint32_t& sq)
 {
-    br.refill();
     uint32_t hi = (uint32_t)(br.W >> 32);
-    uint32_t q = 0;
-    if (hi == 0u) {
-        q = long_run<FWD>(br, limit, ok);
+    int z = __clz(hi);
+    int lam = z + k + 1;
+    if (hi == 0u || lam > br.avail) {
+        br.refill();
         hi = (uint32_t)(br.W >> 32);
-        if (!ok) return 0u;
+        uint32_t q = 0;
+        if (hi == 0u) {
+            q = long_run<FWD>(br, limit, ok);
+            hi = (uint32_t)(br.W >> 32);
+            if (!ok) return 0u;
+        }
+        z = __clz(hi);
+        br.W <<= (z + 1);
+        br.avail -= z + 1;
+        if (br.avail < k) br.refill();
+        const uint32_t r = k ? (uint32_t)(br.W >> (64 - k)) : 0u;
+        br.W <<= k;
+        br.avail -= k;
+        q += (uint32_t)z;
+        sq += q;
+        return (q << k) | r;
     }
-    const int z = __clz(hi);
-    q += (uint32_t)z;
-    br.W <<= (z + 1);
-    br.avail -= z + 1;
-    if (br.avail < k) br.refill();
-    const uint32_t r = k ? (uint32_t)(br.W >> (64 - k)) : 0u;
-    br.W <<= k;
-    br.avail -= k;
-    return (q << k) | r;
+    // fast path: the whole code is in the top 32 bits: 0..0 1 r
+    const uint32_t val = hi >> (32 - lam);      // (1 << k) | r
+    br.W <<= lam;
+    br.avail -= lam;
+    sq += (uint32_t)z;
+    return (uint32_t)z * pow2k + (val - pow2k);  // (z << k) | r
 }
 
 // ------------------------------------------------------------------------------------------------

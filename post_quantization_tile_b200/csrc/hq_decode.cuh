@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
         const int k = (int)(mt & 15u);
         if (ok) {
             const uint32_t sq_meta = mt >> 4;
+            const uint32_t pow2k = 1u << k;
             sq_want = sq_meta;
             const int ch = row_l / kChunkTiles;
             const int tile0 = (int)(sm.chunkbase[ch] * 32u + sm.rowoff[row_l]);
@@ -210,8 +211,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                     uint32_t z[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        z[j] = get_code<true>(br, k, sq_meta, ok);
-                        sq += z[j] >> k;
+                        if ((j & 1) == 0) br.refill();
+                        z[j] = get_code<true>(br, k, pow2k, sq_meta, ok, sq);
                     }
                     *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
                                                           z[4] | (z[5] << 16), z[6] | (z[7] << 16));
@@ -226,8 +227,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                     uint32_t z[8];
 #pragma unroll
                     for (int j = 7; j >= 0; --j) {
-                        z[j] = get_code<false>(br, k, sq_meta, ok);
-                        sq += z[j] >> k;
+                        if ((j & 1) == 1) br.refill();
+                        z[j] = get_code<false>(br, k, pow2k, sq_meta, ok, sq);
                     }
                     *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
                                                           z[4] | (z[5] << 16), z[6] | (z[7] << 16));
@@ -343,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                     for (int q = 0; q < 4; ++q) {
                         const float lo = half ? P[8 * c + 2 * q].y : P[8 * c + 2 * q].x;
                         const float hi = half ? P[8 * c + 2 * q + 1].y : P[8 * c + 2 * q + 1].x;
-                        const uint32_t bits = (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
-                        w[q] = bits ^ sm.mask[e0 / 2 + q];
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);  // one packed RNE conversion
+                        w[q] = *reinterpret_cast<const uint32_t*>(&b2) ^ sm.mask[e0 / 2 + q];
                     }
                     const int cg = e0 / 8;
                     *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =

@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
 #pragma unroll
                     for (int i = 0; i < D; ++i) u[i] = half ? P[g8 * 8 + b * D + i].y : P[g8 * 8 + b * D + i].x;
                     int32_t v[D];
-                    quantize_block<LAT>(u, v);
+                    const uint32_t c = quantize_strip<LAT, SRC == 2>(u, sym + b * D, v);
                     if constexpr (SRC == 2) {
                         if (valid && a.v_out) {
                             int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V + pos;
@@ -380,7 +380,6 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
                             for (int i = 0; i < D; ++i) vo[i] = v[i];
                         }
                     }
-                    const uint32_t c = strip_block<LAT>(v, sym + b * D);
                     if constexpr (LAT == HQ_E8) cosbits |= c << (pos / 8);
                 }
                 uint32_t z[8];

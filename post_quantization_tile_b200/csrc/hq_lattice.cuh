@@ -5,16 +5,30 @@
 // quantizers and codes" (IEEE T-IT 28(2), 1982), in binary32 without contraction:
 //   a = rint(u) via the 1.5*2^23 addition (exact for |u| < 2^22, which the per-tile RMS scaling
 //   and the step range guarantee), e = a - u (exact, never -0), "toward u" = +1 when e < 0;
-//   argmax / argmin of |e| compare max(|e|, 2^-63), ties to the lowest index.
+//   argmax / argmin of |e| compare max(|e|, 2^-31), ties to the lowest index.  The comparison
+//   runs on 32-bit keys (clamped |e| bits << 4 | index << 1 | sign of e): the clamped bits of
+//   |e| in [2^-31, 1/2] all start with 0011, so the shift drops nothing that orders them, and one
+//   integer max / min returns the value, the lowest tied index and the sign together.
 #pragma once
 
 #include "hq_common.cuh"
 
 namespace hq {
 
-constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-constexpr float kTiny = 1.0842021724855044e-19f;  // 2^-63
-constexpr float kA2K = 1.15470053837925153f;      // RN(2/sqrt(3))
+constexpr float kMagic = 12582912.0f;         // 1.5 * 2^23
+constexpr uint32_t kTinyBits = 0x30000000u;   // 2^-31
+constexpr float kA2K = 1.15470053837925153f;  // RN(2/sqrt(3))
+
+template <int LAT>
+struct Lat;
+template <>
+struct Lat<HQ_Z> { static constexpr int d = 1; };
+template <>
+struct Lat<HQ_A2> { static constexpr int d = 2; };
+template <>
+struct Lat<HQ_D4> { static constexpr int d = 4; };
+template <>
+struct Lat<HQ_E8> { static constexpr int d = 8; };
 
 __device__ __forceinline__ float rint_magic(float u, int32_t& ai)
 {
@@ -23,80 +37,93 @@ __device__ __forceinline__ float rint_magic(float u, int32_t& ai)
     return __fadd_rn(t, -kMagic);
 }
 
-__device__ __forceinline__ float clamp_tiny(float v) { return v < kTiny ? kTiny : v; }
+// argmax key of coordinate i of a d-block: clamped |e| bits, then index (d-1-i, so the lowest
+// index wins ties), then the sign of e
+__device__ __forceinline__ uint32_t max_key(float e, int i, int d)
+{
+    const uint32_t eb = __float_as_uint(e);
+    const uint32_t mag = max(eb & 0x7FFFFFFFu, kTinyBits);
+    return (mag << 4) | ((uint32_t)(d - 1 - i) << 1) | (eb >> 31);
+}
+__device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float((key >> 4) | kTinyBits); }
 
-// D4 = {v in Z^4, sum even}; v = the nearest point.
+// D4 = {v in Z^4, sum even}; v = the nearest point: round, and if the sum is odd move the
+// coordinate with the largest rounding error one step toward u.
 __device__ __forceinline__ void q_d4(const float (&u)[4], int32_t (&v)[4])
 {
-    float e[4];
     int32_t sum = 0;
+    uint32_t kmax = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float r = rint_magic(u[i], v[i]);
-        e[i] = __fadd_rn(r, -u[i]);
         sum += v[i];
+        kmax = max(kmax, max_key(__fadd_rn(r, -u[i]), i, 4));
     }
-    if (sum & 1) {
-        int j = 0;
-        float best = clamp_tiny(fabsf(e[0]));
+    const int j = 3 - (int)((kmax >> 1) & 7u);
+    const int32_t delta = (sum & 1) ? ((kmax & 1u) ? 1 : -1) : 0;
 #pragma unroll
-        for (int i = 1; i < 4; ++i) {
-            const float c = clamp_tiny(fabsf(e[i]));
-            if (c > best) { best = c; j = i; }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (i == j) v[i] += (e[i] < 0.0f) ? 1 : -1;
-    }
+    for (int i = 0; i < 4; ++i)
+        if (i == j) v[i] += delta;
 }
 
-// E8 = D8 u (D8 + 1/2): v = twice the nearest point.  The coset choice compares
+// E8 = D8 u (D8 + 1/2), fused with bit-stripping.  Returns the coset bit c and writes the 8
+// symbols (w0 .. w6, (w7 - p)/2) of the nearest point v/2 (v doubled coordinates, w = (v - c)/2);
+// v itself when WANT_V.  The coset choice compares
 // |u-A|^2 - |u-B|^2 = sum(|e| - 1/4) + [A fixed](1 - 2 max|e|) - [B fixed](2 min|e|) in binary32
 // as D = ((S - 2) + cA) - cB, S the pairwise sum of |e|; B only when D > 0.
-__device__ __forceinline__ void q_e8(const float (&u)[8], int32_t (&v)[8])
+//   A: w = a; if sum a is odd the coordinate with max |e| moves toward u.
+//   B: w = a - [e >= 0] (w + 1/2 is the half-integer toward u); if sum w is odd the coordinate
+//      with min |e| moves to its other half-integer neighbour.
+template <bool WANT_V>
+__device__ __forceinline__ uint32_t e8_symbols(const float (&u)[8], int32_t (&s)[8], int32_t* v)
 {
-    float e[8], ae[8];
     int32_t a[8];
-    int32_t sumA = 0, nonneg = 0;
+    float ae[8];
+    uint32_t eb[8];
+    uint32_t kmax = 0u, kmin = 0xFFFFFFFFu, tx = 0u, sx = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float r = rint_magic(u[i], a[i]);
-        e[i] = __fadd_rn(r, -u[i]);
-        ae[i] = fabsf(e[i]);
-        sumA += a[i];
-        nonneg += (e[i] < 0.0f) ? 0 : 1;
+        const float t = __fadd_rn(u[i], kMagic);
+        a[i] = __float_as_int(t) - __float_as_int(kMagic);
+        const float e = __fadd_rn(__fadd_rn(t, -kMagic), -u[i]);
+        ae[i] = fabsf(e);
+        eb[i] = __float_as_uint(e);
+        const uint32_t key = max_key(e, i, 8);
+        kmax = max(kmax, key);
+        kmin = min(kmin, key ^ 0xEu);  // index bits flipped: ties go to the lowest index
+        tx ^= __float_as_uint(t);      // bit 0: parity of sum a (the magic constant is even)
+        sx ^= eb[i];                   // bit 31: parity of #{e < 0} (e is never -0)
     }
-    const int parA = sumA & 1;
-    const int parB = (sumA - nonneg) & 1;
+    const uint32_t parA = tx & 1u;
+    const uint32_t parB = parA ^ (sx >> 31);  // sum w = sum a - #{e >= 0}, and 8 is even
     const float S = __fadd_rn(__fadd_rn(__fadd_rn(ae[0], ae[1]), __fadd_rn(ae[2], ae[3])),
                               __fadd_rn(__fadd_rn(ae[4], ae[5]), __fadd_rn(ae[6], ae[7])));
-    int jA = 0, mB = 0;
-    float emax = clamp_tiny(ae[0]), emin = emax;
-#pragma unroll
-    for (int i = 1; i < 8; ++i) {
-        const float c = clamp_tiny(ae[i]);
-        if (c > emax) { emax = c; jA = i; }
-        if (c < emin) { emin = c; mB = i; }
-    }
-    const float cA = parA ? __fadd_rn(1.0f, -__fmul_rn(2.0f, emax)) : 0.0f;
-    const float cB = parB ? __fmul_rn(2.0f, emin) : 0.0f;
+    const float cA = parA ? __fadd_rn(1.0f, -__fmul_rn(2.0f, key_value(kmax))) : 0.0f;
+    const float cB = parB ? __fmul_rn(2.0f, key_value(kmin)) : 0.0f;
     const float D = __fadd_rn(__fadd_rn(__fadd_rn(S, -2.0f), cA), -cB);
-    if (!(D > 0.0f)) {
+    const bool isB = D > 0.0f;
+    // the coordinate to fix and its direction: A moves toward u (+1 when e < 0), B away from it
+    const uint32_t kf = isB ? kmin : kmax;
+    const int fix = isB ? (int)((kmin >> 1) & 7u) : 7 - (int)((kmax >> 1) & 7u);
+    const uint32_t dofix = isB ? parB : parA;
+    const int32_t delta = dofix ? ((((kf & 1u) != 0u) != isB) ? 1 : -1) : 0;
+    const uint32_t bmask = isB ? 0xFFFFFFFFu : 0u;
+    int32_t w[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            int32_t ai = a[i];
-            if (parA && i == jA) ai += (e[i] < 0.0f) ? 1 : -1;
-            v[i] = 2 * ai;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int32_t toward = (e[i] < 0.0f) ? 1 : -1;
-            int32_t vi = 2 * a[i] + toward;
-            if (parB && i == mB) vi -= 2 * toward;
-            v[i] = vi;
-        }
+    for (int i = 0; i < 8; ++i) {
+        w[i] = a[i] - (int32_t)((~eb[i] & bmask) >> 31);
+        if (i == fix) w[i] += delta;
     }
+    const int32_t p = (w[0] ^ w[1] ^ w[2] ^ w[3] ^ w[4] ^ w[5] ^ w[6]) & 1;
+#pragma unroll
+    for (int i = 0; i < 7; ++i) s[i] = w[i];
+    s[7] = (w[7] - p) >> 1;
+    const uint32_t c = isB ? 1u : 0u;
+    if constexpr (WANT_V) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 2 * w[i] + (int32_t)c;
+    }
+    return c;
 }
 
 // A2 with minimum distance 1 in (P, Q) = (2 u0, u1 K); the even point when |eP| + 3|eQ| <= 1.
@@ -115,45 +142,6 @@ __device__ __forceinline__ void q_a2(const float (&u)[2], int32_t (&v)[2])
     } else {
         v[0] = 2 * aP + ((eP < 0.0f) ? 1 : -1);
         v[1] = 2 * aQ + ((eQ < 0.0f) ? 1 : -1);
-    }
-}
-
-template <int LAT>
-struct Lat;
-template <>
-struct Lat<HQ_Z> { static constexpr int d = 1; };
-template <>
-struct Lat<HQ_A2> { static constexpr int d = 2; };
-template <>
-struct Lat<HQ_D4> { static constexpr int d = 4; };
-template <>
-struct Lat<HQ_E8> { static constexpr int d = 8; };
-
-// nearest point of one block: u[d] -> integer embedding v[d]
-template <int LAT>
-__device__ __forceinline__ void quantize_block(const float* u, int32_t* v)
-{
-    if constexpr (LAT == HQ_Z) {
-        rint_magic(u[0], v[0]);
-    } else if constexpr (LAT == HQ_A2) {
-        const float uu[2] = {u[0], u[1]};
-        int32_t vv[2];
-        q_a2(uu, vv);
-        v[0] = vv[0]; v[1] = vv[1];
-    } else if constexpr (LAT == HQ_D4) {
-        const float uu[4] = {u[0], u[1], u[2], u[3]};
-        int32_t vv[4];
-        q_d4(uu, vv);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = vv[i];
-    } else {
-        float uu[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) uu[i] = u[i];
-        int32_t vv[8];
-        q_e8(uu, vv);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = vv[i];
     }
 }
 
@@ -186,6 +174,45 @@ __device__ __forceinline__ uint32_t strip_block(const int32_t* v, int32_t* s)
     }
 }
 
+// nearest point of one block and its stripped symbols: u[d] -> symbols s[d] (+ E8 coset bit);
+// the integer embedding v[d] is written when WANT_V
+template <int LAT, bool WANT_V>
+__device__ __forceinline__ uint32_t quantize_strip(const float* u, int32_t* s, int32_t* v)
+{
+    if constexpr (LAT == HQ_E8) {
+        float uu[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) uu[i] = u[i];
+        int32_t ss[8];
+        const uint32_t c = e8_symbols<WANT_V>(uu, ss, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i] = ss[i];
+        return c;
+    } else {
+        int32_t vv[Lat<LAT>::d];
+        if constexpr (LAT == HQ_Z) {
+            rint_magic(u[0], vv[0]);
+        } else if constexpr (LAT == HQ_A2) {
+            const float uu[2] = {u[0], u[1]};
+            int32_t t2[2];
+            q_a2(uu, t2);
+            vv[0] = t2[0];
+            vv[1] = t2[1];
+        } else {
+            const float uu[4] = {u[0], u[1], u[2], u[3]};
+            int32_t t4[4];
+            q_d4(uu, t4);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) vv[i] = t4[i];
+        }
+        if constexpr (WANT_V) {
+#pragma unroll
+            for (int i = 0; i < Lat<LAT>::d; ++i) v[i] = vv[i];
+        }
+        return strip_block<LAT>(vv, s);
+    }
+}
+
 // inverse of strip_block: symbols (+ coset bit) -> integer embedding
 template <int LAT>
 __device__ __forceinline__ void unstrip_block(const int32_t* s, uint32_t c, int32_t* v)
@@ -200,7 +227,7 @@ __device__ __forceinline__ void unstrip_block(const int32_t* s, uint32_t c, int3
         v[0] = s[0]; v[1] = s[1]; v[2] = s[2];
         v[3] = 2 * s[3] + p;
     } else {
-        const int32_t p = (s[0] + s[1] + s[2] + s[3] + s[4] + s[5] + s[6]) & 1;
+        const int32_t p = (s[0] ^ s[1] ^ s[2] ^ s[3] ^ s[4] ^ s[5] ^ s[6]) & 1;
 #pragma unroll
         for (int i = 0; i < 7; ++i) v[i] = 2 * s[i] + (int32_t)c;
         v[7] = 2 * (2 * s[7] + p) + (int32_t)c;
