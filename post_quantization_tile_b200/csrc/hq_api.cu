@@ -67,12 +67,13 @@ struct Geometry {
     int TI;
 };
 
-bool geometry(int64_t rows, int64_t cols, int32_t n, Geometry& g)
+// tiles per block item: 128 threads, `tpt` threads per tile (encoder and decoder may differ)
+bool geometry(int64_t rows, int64_t cols, int32_t n, Geometry& g, int tpt = 2)
 {
     if (!valid_tile(n) || rows < 1 || cols < n || cols % n) return false;
     if (rows > (int64_t)1 << 31 || cols > (int64_t)1 << 31) return false;
     const int64_t NT = cols / n;
-    g.TI = kThreads / tpt_for(n);
+    g.TI = kThreads / tpt;
     g.RB = (rows + kChunkTiles - 1) / kChunkTiles;
     g.C = NT * g.RB;
     g.T = NT * rows;
@@ -93,7 +94,8 @@ int64_t bound_words(int64_t rows, int64_t cols, int32_t n)
 size_t ws_bytes_for(int64_t rows, int64_t cols, int32_t n)
 {
     Geometry g;
-    if (!geometry(rows, cols, n, g)) return 0;
+    // the encoder with the most items for this tile (bf16 input shares a tile the most)
+    if (!geometry(rows, cols, n, g, n == 64 ? 1 : (n == 256 ? 2 : enc_tpt(128, 0)))) return 0;
     return sizeof(WsHeader) + (size_t)g.items * 8u;
 }
 
@@ -156,7 +158,8 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
     hq_params_t prm;
     if (!resolve_params(p, prm)) return HQ_ERR_ARG;
     Geometry g;
-    if (!geometry(rows, cols, prm.tile, g)) return HQ_ERR_ARG;
+    const int tpt = prm.tile == 64 ? 1 : (prm.tile == 256 ? 2 : enc_tpt(128, src));
+    if (!geometry(rows, cols, prm.tile, g, tpt)) return HQ_ERR_ARG;
     if (kv && prm.lattice != HQ_D4) return HQ_ERR_UNSUPPORTED;
     if (kv && cols != prm.tile) return HQ_ERR_ARG;
     if (src == 1 && prm.tile == 256) return HQ_ERR_UNSUPPORTED;
@@ -226,7 +229,7 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
     if (!(prm.step >= 0.00390625f && prm.step <= 64.0f)) return HQ_ERR_ARG;
     if (kv && prm.lattice != HQ_D4) return HQ_ERR_UNSUPPORTED;
     Geometry g;
-    if (!geometry(code->rows, code->cols, prm.tile, g)) return HQ_ERR_ARG;
+    if (!geometry(code->rows, code->cols, prm.tile, g, dec_tpt(prm.tile))) return HQ_ERR_ARG;
     if (!code->scale || !code->meta || !code->chunk_word || !code->bits || !aligned16(code->bits)) return HQ_ERR_ARG;
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
     if (!use_device_of(y)) return HQ_ERR_ARG;

@@ -39,8 +39,21 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 64, "workspace header");
 
-// threads per tile: one thread holds n/TPT coefficients in registers
-__host__ __device__ constexpr int tpt_for(int n) { return n == 256 ? 2 : 1; }
+// threads per tile: one thread holds n/TPT coefficients in registers.  Two threads share a tile
+// of 256 (256 registers of coefficients would not fit); for n = 128 the choice is a build option
+// (the bit format does not depend on it).
+#ifndef HQ_ENC_TPT128
+#define HQ_ENC_TPT128 1
+#endif
+#ifndef HQ_DEC_TPT128
+#define HQ_DEC_TPT128 1
+#endif
+// src: 0 bf16 weight, 1 fp32 weight, 2 fp32 coefficients (fp32 weights keep one thread per tile)
+__host__ __device__ constexpr int enc_tpt(int n, int src)
+{
+    return (n == 256 || (n == 128 && src != 1 && HQ_ENC_TPT128 == 2)) ? 2 : 1;
+}
+__host__ __device__ constexpr int dec_tpt(int n) { return (n == 256 || (n == 128 && HQ_DEC_TPT128 == 2)) ? 2 : 1; }
 
 // ------------------------------------------------------------------------------------------------
 // Philox4x32-10 (Salmon et al., SC'11): published multipliers and Weyl key increments.

@@ -30,7 +30,7 @@ struct DecodeArgs {
 
 template <int N, int DST>  // DST: 0 bf16, 1 fp32
 struct DecGeom {
-    static constexpr int TPT = tpt_for(N);
+    static constexpr int TPT = dec_tpt(N);
     static constexpr int V = N / TPT;
     static constexpr int H = V / 2;
     static constexpr int TI = kThreads / TPT;
@@ -202,10 +202,35 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                 cosbits = (uint32_t)(two >> (cpos & 31)) & ((V / 8) >= 32 ? 0xffffffffu : ((1u << (V / 8)) - 1u));
             }
             uint32_t sq = 0;
-            if (tau == 0) {
+            if constexpr (TPT == 1) {
+                // both halves in one loop: independent forward and backward readers
+                BitReader<true> rf;
+                BitReader<false> rb;
+                rf.begin(in, tile0 + COSB, G::IN_WORDS - 1);
+                rb.begin(in, tile0 + (int)L - 1, G::IN_WORDS - 1);
+                uint32_t sqb = 0;
+#pragma unroll 1
+                for (int g = 0; g < N / 16; ++g) {
+                    uint32_t zf[8], zb[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if ((j & 1) == 0) {
+                            rf.refill();
+                            rb.refill();
+                        }
+                        zf[j] = get_code<true>(rf, k, pow2k, sq_meta, ok, sq);
+                        zb[7 - j] = get_code<false>(rb, k, pow2k, sq_meta, ok, sqb);
+                    }
+                    *zz_slot(sm.buf, g, tid) = make_uint4(zf[0] | (zf[1] << 16), zf[2] | (zf[3] << 16),
+                                                          zf[4] | (zf[5] << 16), zf[6] | (zf[7] << 16));
+                    *zz_slot(sm.buf, V / 8 - 1 - g, tid) = make_uint4(zb[0] | (zb[1] << 16), zb[2] | (zb[3] << 16),
+                                                                      zb[4] | (zb[5] << 16), zb[6] | (zb[7] << 16));
+                }
+                sq += sqb;
+            } else if (tau == 0) {
                 BitReader<true> br;
                 br.begin(in, tile0 + COSB, G::IN_WORDS - 1);
-                constexpr int G8 = (TPT == 1 ? N / 2 : V) / 8;
+                constexpr int G8 = V / 8;
 #pragma unroll 1
                 for (int g = 0; g < G8; ++g) {
                     uint32_t z[8];
@@ -218,10 +243,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                                                           z[4] | (z[5] << 16), z[6] | (z[7] << 16));
                 }
             }
-            if (TPT == 1 || tau == 1) {
+            else {
                 BitReader<false> br;
                 br.begin(in, tile0 + (int)L - 1, G::IN_WORDS - 1);
-                constexpr int G0 = (TPT == 1 ? N / 2 : 0) / 8;
+                constexpr int G0 = 0;
 #pragma unroll 1
                 for (int g = V / 8 - 1; g >= G0; --g) {
                     uint32_t z[8];

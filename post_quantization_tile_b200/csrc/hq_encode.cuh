@@ -35,7 +35,7 @@ struct EncodeArgs {
 // SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
 template <int N, int SRC>
 struct EncGeom {
-    static constexpr int TPT = tpt_for(N);
+    static constexpr int TPT = enc_tpt(N, SRC);
     static constexpr int V = N / TPT;      // coefficients per thread
     static constexpr int H = V / 2;        // float2 pairs per thread: P[m] = (c[m], c[m + H])
     static constexpr int TI = kThreads / TPT;  // tiles (rows) per item
@@ -146,17 +146,18 @@ __device__ __forceinline__ void load_row(const unsigned char* stage, const uint3
                 for (int m = 0; m < H; m += 2 * h) Q[m] = f2add(Q[m], Q[m + h]);
             sumsq = __fadd_rn(Q[0].x, Q[0].y);
         } else {
-            // N = 256, V = 128, H = 64: quarter k (0..3) of the row = elements 64k .. 64k+63
+            // quarter k (0..3) of the row = elements k n/4 .. (k+1) n/4 - 1 = chunks k QC .. (k+1) QC - 1
+            constexpr int QC = N / 32;
             float2 Q[H];
             const float2 sgn = tau ? make_float2(-1.0f, -1.0f) : make_float2(1.0f, 1.0f);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < QC; ++c) {
                 uint4 X[4];
                 uint32_t x[4][4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    X[k] = *chunk_ptr(c + 8 * k);
-                    const uint4 M = *reinterpret_cast<const uint4*>(mask + 4 * (c + 8 * k));
+                    X[k] = *chunk_ptr(c + QC * k);
+                    const uint4 M = *reinterpret_cast<const uint4*>(mask + 4 * (c + QC * k));
                     x[k][0] = X[k].x ^ M.x; x[k][1] = X[k].y ^ M.y; x[k][2] = X[k].z ^ M.z; x[k][3] = X[k].w ^ M.w;
                 }
 #pragma unroll
@@ -168,7 +169,7 @@ __device__ __forceinline__ void load_row(const unsigned char* stage, const uint3
                                              : make_float2(bf16lo_to_f32(x[0][q]), bf16lo_to_f32(x[1][q]));
                         const float2 hi = hh ? make_float2(bf16hi_to_f32(x[2][q]), bf16hi_to_f32(x[3][q]))
                                              : make_float2(bf16lo_to_f32(x[2][q]), bf16lo_to_f32(x[3][q]));
-                        // this thread's half of the RMS: tau 0 sums x[0..128), tau 1 x[128..256)
+                        // this thread's half of the RMS: tau 0 sums x[0, n/2), tau 1 x[n/2, n)
                         Q[m] = tau ? f2mul(hi, hi) : f2mul(lo, lo);
                         // first butterfly, stride n/2: tau 0 keeps sums, tau 1 differences
                         P[m] = __ffma2_rn(hi, sgn, lo);
@@ -213,11 +214,11 @@ __device__ __forceinline__ void load_row(const unsigned char* stage, const uint3
                 sumsq = 0.0f;
             }
         } else {
-            // coefficients with n = 256: thread tau holds positions tau*128 + [0, 128)
+            // coefficients, two threads per tile: thread tau holds positions tau V + [0, V)
 #pragma unroll
             for (int c = 0; c < H / 4; ++c) {
-                const uint4 A = *chunk_ptr(tau * 32 + c);
-                const uint4 B = *chunk_ptr(tau * 32 + c + H / 4);
+                const uint4 A = *chunk_ptr(tau * (G::V / 4) + c);
+                const uint4 B = *chunk_ptr(tau * (G::V / 4) + c + H / 4);
                 P[4 * c + 0] = make_float2(__uint_as_float(A.x), __uint_as_float(B.x));
                 P[4 * c + 1] = make_float2(__uint_as_float(A.y), __uint_as_float(B.y));
                 P[4 * c + 2] = make_float2(__uint_as_float(A.z), __uint_as_float(B.z));
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
     const int row_l = tid / TPT;   // row within the item
     const int tau = tid % TPT;
 
+    for (int w = tid; w < G::STG_WORDS; w += kThreads) sm.stg[w] = 0u;
     if (tid == 0) {
         mbar_init(&sm.bar, 1);
         fence_mbar_init();
@@ -464,9 +466,8 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
             continue;
         }
 
+        // the staging stream is all zero here: cleared once at start, then by each copy-out
         const uint32_t item_words = sm.item_words;
-        for (uint32_t w = tid; w < item_words + 2; w += kThreads) sm.stg[w] = 0u;
-        __syncthreads();  // [D]
 
         // ---------------- Rice bits into the staging stream ----------------
         if (emit) {
@@ -481,11 +482,29 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
             }
             const uint32_t km = (1u << k) - 1u;
             const uint32_t one = 1u << k;
-            if (tau == 0) {
+            if constexpr (TPT == 1) {
+                // both halves in one loop: the forward writer (first half, from the tile start)
+                // and the backward writer (second half, from the tile's last bit) are independent
+                BitWriter<true> bf;
+                BitWriter<false> bb;
+                bf.begin(sm.stg, tile0 + COSB);
+                bb.begin(sm.stg, tile0 + (int)L - 1);
+#pragma unroll 1
+                for (int g = 0; g < N / 16; ++g) {
+                    const uint4 wf = *zz_slot(sm.buf, g, tid);
+                    const uint4 wb = *zz_slot(sm.buf, V / 8 - 1 - g, tid);
+                    put4<true>(bf, wf.x & 0xFFFFu, wf.x >> 16, wf.y & 0xFFFFu, wf.y >> 16, k, km, one);
+                    put4<false>(bb, wb.w >> 16, wb.w & 0xFFFFu, wb.z >> 16, wb.z & 0xFFFFu, k, km, one);
+                    put4<true>(bf, wf.z & 0xFFFFu, wf.z >> 16, wf.w & 0xFFFFu, wf.w >> 16, k, km, one);
+                    put4<false>(bb, wb.y >> 16, wb.y & 0xFFFFu, wb.x >> 16, wb.x & 0xFFFFu, k, km, one);
+                }
+                bf.finish();
+                bb.finish();
+            } else if (tau == 0) {
                 // first half, forward from the tile start
                 BitWriter<true> bw;
                 bw.begin(sm.stg, tile0 + COSB);
-                constexpr int G8 = (TPT == 1 ? N / 2 : V) / 8;
+                constexpr int G8 = V / 8;
 #pragma unroll 1
                 for (int g = 0; g < G8; ++g) {
                     const uint4 w = *zz_slot(sm.buf, g, tid);
@@ -494,11 +513,11 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
                 }
                 bw.finish();
             }
-            if (TPT == 1 || tau == 1) {
+            else {
                 // second half, backward from the tile's last bit (symbols in decreasing order)
                 BitWriter<false> bw;
                 bw.begin(sm.stg, tile0 + (int)L - 1);
-                constexpr int G0 = (TPT == 1 ? N / 2 : 0) / 8;
+                constexpr int G0 = 0;
 #pragma unroll 1
                 for (int g = V / 8 - 1; g >= G0; --g) {
                     const uint4 w = *zz_slot(sm.buf, g, tid);
@@ -555,9 +574,13 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
         const uint32_t base = sm.base;
         const bool fits = (int64_t)base + (int64_t)item_words <= a.cap_words;
         if (fits) {
-            for (uint32_t w = tid; w < item_words; w += kThreads) a.bits[base + w] = sm.stg[w];
-        } else if (tid == 0) {
-            status_set(a.ws, kStCapacity);
+            for (uint32_t w = tid; w < item_words; w += kThreads) {
+                a.bits[base + w] = sm.stg[w];
+                sm.stg[w] = 0u;
+            }
+        } else {
+            for (uint32_t w = tid; w < item_words; w += kThreads) sm.stg[w] = 0u;
+            if (tid == 0) status_set(a.ws, kStCapacity);
         }
         const int nch = (rows_valid + kChunkTiles - 1) / kChunkTiles;
         const int64_t c0 = jt * a.RB + ib * G::CH;
