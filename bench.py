@@ -65,6 +65,22 @@ def oracle_sample(inputs, rows_per_matrix: int, steps: int):
     return gbs, t_total, elems
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The slowest rank's time: every multi-GPU number is the max over ranks."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(bytes_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job GB/s: every rank processes its own copy of the batch in ms_max."""
+    return world * bytes_per_rank / (ms_max * 1e-3) / 1e9
+
+
 def kernel_sources_hash() -> str:
     import glob
     import hashlib
@@ -258,11 +274,7 @@ def run_gpu(args):
         clk.mark(False)
     if world > 1:
         dist.barrier()
-    ms = t0.elapsed_time(t1) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
     enc_ms = [statistics.mean(enc_ev[k * len(SHAPES) + i][0].elapsed_time(enc_ev[k * len(SHAPES) + i][1])
                               for k in range(args.steps)) for i in range(len(SHAPES))]
     dec_ms = [statistics.mean(dec_ev[k * len(SHAPES) + i][0].elapsed_time(dec_ev[k * len(SHAPES) + i][1])
@@ -287,11 +299,7 @@ def run_gpu(args):
     c1 = torch.cuda.Event(enable_timing=True)
     c1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = c0.elapsed_time(c1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(c0.elapsed_time(c1) / e2e_steps, dev)
     st, _ = hq.status(ws)
 
     peak, peak_kind = load_peaks()
@@ -304,7 +312,7 @@ def run_gpu(args):
     else:
         kname, kms, kbytes = "decode", dec_ms[i_big], dec_bytes
     achieved = kbytes / (kms * 1e-3) / 1e9
-    value = world * bf16_bytes / (ms * 1e-3) / 1e9
+    value = weak_scaling_value(bf16_bytes, world, ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -331,7 +339,7 @@ def run_gpu(args):
                          "bytes_per_launch": kbytes,
                          "traffic": measured_traffic(kname, SHAPES[i_big][0] * SHAPES[i_big][1])},
             "cpu_baseline": cpu,
-            "e2e": {"value": world * bf16_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": {"value": weak_scaling_value(bf16_bytes, world, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": bf16_bytes, "d2h_bytes_per_step": bf16_bytes},
             "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),

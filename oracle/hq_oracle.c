@@ -558,12 +558,13 @@ static int valid_kv(int kv, int lattice) { return !kv || lattice == HQO_D4; }
  *   outputs : scale[T] (bf16 bits of the per-tile RMS), meta[T] = k | (sum q << 4),
  *             chunk_word[C+1], bits[cap_words]; optional v_out[T*n] (integer codes) and
  *             u_out[T*n] (normalised coefficients before dither)
+ *   row0    : KV only: global row of x's first row (a slice of a larger KV tensor)
  * Returns a bitmask of status bits (0 = ok).
  */
 uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n, int lattice, float beta,
                     uint64_t seed, int kv, int64_t kv_S, uint16_t* scale, uint16_t* meta,
                     uint32_t* chunk_word, uint32_t* bits, int64_t cap_words, int32_t* v_out,
-                    float* u_out)
+                    float* u_out, int64_t row0)
 {
     if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || rows <= 0 || cols <= 0 || cols % n) return 1u << 1;
     uint32_t status = 0;
@@ -608,7 +609,7 @@ uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n,
                     for (int j = 0; j < n; ++j) u[j] = xt[j] * g;
                 }
                 int64_t bh = 0, sidx = r;
-                if (kv) kv_row(r, kv_S, &bh, &sidx);
+                if (kv) kv_row(row0 + r, kv_S, &bh, &sidx);
                 int32_t v[HQO_MAXN];
                 quantize_tile(u, n, lattice, kv, seed, bh, sidx, v);
                 int k, sumq;
@@ -754,7 +755,7 @@ static void reconstruct_tile(const int32_t* v, int n, int lattice, int kv, uint6
 /* Full decode to binary64 out[rows, cols].  Returns status bits. */
 uint32_t hqo_decode(const uint16_t* scale, const uint16_t* meta, const uint32_t* chunk_word, const uint32_t* bits,
                     int64_t rows, int64_t cols, int n, int lattice, float beta, uint64_t seed, int kv,
-                    int64_t kv_S, double* out)
+                    int64_t kv_S, double* out, int64_t row0)
 {
     if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || rows <= 0 || cols % n) return 1u << 1;
     const int64_t NT = cols / n;
@@ -765,7 +766,7 @@ uint32_t hqo_decode(const uint16_t* scale, const uint16_t* meta, const uint32_t*
         for (int64_t r = 0; r < rows; ++r) {
             int64_t t = jt * rows + r;
             int64_t bh = 0, sidx = r;
-            if (kv) kv_row(r, kv_S, &bh, &sidx);
+            if (kv) kv_row(row0 + r, kv_S, &bh, &sidx);
             double tile[HQO_MAXN];
             reconstruct_tile(v + t * n, n, lattice, kv, seed, bh, sidx, scale[t], beta, jt * n, tile);
             memcpy(out + r * cols + jt * n, tile, sizeof(double) * (size_t)n);
