@@ -48,6 +48,12 @@ static_assert(sizeof(WsHeader) == 64, "workspace header");
 #ifndef HQ_DEC_TPT128
 #define HQ_DEC_TPT128 1
 #endif
+#ifndef HQ_ENC_SEPARATE_ZZ
+#define HQ_ENC_SEPARATE_ZZ 0
+#endif
+#ifndef HQ_DEC_STAGES
+#define HQ_DEC_STAGES 1
+#endif
 // src: 0 bf16 weight, 1 fp32 weight, 2 fp32 coefficients (fp32 weights keep one thread per tile)
 __host__ __device__ constexpr int enc_tpt(int n, int src)
 {
@@ -342,7 +348,7 @@ __device__ __forceinline__ uint32_t long_run(BitReader<FWD>& br, uint32_t limit,
 }
 
 // one Rice code: q zeros, a one, r (k bits MSB-first); returns the zig-zag value q << k | r and
-// adds q to sq.  The caller keeps at least 33 valid bits in the window before a pair of codes;
+// adds q to sq.  The caller tops the window up to at least 33 bits every four codes;
 // a code that is longer than the bits at hand takes the slow path (refill, long runs).
 template <bool FWD>
 __device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t pow2k, uint32_t limit, bool& ok,

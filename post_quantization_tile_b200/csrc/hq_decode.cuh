@@ -48,21 +48,24 @@ struct DecGeom {
     static constexpr int IN_WORDS = (TI * ((LMAX + 31) / 32) + CH + 8 + 2 * GUARD + 3) / 4 * 4;
     static constexpr int MASKS = DST == 0 ? N / 2 : N;
     static constexpr int LOG2N = N == 64 ? 6 : (N == 128 ? 7 : 8);
+    // input stages: one (the next item is fetched once this one is parsed) or two (fetched a
+    // whole item ahead, at the cost of shared memory)
+    static constexpr int STAGES = HQ_DEC_STAGES;
 };
 
 template <int N, int DST>
 struct DecSmem {
     using G = DecGeom<N, DST>;
-    alignas(1024) unsigned char buf[G::BUF];   // zig-zag scratch, then the output TMA box
-    alignas(16) uint32_t in[G::IN_WORDS];      // the item's words (one stage)
+    alignas(1024) unsigned char buf[G::BUF];       // zig-zag scratch, then the output TMA box
+    alignas(16) uint32_t in[G::STAGES][G::IN_WORDS];  // the items' words
     alignas(16) uint32_t mask[G::MASKS];
     uint32_t Ls[G::TI];
     uint32_t rowoff[G::TI];
-    uint32_t chunkbase[G::CH + 1];  // chunk start word relative to the copied range
-    int64_t item_cur;
-    int32_t ok_cur;
+    uint32_t chunkbase[G::STAGES][G::CH + 1];  // chunk start word relative to the copied range
+    int64_t item_ring[G::STAGES];
+    int32_t ok_ring[G::STAGES];
     int64_t mask_jt;
-    alignas(8) uint64_t bar;
+    alignas(8) uint64_t bar[G::STAGES];
 };
 
 template <int N, int DST>
@@ -88,11 +91,11 @@ __device__ __forceinline__ void build_masks_out(uint32_t* mask, int64_t jt, uint
 // Producer (one thread): copy the words of item `it` into the input stage.  An item whose
 // chunk offsets are inconsistent with the buffers is flagged and decoded as zeros.
 template <int N, int DST>
-__device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs& a, int64_t it)
+__device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs& a, int s, int64_t it)
 {
     using G = DecGeom<N, DST>;
-    sm.item_cur = it;
-    sm.ok_cur = 0;
+    sm.item_ring[s] = it;
+    sm.ok_ring[s] = 0;
     if (it >= a.items) return;
     const int64_t jt = it / a.IB, ib = it % a.IB;
     const int64_t r0 = ib * G::TI;
@@ -104,16 +107,16 @@ __device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs
     const int64_t lo = w0 & ~(int64_t)3;
     const int64_t hi = (w1 + 3) & ~(int64_t)3;
     const bool good = w1 >= w0 && hi <= a.cap_words && (hi - lo) <= (int64_t)(G::IN_WORDS - 2 * G::GUARD);
-    for (int ch = 0; ch <= nch; ++ch) sm.chunkbase[ch] = (uint32_t)(a.chunk_word[c0 + ch] - lo + G::GUARD);
+    for (int ch = 0; ch <= nch; ++ch) sm.chunkbase[s][ch] = (uint32_t)(a.chunk_word[c0 + ch] - lo + G::GUARD);
     if (!good) status_set(a.ws, kStCorrupt);
     const uint32_t bytes = (uint32_t)((hi - lo) * 4);
     if (good && bytes) {
-        sm.ok_cur = 1;
-        mbar_arrive_expect_tx(&sm.bar, bytes);
-        bulk_load_1d(sm.in + G::GUARD, a.bits + lo, bytes, &sm.bar);
+        sm.ok_ring[s] = 1;
+        mbar_arrive_expect_tx(&sm.bar[s], bytes);
+        bulk_load_1d(sm.in[s] + G::GUARD, a.bits + lo, bytes, &sm.bar[s]);
     } else {
-        sm.ok_cur = good ? 1 : 0;
-        mbar_arrive(&sm.bar);  // complete the phase without data
+        sm.ok_ring[s] = good ? 1 : 0;
+        mbar_arrive(&sm.bar[s]);  // complete the phase without data
     }
 }
 
@@ -134,21 +137,23 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
     const int tau = tid % TPT;
 
     if (tid == 0) {
-        mbar_init(&sm.bar, 1);
+        for (int s = 0; s < G::STAGES; ++s) mbar_init(&sm.bar[s], 1);
         fence_mbar_init();
         sm.mask_jt = -1;
-        issue_item<N, DST>(sm, a, (int64_t)blockIdx.x);
+        for (int s = 0; s < G::STAGES; ++s) issue_item<N, DST>(sm, a, s, (int64_t)blockIdx.x + (int64_t)s * gridDim.x);
     }
     __syncthreads();
 
     for (int iter = 0;; ++iter) {
-        const int64_t item = sm.item_cur;
+        const int st = iter % G::STAGES;
+        const uint32_t parity = (uint32_t)((iter / G::STAGES) & 1);
+        const int64_t item = sm.item_ring[st];
         if (item >= a.items) break;
         const int64_t jt = item / a.IB, ib = item % a.IB;
         const int64_t r0 = ib * TI;
         const int rows_valid = (int)min((int64_t)TI, a.rows - r0);
         const bool valid = row_l < rows_valid;
-        const bool stage_ok = sm.ok_cur != 0;
+        const bool stage_ok = sm.ok_ring[st] != 0;
 
         if (sm.mask_jt != jt) {
             build_masks_out<N, DST>(sm.mask, jt, a.seed);
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                 sm.rowoff[ch * 32 + lane] = incl - v;
             }
         }
-        if (!mbar_wait(&sm.bar, (uint32_t)(iter & 1))) status_set(a.ws, kStTimeout);
+        if (!mbar_wait(&sm.bar[st], parity)) status_set(a.ws, kStTimeout);
         __syncthreads();
 
         // ---------------- parse: Rice codes -> zig-zag scratch ----------------
@@ -193,8 +198,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
             const uint32_t pow2k = 1u << k;
             sq_want = sq_meta;
             const int ch = row_l / kChunkTiles;
-            const int tile0 = (int)(sm.chunkbase[ch] * 32u + sm.rowoff[row_l]);
-            const uint32_t* in = sm.in;
+            const int tile0 = (int)(sm.chunkbase[st][ch] * 32u + sm.rowoff[row_l]);
+            const uint32_t* in = sm.in[st];
             if constexpr (LAT == HQ_E8) {
                 const int cpos = tile0 + tau * (V / 8);
                 const int cw = min(max(cpos >> 5, 0), G::IN_WORDS - 2);
@@ -214,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                     uint32_t zf[8], zb[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        if ((j & 1) == 0) {
+                        if ((j & 3) == 0) {
                             rf.refill();
                             rb.refill();
                         }
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                     uint32_t z[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        if ((j & 1) == 0) br.refill();
+                        if ((j & 3) == 0) br.refill();
                         z[j] = get_code<true>(br, k, pow2k, sq_meta, ok, sq);
                     }
                     *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
                     uint32_t z[8];
 #pragma unroll
                     for (int j = 7; j >= 0; --j) {
-                        if ((j & 1) == 1) br.refill();
+                        if ((j & 3) == 3) br.refill();
                         z[j] = get_code<false>(br, k, pow2k, sq_meta, ok, sq);
                     }
                     *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
@@ -269,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a,
         }
         if (valid && stage_ok && !ok) status_set(a.ws, kStCorrupt);
         __syncthreads();  // the input stage is consumed: fetch the next item's words
-        if (tid == 0) issue_item<N, DST>(sm, a, item + (int64_t)gridDim.x);
+        if (tid == 0) issue_item<N, DST>(sm, a, st, item + (int64_t)G::STAGES * gridDim.x);
 
         // ---------------- codes -> lattice point (float pairs) ----------------
         float2 P[H];

@@ -43,8 +43,12 @@ struct EncGeom {
     static constexpr int ROWB = N * ES;    // bytes per tile row
     static constexpr int NB = ROWB / 128;  // 128-byte boxes per row
     static constexpr int STAGE = NB * TI * 128;
-    static constexpr int ZZ = V * 2 * kThreads;  // zig-zag symbol scratch (uint16), aliases the stage
-    static constexpr int BUF = STAGE > ZZ ? STAGE : ZZ;
+    static constexpr int ZZ = V * 2 * kThreads;  // zig-zag symbol scratch (uint16)
+    // the scratch aliases the TMA stage (smaller footprint, 3 blocks per SM, the next item is
+    // loaded after packing) or has its own buffer (next item loaded as soon as the stage is read)
+    static constexpr bool SEPARATE_ZZ = HQ_ENC_SEPARATE_ZZ != 0;
+    static constexpr int BUF = SEPARATE_ZZ ? STAGE : (STAGE > ZZ ? STAGE : ZZ);
+    static constexpr int ZZBUF = SEPARATE_ZZ ? ZZ : 16;
     static constexpr int CH = TI / kChunkTiles;  // chunks per item
     // staging bound per tile: n/8 coset bits + n (k + 1) + sum q with k <= 11 and sum q < 2n.
     // The step range keeps k <= 9; longer tiles are reported (HQ_ERR_RANGE) and left out.
@@ -58,7 +62,8 @@ struct EncGeom {
 template <int N, int SRC>
 struct EncSmem {
     using G = EncGeom<N, SRC>;
-    alignas(1024) unsigned char buf[G::BUF];  // TMA stage, then the zig-zag scratch
+    alignas(1024) unsigned char buf[G::BUF];  // TMA stage (and the zig-zag scratch when aliased)
+    alignas(16) unsigned char zzbuf[G::ZZBUF];
     uint32_t stg[G::STG_WORDS];
     alignas(16) uint32_t mask[G::MASKS];
     uint32_t Ls[G::TI];
@@ -274,6 +279,7 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
     const int lane = tid & 31, warp = tid >> 5;
     const int row_l = tid / TPT;   // row within the item
     const int tau = tid % TPT;
+    unsigned char* const zzs = G::SEPARATE_ZZ ? sm.zzbuf : sm.buf;
 
     for (int w = tid; w < G::STG_WORDS; w += kThreads) sm.stg[w] = 0u;
     if (tid == 0) {
@@ -308,7 +314,13 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
         load_row<N, SRC>(sm.buf, sm.mask, row_l, tau, P, sumsq);
         unsigned int next_claim = 0;
         if (tid == 0) next_claim = atomicAdd(&a.ws->counter, 1u);  // used once the stage is free
-        __syncthreads();  // [A] the stage is consumed: sm.buf becomes the zig-zag scratch
+        __syncthreads();  // [A] the stage is consumed (and, aliased, becomes the zig-zag scratch)
+        if constexpr (G::SEPARATE_ZZ) {
+            if (tid == 0) {
+                sm.item_cur = next_claim;
+                issue_tma<N, SRC>(sm, &tmap, a, next_claim);
+            }
+        }
 
         // ---------------- per-tile scale, RHT, normalisation ----------------
         uint16_t sbits = 0;
@@ -362,6 +374,42 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
         // ---------------- lattice + strip -> zig-zag scratch ----------------
         uint32_t A = 0, zor = 0;
         uint32_t cosbits = 0;  // coset bit of local block lb at bit lb (E8)
+        auto store_group = [&](int group, const int32_t (&sym)[8]) {
+            uint32_t z[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                z[i] = zigzag(sym[i]);
+                A += z[i];
+                if constexpr (SRC == 2) zor |= z[i];
+            }
+            *zz_slot(zzs, group, tid) =
+                make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16), z[4] | (z[5] << 16), z[6] | (z[7] << 16));
+        };
+        if constexpr (LAT == HQ_E8) {
+            // pair-block g8: lane x is block g8 (positions 8 g8 ..), lane y block g8 + H/8
+#pragma unroll
+            for (int g8 = 0; g8 < H / 8; ++g8) {
+                float2 p8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) p8[i] = P[g8 * 8 + i];
+                int32_t sx[8], sy[8], vx[8], vy[8];
+                uint32_t cx, cy;
+                e8_pair_symbols<SRC == 2>(p8, sx, sy, cx, cy, vx, vy);
+                if constexpr (SRC == 2) {
+                    if (valid && a.v_out) {
+                        int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            vo[g8 * 8 + i] = vx[i];
+                            vo[H + g8 * 8 + i] = vy[i];
+                        }
+                    }
+                }
+                cosbits |= (cx << g8) | (cy << (H / 8 + g8));
+                store_group(g8, sx);
+                store_group(H / 8 + g8, sy);
+            }
+        } else {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -382,18 +430,11 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
                             for (int i = 0; i < D; ++i) vo[i] = v[i];
                         }
                     }
-                    if constexpr (LAT == HQ_E8) cosbits |= c << (pos / 8);
+                    (void)c;
                 }
-                uint32_t z[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    z[i] = zigzag(sym[i]);
-                    A += z[i];
-                    if constexpr (SRC == 2) zor |= z[i];
-                }
-                *zz_slot(sm.buf, half * (H / 8) + g8, tid) =
-                    make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16), z[4] | (z[5] << 16), z[6] | (z[7] << 16));
+                store_group(half * (H / 8) + g8, sym);
             }
+        }
         }
 
         // ---------------- Rice parameter and tile length ----------------
@@ -402,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
         uint32_t sq = 0;
 #pragma unroll 4
         for (int g = 0; g < V / 8; ++g) {
-            const uint4 w = *zz_slot(sm.buf, g, tid);
+            const uint4 w = *zz_slot(zzs, g, tid);
             sq += ((w.x & 0xFFFFu) >> k) + ((w.x >> 16) >> k) + ((w.y & 0xFFFFu) >> k) + ((w.y >> 16) >> k) +
                   ((w.z & 0xFFFFu) >> k) + ((w.z >> 16) >> k) + ((w.w & 0xFFFFu) >> k) + ((w.w >> 16) >> k);
         }
@@ -458,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
         }
         __syncthreads();  // [C]
         if constexpr (COUNT) {
-            if (tid == 0) {
+            if (!G::SEPARATE_ZZ && tid == 0) {
                 sm.item_cur = next_claim;
                 issue_tma<N, SRC>(sm, &tmap, a, next_claim);
             }
@@ -491,8 +532,8 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
                 bb.begin(sm.stg, tile0 + (int)L - 1);
 #pragma unroll 1
                 for (int g = 0; g < N / 16; ++g) {
-                    const uint4 wf = *zz_slot(sm.buf, g, tid);
-                    const uint4 wb = *zz_slot(sm.buf, V / 8 - 1 - g, tid);
+                    const uint4 wf = *zz_slot(zzs, g, tid);
+                    const uint4 wb = *zz_slot(zzs, V / 8 - 1 - g, tid);
                     put4<true>(bf, wf.x & 0xFFFFu, wf.x >> 16, wf.y & 0xFFFFu, wf.y >> 16, k, km, one);
                     put4<false>(bb, wb.w >> 16, wb.w & 0xFFFFu, wb.z >> 16, wb.z & 0xFFFFu, k, km, one);
                     put4<true>(bf, wf.z & 0xFFFFu, wf.z >> 16, wf.w & 0xFFFFu, wf.w >> 16, k, km, one);
@@ -507,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
                 constexpr int G8 = V / 8;
 #pragma unroll 1
                 for (int g = 0; g < G8; ++g) {
-                    const uint4 w = *zz_slot(sm.buf, g, tid);
+                    const uint4 w = *zz_slot(zzs, g, tid);
                     put4<true>(bw, w.x & 0xFFFFu, w.x >> 16, w.y & 0xFFFFu, w.y >> 16, k, km, one);
                     put4<true>(bw, w.z & 0xFFFFu, w.z >> 16, w.w & 0xFFFFu, w.w >> 16, k, km, one);
                 }
@@ -520,15 +561,15 @@ __global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a,
                 constexpr int G0 = 0;
 #pragma unroll 1
                 for (int g = V / 8 - 1; g >= G0; --g) {
-                    const uint4 w = *zz_slot(sm.buf, g, tid);
+                    const uint4 w = *zz_slot(zzs, g, tid);
                     put4<false>(bw, w.w >> 16, w.w & 0xFFFFu, w.z >> 16, w.z & 0xFFFFu, k, km, one);
                     put4<false>(bw, w.y >> 16, w.y & 0xFFFFu, w.x >> 16, w.x & 0xFFFFu, k, km, one);
                 }
                 bw.finish();
             }
         }
-        __syncthreads();  // [E] scratch free: load the next item
-        if (tid == 0) {
+        __syncthreads();  // [E] scratch free: load the next item (aliased scratch)
+        if (!G::SEPARATE_ZZ && tid == 0) {
             sm.item_cur = next_claim;
             issue_tma<N, SRC>(sm, &tmap, a, next_claim);
         }

@@ -74,8 +74,9 @@ __device__ __forceinline__ void q_d4(const float (&u)[4], int32_t (&v)[4])
 //   A: w = a; if sum a is odd the coordinate with max |e| moves toward u.
 //   B: w = a - [e >= 0] (w + 1/2 is the half-integer toward u); if sum w is odd the coordinate
 //      with min |e| moves to its other half-integer neighbour.
+// E8 decision from t = u + 1.5*2^23 and e = (t - 1.5*2^23) - u (computed by the caller)
 template <bool WANT_V>
-__device__ __forceinline__ uint32_t e8_symbols(const float (&u)[8], int32_t (&s)[8], int32_t* v)
+__device__ __forceinline__ uint32_t e8_from_te(const float (&tv)[8], const float (&ev)[8], int32_t (&s)[8], int32_t* v)
 {
     int32_t a[8];
     float ae[8];
@@ -83,9 +84,9 @@ __device__ __forceinline__ uint32_t e8_symbols(const float (&u)[8], int32_t (&s)
     uint32_t kmax = 0u, kmin = 0xFFFFFFFFu, tx = 0u, sx = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float t = __fadd_rn(u[i], kMagic);
+        const float t = tv[i];
         a[i] = __float_as_int(t) - __float_as_int(kMagic);
-        const float e = __fadd_rn(__fadd_rn(t, -kMagic), -u[i]);
+        const float e = ev[i];
         ae[i] = fabsf(e);
         eb[i] = __float_as_uint(e);
         const uint32_t key = max_key(e, i, 8);
@@ -124,6 +125,40 @@ __device__ __forceinline__ uint32_t e8_symbols(const float (&u)[8], int32_t (&s)
         for (int i = 0; i < 8; ++i) v[i] = 2 * w[i] + (int32_t)c;
     }
     return c;
+}
+
+template <bool WANT_V>
+__device__ __forceinline__ uint32_t e8_symbols(const float (&u)[8], int32_t (&s)[8], int32_t* v)
+{
+    float t[8], e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        t[i] = __fadd_rn(u[i], kMagic);
+        e[i] = __fadd_rn(__fadd_rn(t[i], -kMagic), -u[i]);
+    }
+    return e8_from_te<WANT_V>(t, e, s, v);
+}
+
+// two E8 blocks at once, one in each lane of eight float2 pairs: the rounding arithmetic runs on
+// paired binary32 operations (the same roundings as e8_symbols), the decisions per lane
+template <bool WANT_V>
+__device__ __forceinline__ void e8_pair_symbols(const float2 (&p)[8], int32_t (&sx)[8], int32_t (&sy)[8],
+                                                uint32_t& cx, uint32_t& cy, int32_t* vx, int32_t* vy)
+{
+    float tx[8], ty[8], ex[8], ey[8];
+    const float2 m2 = make_float2(kMagic, kMagic);
+    const float2 nm2 = make_float2(-kMagic, -kMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 t = __fadd2_rn(p[i], m2);
+        const float2 r = __fadd2_rn(t, nm2);
+        const float2 e = __ffma2_rn(p[i], neg1, r);  // r - u, exact product
+        tx[i] = t.x; ty[i] = t.y;
+        ex[i] = e.x; ey[i] = e.y;
+    }
+    cx = e8_from_te<WANT_V>(tx, ex, sx, vx);
+    cy = e8_from_te<WANT_V>(ty, ey, sy, vy);
 }
 
 // A2 with minimum distance 1 in (P, Q) = (2 u0, u1 K); the even point when |eP| + 3|eQ| <= 1.
