@@ -119,10 +119,11 @@ size_t hq_workspace_bytes(int64_t rows, int64_t cols, const hq_params_t* p);
 
 /*
  * Step for a target payload rate from the high-resolution approximation of an entropy-coded
- * lattice quantizer on Gaussian coefficients (RHT output, Methodology step 1 "approximately
- * Gaussian"): beta = 2^(h - R) / V^(1/d) with h = log2(sqrt(2 pi e)) and V, d the cell volume
+ * lattice quantizer on Gaussian coefficients (the RHT output is close to Gaussian, Methodology
+ * step 1): beta = 2^(h - R) / V^(1/d) with h = log2(sqrt(2 pi e)) and V, d the cell volume
  * and dimension of the lattice.  A starting point; hq_encode_count gives the realised rate for
- * an exact search ("within ~0.01 bps of any target", Methodology step 3).
+ * an exact search (the method lands the realised rate about 0.01 bps from its target,
+ * Methodology step 3).
  */
 float hq_step_for_rate(int32_t lattice, int32_t tile, float bps);
 

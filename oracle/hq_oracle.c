@@ -127,7 +127,7 @@ static float inv_sqrt_n(int n)
 
 /* ------------------------------------------------------------------------------------------ */
 /* Per-tile RMS: q_i = x_i * x_i, summed by the ascending pairwise tree (h = 1, 2, ..., n/2;   */
-/* q[i] += q[i+h] for i = 0 mod 2h), s = sqrt(q[0] * (1/n)).  "per-tile scaling" (Methodology  */
+/* q[i] += q[i+h] for i = 0 mod 2h), s = sqrt(q[0] * (1/n)).  per-tile scaling (Methodology    */
 /* step 2), RMS statistic as the workload description fixes it.                                */
 /* ------------------------------------------------------------------------------------------ */
 float hqo_rms(const float* x, int n)
@@ -370,7 +370,7 @@ static void unstrip_block(int lattice, const int32_t* sym, int coset, int32_t* v
 
 /* ------------------------------------------------------------------------------------------ */
 /* Rice coding (Methodology step 3).  zz = 2m (m >= 0) or -2m-1 (m < 0); the tile parameter   */
-/* k = min{k >= 0 : sum zz < n 2^(k+1)}, capped at 15 -- "k from the mean index": k is the     */
+/* k = min{k >= 0 : sum zz < n 2^(k+1)}, capped at 15 -- k follows the mean index: k is the   */
 /* smallest k with mean(zz) < 2^(k+1), the rational form of the mean-based Rice parameter that  */
 /* is optimal for geometric sources (it codes Gaussian-like symbols within ~0.06 bit of their  */
 /* entropy, where k = ceil(log2 mean) loses ~0.3 bit).  q = zz >> k, r = zz & (2^k - 1).  Below */

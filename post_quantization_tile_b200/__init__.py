@@ -297,7 +297,7 @@ def encode_count(x: torch.Tensor, tile: int, lattice: int | str, step: float, se
 def calibrate_step(x: torch.Tensor, tile: int, lattice: int | str, target_bps: float, seed: int = 0,
                    kv: bool = False, kv_S: int = 0, iters: int = 24) -> float:
     """Bisection on log(step) with count-only encodes so the payload rate hits target_bps
-    ("within ~0.01 bps of any target", Methodology step 3)."""
+    (the method lands the realised rate about 0.01 bps from its target, Methodology step 3)."""
     import math
     n = x.numel()
     lo, hi = math.log(2.0 ** -8), math.log(2.0 ** 6)

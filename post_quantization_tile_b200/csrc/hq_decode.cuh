@@ -121,7 +121,7 @@ __device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs
 }
 
 template <int N, int LAT, bool KV, int DST>
-__global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap)
+__global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap)
 {
     using G = DecGeom<N, DST>;
     using SM = DecSmem<N, DST>;

@@ -265,7 +265,7 @@ __device__ __forceinline__ void issue_tma(EncSmem<N, SRC>& sm, const CUtensorMap
 }
 
 template <int N, int LAT, bool KV, int SRC, bool COUNT>
-__global__ void __launch_bounds__(kThreads, 3) encode_kernel(const EncodeArgs a, const __grid_constant__ CUtensorMap tmap)
+__global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const EncodeArgs a, const __grid_constant__ CUtensorMap tmap)
 {
     using G = EncGeom<N, SRC>;
     using SM = EncSmem<N, SRC>;
