@@ -187,6 +187,7 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
     a.cols = cols;
     a.beta = prm.step;
     a.seed = prm.seed;
+    hq::philox_round_keys(prm.seed, a.rk);
     a.kv_S = kv ? kv_S : 0;
     a.items = g.items;
     a.IB = g.IB;
@@ -243,6 +244,7 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
     a.cols = code->cols;
     a.beta = prm.step;
     a.seed = prm.seed;
+    hq::philox_round_keys(prm.seed, a.rk);
     a.kv_S = code->kv_S;
     a.items = g.items;
     a.IB = g.IB;

@@ -14,6 +14,9 @@ namespace hq {
 // ------------------------------------------------------------------------------------------------
 // Kernel configuration
 // ------------------------------------------------------------------------------------------------
+#ifndef HQ_QUANT_ROT
+#define HQ_QUANT_ROT 2  // rounds of the quantizer body per tile (encode_kernel)
+#endif
 #ifndef HQ_THREADS
 #define HQ_THREADS 128
 #endif
@@ -81,6 +84,32 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
         const uint32_t lo1 = 0xCD9E8D57u * c.z;
         const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
         c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    }
+    return c;
+}
+
+// round keys of a 64-bit seed: rk[2 r], rk[2 r + 1] are the key words of round r
+__host__ __device__ inline void philox_round_keys(uint64_t seed, uint32_t (&rk)[20])
+{
+    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        rk[2 * r] = k0;
+        rk[2 * r + 1] = k1;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+}
+
+// the same generator with precomputed round keys (kernel parameters: no registers held for them)
+__device__ __forceinline__ uint4 philox4x32_10_rk(uint4 c, const uint32_t (&rk)[20])
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ rk[2 * r], lo1, hi0 ^ c.w ^ rk[2 * r + 1], lo0);
     }
     return c;
 }
@@ -276,12 +305,13 @@ __device__ __forceinline__ void put4(BitWriter<FWD>& bw, uint32_t z0, uint32_t z
     const uint32_t l0 = q0 + k1, l1 = q1 + k1, l2 = q2 + k1, l3 = q3 + k1;
     const uint32_t L = l0 + l1 + l2 + l3;
     if (L <= 32u) {
-        // codes are (k+1)-bit values with the zero runs implied by the shifts
-        unsigned long long c = c0;
+        // codes are (k+1)-bit values with the zero runs implied by the shifts; every partial
+        // result has at most L <= 32 bits and every shift is at most 29, so 32 bits suffice
+        uint32_t c = c0;
         c = (c << l1) | c1;
         c = (c << l2) | c2;
         c = (c << l3) | c3;
-        bw.put((uint32_t)c, (int)L);
+        bw.put(c, (int)L);
     } else {
         const uint32_t cs[4] = {c0, c1, c2, c3};
         const uint32_t qs[4] = {q0, q1, q2, q3};

@@ -26,6 +26,7 @@ struct DecodeArgs {
     const uint32_t* bits;
     int64_t cap_words;
     WsHeader* ws;
+    uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
 };
 
 template <int N, int DST>  // DST: 0 bf16, 1 fp32
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 for (int half = 0; half < 2; ++half) {
                     float U[4];
                     const uint32_t blk = (uint32_t)(tau * (V / 4) + half * (H / 4) + b);
-                    dither_d4(a.seed, bh, sidx, blk, U);
+                    dither_d4(a.rk, bh, sidx, blk, U);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         if (half) P[4 * b + i].y = __fadd_rn(P[4 * b + i].y, -U[i]);

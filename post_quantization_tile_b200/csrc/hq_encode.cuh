@@ -30,6 +30,7 @@ struct EncodeArgs {
     int32_t* v_out;
     WsHeader* ws;
     unsigned long long* states;
+    uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
 };
 
 // SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
@@ -349,29 +350,21 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
             for (int m = 0; m < H; ++m) P[m] = zero_tile ? make_float2(0.0f, 0.0f) : f2mul(P[m], g2);
         }
 
-        // ---------------- dither (KV) ----------------
+        // ---------------- KV dither counters ----------------
+        uint64_t sidx = 0;
+        uint32_t bh = 0;
         if constexpr (KV) {
             const int64_t r = r0 + row_l;
             const uint64_t Sv = (uint64_t)a.kv_S;
-            const uint64_t sidx = Sv ? (uint64_t)r % Sv : (uint64_t)r;
-            const uint32_t bh = Sv ? (uint32_t)((uint64_t)r / Sv) : 0u;
-#pragma unroll
-            for (int b = 0; b < H / 4; ++b) {
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float U[4];
-                    const uint32_t blk = (uint32_t)(tau * (V / 4) + half * (H / 4) + b);
-                    dither_d4(a.seed, bh, sidx, blk, U);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (half) P[4 * b + i].y = __fadd_rn(P[4 * b + i].y, U[i]);
-                        else P[4 * b + i].x = __fadd_rn(P[4 * b + i].x, U[i]);
-                    }
-                }
-            }
+            sidx = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+            bh = Sv ? (uint32_t)((uint64_t)r / Sv) : 0u;
         }
 
-        // ---------------- lattice + strip -> zig-zag scratch ----------------
+        // ---------------- (dither,) lattice + strip -> zig-zag scratch ----------------
+        // Pair-block g8 is P[8 g8 .. 8 g8 + 8): lane x holds positions 8 g8 .., lane y positions
+        // H + 8 g8 ...  The pair-blocks run in ROT rounds of one unrolled body over P[0 .. H/ROT):
+        // after each round the next part of P moves down, so the instruction stream of the
+        // quantizer is 1/ROT as long (unrolled over a whole tile it overflows the instruction cache).
         uint32_t A = 0, zor = 0;
         uint32_t cosbits = 0;  // coset bit of local block lb at bit lb (E8)
         auto store_group = [&](int group, const int32_t (&sym)[8]) {
@@ -385,56 +378,81 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
             *zz_slot(zzs, group, tid) =
                 make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16), z[4] | (z[5] << 16), z[6] | (z[7] << 16));
         };
-        if constexpr (LAT == HQ_E8) {
-            // pair-block g8: lane x is block g8 (positions 8 g8 ..), lane y block g8 + H/8
+        constexpr int ROT = (H >= 16 && !KV) ? HQ_QUANT_ROT : 1;
+        constexpr int PB = H / 8 / ROT;  // pair-blocks per round
+#pragma unroll 1
+        for (int rr = 0; rr < ROT; ++rr) {
 #pragma unroll
-            for (int g8 = 0; g8 < H / 8; ++g8) {
-                float2 p8[8];
+            for (int gb = 0; gb < PB; ++gb) {
+                const int g8 = rr * PB + gb;
+                if constexpr (LAT == HQ_E8) {
+                    float2 p8[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) p8[i] = P[g8 * 8 + i];
-                int32_t sx[8], sy[8], vx[8], vy[8];
-                uint32_t cx, cy;
-                e8_pair_symbols<SRC == 2>(p8, sx, sy, cx, cy, vx, vy);
-                if constexpr (SRC == 2) {
-                    if (valid && a.v_out) {
-                        int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            vo[g8 * 8 + i] = vx[i];
-                            vo[H + g8 * 8 + i] = vy[i];
-                        }
-                    }
-                }
-                cosbits |= (cx << g8) | (cy << (H / 8 + g8));
-                store_group(g8, sx);
-                store_group(H / 8 + g8, sy);
-            }
-        } else {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-            for (int g8 = 0; g8 < H / 8; ++g8) {
-                int32_t sym[8];
-#pragma unroll
-                for (int b = 0; b < 8 / D; ++b) {
-                    const int pos = half * H + g8 * 8 + b * D;
-                    float u[D];
-#pragma unroll
-                    for (int i = 0; i < D; ++i) u[i] = half ? P[g8 * 8 + b * D + i].y : P[g8 * 8 + b * D + i].x;
-                    int32_t v[D];
-                    const uint32_t c = quantize_strip<LAT, SRC == 2>(u, sym + b * D, v);
+                    for (int i = 0; i < 8; ++i) p8[i] = P[gb * 8 + i];
+                    int32_t sx[8], sy[8], vx[8], vy[8];
+                    uint32_t cx, cy;
+                    e8_pair_symbols<SRC == 2>(p8, sx, sy, cx, cy, vx, vy);
                     if constexpr (SRC == 2) {
                         if (valid && a.v_out) {
-                            int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V + pos;
+                            int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V;
 #pragma unroll
-                            for (int i = 0; i < D; ++i) vo[i] = v[i];
+                            for (int i = 0; i < 8; ++i) {
+                                vo[g8 * 8 + i] = vx[i];
+                                vo[H + g8 * 8 + i] = vy[i];
+                            }
                         }
                     }
-                    (void)c;
+                    cosbits |= (cx << g8) | (cy << (H / 8 + g8));
+                    store_group(g8, sx);
+                    store_group(H / 8 + g8, sy);
+                } else {
+                    if constexpr (KV) {
+                        // dither: the D4 block of lane `half` at pairs 4 b .. 4 b + 4 takes
+                        // block counter tau V/4 + half H/4 + b
+#pragma unroll
+                        for (int bb = 0; bb < 2; ++bb) {
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                float U[4];
+                                const uint32_t blk = (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8 + bb);
+                                dither_d4(a.rk, bh, sidx, blk, U);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    float2& q = P[gb * 8 + 4 * bb + i];
+                                    if (half) q.y = __fadd_rn(q.y, U[i]);
+                                    else q.x = __fadd_rn(q.x, U[i]);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        int32_t sym[8];
+#pragma unroll
+                        for (int b = 0; b < 8 / D; ++b) {
+                            float u[D];
+#pragma unroll
+                            for (int i = 0; i < D; ++i) u[i] = half ? P[gb * 8 + b * D + i].y : P[gb * 8 + b * D + i].x;
+                            int32_t v[D];
+                            const uint32_t c = quantize_strip<LAT, SRC == 2>(u, sym + b * D, v);
+                            if constexpr (SRC == 2) {
+                                if (valid && a.v_out) {
+                                    int32_t* vo =
+                                        a.v_out + (r0 + row_l) * (int64_t)N + tau * V + half * H + g8 * 8 + b * D;
+#pragma unroll
+                                    for (int i = 0; i < D; ++i) vo[i] = v[i];
+                                }
+                            }
+                            (void)c;
+                        }
+                        store_group(half * (H / 8) + g8, sym);
+                    }
                 }
-                store_group(half * (H / 8) + g8, sym);
             }
-        }
+            if (ROT > 1 && rr + 1 < ROT) {
+#pragma unroll
+                for (int m = 0; m < H - H / ROT; ++m) P[m] = P[m + H / ROT];
+            }
         }
 
         // ---------------- Rice parameter and tile length ----------------

@@ -271,16 +271,16 @@ __device__ __forceinline__ void unstrip_block(const int32_t* s, uint32_t c, int3
 
 // KV dither for D4 block `blk` of token (bh, s): U uniform on the Voronoi cell of D4
 // ("Subtractive Dither", Methodology step 4).  r = 2 (w >> 8) 2^-24 is uniform on [0,2)^4, a union
-// of D4 cells (2Z^4 is a sublattice of D4); U = r - Q_D4(r).
-__device__ __forceinline__ void dither_d4(uint64_t seed, uint32_t bh, uint64_t s, uint32_t blk, float (&U)[4])
+// of D4 cells (2Z^4 is a sublattice of D4); U = r - Q_D4(r).  rk: the round keys of the seed.
+__device__ __forceinline__ void dither_d4(const uint32_t (&rk)[20], uint32_t bh, uint64_t s, uint32_t blk, float (&U)[4])
 {
-    const uint4 w = philox4x32_10(make_uint4((uint32_t)s, bh, 0x80000000u | blk, (uint32_t)(s >> 32)),
-                                  (uint32_t)seed, (uint32_t)(seed >> 32));
+    const uint4 w = philox4x32_10_rk(make_uint4((uint32_t)s, bh, 0x80000000u | blk, (uint32_t)(s >> 32)), rk);
+    // 2 (w >> 8) 2^-24 = (w >> 8) 2^-23: every step is exact (24-bit integers, power-of-two scale)
     float r[4];
-    r[0] = __fmul_rn(2.0f, __fmul_rn((float)(w.x >> 8), 5.9604644775390625e-08f));
-    r[1] = __fmul_rn(2.0f, __fmul_rn((float)(w.y >> 8), 5.9604644775390625e-08f));
-    r[2] = __fmul_rn(2.0f, __fmul_rn((float)(w.z >> 8), 5.9604644775390625e-08f));
-    r[3] = __fmul_rn(2.0f, __fmul_rn((float)(w.w >> 8), 5.9604644775390625e-08f));
+    r[0] = __fmul_rn((float)(w.x >> 8), 1.1920928955078125e-07f);
+    r[1] = __fmul_rn((float)(w.y >> 8), 1.1920928955078125e-07f);
+    r[2] = __fmul_rn((float)(w.z >> 8), 1.1920928955078125e-07f);
+    r[3] = __fmul_rn((float)(w.w >> 8), 1.1920928955078125e-07f);
     int32_t q[4];
     q_d4(r, q);
 #pragma unroll
