@@ -243,6 +243,8 @@ struct BitWriter {
     unsigned long long acc;  // valid bits are the low `nb` bits, earliest read bit highest
     int nb;
     int wi;                  // stored word index of the next emitted word
+    int wi0;                 // word index of the first (head) word
+    uint32_t head;           // the head word, merged into the stream by finish()
     bool first;
     uint32_t* stg;
 
@@ -251,14 +253,19 @@ struct BitWriter {
         stg = s;
         acc = 0ull;
         wi = start_or_end_bit >> 5;
+        wi0 = wi;
+        head = 0u;
         nb = FWD ? (start_or_end_bit & 31) : (31 - (start_or_end_bit & 31));
         first = true;
     }
+    // The head word may share bits with a neighbouring tile (or the coset bits), so it is kept in
+    // a register and OR-ed in by finish(); every later word belongs to this writer alone and is a
+    // plain store.
     __device__ __forceinline__ void emit(uint32_t rw)
     {
         const uint32_t w = FWD ? __brev(rw) : rw;
         if (first) {
-            atomicOr(stg + wi, w);
+            head = w;
             first = false;
         } else {
             stg[wi] = w;
@@ -275,9 +282,11 @@ struct BitWriter {
             nb -= 32;
         }
     }
+    // the partial last word and the head word meet other writers' bits: OR them in
     __device__ __forceinline__ void finish()
     {
         if (nb > 0) atomicOr(stg + wi, FWD ? __brev((uint32_t)(acc << (32 - nb))) : (uint32_t)(acc << (32 - nb)));
+        if (!first) atomicOr(stg + wi0, head);
     }
 };
 

@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 const uint32_t zw[4] = {w.x, w.y, w.z, w.w};
                 int32_t sym[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) sym[j] = ok ? unzigzag((zw[j >> 1] >> (16 * (j & 1))) & 0xFFFFu) : 0;
+                for (int j = 0; j < 8; ++j) sym[j] = unzigzag((zw[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);  // !ok: zeroed below
 #pragma unroll
                 for (int b = 0; b < 8 / D; ++b) {
                     const int pos = half * H + g8 * 8 + b * D;
@@ -323,9 +323,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 }
             }
         }
-        if (!ok) {
+        if (__any_sync(0xffffffffu, !ok)) {
 #pragma unroll
-            for (int m = 0; m < H; ++m) P[m] = make_float2(0.0f, 0.0f);
+            for (int m = 0; m < H; ++m) P[m] = ok ? P[m] : make_float2(0.0f, 0.0f);
         }
 
         // ---------------- inverse transform: H_n p, exact for integer points ----------------

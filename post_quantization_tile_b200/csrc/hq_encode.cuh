@@ -347,7 +347,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
             const float g = zero_tile ? 0.0f : __fmul_rn(cn, rinv);
             const float2 g2 = make_float2(g, g);
 #pragma unroll
-            for (int m = 0; m < H; ++m) P[m] = zero_tile ? make_float2(0.0f, 0.0f) : f2mul(P[m], g2);
+            for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], g2);
+            // zero (and non-finite) tiles code as all zeros; a warp-uniform test keeps the
+            // per-coefficient selects off the common path
+            if (__any_sync(0xffffffffu, zero_tile)) {
+#pragma unroll
+                for (int m = 0; m < H; ++m) P[m] = zero_tile ? make_float2(0.0f, 0.0f) : P[m];
+            }
         }
 
         // ---------------- KV dither counters ----------------
@@ -458,13 +464,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
         // ---------------- Rice parameter and tile length ----------------
         if constexpr (TPT == 2) A += __shfl_xor_sync(0xffffffffu, A, 1);
         const int k = rice_k(A, G::LOG2N);
-        uint32_t sq = 0;
+        // sum q = sum (zz >> k) on both 16-bit halves of the packed scratch words at once: the k rule
+        // keeps the tile's sum below 2n (at most n when k is capped), so neither half carries over
+        const uint32_t hm = (0xFFFFu >> k) * 0x00010001u;
+        uint32_t sq2 = 0;
 #pragma unroll 4
         for (int g = 0; g < V / 8; ++g) {
             const uint4 w = *zz_slot(zzs, g, tid);
-            sq += ((w.x & 0xFFFFu) >> k) + ((w.x >> 16) >> k) + ((w.y & 0xFFFFu) >> k) + ((w.y >> 16) >> k) +
-                  ((w.z & 0xFFFFu) >> k) + ((w.z >> 16) >> k) + ((w.w & 0xFFFFu) >> k) + ((w.w >> 16) >> k);
+            sq2 += ((w.x >> k) & hm) + ((w.y >> k) & hm) + ((w.z >> k) & hm) + ((w.w >> k) & hm);
         }
+        const uint32_t sq = (sq2 & 0xFFFFu) + (sq2 >> 16);
         uint32_t sq_tile = sq;
         if constexpr (TPT == 2) sq_tile += __shfl_xor_sync(0xffffffffu, sq, 1);
         const uint32_t L = (uint32_t)COSB + (uint32_t)N * (uint32_t)(k + 1) + sq_tile;
