@@ -275,10 +275,12 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
-    enc_ms = [statistics.mean(enc_ev[k * len(SHAPES) + i][0].elapsed_time(enc_ev[k * len(SHAPES) + i][1])
-                              for k in range(args.steps)) for i in range(len(SHAPES))]
-    dec_ms = [statistics.mean(dec_ev[k * len(SHAPES) + i][0].elapsed_time(dec_ev[k * len(SHAPES) + i][1])
-                              for k in range(args.steps)) for i in range(len(SHAPES))]
+    enc_calls = [[enc_ev[k * len(SHAPES) + i][0].elapsed_time(enc_ev[k * len(SHAPES) + i][1])
+                  for k in range(args.steps)] for i in range(len(SHAPES))]
+    dec_calls = [[dec_ev[k * len(SHAPES) + i][0].elapsed_time(dec_ev[k * len(SHAPES) + i][1])
+                  for k in range(args.steps)] for i in range(len(SHAPES))]
+    enc_ms = [statistics.mean(c) for c in enc_calls]
+    dec_ms = [statistics.mean(c) for c in dec_calls]
 
     # e2e through the public API with host buffers: pinned H2D of the inputs, encode, decode,
     # D2H of the reconstruction, every step
@@ -314,6 +316,8 @@ def run_gpu(args):
     achieved = kbytes / (kms * 1e-3) / 1e9
     value = weak_scaling_value(bf16_bytes, world, ms)
 
+    kv = None if args.no_kv else run_kv(hq, dev, stream, peak)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = max(r for r, _ in SHAPES)
@@ -334,6 +338,8 @@ def run_gpu(args):
             "encode_gbs": [SHAPES[i][0] * SHAPES[i][1] * 2 / (enc_ms[i] * 1e-3) / 1e9 for i in range(len(SHAPES))],
             "decode_gbs": [SHAPES[i][0] * SHAPES[i][1] * 2 / (dec_ms[i] * 1e-3) / 1e9 for i in range(len(SHAPES))],
             "encode_ms": enc_ms, "decode_ms": dec_ms,
+            "encode_ms_p10_p50_p90": [percentiles(c) for c in enc_calls],
+            "decode_ms_p10_p50_p90": [percentiles(c) for c in dec_calls],
             "roofline": {"bound": "hbm", "kernel": f"{kname} 11008x4096", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "bytes_per_launch": kbytes,
@@ -342,6 +348,7 @@ def run_gpu(args):
             "e2e": {"value": weak_scaling_value(bf16_bytes, world, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": bf16_bytes, "d2h_bytes_per_step": bf16_bytes},
             "gpu_launches": 4 * args.steps,
+            "kv_cache": kv,
             "clocks": clk.summary(),
             "status": st,
         }
@@ -349,6 +356,55 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def percentiles(calls):
+    """p10, p50, p90 of per-call times (ms)."""
+    q = np.percentile(np.asarray(calls, dtype=np.float64), [10, 50, 90])
+    return [float(v) for v in q]
+
+
+def run_kv(hq, dev, stream, peak):
+    """Dithered D4 KV-cache codec on one K tensor [8, 32, 8192, 128] bf16 (268 M scalars, 537 MB)
+    at 2 bps payload: per-call encode and decode times, outside the timed step.  Calls alternate
+    between two tensors (and two codes), 1.07 GB in all, so no call finds its input in L2."""
+    import torch
+
+    from post_quantization_tile_b200 import workloads as W
+    B, H, S, D = 8, 32, 8192, 128
+    keys = [torch.from_numpy(W.kv_keys(B, H, S, D, seed=2 + i).view(np.int16)).view(torch.bfloat16).to(dev)
+            for i in range(2)]
+    beta = hq.calibrate_step(keys[0], D, hq.D4, 2.0, seed=SEED, kv=True, kv_S=S)
+    codes = [hq.kv_encode(keys[i], step=beta, seed=SEED) for i in range(2)]
+    out = torch.empty_like(keys[0])
+    calls = 10
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(calls)]
+    for k in range(3):
+        hq.kv_encode(keys[k % 2], step=beta, seed=SEED, out=codes[k % 2], ws=codes[k % 2].ws)
+        hq.decode(codes[(k + 1) % 2], out=out.view(-1, D), ws=codes[(k + 1) % 2].ws)
+    for k in range(calls):
+        a, b = k % 2, (k + 1) % 2
+        ev[k][0].record(stream)
+        hq.kv_encode(keys[a], step=beta, seed=SEED, out=codes[a], ws=codes[a].ws)
+        ev[k][1].record(stream)
+        ev[k][2].record(stream)
+        hq.decode(codes[b], out=out.view(-1, D), ws=codes[b].ws)
+        ev[k][3].record(stream)
+    torch.cuda.synchronize()
+    st, _ = hq.status(codes[0].ws)
+    enc = [e[0].elapsed_time(e[1]) for e in ev]
+    dec = [e[2].elapsed_time(e[3]) for e in ev]
+    n = B * H * S * D
+    code_bytes = 4 * codes[0].total_words() + 4 * codes[0].scale.numel() + 4 * codes[0].chunk_word.numel()
+    moved = 2 * n + code_bytes
+    e50, d50 = statistics.median(enc), statistics.median(dec)
+    return {"workload": "kv_keys_8x32x8192x128_bf16_D4_dither_n128_2bps", "step": beta,
+            "payload_bps": codes[0].payload_bps(), "total_bps": codes[0].total_bps(),
+            "encode_ms_p10_p50_p90": percentiles(enc), "decode_ms_p10_p50_p90": percentiles(dec),
+            "encode_gbs_bf16": 2 * n / (e50 * 1e-3) / 1e9, "decode_gbs_bf16": 2 * n / (d50 * 1e-3) / 1e9,
+            "encode_roofline_frac": moved / (e50 * 1e-3) / 1e9 / peak,
+            "decode_roofline_frac": moved / (d50 * 1e-3) / 1e9 / peak,
+            "bytes_per_call": moved, "status": st}
 
 
 def run_profile(args):
@@ -389,6 +445,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kv", action="store_true", help="skip the KV-cache codec fields")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)
