@@ -174,6 +174,33 @@ hq_status_t hq_quantize_coeffs(const float* u, int64_t tiles, const hq_params_t*
 hq_status_t hq_encode_count(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
                             int32_t kv, int64_t kv_S, uint64_t* bits_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Result of a step search, written to device memory. */
+typedef struct {
+    float step;            /* the chosen step beta                                          */
+    int32_t probes;        /* count-only passes made                                        */
+    uint64_t payload_bits; /* payload bits of encoding x at `step` (Methodology step 3 rate) */
+} hq_rate_result_t;
+
+/*
+ * Exact-rate mode: search the step whose payload rate is p->bps (in [1, 8]) on this tensor, the
+ * per-tensor counterpart of the method's claim that the realised rate lands about 0.01 bps from
+ * any target (Methodology step 3, Rice coding).  Up to `max_probes` (1 .. 64; 0 means 16)
+ * count-only encodes, each followed by a one-thread update on the device: the first probe is
+ * p->step if it is > 0, else hq_step_for_rate; while only one side of the target has been seen
+ * the next probe is a Newton step in log2(step) with slope -1 bit per scalar per doubling; once
+ * the target is bracketed, regula falsi on the binary32 bit patterns of the step, with a
+ * bisection whenever the same side moves twice in a row.  The search stops at the first probe
+ * within tol_bps of the target (tol_bps <= 0 means 0.005; at most 1), when the bracket closes to
+ * adjacent binary32 steps, at the
+ * ends of the step range [2^-8, 64], or after max_probes passes; `result` (device) then holds
+ * the probe closest to the target.  Everything runs on `stream` without a host synchronisation
+ * (a CUDA graph may capture it).  ws: at least hq_workspace_bytes(rows, cols, p) bytes.
+ * Errors: HQ_ERR_ARG for invalid arguments, as hq_encode_count; device errors in ws.
+ */
+hq_status_t hq_step_search(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                           int32_t kv, int64_t kv_S, int32_t max_probes, float tol_bps, hq_rate_result_t* result,
+                           void* ws, size_t ws_bytes, void* stream);
+
 /*
  * Synchronise `stream`, then read the status word of `ws`: returns HQ_OK or the most severe
  * device error (TIMEOUT, CORRUPT, CAPACITY, NONFINITE in that order) and, if detail is not NULL,

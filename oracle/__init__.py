@@ -319,3 +319,80 @@ def calibrate_step(x: np.ndarray, n: int, lattice: int, target_bps: float, seed:
         else:
             hi = mid
     return float(np.float32(np.exp(0.5 * (lo + hi))))
+
+
+STEP_BITS_MIN, STEP_BITS_MAX = 0x3B800000, 0x42800000  # binary32 bit patterns of 2^-8 and 64
+
+
+def _f32_bits(x: float) -> int:
+    return int(np.array([x], dtype=np.float32).view(np.int32)[0])
+
+
+def _bits_f32(b: int) -> float:
+    return float(np.array([b], dtype=np.int32).view(np.float32)[0])
+
+
+def step_search(x: np.ndarray, n: int, lattice: int, target_bps: float, seed: int = 0, kv: bool = False,
+                kv_S: int = 0, step0: float = 0.0, max_probes: int = 16, tol_bps: float = 0.005):
+    """Exact-rate mode: the step whose payload rate on x is target_bps, within tol_bps (the
+    method lands the realised rate about 0.01 bps from any target, Methodology step 3, Rice
+    coding).  Written from the rule as stated, with every quantity in binary64:
+
+    * probe 1 is step0;
+    * after each probe (payload bits c): keep the probe closest to the target; stop if
+      |c - target| <= tol_bps n (tol_bps as binary32, widened); else the probe becomes the low
+      end of the bracket (rate too high, c > target) or the high end;
+    * with both ends known: stop when they are adjacent binary32 values; else the next probe is
+      the regula-falsi point lo + floor(t (hi - lo)), t = (c_lo - target) / (c_lo - c_hi), on the
+      bit patterns, or the midpoint when the same end moved twice in a row, kept strictly inside;
+    * with one end known: a Newton step of floor(excess 2^23 + 1/2) bit patterns (excess = bps
+      above the target, slope -1 bit per doubling of the step), at least one, clamped to
+      [2^-8, 64]; stop if it cannot move;
+    * stop after max_probes probes.
+
+    Returns (step, probes, payload bits at step)."""
+    N = float(x.shape[0] * x.shape[1])
+    target = float(np.float32(target_bps)) * N
+    tol = float(np.float32(tol_bps)) * N
+    b = _f32_bits(step0)
+    lo = hi = -1
+    c_lo = c_hi = 0
+    last_side = 0
+    probes = 0
+    best, c_best = b, 0
+    while True:
+        c = encode(x, n, lattice, _bits_f32(b), seed, kv, kv_S).payload_bits()
+        probes += 1
+        err = abs(float(c) - target)
+        if probes == 1 or err < abs(float(c_best) - target):
+            best, c_best = b, c
+        if err <= tol:
+            break
+        if float(c) > target:
+            lo, c_lo, side = b, c, 1
+        else:
+            hi, c_hi, side = b, c, 2
+        if lo >= 0 and hi >= 0:
+            if hi - lo <= 1:
+                break
+            if side == last_side:
+                nb = lo + (hi - lo) // 2
+            else:
+                t = (float(c_lo) - target) / (float(c_lo) - float(c_hi))
+                nb = lo + int(np.floor(t * float(hi - lo)))
+            nb = min(max(nb, lo + 1), hi - 1)
+        else:
+            excess = (float(c) - target) / N
+            d = float(np.floor(excess * 8388608.0 + 0.5))
+            d = min(max(d, -134217728.0), 134217728.0)
+            nb = b + int(d)
+            if nb == b:
+                nb += 1 if side == 1 else -1
+            nb = min(max(nb, STEP_BITS_MIN), STEP_BITS_MAX)
+            if nb == b:
+                break
+        last_side = side
+        if probes >= max_probes:
+            break
+        b = nb
+    return _bits_f32(best), probes, c_best

@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import struct
 from dataclasses import dataclass
 
 import torch
@@ -72,12 +73,14 @@ def lib():
         L.hq_quantize_coeffs.argtypes = [P, i64, ctypes.POINTER(Params), i32, i64, P, ctypes.POINTER(CodeStruct), P,
                                          ctypes.c_size_t, P]
         L.hq_encode_count.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, P, P, ctypes.c_size_t, P]
+        L.hq_step_search.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, i32, ctypes.c_float, P, P,
+                                     ctypes.c_size_t, P]
         L.hq_status_read.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
         L.hq_status_str.argtypes = [i32]
         L.hq_status_str.restype = ctypes.c_char_p
         L.hq_version.restype = i32
         for f in ["hq_encode", "hq_decode", "hq_kv_encode", "hq_kv_decode", "hq_quantize_coeffs", "hq_encode_count",
-                  "hq_status_read"]:
+                  "hq_step_search", "hq_status_read"]:
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -294,22 +297,33 @@ def encode_count(x: torch.Tensor, tile: int, lattice: int | str, step: float, se
     return outb
 
 
+def step_search(x: torch.Tensor, tile: int, lattice: int | str, target_bps: float, seed: int = 0, kv: bool = False,
+                kv_S: int = 0, step0: float = 0.0, max_probes: int = 0, tol_bps: float = 0.0,
+                ws: Workspace | None = None) -> tuple[float, int, int]:
+    """Exact-rate mode on the device (hq_step_search): (step, probes, payload bits at step).
+    x: 2-D [rows, cols] or KV [B, H, S, D]; reading the result synchronises the stream."""
+    _require_cuda(x, "x")
+    if x.dim() == 4:
+        rows, cols = x.shape[0] * x.shape[1] * x.shape[2], x.shape[3]
+        kv, kv_S = True, x.shape[2]
+    else:
+        rows, cols = x.shape
+    p = params(tile, lattice, step0, target_bps, seed)
+    L = lib()
+    w = ws or workspace(L.hq_workspace_bytes(rows, cols, ctypes.byref(p)))
+    res = torch.zeros(2, dtype=torch.int64, device=x.device)  # {float step, int32 probes}, uint64 bits
+    _check(L.hq_step_search(_ptr(x), _dtype_code(x), rows, cols, ctypes.byref(p), int(kv), int(kv_S), int(max_probes),
+                            float(tol_bps), _ptr(res), w.ptr(), w.nbytes, _stream()), "hq_step_search")
+    r = res.cpu().tolist()
+    step = struct.unpack("<f", struct.pack("<I", r[0] & 0xFFFFFFFF))[0]
+    return step, int(r[0] >> 32), int(r[1])
+
+
 def calibrate_step(x: torch.Tensor, tile: int, lattice: int | str, target_bps: float, seed: int = 0,
-                   kv: bool = False, kv_S: int = 0, iters: int = 24) -> float:
-    """Bisection on log(step) with count-only encodes so the payload rate hits target_bps
-    (the method lands the realised rate about 0.01 bps from its target, Methodology step 3)."""
-    import math
-    n = x.numel()
-    lo, hi = math.log(2.0 ** -8), math.log(2.0 ** 6)
-    for _ in range(iters):
-        mid = 0.5 * (lo + hi)
-        b = float(torch.tensor(math.exp(mid), dtype=torch.float32))
-        r = encode_count(x, tile, lattice, b, seed, kv, kv_S).item() / n
-        if r > target_bps:
-            lo = mid
-        else:
-            hi = mid
-    return float(torch.tensor(math.exp(0.5 * (lo + hi)), dtype=torch.float32))
+                   kv: bool = False, kv_S: int = 0) -> float:
+    """A step whose payload rate is target_bps to 1e-4 bps where the rate allows it: the device
+    step search with a tight tolerance (Methodology step 3)."""
+    return step_search(x, tile, lattice, target_bps, seed, kv, kv_S, max_probes=64, tol_bps=1e-4)[0]
 
 
 def status(ws: Workspace) -> tuple[int, int]:

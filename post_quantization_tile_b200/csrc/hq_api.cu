@@ -150,14 +150,23 @@ cudaError_t run_decode(int lattice, int n, bool kv, int dst, const DecodeArgs& a
     }
 }
 
-// common body of the encode entry points (src 0/1 dense input, src 2 coefficients)
-hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, const hq_params_t* p, int32_t kv,
-                          int64_t kv_S, int32_t* v_out, hq_code_t* out, unsigned long long* count_out, void* ws,
-                          size_t ws_bytes, void* stream)
-{
+// arguments, tensor map and geometry of one encode launch (src 0/1 dense input, src 2 coefficients)
+struct EncodePlan {
     hq_params_t prm;
-    if (!resolve_params(p, prm)) return HQ_ERR_ARG;
     Geometry g;
+    CUtensorMap map;
+    EncodeArgs a;
+    bool kv;
+    int src;
+};
+
+hq_status_t plan_encode(const void* x, int src, int64_t rows, int64_t cols, const hq_params_t* p, int32_t kv,
+                        int64_t kv_S, int32_t* v_out, hq_code_t* out, bool count, void* ws, size_t ws_bytes,
+                        EncodePlan& pl)
+{
+    hq_params_t& prm = pl.prm;
+    if (!resolve_params(p, prm)) return HQ_ERR_ARG;
+    Geometry& g = pl.g;
     const int tpt = prm.tile == 64 ? 1 : (prm.tile == 256 ? 2 : enc_tpt(128, src));
     if (!geometry(rows, cols, prm.tile, g, tpt)) return HQ_ERR_ARG;
     if (kv && prm.lattice != HQ_D4) return HQ_ERR_UNSUPPORTED;
@@ -166,7 +175,6 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
     if (src == 2 && cols != prm.tile) return HQ_ERR_ARG;
     if (!x || !aligned16(x) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
     if (ws_bytes < ws_bytes_for(rows, cols, prm.tile)) return HQ_ERR_ARG;
-    const bool count = count_out != nullptr;
     if (!count) {
         if (!out || !out->meta || !out->chunk_word || !out->bits || out->cap_words < 1) return HQ_ERR_ARG;
         if (src != 2 && !out->scale) return HQ_ERR_ARG;
@@ -175,14 +183,10 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
 
     if (!use_device_of(x)) return HQ_ERR_ARG;
     const int es = src == 0 ? 2 : 4;
-    CUtensorMap map;
-    if (!make_map(&map, x, rows, cols, es, g.TI)) return HQ_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t clear = count ? sizeof(WsHeader) : sizeof(WsHeader) + (size_t)g.items * 8u;
-    cudaError_t e = cudaMemsetAsync(ws, 0, clear, st);
-    if (e != cudaSuccess) return HQ_ERR_CUDA;
+    if (!make_map(&pl.map, x, rows, cols, es, g.TI)) return HQ_ERR_CUDA;
 
-    EncodeArgs a{};
+    EncodeArgs& a = pl.a;
+    a = EncodeArgs{};
     a.rows = rows;
     a.cols = cols;
     a.beta = prm.step;
@@ -203,20 +207,169 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
     a.v_out = v_out;
     a.ws = static_cast<WsHeader*>(ws);
     a.states = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + sizeof(WsHeader));
-    e = run_encode(prm.lattice, prm.tile, kv != 0, src, count, a, map, st);
+    a.search = nullptr;
+    pl.kv = kv != 0;
+    pl.src = src;
+    return HQ_OK;
+}
+
+// common body of the encode entry points
+hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, const hq_params_t* p, int32_t kv,
+                          int64_t kv_S, int32_t* v_out, hq_code_t* out, unsigned long long* count_out, void* ws,
+                          size_t ws_bytes, void* stream)
+{
+    const bool count = count_out != nullptr;
+    EncodePlan pl;
+    const hq_status_t ps = plan_encode(x, src, rows, cols, p, kv, kv_S, v_out, out, count, ws, ws_bytes, pl);
+    if (ps != HQ_OK) return ps;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t clear = count ? sizeof(WsHeader) : sizeof(WsHeader) + (size_t)pl.g.items * 8u;
+    cudaError_t e = cudaMemsetAsync(ws, 0, clear, st);
+    if (e != cudaSuccess) return HQ_ERR_CUDA;
+    e = run_encode(pl.prm.lattice, pl.prm.tile, pl.kv, src, count, pl.a, pl.map, st);
     if (e != cudaSuccess) return HQ_ERR_CUDA;
     if (count) {
-        e = cudaMemcpyAsync(count_out, &a.ws->count_bits, sizeof(unsigned long long), cudaMemcpyDeviceToDevice, st);
+        e = cudaMemcpyAsync(count_out, &pl.a.ws->count_bits, sizeof(unsigned long long), cudaMemcpyDeviceToDevice, st);
         if (e != cudaSuccess) return HQ_ERR_CUDA;
     } else {
         out->rows = rows;
         out->cols = cols;
         out->kv_S = kv ? kv_S : 0;
-        out->p = prm;
+        out->p = pl.prm;
         out->kv = kv ? 1 : 0;
         out->version = HQ_FORMAT_VERSION;
     }
     return HQ_OK;
+}
+
+// ---------------- step search (exact-rate mode) ----------------
+constexpr int32_t kStepBitsMin = 0x3B800000;  // 2^-8
+constexpr int32_t kStepBitsMax = 0x42800000;  // 64
+
+__global__ void rate_search_init(RateSearch* s, WsHeader* h, float probe, double target, double tol, double n)
+{
+    h->counter = 0u;
+    h->count_bits = 0ull;
+    s->probe = probe;
+    s->done = 0;
+    s->lo = -1;
+    s->hi = -1;
+    s->c_lo = 0;
+    s->c_hi = 0;
+    s->last_side = 0;
+    s->probes = 0;
+    s->best = __float_as_int(probe);
+    s->c_best = 0;
+    s->target = target;
+    s->tol = tol;
+    s->n = n;
+}
+
+// one step of the search after a count-only pass (one thread).  The arithmetic is binary64 with
+// explicit roundings, so that any implementation of the same rule takes the same probes.
+__global__ void rate_search_update(RateSearch* s, WsHeader* h, int32_t max_probes)
+{
+    if (s->done) return;
+    const long long c = (long long)h->count_bits;
+    h->count_bits = 0ull;  // the next pass starts from a clean header
+    h->counter = 0u;
+    const int32_t b = __float_as_int(s->probe);
+    s->probes += 1;
+    const double err = fabs(__dadd_rn((double)c, -s->target));
+    if (s->probes == 1 || err < fabs(__dadd_rn((double)s->c_best, -s->target))) {
+        s->best = b;
+        s->c_best = c;
+    }
+    if (err <= s->tol) {
+        s->done = 1;
+        return;
+    }
+    int side;
+    if ((double)c > s->target) {
+        s->lo = b;
+        s->c_lo = c;
+        side = 1;
+    } else {
+        s->hi = b;
+        s->c_hi = c;
+        side = 2;
+    }
+    long long nb;
+    if (s->lo >= 0 && s->hi >= 0) {
+        const int32_t lo = s->lo, hi = s->hi;
+        if (hi - lo <= 1) {
+            s->done = 1;
+            return;
+        }
+        if (side == s->last_side) {
+            nb = lo + (hi - lo) / 2;
+        } else {
+            const double t = __ddiv_rn(__dadd_rn((double)s->c_lo, -s->target), __dadd_rn((double)s->c_lo, -(double)s->c_hi));
+            nb = lo + (long long)floor(__dmul_rn(t, (double)(hi - lo)));
+        }
+        nb = nb < lo + 1 ? lo + 1 : (nb > hi - 1 ? hi - 1 : nb);
+    } else {
+        // bps above the target times 2^23 binary32 steps per doubling of the step
+        const double excess = __ddiv_rn(__dadd_rn((double)c, -s->target), s->n);
+        double d = floor(__dadd_rn(__dmul_rn(excess, 8388608.0), 0.5));
+        d = d > 134217728.0 ? 134217728.0 : (d < -134217728.0 ? -134217728.0 : d);
+        nb = (long long)b + (long long)d;
+        if (nb == b) nb += side == 1 ? 1 : -1;
+        nb = nb < kStepBitsMin ? kStepBitsMin : (nb > kStepBitsMax ? kStepBitsMax : nb);
+        if (nb == b) {
+            s->done = 1;
+            return;
+        }
+    }
+    s->last_side = side;
+    if (s->probes >= max_probes) {
+        s->done = 1;
+        return;
+    }
+    s->probe = __int_as_float((int32_t)nb);
+}
+
+__global__ void rate_search_finish(const RateSearch* s, hq_rate_result_t* r)
+{
+    r->step = __int_as_float(s->best);
+    r->probes = s->probes;
+    r->payload_bits = (uint64_t)s->c_best;
+}
+
+hq_status_t step_search_common(const void* x, int src, int64_t rows, int64_t cols, const hq_params_t* p, int32_t kv,
+                               int64_t kv_S, int32_t max_probes, float tol_bps, hq_rate_result_t* result, void* ws,
+                               size_t ws_bytes, void* stream)
+{
+    if (!(tol_bps <= 1.0f)) return HQ_ERR_ARG;
+    if (!(tol_bps > 0.0f)) tol_bps = 0.005f;
+    if (!p || !result || !aligned16(result)) return HQ_ERR_ARG;
+    if (!(p->bps >= 1.0f && p->bps <= 8.0f)) return HQ_ERR_ARG;
+    if (max_probes == 0) max_probes = 16;
+    if (max_probes < 1 || max_probes > 64) return HQ_ERR_ARG;
+    if (ws_bytes < sizeof(WsHeader) + sizeof(RateSearch)) return HQ_ERR_ARG;
+    hq_params_t q = *p;
+    if (!(q.step > 0.0f)) q.step = hq_step_for_rate(q.lattice, q.tile, q.bps);
+    if (!(q.step >= 0.00390625f && q.step <= 64.0f)) return HQ_ERR_ARG;
+    EncodePlan pl;
+    const hq_status_t ps = plan_encode(x, src, rows, cols, &q, kv, kv_S, nullptr, nullptr, true, ws, ws_bytes, pl);
+    if (ps != HQ_OK) return ps;
+    if (!use_device_of(result)) return HQ_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    RateSearch* s = reinterpret_cast<RateSearch*>(static_cast<char*>(ws) + sizeof(WsHeader));
+    pl.a.search = s;
+    const double n = (double)rows * (double)cols;
+    const double target = (double)q.bps * n;
+    const double tol = (double)tol_bps * n;
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
+    rate_search_init<<<1, 1, 0, st>>>(s, pl.a.ws, q.step, target, tol, n);
+    if (cudaGetLastError() != cudaSuccess) return HQ_ERR_CUDA;
+    for (int i = 0; i < max_probes; ++i) {
+        if (run_encode(pl.prm.lattice, pl.prm.tile, pl.kv, src, true, pl.a, pl.map, st) != cudaSuccess) return HQ_ERR_CUDA;
+        rate_search_update<<<1, 1, 0, st>>>(s, pl.a.ws, max_probes);
+        if (cudaGetLastError() != cudaSuccess) return HQ_ERR_CUDA;
+    }
+    rate_search_finish<<<1, 1, 0, st>>>(s, result);
+    return cuda_status(cudaGetLastError());
 }
 
 hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int32_t kv, void* ws, size_t ws_bytes,
@@ -351,6 +504,15 @@ hq_status_t hq_encode_count(const void* x, hq_dtype_t dtype, int64_t rows, int64
     if (!bits_out) return HQ_ERR_ARG;
     return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, kv, kv ? kv_S : 0, nullptr, nullptr,
                          reinterpret_cast<unsigned long long*>(bits_out), ws, ws_bytes, stream);
+}
+
+hq_status_t hq_step_search(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                           int32_t kv, int64_t kv_S, int32_t max_probes, float tol_bps, hq_rate_result_t* result,
+                           void* ws, size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    return step_search_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, kv, kv ? kv_S : 0, max_probes, tol_bps,
+                              result, ws, ws_bytes, stream);
 }
 
 hq_status_t hq_status_read(const void* ws, void* stream, int64_t* detail)

@@ -46,6 +46,23 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 64, "workspace header");
 
+// Step search (exact-rate mode), kept in the workspace right after the header.  Count-only encodes
+// read the probe step from here; a one-thread update kernel between them moves the bracket.
+struct RateSearch {
+    float probe;                   // step of the next count-only pass
+    int32_t done;                  // 1: the search has ended, later passes return at once
+    int32_t lo, hi;                // bracket as binary32 bit patterns (-1: side not seen yet)
+    long long c_lo, c_hi;          // payload bits at lo (above target) and hi (at or below target)
+    int32_t last_side;             // 0 none, 1 lo moved, 2 hi moved (last update)
+    int32_t probes;                // count-only passes made
+    int32_t best;                  // bits of the step with the smallest |bits - target| so far
+    int32_t pad0;
+    long long c_best;
+    double target, tol;            // payload bits wanted, accepted distance
+    double n;                      // scalars in the tensor
+};
+static_assert(sizeof(RateSearch) <= 192, "rate search state");
+
 // threads per tile: one thread holds n/TPT coefficients in registers.  Two threads share a tile
 // of 256 (256 registers of coefficients would not fit); for n = 128 the choice is a build option
 // (the bit format does not depend on it).

@@ -31,6 +31,7 @@ struct EncodeArgs {
     WsHeader* ws;
     unsigned long long* states;
     uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
+    const RateSearch* search;  // count-only passes of a step search: the step comes from here
 };
 
 // SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
@@ -282,6 +283,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
     const int tau = tid % TPT;
     unsigned char* const zzs = G::SEPARATE_ZZ ? sm.zzbuf : sm.buf;
 
+    // a count-only pass of a finished step search does nothing (block-uniform)
+    float beta = a.beta;
+    if constexpr (COUNT) {
+        if (a.search) {
+            if (*(volatile const int32_t*)&a.search->done) return;
+            beta = *(volatile const float*)&a.search->probe;
+        }
+    }
+
     for (int w = tid; w < G::STG_WORDS; w += kThreads) sm.stg[w] = 0u;
     if (tid == 0) {
         mbar_init(&sm.bar, 1);
@@ -341,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
             const bool zero_tile = !finite || sh < 1.2621774483536189e-29f;  // 2^-96
             if (zero_tile) sbits = 0;
             fwht_pairs<H>(P);
-            const float t = __fmul_rn(sh, a.beta);
+            const float t = __fmul_rn(sh, beta);
             const float rinv = __frcp_rn(t);
             const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
             const float g = zero_tile ? 0.0f : __fmul_rn(cn, rinv);
