@@ -62,6 +62,7 @@ def lib():
         L.hqo_strip_block.argtypes = [i32, P, P, P]
         L.hqo_unstrip_block.argtypes = [i32, P, i32, P]
         L.hqo_dither_d4.argtypes = [u64, i64, i64, i32, P]
+        L.hqo_dither.argtypes = [i32, u64, i64, i64, i32, P]
         L.hqo_rice_tile.argtypes = [P, i32, i32, P, i64, P, P]
         L.hqo_rice_tile.restype = i64
         L.hqo_parse_tile.argtypes = [P, i64, i32, i32, ctypes.c_uint16, P, P]
@@ -136,6 +137,13 @@ def quantize_blocks(lattice: int, u: np.ndarray) -> np.ndarray:
 def dither_d4(seed: int, bh: int, s: int, blk: int) -> np.ndarray:
     U = np.zeros(4, dtype=np.float32)
     lib().hqo_dither_d4(seed, bh, s, blk, _p(U))
+    return U
+
+
+def dither(lattice: int, seed: int, c1: int, c: int, n: int) -> np.ndarray:
+    """The subtractive dither of one tile (float32 [n], quantizer coordinates: (P, Q) for A2)."""
+    U = np.zeros(n, dtype=np.float32)
+    lib().hqo_dither(lattice, seed, c1, c, n, _p(U))
     return U
 
 

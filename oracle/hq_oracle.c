@@ -278,10 +278,9 @@ void hqo_q_e8(const float* u, int32_t* v)
  * |eP| + 3|eQ| - 1, so the even point is taken when RN(|eP| + RN(3|eQ|)) <= 1. */
 static const float A2_K = 1.15470053837925153f; /* RN(2/sqrt(3)) */
 
-void hqo_q_a2(const float* u, int32_t* v)
+/* A2 nearest point given (P, Q) directly (the dither is added in these coordinates). */
+void hqo_q_a2_pq(float P, float Q, int32_t* v)
 {
-    float P = 2.0f * u[0];
-    float Q = u[1] * A2_K;
     float hP = P * 0.5f, hQ = Q * 0.5f;
     float rP = rintf(hP), rQ = rintf(hQ);
     float eP = rP - hP, eQ = rQ - hQ;
@@ -295,6 +294,8 @@ void hqo_q_a2(const float* u, int32_t* v)
         v[1] = 2 * aQ + ((eQ < 0.0f) ? 1 : -1);
     }
 }
+
+void hqo_q_a2(const float* u, int32_t* v) { hqo_q_a2_pq(2.0f * u[0], u[1] * A2_K, v); }
 
 static int lattice_dim(int lattice)
 {
@@ -454,19 +455,63 @@ static int get_code(bitr_t* rd, int64_t* pos, int step, int k, uint32_t limit, u
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* KV dither (Methodology step 4): U uniform on the Voronoi cell of D4.  Philox block with    */
-/* key = seed and counter (s_lo, b*H + h, 0x80000000 | block, s_hi) gives four words w_i;     */
-/* r_i = 2 (w_i >> 8) 2^-24 is uniform on [0,2)^4, a union of D4 fundamental domains since     */
-/* 2Z^4 is a sublattice of D4; U = r - Q_D4(r) is then uniform on V(D4).                       */
+/* Subtractive dither (Methodology step 4): U uniform on the Voronoi cell of the lattice, in   */
+/* the coordinates its quantizer works in (u for Z, D4, E8; (P, Q) = (2 u0, u1 K) for A2).     */
+/* Group g of four consecutive coefficients of a tile draws one Philox block: key = seed,      */
+/* counter (c_lo, c1, 0x80000000 | g, c_hi) with c = s for the KV row (b H + h, s), c1 = b H + h */
+/* (the weight-path option uses c = row, c1 = tile column).  The words w_i give                */
+/* r_i = box (w_i >> 8) 2^-24, uniform on [0, box)^d: box 1 for Z, 2 for the others.  Each box */
+/* is a union of fundamental domains (Z^1; 2Z^4 in D4; 2Z^8 in E8, which holds D8; 2Z^2 in the */
+/* (P, Q) lattice P = Q mod 2), so U = r - Q(r) is uniform on the Voronoi cell.  E8 blocks     */
+/* take groups 2b and 2b+1.                                                                    */
 /* ------------------------------------------------------------------------------------------ */
-void hqo_dither_d4(uint64_t seed, int64_t bh, int64_t s, int blk, float U[4])
+static void dither_group(uint64_t seed, int64_t c1, int64_t c, int g, float box, float r[4])
 {
-    uint32_t ctr[4] = {(uint32_t)(uint64_t)s, (uint32_t)(uint64_t)bh, 0x80000000u | (uint32_t)blk,
-                       (uint32_t)((uint64_t)s >> 32)};
+    uint32_t ctr[4] = {(uint32_t)(uint64_t)c, (uint32_t)(uint64_t)c1, 0x80000000u | (uint32_t)g,
+                       (uint32_t)((uint64_t)c >> 32)};
     uint32_t w[4];
     hqo_philox4x32_10(ctr, (uint32_t)seed, (uint32_t)(seed >> 32), w);
+    for (int i = 0; i < 4; ++i) r[i] = box * ((float)(w[i] >> 8) * 5.9604644775390625e-08f);
+}
+
+/* U for all n coefficients of one tile */
+void hqo_dither(int lattice, uint64_t seed, int64_t c1, int64_t c, int n, float* U)
+{
+    const float box = lattice == HQO_Z ? 1.0f : 2.0f;
+    float r[HQO_MAXN];
+    for (int g = 0; g < n / 4; ++g) dither_group(seed, c1, c, g, box, r + 4 * g);
+    int32_t v[8];
+    switch (lattice) {
+    case HQO_Z:
+        for (int i = 0; i < n; ++i) U[i] = r[i] - rintf(r[i]);
+        break;
+    case HQO_A2:
+        for (int b = 0; b < n / 2; ++b) {
+            hqo_q_a2_pq(r[2 * b], r[2 * b + 1], v);
+            U[2 * b] = r[2 * b] - (float)v[0];
+            U[2 * b + 1] = r[2 * b + 1] - (float)v[1];
+        }
+        break;
+    case HQO_D4:
+        for (int b = 0; b < n / 4; ++b) {
+            hqo_q_d4(r + 4 * b, v);
+            for (int i = 0; i < 4; ++i) U[4 * b + i] = r[4 * b + i] - (float)v[i];
+        }
+        break;
+    default:
+        for (int b = 0; b < n / 8; ++b) {
+            hqo_q_e8(r + 8 * b, v);  /* twice the point */
+            for (int i = 0; i < 8; ++i) U[8 * b + i] = r[8 * b + i] - 0.5f * (float)v[i];
+        }
+        break;
+    }
+}
+
+/* the D4 dither of one block (group), kept for the pins */
+void hqo_dither_d4(uint64_t seed, int64_t bh, int64_t s, int blk, float U[4])
+{
     float r[4];
-    for (int i = 0; i < 4; ++i) r[i] = 2.0f * ((float)(w[i] >> 8) * 5.9604644775390625e-08f);
+    dither_group(seed, bh, s, blk, 2.0f, r);
     int32_t q[4];
     hqo_q_d4(r, q);
     for (int i = 0; i < 4; ++i) U[i] = r[i] - (float)q[i];
@@ -479,21 +524,28 @@ void hqo_dither_d4(uint64_t seed, int64_t bh, int64_t s, int blk, float U[4])
 /* boundaries; chunk_word[c] is the word offset of chunk c, chunk_word[C] the total.          */
 /* ------------------------------------------------------------------------------------------ */
 
-/* One tile from lattice-unit coefficients u (already normalised, before dither) to symbols.
- * kv: add the D4 dither of row (bh, s) first.  Returns codes v (integer embedding). */
-static void quantize_tile(const float* u_in, int n, int lattice, int kv, uint64_t seed, int64_t bh,
-                          int64_t s, int32_t* v)
+/* One tile from lattice-unit coefficients u (already normalised, before dither) to codes v
+ * (integer embedding).  dither: add the tile's dither (counter words c1, c) first. */
+static void quantize_tile(const float* u_in, int n, int lattice, int dither, uint64_t seed, int64_t c1,
+                          int64_t c, int32_t* v)
 {
     int d = lattice_dim(lattice);
     float z[HQO_MAXN];
     for (int i = 0; i < n; ++i) z[i] = u_in[i];
-    if (kv) {
-        for (int b = 0; b < n / 4; ++b) {
-            float U[4];
-            hqo_dither_d4(seed, bh, s, b, U);
-            for (int i = 0; i < 4; ++i) z[4 * b + i] = z[4 * b + i] + U[i];
-        }
+    if (!dither) {
+        for (int b = 0; b < n / d; ++b) quantize_block(lattice, z + b * d, v + b * d);
+        return;
     }
+    float U[HQO_MAXN];
+    hqo_dither(lattice, seed, c1, c, n, U);
+    if (lattice == HQO_A2) {
+        for (int b = 0; b < n / 2; ++b) {
+            float P = 2.0f * z[2 * b], Q = z[2 * b + 1] * A2_K;
+            hqo_q_a2_pq(P + U[2 * b], Q + U[2 * b + 1], v + 2 * b);
+        }
+        return;
+    }
+    for (int i = 0; i < n; ++i) z[i] = z[i] + U[i];
     for (int b = 0; b < n / d; ++b) quantize_block(lattice, z + b * d, v + b * d);
 }
 
@@ -547,14 +599,26 @@ static int valid_common(int n, int lattice)
     return (n == 64 || n == 128 || n == 256) && lattice >= 0 && lattice <= 3;
 }
 
-/* the KV dither is defined for D4 only (its Voronoi cell) */
-static int valid_kv(int kv, int lattice) { return !kv || lattice == HQO_D4; }
+/* kv: 0 no dither; 1 KV rows (b H + h, s) with the dither; 2 weights with the dither (option) */
+static int valid_kv(int kv, int lattice) { return (kv >= 0 && kv <= 2) && lattice >= 0 && lattice <= 3; }
+
+/* dither counter words of tile (row r of the call, tile column jt) */
+static void dither_words(int kv, int64_t r, int64_t kv_S, int64_t jt, int64_t* c1, int64_t* c)
+{
+    if (kv == 1) {
+        kv_row(r, kv_S, c1, c);
+    } else {
+        *c1 = jt;
+        *c = r;
+    }
+}
 
 /*
  * Full encode.
  *   x       : [rows, cols] bf16 (dtype 0) or fp32 (dtype 1), row-major
  *   beta    : step (lattice units per normalised coefficient), > 0
- *   kv      : 1 = KV path (D4 dither), kv_S = S of the [B,H,S,D] layout (rows = B*H*S)
+ *   kv      : 1 = KV path (dither of row (b H + h, s)), kv_S = S of the [B,H,S,D] layout
+ *             (rows = B*H*S); 2 = weights with the dither of tile (row, tile column); 0 none
  *   outputs : scale[T] (bf16 bits of the per-tile RMS), meta[T] = k | (sum q << 4),
  *             chunk_word[C+1], bits[cap_words]; optional v_out[T*n] (integer codes) and
  *             u_out[T*n] (normalised coefficients before dither)
@@ -608,10 +672,10 @@ uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n,
                     float g = cn * rinv;
                     for (int j = 0; j < n; ++j) u[j] = xt[j] * g;
                 }
-                int64_t bh = 0, sidx = r;
-                if (kv) kv_row(row0 + r, kv_S, &bh, &sidx);
+                int64_t c1 = 0, cw = 0;
+                if (kv) dither_words(kv, row0 + r, kv_S, jt, &c1, &cw);
                 int32_t v[HQO_MAXN];
-                quantize_tile(u, n, lattice, kv, seed, bh, sidx, v);
+                quantize_tile(u, n, lattice, kv != 0, seed, c1, cw, v);
                 int k, sumq;
                 rice_tile(v, n, lattice, &w, &k, &sumq);
                 scale[t] = sh;
@@ -629,8 +693,9 @@ uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n,
 
 /*
  * Quantize caller-given normalised coefficients u[tiles, n] (lattice units): lattice + strip +
- * Rice + chunk layout with rows = tiles and one tile column.  For kv, the dither of row
- * (t / kv_S, t % kv_S) is added first.  Outputs as for hqo_encode (no scale).
+ * Rice + chunk layout with rows = tiles and one tile column.  kv = 1: the dither of KV row
+ * (t / kv_S, t % kv_S) is added first; kv = 2: the dither of tile (t, 0).  Outputs as for
+ * hqo_encode (no scale).
  */
 uint32_t hqo_quantize_coeffs(const float* u, int64_t tiles, int n, int lattice, int kv, int64_t kv_S,
                              uint64_t seed, int32_t* v_out, uint16_t* meta, uint32_t* chunk_word,
@@ -644,10 +709,10 @@ uint32_t hqo_quantize_coeffs(const float* u, int64_t tiles, int n, int lattice, 
         chunk_word[c] = (uint32_t)(w.bitpos >> 5);
         int64_t t_end = (c + 1) * 32 < tiles ? (c + 1) * 32 : tiles;
         for (int64_t t = c * 32; t < t_end; ++t) {
-            int64_t bh = 0, sidx = t;
-            if (kv) kv_row(t, kv_S, &bh, &sidx);
+            int64_t c1 = 0, cw = 0;
+            if (kv) dither_words(kv, t, kv_S, 0, &c1, &cw);
             int32_t v[HQO_MAXN];
-            quantize_tile(u + t * n, n, lattice, kv, seed, bh, sidx, v);
+            quantize_tile(u + t * n, n, lattice, kv != 0, seed, c1, cw, v);
             int k, sumq;
             rice_tile(v, n, lattice, &w, &k, &sumq);
             meta[t] = (uint16_t)(k | (sumq << 4));
@@ -724,25 +789,21 @@ uint32_t hqo_parse(const uint16_t* meta, const uint32_t* chunk_word, const uint3
 
 /*
  * Reconstruct one tile (binary64) from its integer codes: lattice point p (u units) from the
- * codes, minus the dither for KV, then x_hat = D H_n p * (s_hat * beta * c_n).
- *   E8: p = v / 2;  D4, Z: p = v;  A2: p = (P/2, Q sqrt(3)/2).
+ * codes, minus the dither when there is one, then x_hat = D H_n p * (s_hat * beta * c_n).
+ *   E8: p = v / 2;  D4, Z: p = v;  A2: p = (P/2, Q sqrt(3)/2), the dither taken off P and Q.
  * H_n H_n = n I and u = (H D x) c_n / (s_hat beta) give x = D H u (s_hat beta) c_n.
  */
-static void reconstruct_tile(const int32_t* v, int n, int lattice, int kv, uint64_t seed, int64_t bh,
-                             int64_t s, uint16_t sh, float beta, int64_t col0, double* out)
+static void reconstruct_tile(const int32_t* v, int n, int lattice, int dither, uint64_t seed, int64_t c1,
+                             int64_t c, uint16_t sh, float beta, int64_t col0, double* out)
 {
     double p[HQO_MAXN];
+    float U[HQO_MAXN];
+    if (dither) hqo_dither(lattice, seed, c1, c, n, U);
     for (int i = 0; i < n; ++i) {
-        if (lattice == HQO_E8) p[i] = 0.5 * (double)v[i];
-        else if (lattice == HQO_A2) p[i] = (i & 1) ? (double)v[i] * (sqrt(3.0) / 2.0) : 0.5 * (double)v[i];
-        else p[i] = (double)v[i];
-    }
-    if (kv) {
-        for (int b = 0; b < n / 4; ++b) {
-            float U[4];
-            hqo_dither_d4(seed, bh, s, b, U);
-            for (int i = 0; i < 4; ++i) p[4 * b + i] -= (double)U[i];
-        }
+        double Ui = dither ? (double)U[i] : 0.0;
+        if (lattice == HQO_E8) p[i] = 0.5 * (double)v[i] - Ui;
+        else if (lattice == HQO_A2) p[i] = (i & 1) ? ((double)v[i] - Ui) * (sqrt(3.0) / 2.0) : 0.5 * ((double)v[i] - Ui);
+        else p[i] = (double)v[i] - Ui;
     }
     hqo_fwht_f64(p, n);
     double h = (double)hqo_bf16_to_f32(sh) * (double)beta / sqrt((double)n);
@@ -765,10 +826,10 @@ uint32_t hqo_decode(const uint16_t* scale, const uint16_t* meta, const uint32_t*
     for (int64_t jt = 0; jt < NT; ++jt)
         for (int64_t r = 0; r < rows; ++r) {
             int64_t t = jt * rows + r;
-            int64_t bh = 0, sidx = r;
-            if (kv) kv_row(row0 + r, kv_S, &bh, &sidx);
+            int64_t c1 = 0, cw = 0;
+            if (kv) dither_words(kv, row0 + r, kv_S, jt, &c1, &cw);
             double tile[HQO_MAXN];
-            reconstruct_tile(v + t * n, n, lattice, kv, seed, bh, sidx, scale[t], beta, jt * n, tile);
+            reconstruct_tile(v + t * n, n, lattice, kv != 0, seed, c1, cw, scale[t], beta, jt * n, tile);
             memcpy(out + r * cols + jt * n, tile, sizeof(double) * (size_t)n);
         }
     free(v);

@@ -1,0 +1,100 @@
+"""Subtractive dither for every lattice (Methodology step 4: U ~ Uniform(V(Lambda)), added before
+quantization and subtracted after).  Pins that do not reuse the oracle's own arithmetic:
+
+* every dither vector lies in the Voronoi cell of the lattice point 0 (its nearest point is 0, by
+  brute force over the lattice points around it);
+* the dithered error per dimension is the lattice's normalised second moment times V^(2/d), a
+  closed form: Z 1/12, A2 (minimum distance 1) 5/72, D4 13/120, E8 929/12960;
+* the reconstruction is unbiased per vector over independent seeds;
+* the D4 dither is unchanged from the KV path's group definition.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+
+SQ3 = np.sqrt(3.0)
+SECOND_MOMENT = {oracle.Z: 1.0 / 12.0, oracle.A2: 5.0 / 72.0, oracle.D4: 13.0 / 120.0, oracle.E8: 929.0 / 12960.0}
+
+
+def _to_u(lattice, P):
+    """quantizer coordinates -> u coordinates (only A2 differs: (P, Q) -> (P/2, Q sqrt(3)/2))"""
+    P = np.asarray(P, dtype=np.float64)
+    if lattice != oracle.A2:
+        return P
+    out = P.copy()
+    out[..., 0::2] *= 0.5
+    out[..., 1::2] *= SQ3 / 2.0
+    return out
+
+
+def _points(lattice, v):
+    """integer embedding -> lattice point in u coordinates"""
+    v = np.asarray(v, dtype=np.float64)
+    if lattice == oracle.E8:
+        return 0.5 * v
+    return _to_u(lattice, v)
+
+
+def _near_points(lattice):
+    """lattice points (u coordinates) of one block within distance 1.5 of the origin"""
+    d = oracle.LATTICE_DIM[lattice]
+    if lattice == oracle.Z:
+        return np.array([[-1.0], [0.0], [1.0]])
+    if lattice == oracle.A2:
+        pts = [(P / 2.0, Q * SQ3 / 2.0) for P in range(-3, 4) for Q in range(-2, 3) if (P - Q) % 2 == 0]
+        return np.array(pts)
+    if lattice == oracle.D4:
+        pts = [p for p in itertools.product(range(-1, 2), repeat=4) if sum(p) % 2 == 0]
+        return np.array(pts, dtype=np.float64)
+    pts = [p for p in itertools.product(range(-1, 2), repeat=8) if sum(p) % 2 == 0]
+    half = [tuple(x / 2.0 for x in p) for p in itertools.product((-1, 1), repeat=8) if sum(p) % 4 == 0]
+    return np.array(pts + half, dtype=np.float64)
+
+
+@pytest.mark.parametrize("lattice", [oracle.Z, oracle.A2, oracle.D4, oracle.E8])
+def test_dither_lies_in_the_voronoi_cell(lattice):
+    d = oracle.LATTICE_DIM[lattice]
+    near = _near_points(lattice)
+    for c in range(40):
+        U = _to_u(lattice, oracle.dither(lattice, 11, 3, c, 128)).reshape(-1, d)
+        dist = ((U[:, None, :] - near[None, :, :]) ** 2).sum(-1)
+        d0 = (U ** 2).sum(-1)
+        assert np.all(d0 <= dist.min(1) + 1e-6)
+        assert np.max(np.abs(U)) <= 1.0
+
+
+@pytest.mark.parametrize("lattice", [oracle.Z, oracle.A2, oracle.D4, oracle.E8])
+def test_dithered_error_has_the_cells_second_moment(lattice):
+    rng = np.random.default_rng(5)
+    tiles, n = 2048, 128
+    u = (rng.standard_normal((tiles, n)) * 3.0).astype(np.float32)
+    v, *_ = oracle.quantize_coeffs(u, n, lattice, seed=9, kv=True, kv_S=tiles)
+    U = np.stack([_to_u(lattice, oracle.dither(lattice, 9, 0, t, n)) for t in range(tiles)])
+    err = _points(lattice, v) - U - u.astype(np.float64)
+    mse = np.mean(err ** 2)
+    assert abs(mse / SECOND_MOMENT[lattice] - 1.0) < 0.01, mse
+
+
+@pytest.mark.parametrize("lattice", [oracle.Z, oracle.A2, oracle.E8])
+def test_dithered_reconstruction_is_unbiased_per_vector(lattice):
+    rng = np.random.default_rng(8)
+    tiles, n, M = 16, 64, 400
+    u = (rng.standard_normal((tiles, n)) * 1.5).astype(np.float32)
+    acc = np.zeros((M, tiles, n))
+    for m in range(M):
+        v, *_ = oracle.quantize_coeffs(u, n, lattice, seed=1000 + m, kv=True, kv_S=tiles)
+        U = np.stack([_to_u(lattice, oracle.dither(lattice, 1000 + m, 0, t, n)) for t in range(tiles)])
+        acc[m] = _points(lattice, v) - U - u
+    z = acc.mean(0) / (acc.std(0) / np.sqrt(M))
+    assert np.mean(np.abs(z) > 4.0) < 1e-3
+    # the same inputs without the dither: rounding errors are a fixed function of u
+    v0, *_ = oracle.quantize_coeffs(u, n, lattice, seed=1000, kv=False)
+    assert np.max(np.abs(_points(lattice, v0) - u)) > 0.1
+
+
+def test_d4_group_dither_is_the_kv_block_dither():
+    for g in range(8):
+        assert np.array_equal(oracle.dither(oracle.D4, 7, 5, 99, 32)[4 * g:4 * g + 4], oracle.dither_d4(7, 5, 99, g))
