@@ -29,7 +29,13 @@
  *     offset in `bits`, chunk_word[C] the total number of words.
  *   - A KV tensor [B, H, S, D] (contiguous) is coded as rows = B*H*S, cols = n = D: one tile per
  *     head vector, the random signs shared by every head and token (per-layer seed), the dither
- *     fresh per (b, h, s) and D4 block.
+ *     fresh per (b, h, s) and group of four coefficients.
+ *   - Dither (Methodology step 4, "Subtractive Dither"): U uniform on the Voronoi cell of the
+ *     lattice, in its quantizer's coordinates (u for Z, D4, E8; (P, Q) = (2 u0, u1 2/sqrt3) for
+ *     A2).  Group g of four consecutive coefficients of a tile draws one Philox4x32-10 block, key
+ *     = seed, counter (c_lo, c1, 0x80000000 | g, c_hi): c = s, c1 = b*H + h for KV row (b, h, s);
+ *     c = row, c1 = tile column for dithered weights.  r_i = box (w_i >> 8) 2^-24 with box 1 (Z)
+ *     or 2, and U = r - Q(r) per lattice block (E8 blocks take groups 2b, 2b+1).
  */
 #ifndef HQ_H
 #define HQ_H
@@ -52,7 +58,7 @@ typedef enum { HQ_BF16 = 0, HQ_F32 = 1 } hq_dtype_t;
 typedef enum {
     HQ_OK = 0,
     HQ_ERR_ARG = 1,          /* bad argument (null pointer, size, alignment, range)          */
-    HQ_ERR_UNSUPPORTED = 2,  /* valid but not provided (e.g. KV dither on a lattice != D4)  */
+    HQ_ERR_UNSUPPORTED = 2,  /* valid but not provided (e.g. fp32 input with n = 256)       */
     HQ_ERR_CAPACITY = 3,     /* device: `bits` too small; detail = words needed              */
     HQ_ERR_NONFINITE = 4,    /* device: a tile held NaN/Inf (coded as zeros); detail = count */
     HQ_ERR_CORRUPT = 5,      /* device: stream inconsistent with meta / chunk_word            */
@@ -86,7 +92,7 @@ typedef struct {
  *   rows, cols  dense shape (KV: rows = B*H*S, cols = D)
  *   kv_S        S of the KV layout (dither counter); 0 for weights
  *   p           parameters with the step resolved (never 0 after encode)
- *   kv          1 for the KV path (dithered D4), else 0
+ *   kv          0 plain; 1 KV rows with the dither; 2 weights with the dither (hq_encode_dither)
  *   version     HQ_FORMAT_VERSION
  *   scale       [T] bf16 bit patterns of the per-tile RMS (0 = all-zero tile)
  *   meta        [T] k | (sum q << 4): the tile's Rice parameter and unary total
@@ -138,16 +144,25 @@ hq_status_t hq_encode(const void* x, hq_dtype_t dtype, int64_t rows, int64_t col
                       hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Weight-path dither option: as hq_encode, with the dither of tile (row, tile column) added
+ * before quantization (the method applies the dither to the KV cache; here any lattice, any
+ * shape).  out->kv = 2; hq_decode takes the dither off again.
+ */
+hq_status_t hq_encode_dither(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                             hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Decode a weight: y[rows, cols] (device, dtype, 16-byte aligned) = D H_n p * (bf16(s) beta /
- * sqrt(n)) per tile, p the lattice point; bf16 output is the binary32 value rounded to nearest
- * even.  Device errors: HQ_ERR_CORRUPT (tile written as zeros).
+ * sqrt(n)) per tile, p the lattice point (minus the dither for codes with kv = 2); bf16 output
+ * is the binary32 value rounded to nearest even.  Device errors: HQ_ERR_CORRUPT (tile written
+ * as zeros).
  */
 hq_status_t hq_decode(const hq_code_t* code, void* y, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Encode a KV tensor kv[B, H, S, D] (device, contiguous) with D == p->tile and the dithered D4
- * lattice (Methodology step 4): for each D4 block the dither U, uniform on the Voronoi cell of
- * D4, is added before quantization.  Other lattices return HQ_ERR_UNSUPPORTED.
+ * Encode a KV tensor kv[B, H, S, D] (device, contiguous) with D == p->tile and the dither
+ * (Methodology step 4): the dither U of each head vector, uniform on the Voronoi cell of
+ * p->lattice (any of the four; the method's choice is D4), is added before quantization.
  */
 hq_status_t hq_kv_encode(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D,
                          const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
@@ -158,10 +173,11 @@ hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void
 
 /*
  * Lattice quantization, bit-stripping and Rice coding of caller-given normalised coefficients
- * (Methodology steps 2-3, and step 4's dither when kv = 1): u[tiles, tile] fp32 device array in
+ * (Methodology steps 2-3, and step 4's dither when kv != 0): u[tiles, tile] fp32 device array in
  * lattice units, one tile per row, chunks of 32 consecutive rows.  v_out (device, optional,
  * int32 [tiles, tile]) receives the integer codes: Z and D4 the point itself, E8 twice the point,
- * A2 (P, Q) with the point at (P/2, Q sqrt(3)/2).  For kv, row t is token (t / kv_S, t % kv_S).
+ * A2 (P, Q) with the point at (P/2, Q sqrt(3)/2).  kv = 1: row t is token (t / kv_S, t % kv_S)
+ * (kv_S <= 0: one head); kv = 2: row t is the weight tile (t, 0).
  * out->scale may be NULL.  This entry point checks codes and bitstreams bit for bit.
  */
 hq_status_t hq_quantize_coeffs(const float* u, int64_t tiles, const hq_params_t* p, int32_t kv, int64_t kv_S,

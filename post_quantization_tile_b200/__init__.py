@@ -66,6 +66,8 @@ def lib():
         L.hq_step_for_rate.restype = ctypes.c_float
         L.hq_encode.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), ctypes.POINTER(CodeStruct), P,
                                 ctypes.c_size_t, P]
+        L.hq_encode_dither.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), ctypes.POINTER(CodeStruct), P,
+                                       ctypes.c_size_t, P]
         L.hq_decode.argtypes = [ctypes.POINTER(CodeStruct), P, i32, P, ctypes.c_size_t, P]
         L.hq_kv_encode.argtypes = [P, i32, i64, i64, i64, i64, ctypes.POINTER(Params), ctypes.POINTER(CodeStruct), P,
                                    ctypes.c_size_t, P]
@@ -79,8 +81,8 @@ def lib():
         L.hq_status_str.argtypes = [i32]
         L.hq_status_str.restype = ctypes.c_char_p
         L.hq_version.restype = i32
-        for f in ["hq_encode", "hq_decode", "hq_kv_encode", "hq_kv_decode", "hq_quantize_coeffs", "hq_encode_count",
-                  "hq_step_search", "hq_status_read"]:
+        for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_decode", "hq_quantize_coeffs",
+                  "hq_encode_count", "hq_step_search", "hq_status_read"]:
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -204,8 +206,9 @@ def _fill(code: Code, cs: CodeStruct):
 
 
 def encode(x: torch.Tensor, tile: int = 128, lattice: int | str = E8, step: float = 0.0, bps: float = 4.0,
-           seed: int = 0, out: Code | None = None, ws: Workspace | None = None) -> Code:
-    """Encode a 2-D bf16/fp32 CUDA tensor (Methodology steps 1-3)."""
+           seed: int = 0, out: Code | None = None, ws: Workspace | None = None, dither: bool = False) -> Code:
+    """Encode a 2-D bf16/fp32 CUDA tensor (Methodology steps 1-3); dither=True adds the
+    subtractive dither of each tile (the weight-path option of step 4)."""
     _require_cuda(x, "x")
     if x.dim() != 2:
         raise ValueError("x must be 2-D [rows, cols]")
@@ -216,8 +219,9 @@ def encode(x: torch.Tensor, tile: int = 128, lattice: int | str = E8, step: floa
     need = L.hq_workspace_bytes(rows, cols, ctypes.byref(p))
     w = ws or workspace(need)
     cs = code.struct()
-    _check(L.hq_encode(_ptr(x), _dtype_code(x), rows, cols, ctypes.byref(p), ctypes.byref(cs), w.ptr(), w.nbytes,
-                       _stream()), "hq_encode")
+    fn = L.hq_encode_dither if dither else L.hq_encode
+    _check(fn(_ptr(x), _dtype_code(x), rows, cols, ctypes.byref(p), ctypes.byref(cs), w.ptr(), w.nbytes, _stream()),
+           "hq_encode")
     _fill(code, cs)
     code.ws = w
     return code
@@ -231,7 +235,7 @@ def decode(code: Code, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | 
     L = lib()
     w = ws or workspace(4096)
     cs = code.struct()
-    fn = L.hq_kv_decode if code.kv else L.hq_decode
+    fn = L.hq_kv_decode if code.kv == 1 else L.hq_decode
     _check(fn(ctypes.byref(cs), _ptr(y), _dtype_code(y), w.ptr(), w.nbytes, _stream()), "hq_decode")
     code.ws = w
     return y
@@ -239,7 +243,7 @@ def decode(code: Code, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | 
 
 def kv_encode(kv: torch.Tensor, step: float = 0.0, bps: float = 4.0, seed: int = 0, lattice: int | str = D4,
               out: Code | None = None, ws: Workspace | None = None) -> Code:
-    """Encode a KV tensor [B, H, S, D] with the dithered D4 lattice (Methodology step 4)."""
+    """Encode a KV tensor [B, H, S, D] with the dither (Methodology step 4; D4 by default, any lattice)."""
     _require_cuda(kv, "kv")
     if kv.dim() != 4:
         raise ValueError("kv must be [B, H, S, D]")

@@ -169,8 +169,8 @@ hq_status_t plan_encode(const void* x, int src, int64_t rows, int64_t cols, cons
     Geometry& g = pl.g;
     const int tpt = prm.tile == 64 ? 1 : (prm.tile == 256 ? 2 : enc_tpt(128, src));
     if (!geometry(rows, cols, prm.tile, g, tpt)) return HQ_ERR_ARG;
-    if (kv && prm.lattice != HQ_D4) return HQ_ERR_UNSUPPORTED;
-    if (kv && cols != prm.tile) return HQ_ERR_ARG;
+    if (kv < 0 || kv > 2) return HQ_ERR_ARG;
+    if (kv == 1 && cols != prm.tile) return HQ_ERR_ARG;
     if (src == 1 && prm.tile == 256) return HQ_ERR_UNSUPPORTED;
     if (src == 2 && cols != prm.tile) return HQ_ERR_ARG;
     if (!x || !aligned16(x) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
@@ -192,7 +192,7 @@ hq_status_t plan_encode(const void* x, int src, int64_t rows, int64_t cols, cons
     a.beta = prm.step;
     a.seed = prm.seed;
     hq::philox_round_keys(prm.seed, a.rk);
-    a.kv_S = kv ? kv_S : 0;
+    a.kv_S = kv == 1 ? kv_S : 0;  // 0: dither counter words (row, tile column)
     a.items = g.items;
     a.IB = g.IB;
     a.RB = g.RB;
@@ -234,9 +234,9 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
     } else {
         out->rows = rows;
         out->cols = cols;
-        out->kv_S = kv ? kv_S : 0;
+        out->kv_S = kv == 1 ? kv_S : 0;
         out->p = pl.prm;
-        out->kv = kv ? 1 : 0;
+        out->kv = kv;
         out->version = HQ_FORMAT_VERSION;
     }
     return HQ_OK;
@@ -376,12 +376,12 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
                           void* stream)
 {
     if (!code || !y || !aligned16(y) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
-    if (code->version != HQ_FORMAT_VERSION || code->kv != kv) return HQ_ERR_ARG;
+    if (code->version != HQ_FORMAT_VERSION) return HQ_ERR_ARG;
+    if (kv ? code->kv != 1 : (code->kv != 0 && code->kv != 2)) return HQ_ERR_ARG;
     if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
     const hq_params_t& prm = code->p;
     if (!valid_tile(prm.tile) || prm.lattice < HQ_Z || prm.lattice > HQ_E8) return HQ_ERR_ARG;
     if (!(prm.step >= 0.00390625f && prm.step <= 64.0f)) return HQ_ERR_ARG;
-    if (kv && prm.lattice != HQ_D4) return HQ_ERR_UNSUPPORTED;
     Geometry g;
     if (!geometry(code->rows, code->cols, prm.tile, g, dec_tpt(prm.tile))) return HQ_ERR_ARG;
     if (!code->scale || !code->meta || !code->chunk_word || !code->bits || !aligned16(code->bits)) return HQ_ERR_ARG;
@@ -398,7 +398,7 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
     a.beta = prm.step;
     a.seed = prm.seed;
     hq::philox_round_keys(prm.seed, a.rk);
-    a.kv_S = code->kv_S;
+    a.kv_S = code->kv == 1 ? code->kv_S : 0;
     a.items = g.items;
     a.IB = g.IB;
     a.RB = g.RB;
@@ -409,7 +409,7 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
     a.bits = code->bits;
     a.cap_words = code->cap_words;
     a.ws = static_cast<WsHeader*>(ws);
-    return cuda_status(run_decode(prm.lattice, prm.tile, kv != 0, es == 2 ? 0 : 1, a, map, st));
+    return cuda_status(run_decode(prm.lattice, prm.tile, code->kv != 0, es == 2 ? 0 : 1, a, map, st));
 }
 
 }  // namespace
@@ -465,6 +465,13 @@ hq_status_t hq_encode(const void* x, hq_dtype_t dtype, int64_t rows, int64_t col
 {
     if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
     return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, 0, 0, nullptr, out, nullptr, ws, ws_bytes, stream);
+}
+
+hq_status_t hq_encode_dither(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
+                             hq_code_t* out, void* ws, size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, 2, 0, nullptr, out, nullptr, ws, ws_bytes, stream);
 }
 
 hq_status_t hq_decode(const hq_code_t* code, void* y, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream)

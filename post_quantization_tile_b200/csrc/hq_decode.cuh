@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
 #pragma unroll
                     for (int i = 0; i < D; ++i) {
                         float f = __int_as_float(v[i] + __float_as_int(kMagic)) - kMagic;  // exact, |v| < 2^22
-                        if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
+                        // A2: (P, Q) -> u after the dither is taken off (in P, Q coordinates)
+                        if constexpr (LAT == HQ_A2 && !KV) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
                         if (half) P[g8 * 8 + b * D + i].y = f;
                         else P[g8 * 8 + b * D + i].x = f;
                     }
@@ -304,21 +305,42 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
             }
         }
         if constexpr (KV) {
+            // the dither of this tile, taken off in the quantizer's coordinates: doubled u for E8
+            // (minus 2U), (P, Q) for A2 (then scaled to u), u for Z and D4
             const int64_t r = r0 + row_l;
             const uint64_t Sv = (uint64_t)a.kv_S;
-            const uint64_t sidx = Sv ? (uint64_t)r % Sv : (uint64_t)r;
-            const uint32_t bh = Sv ? (uint32_t)((uint64_t)r / Sv) : 0u;
+            const uint64_t dc = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+            const uint32_t dc1 = Sv ? (uint32_t)((uint64_t)r / Sv) : (uint32_t)jt;
+            if constexpr (LAT == HQ_E8) {
 #pragma unroll
-            for (int b = 0; b < H / 4; ++b) {
+                for (int g8 = 0; g8 < H / 8; ++g8) {
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float U[4];
-                    const uint32_t blk = (uint32_t)(tau * (V / 4) + half * (H / 4) + b);
-                    dither_d4(a.rk, bh, sidx, blk, U);
+                    for (int half = 0; half < 2; ++half) {
+                        float U[8];
+                        dither_e8(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8), U);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (half) P[4 * b + i].y = __fadd_rn(P[4 * b + i].y, -U[i]);
-                        else P[4 * b + i].x = __fadd_rn(P[4 * b + i].x, -U[i]);
+                        for (int i = 0; i < 8; ++i) {
+                            float2& q = P[8 * g8 + i];
+                            if (half) q.y = __fadd_rn(q.y, -__fmul_rn(2.0f, U[i]));
+                            else q.x = __fadd_rn(q.x, -__fmul_rn(2.0f, U[i]));
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int b = 0; b < H / 4; ++b) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float U[4];
+                        dither_group<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + b), U);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            float2& q = P[4 * b + i];
+                            float f = __fadd_rn(half ? q.y : q.x, -U[i]);
+                            if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
+                            if (half) q.y = f;
+                            else q.x = f;
+                        }
                     }
                 }
             }

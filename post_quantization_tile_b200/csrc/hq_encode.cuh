@@ -366,14 +366,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
             }
         }
 
-        // ---------------- KV dither counters ----------------
-        uint64_t sidx = 0;
-        uint32_t bh = 0;
+        // ---------------- dither counter words: KV row (b H + h, s), or (row, tile column) ----------------
+        uint64_t dc = 0;
+        uint32_t dc1 = 0;
         if constexpr (KV) {
             const int64_t r = r0 + row_l;
             const uint64_t Sv = (uint64_t)a.kv_S;
-            sidx = Sv ? (uint64_t)r % Sv : (uint64_t)r;
-            bh = Sv ? (uint32_t)((uint64_t)r / Sv) : 0u;
+            dc = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+            dc1 = Sv ? (uint32_t)((uint64_t)r / Sv) : (uint32_t)jt;
         }
 
         // ---------------- (dither,) lattice + strip -> zig-zag scratch ----------------
@@ -405,6 +405,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                     float2 p8[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) p8[i] = P[gb * 8 + i];
+                    if constexpr (KV) {
+                        // dither: the block of lane x is groups 2 g8, 2 g8 + 1 of this thread's
+                        // positions, lane y the same H/4 groups further on
+                        float Ux[8], Uy[8];
+                        dither_e8(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + 2 * g8), Ux);
+                        dither_e8(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + H / 4 + 2 * g8), Uy);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) p8[i] = make_float2(__fadd_rn(p8[i].x, Ux[i]), __fadd_rn(p8[i].y, Uy[i]));
+                    }
                     int32_t sx[8], sy[8], vx[8], vy[8];
                     uint32_t cx, cy;
                     e8_pair_symbols<SRC == 2>(p8, sx, sy, cx, cy, vx, vy);
@@ -422,35 +431,41 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                     store_group(g8, sx);
                     store_group(H / 8 + g8, sy);
                 } else {
-                    if constexpr (KV) {
-                        // dither: the D4 block of lane `half` at pairs 4 b .. 4 b + 4 takes
-                        // block counter tau V/4 + half H/4 + b
-#pragma unroll
-                        for (int bb = 0; bb < 2; ++bb) {
-#pragma unroll
-                            for (int half = 0; half < 2; ++half) {
-                                float U[4];
-                                const uint32_t blk = (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8 + bb);
-                                dither_d4(a.rk, bh, sidx, blk, U);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    float2& q = P[gb * 8 + 4 * bb + i];
-                                    if (half) q.y = __fadd_rn(q.y, U[i]);
-                                    else q.x = __fadd_rn(q.x, U[i]);
-                                }
-                            }
-                        }
-                    }
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
+                        float u8[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) u8[i] = half ? P[gb * 8 + i].y : P[gb * 8 + i].x;
+                        // dither of the two groups (positions half H + 8 g8 + 4 bb ..): added to u,
+                        // or for A2 to (P, Q) = (2 u0, u1 K), the coordinates of its quantizer
+                        float U8[8];
+                        if constexpr (KV) {
+#pragma unroll
+                            for (int bb = 0; bb < 2; ++bb) {
+                                float U4[4];
+                                dither_group<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8 + bb), U4);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) U8[4 * bb + i] = U4[i];
+                            }
+                            if constexpr (LAT != HQ_A2) {
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) u8[i] = __fadd_rn(u8[i], U8[i]);
+                            }
+                        }
                         int32_t sym[8];
 #pragma unroll
                         for (int b = 0; b < 8 / D; ++b) {
-                            float u[D];
-#pragma unroll
-                            for (int i = 0; i < D; ++i) u[i] = half ? P[gb * 8 + b * D + i].y : P[gb * 8 + b * D + i].x;
                             int32_t v[D];
-                            const uint32_t c = quantize_strip<LAT, SRC == 2>(u, sym + b * D, v);
+                            if constexpr (KV && LAT == HQ_A2) {
+                                int32_t v2[2];
+                                q_a2_pq(__fadd_rn(__fmul_rn(2.0f, u8[2 * b]), U8[2 * b]),
+                                        __fadd_rn(__fmul_rn(u8[2 * b + 1], kA2K), U8[2 * b + 1]), v2);
+                                v[0] = v2[0];
+                                v[1] = v2[1];
+                                strip_block<LAT>(v, sym + b * D);
+                            } else {
+                                quantize_strip<LAT, SRC == 2>(u8 + b * D, sym + b * D, v);
+                            }
                             if constexpr (SRC == 2) {
                                 if (valid && a.v_out) {
                                     int32_t* vo =
@@ -459,7 +474,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                                     for (int i = 0; i < D; ++i) vo[i] = v[i];
                                 }
                             }
-                            (void)c;
                         }
                         store_group(half * (H / 8) + g8, sym);
                     }

@@ -58,14 +58,10 @@ template <int LAT>
 static cudaError_t enc_dispatch(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m,
                                 cudaStream_t st)
 {
-    if constexpr (LAT == HQ_D4) {
-        if (kv) {
-            if (n == 64) return enc_src<64, LAT, true>(src, count, a, m, st);
-            if (n == 128) return enc_src<128, LAT, true>(src, count, a, m, st);
-            return enc_src<256, LAT, true>(src, count, a, m, st);
-        }
-    } else {
-        if (kv) return cudaErrorInvalidValue;
+    if (kv) {  // with the subtractive dither
+        if (n == 64) return enc_src<64, LAT, true>(src, count, a, m, st);
+        if (n == 128) return enc_src<128, LAT, true>(src, count, a, m, st);
+        return enc_src<256, LAT, true>(src, count, a, m, st);
     }
     if (n == 64) return enc_src<64, LAT, false>(src, count, a, m, st);
     if (n == 128) return enc_src<128, LAT, false>(src, count, a, m, st);
@@ -87,14 +83,10 @@ static cudaError_t dec_dst(int dst, const DecodeArgs& a, const CUtensorMap& m, c
 template <int LAT>
 static cudaError_t dec_dispatch(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st)
 {
-    if constexpr (LAT == HQ_D4) {
-        if (kv) {
-            if (n == 64) return dec_dst<64, LAT, true>(dst, a, m, st);
-            if (n == 128) return dec_dst<128, LAT, true>(dst, a, m, st);
-            return dec_dst<256, LAT, true>(dst, a, m, st);
-        }
-    } else {
-        if (kv) return cudaErrorInvalidValue;
+    if (kv) {  // with the subtractive dither
+        if (n == 64) return dec_dst<64, LAT, true>(dst, a, m, st);
+        if (n == 128) return dec_dst<128, LAT, true>(dst, a, m, st);
+        return dec_dst<256, LAT, true>(dst, a, m, st);
     }
     if (n == 64) return dec_dst<64, LAT, false>(dst, a, m, st);
     if (n == 128) return dec_dst<128, LAT, false>(dst, a, m, st);

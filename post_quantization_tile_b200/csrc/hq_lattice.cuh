@@ -162,10 +162,8 @@ __device__ __forceinline__ void e8_pair_symbols(const float2 (&p)[8], int32_t (&
 }
 
 // A2 with minimum distance 1 in (P, Q) = (2 u0, u1 K); the even point when |eP| + 3|eQ| <= 1.
-__device__ __forceinline__ void q_a2(const float (&u)[2], int32_t (&v)[2])
+__device__ __forceinline__ void q_a2_pq(const float P, const float Q, int32_t (&v)[2])
 {
-    const float P = __fmul_rn(2.0f, u[0]);
-    const float Q = __fmul_rn(u[1], kA2K);
     const float hP = __fmul_rn(P, 0.5f), hQ = __fmul_rn(Q, 0.5f);
     int32_t aP, aQ;
     const float rP = rint_magic(hP, aP), rQ = rint_magic(hQ, aQ);
@@ -178,6 +176,11 @@ __device__ __forceinline__ void q_a2(const float (&u)[2], int32_t (&v)[2])
         v[0] = 2 * aP + ((eP < 0.0f) ? 1 : -1);
         v[1] = 2 * aQ + ((eQ < 0.0f) ? 1 : -1);
     }
+}
+
+__device__ __forceinline__ void q_a2(const float (&u)[2], int32_t (&v)[2])
+{
+    q_a2_pq(__fmul_rn(2.0f, u[0]), __fmul_rn(u[1], kA2K), v);
 }
 
 // bit-stripping of one block: integer embedding v[d] -> d symbols (+ the E8 coset bit)
@@ -269,22 +272,70 @@ __device__ __forceinline__ void unstrip_block(const int32_t* s, uint32_t c, int3
     }
 }
 
-// KV dither for D4 block `blk` of token (bh, s): U uniform on the Voronoi cell of D4
-// ("Subtractive Dither", Methodology step 4).  r = 2 (w >> 8) 2^-24 is uniform on [0,2)^4, a union
-// of D4 cells (2Z^4 is a sublattice of D4); U = r - Q_D4(r).  rk: the round keys of the seed.
-__device__ __forceinline__ void dither_d4(const uint32_t (&rk)[20], uint32_t bh, uint64_t s, uint32_t blk, float (&U)[4])
+// Subtractive dither ("Subtractive Dither", Methodology step 4): U uniform on the Voronoi cell,
+// in the coordinates the quantizer works in (u for Z, D4, E8; (P, Q) for A2).  Group g of four
+// consecutive coefficients of a tile draws one Philox block with counter (c_lo, c1, 0x80000000 | g,
+// c_hi) under the seed's round keys rk: c = s and c1 = b H + h for KV row (b H + h, s); c = row and
+// c1 = tile column for the weight-path option.  r_i = box (w_i >> 8) 2^-24 is uniform on
+// [0, box)^4 (box 1 for Z, 2 otherwise), a union of fundamental domains (2Z^d lies in D4, in E8
+// and in the (P, Q) lattice), so U = r - Q(r) is uniform on the cell.  E8 blocks take two groups.
+__device__ __forceinline__ void dither_r(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t g, float box,
+                                         float (&r)[4])
 {
-    const uint4 w = philox4x32_10_rk(make_uint4((uint32_t)s, bh, 0x80000000u | blk, (uint32_t)(s >> 32)), rk);
-    // 2 (w >> 8) 2^-24 = (w >> 8) 2^-23: every step is exact (24-bit integers, power-of-two scale)
+    const uint4 w = philox4x32_10_rk(make_uint4((uint32_t)c, c1, 0x80000000u | g, (uint32_t)(c >> 32)), rk);
+    // box (w >> 8) 2^-24: every step is exact (24-bit integers, power-of-two scales)
+    const float sc = box == 1.0f ? 5.9604644775390625e-08f : 1.1920928955078125e-07f;
+    r[0] = __fmul_rn((float)(w.x >> 8), sc);
+    r[1] = __fmul_rn((float)(w.y >> 8), sc);
+    r[2] = __fmul_rn((float)(w.z >> 8), sc);
+    r[3] = __fmul_rn((float)(w.w >> 8), sc);
+}
+
+// U for the four coefficients of group g (Z, A2: two blocks, D4: one block)
+template <int LAT>
+__device__ __forceinline__ void dither_group(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t g,
+                                             float (&U)[4])
+{
+    static_assert(LAT != HQ_E8, "E8 blocks span two groups: dither_e8");
     float r[4];
-    r[0] = __fmul_rn((float)(w.x >> 8), 1.1920928955078125e-07f);
-    r[1] = __fmul_rn((float)(w.y >> 8), 1.1920928955078125e-07f);
-    r[2] = __fmul_rn((float)(w.z >> 8), 1.1920928955078125e-07f);
-    r[3] = __fmul_rn((float)(w.w >> 8), 1.1920928955078125e-07f);
-    int32_t q[4];
-    q_d4(r, q);
+    dither_r(rk, c1, c, g, LAT == HQ_Z ? 1.0f : 2.0f, r);
+    if constexpr (LAT == HQ_Z) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) U[i] = __fadd_rn(r[i], -(float)q[i]);
+        for (int i = 0; i < 4; ++i) {
+            int32_t a;
+            U[i] = __fadd_rn(r[i], -rint_magic(r[i], a));
+        }
+    } else if constexpr (LAT == HQ_A2) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            int32_t v[2];
+            q_a2_pq(r[2 * b], r[2 * b + 1], v);
+            U[2 * b] = __fadd_rn(r[2 * b], -(float)v[0]);
+            U[2 * b + 1] = __fadd_rn(r[2 * b + 1], -(float)v[1]);
+        }
+    } else {
+        int32_t q[4];
+        q_d4(r, q);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) U[i] = __fadd_rn(r[i], -(float)q[i]);
+    }
+}
+
+// U for the E8 block made of groups g0, g0 + 1 (u units)
+__device__ __forceinline__ void dither_e8(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t g0, float (&U)[8])
+{
+    float r[8], r0[4], r1[4];
+    dither_r(rk, c1, c, g0, 2.0f, r0);
+    dither_r(rk, c1, c, g0 + 1, 2.0f, r1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        r[i] = r0[i];
+        r[4 + i] = r1[i];
+    }
+    int32_t s[8], v[8];
+    e8_symbols<true>(r, s, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) U[i] = __fadd_rn(r[i], -__fmul_rn(0.5f, (float)v[i]));
 }
 
 }  // namespace hq

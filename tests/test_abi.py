@@ -61,5 +61,10 @@ def test_calls_reject_bad_arguments_without_a_gpu(libhq):
     assert L.hq_encode(ctypes.c_void_p(16), 0, 64, 128, ctypes.byref(p), ctypes.byref(cs), ctypes.c_void_p(256),
                        1 << 20, None) == 1
     p = hq.params(128, hq.E8, 0.3)
-    assert L.hq_kv_encode(ctypes.c_void_p(16), 0, 1, 1, 8, 128, ctypes.byref(p), ctypes.byref(cs), ctypes.c_void_p(256),
-                          1 << 20, None) == 2   # dither is defined for D4 only
+    assert L.hq_kv_encode(ctypes.c_void_p(16), 0, 1, 1, 8, 64, ctypes.byref(p), ctypes.byref(cs), ctypes.c_void_p(256),
+                          1 << 20, None) == 1   # head dimension != tile
+    p = hq.params(100, hq.A2, 0.3)
+    assert L.hq_encode_dither(None, 0, 64, 128, ctypes.byref(p), ctypes.byref(cs), None, 0, None) == 1
+    p = hq.params(128, hq.Z, 0.3)
+    assert L.hq_quantize_coeffs(ctypes.c_void_p(16), 8, ctypes.byref(p), 3, 0, None, ctypes.byref(cs),
+                                ctypes.c_void_p(256), 1 << 20, None) == 1   # kv must be 0, 1 or 2
