@@ -63,6 +63,12 @@ def lib():
         L.hqo_unstrip_block.argtypes = [i32, P, i32, P]
         L.hqo_dither_d4.argtypes = [u64, i64, i64, i32, P]
         L.hqo_dither.argtypes = [i32, u64, i64, i64, i32, P]
+        L.hqo_group_scale.argtypes = [ctypes.c_uint16, ctypes.c_float, i32, i32]
+        L.hqo_group_scale.restype = ctypes.c_float
+        L.hqo_decode_int8.argtypes = [P, P, P, P, i64, i64, i32, i32, ctypes.c_float, P, P]
+        L.hqo_decode_int8.restype = ctypes.c_uint32
+        L.hqo_gemm_grouped.argtypes = [P, P, i64, P, P, i64, i64, i32, P]
+        L.hqo_gemm_grouped_sample.argtypes = [P, P, P, P, i64, i64, i32, P, P, i64, P]
         L.hqo_rice_tile.argtypes = [P, i32, i32, P, i64, P, P]
         L.hqo_rice_tile.restype = i64
         L.hqo_parse_tile.argtypes = [P, i64, i32, i32, ctypes.c_uint16, P, P]
@@ -404,3 +410,48 @@ def step_search(x: np.ndarray, n: int, lattice: int, target_bps: float, seed: in
             break
         b = nb
     return _bits_f32(best), probes, c_best
+
+
+ST_RANGE = 1 << 6
+
+
+def decode_int8(code: Code):
+    """The weight's integer codes as int8 [rows, cols] (RHT domain) and its group scales
+    g[cols / n, rows] (binary32 ((s_hat beta) c_n) c_L); tiles with a code outside [-127, 127]
+    come back as zeros with status bit ST_RANGE.  Returns (v8, g, status)."""
+    v8 = np.zeros((code.rows, code.cols), dtype=np.int8)
+    g = np.zeros((code.cols // code.n, code.rows), dtype=np.float32)
+    bits = np.ascontiguousarray(code.bits, dtype=np.uint32)
+    if bits.size == 0:
+        bits = np.zeros(1, dtype=np.uint32)
+    st = lib().hqo_decode_int8(_p(code.scale), _p(code.meta), _p(code.chunk_word), _p(bits), code.rows, code.cols,
+                               code.n, code.lattice, ctypes.c_float(code.beta), _p(v8), _p(g))
+    if st & 2:
+        raise ValueError("oracle rejected the arguments")
+    return v8, g, int(st)
+
+
+def gemm_grouped(A: np.ndarray, sa: np.ndarray, V: np.ndarray, g: np.ndarray, n: int) -> np.ndarray:
+    """Y[m, r] = sa_m * sum_t g[t, r] S_{m,r,t} with exact int8 group sums S, binary32 fma over t."""
+    A = np.ascontiguousarray(A, dtype=np.int8)
+    V = np.ascontiguousarray(V, dtype=np.int8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    M, K = A.shape
+    N = V.shape[0]
+    Y = np.zeros((M, N), dtype=np.float32)
+    lib().hqo_gemm_grouped(_p(A), _p(sa), M, _p(V), _p(g), N, K, n, _p(Y))
+    return Y
+
+
+def gemm_grouped_sample(A, sa, V, g, n, idx_m, idx_r) -> np.ndarray:
+    A = np.ascontiguousarray(A, dtype=np.int8)
+    V = np.ascontiguousarray(V, dtype=np.int8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    im = np.ascontiguousarray(idx_m, dtype=np.int64)
+    ir = np.ascontiguousarray(idx_r, dtype=np.int64)
+    out = np.zeros(im.size, dtype=np.float32)
+    lib().hqo_gemm_grouped_sample(_p(A), _p(sa), _p(V), _p(g), V.shape[0], A.shape[1], n, _p(im), _p(ir), im.size,
+                                  _p(out))
+    return out

@@ -859,3 +859,75 @@ int hqo_parse_tile(const uint32_t* words, int64_t nwords, int n, int lattice, ui
     *bitlen = L;
     return L >= 0;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Decode-fused int8 GEMM (a next step of the method's tensor-core integration: the abstract's */
+/* 8-bit MMA paths, "int8 beats fp8 on the post-RHT lattice output").  The weight's integer     */
+/* codes v (RHT domain) multiply int8 activations that went through the same RHT:              */
+/*   (W x)_r = sum_t h_{r,t} c_L sum_{j in t} v_{r,j} (H D x)_j / n    (H H = n I),             */
+/* so with a = int8 (H D x) and a per-row activation scale sa_m:                               */
+/*   Y[m, r] = sa_m * sum_t g_{r,t} S_{m,r,t},  S = sum_{j in t} a_{m,j} v_{r,j}  (exact int),  */
+/*   g_{r,t} = ((s_hat beta) c_n) c_L,  c_L = 1/2 for E8 (doubled codes), 1 for Z and D4.       */
+/* The group sums are exact; the scales are applied in binary32 as acc = fma(S, g, acc) over   */
+/* t ascending from acc = 0, then y = acc * sa_m.                                              */
+/* ------------------------------------------------------------------------------------------ */
+
+/* group scale of one tile, binary32 as written above */
+float hqo_group_scale(uint16_t sh, float beta, int n, int lattice)
+{
+    float cn = inv_sqrt_n(n);
+    float h = (hqo_bf16_to_f32(sh) * beta) * cn;
+    return lattice == HQO_E8 ? h * 0.5f : h;
+}
+
+/* codes of a weight code -> v8[rows, cols] (int8, tile (r, jt) at columns jt n ..) and
+ * g[cols / n, rows]; tiles with a code outside [-127, 127] are written as zeros and flagged
+ * (status bit 6, range).  Only Z, D4 and E8 without dither. */
+uint32_t hqo_decode_int8(const uint16_t* scale, const uint16_t* meta, const uint32_t* chunk_word, const uint32_t* bits,
+                         int64_t rows, int64_t cols, int n, int lattice, float beta, int8_t* v8, float* g)
+{
+    if (!valid_common(n, lattice) || lattice == HQO_A2 || rows <= 0 || cols % n) return 1u << 1;
+    const int64_t NT = cols / n;
+    int32_t* v = (int32_t*)malloc(sizeof(int32_t) * (size_t)(rows * cols));
+    if (!v) return 1u << 1;
+    uint32_t status = hqo_parse(meta, chunk_word, bits, rows, cols, n, lattice, v);
+    for (int64_t jt = 0; jt < NT; ++jt)
+        for (int64_t r = 0; r < rows; ++r) {
+            int64_t t = jt * rows + r;
+            int ok = 1;
+            for (int i = 0; i < n; ++i)
+                if (v[t * n + i] < -127 || v[t * n + i] > 127) ok = 0;
+            if (!ok) status |= 1u << 6;
+            for (int i = 0; i < n; ++i) v8[r * cols + jt * n + i] = ok ? (int8_t)v[t * n + i] : 0;
+            g[jt * rows + r] = hqo_group_scale(scale[t], beta, n, lattice);
+        }
+    free(v);
+    return status;
+}
+
+/* one output of the grouped GEMM: A[M, K], V[N, K] int8 row-major, g[K / n, N], sa[M] */
+float hqo_gemm_one(const int8_t* A, const float* sa, const int8_t* V, const float* g, int64_t N, int64_t K, int n,
+                   int64_t m, int64_t r)
+{
+    float acc = 0.0f;
+    for (int64_t t = 0; t < K / n; ++t) {
+        int64_t S = 0;
+        for (int j = 0; j < n; ++j) S += (int64_t)A[m * K + t * n + j] * (int64_t)V[r * K + t * n + j];
+        acc = fmaf((float)S, g[t * N + r], acc);
+    }
+    return acc * sa[m];
+}
+
+void hqo_gemm_grouped(const int8_t* A, const float* sa, int64_t M, const int8_t* V, const float* g, int64_t N,
+                      int64_t K, int n, float* Y)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t r = 0; r < N; ++r) Y[m * N + r] = hqo_gemm_one(A, sa, V, g, N, K, n, m, r);
+}
+
+/* sampled outputs Y[idx_m[i], idx_r[i]] */
+void hqo_gemm_grouped_sample(const int8_t* A, const float* sa, const int8_t* V, const float* g, int64_t N, int64_t K,
+                             int n, const int64_t* idx_m, const int64_t* idx_r, int64_t count, float* out)
+{
+    for (int64_t i = 0; i < count; ++i) out[i] = hqo_gemm_one(A, sa, V, g, N, K, n, idx_m[i], idx_r[i]);
+}
