@@ -190,6 +190,32 @@ hq_status_t hq_quantize_coeffs(const float* u, int64_t tiles, const hq_params_t*
 hq_status_t hq_encode_count(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,
                             int32_t kv, int64_t kv_S, uint64_t* bits_out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * The weight's integer lattice codes, for an int8 tensor-core GEMM in the RHT domain: v_out
+ * [rows, cols] int8 (device, 16-byte aligned) holds the codes of tile (r, jt) at columns jt n ..
+ * (E8: twice the lattice point; Z, D4: the point), g_out [cols / n, rows] fp32 (device) the tile's
+ * scale ((s_hat beta) c_n) c_L with c_L = 1/2 for E8, 1 otherwise, in binary32, so that the tile
+ * decodes to D H_n (v g).  Tiles with a code outside [-127, 127] are written as zeros and
+ * reported as HQ_ERR_RANGE; tiles of a corrupt stream as zeros with HQ_ERR_CORRUPT.
+ * Supported: Z, D4, E8 codes without dither, n = 128 or 256 (HQ_ERR_UNSUPPORTED otherwise).
+ */
+hq_status_t hq_decode_int8(const hq_code_t* code, int8_t* v_out, float* g_out, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/*
+ * Grouped int8 GEMM on the tensor cores (the method's int8 MMA path on the post-RHT lattice
+ * codes; abstract and "Experimental Results"):
+ *   Y[m, r] = sa[m] * sum_t g[t, r] S(m, r, t),  S(m, r, t) = sum_{j = 128 t}^{128 t + 127} A[m, j] V[r, j]
+ * A int8 [M, K] (activations after the same RHT, D H_n per tile of 128), sa fp32 [M], V int8
+ * [N, K] and g fp32 [K / 128, N] as written by hq_decode_int8, Y fp32 [M, N]; all device,
+ * row-major, 16-byte aligned.  The group sums are exact; the scales are applied in binary32 as
+ * acc = fma(S, g, acc) over t = 0, 1, ... from acc = 0, then Y = acc * sa[m].  group must be 128;
+ * M and N multiples of 128, K a multiple of 128 up to 8192 (HQ_ERR_UNSUPPORTED / HQ_ERR_ARG
+ * otherwise).  ws: at least 64 bytes; a bounded wait that ran out reports HQ_ERR_TIMEOUT there.
+ */
+hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8_t* V, const float* g, int64_t N,
+                         int64_t K, int32_t group, float* Y, void* ws, size_t ws_bytes, void* stream);
+
 /* Result of a step search, written to device memory. */
 typedef struct {
     float step;            /* the chosen step beta                                          */

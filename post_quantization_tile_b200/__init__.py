@@ -75,6 +75,8 @@ def lib():
         L.hq_quantize_coeffs.argtypes = [P, i64, ctypes.POINTER(Params), i32, i64, P, ctypes.POINTER(CodeStruct), P,
                                          ctypes.c_size_t, P]
         L.hq_encode_count.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, P, P, ctypes.c_size_t, P]
+        L.hq_decode_int8.argtypes = [ctypes.POINTER(CodeStruct), P, P, P, ctypes.c_size_t, P]
+        L.hq_gemm_int8.argtypes = [P, P, i64, P, P, i64, i64, i32, P, P, ctypes.c_size_t, P]
         L.hq_step_search.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, i32, ctypes.c_float, P, P,
                                      ctypes.c_size_t, P]
         L.hq_status_read.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
@@ -82,7 +84,7 @@ def lib():
         L.hq_status_str.restype = ctypes.c_char_p
         L.hq_version.restype = i32
         for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_decode", "hq_quantize_coeffs",
-                  "hq_encode_count", "hq_step_search", "hq_status_read"]:
+                  "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_status_read"]:
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -299,6 +301,33 @@ def encode_count(x: torch.Tensor, tile: int, lattice: int | str, step: float, se
     _check(L.hq_encode_count(_ptr(x), _dtype_code(x), rows, cols, ctypes.byref(p), int(kv), int(kv_S), _ptr(outb),
                              w.ptr(), w.nbytes, _stream()), "hq_encode_count")
     return outb
+
+
+def decode_int8(code: Code, ws: Workspace | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """The code's integer lattice codes int8 [rows, cols] and tile scales fp32 [cols / n, rows]
+    (hq_decode_int8), the operands of gemm_int8."""
+    dev = code.bits.device
+    v = torch.empty(code.rows, code.cols, dtype=torch.int8, device=dev)
+    g = torch.empty(code.cols // code.p.tile, code.rows, dtype=torch.float32, device=dev)
+    w = ws or workspace(4096)
+    cs = code.struct()
+    _check(lib().hq_decode_int8(ctypes.byref(cs), _ptr(v), _ptr(g), w.ptr(), w.nbytes, _stream()), "hq_decode_int8")
+    code.ws = w
+    return v, g
+
+
+def gemm_int8(A: torch.Tensor, sa: torch.Tensor, V: torch.Tensor, g: torch.Tensor, out: torch.Tensor | None = None,
+              ws: Workspace | None = None) -> torch.Tensor:
+    """Y = sa * sum_t g[t] (A V^T restricted to group t) on the tensor cores (hq_gemm_int8)."""
+    for t, name in ((A, "A"), (sa, "sa"), (V, "V"), (g, "g")):
+        _require_cuda(t, name)
+    M, K = A.shape
+    N = V.shape[0]
+    Y = out if out is not None else torch.empty(M, N, dtype=torch.float32, device=A.device)
+    w = ws or workspace(4096)
+    _check(lib().hq_gemm_int8(_ptr(A), _ptr(sa), M, _ptr(V), _ptr(g), N, K, 128, _ptr(Y), w.ptr(), w.nbytes,
+                              _stream()), "hq_gemm_int8")
+    return Y
 
 
 def step_search(x: torch.Tensor, tile: int, lattice: int | str, target_bps: float, seed: int = 0, kv: bool = False,

@@ -50,7 +50,8 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
 {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
-    const CUtensorMapDataType dt = es == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapDataType dt = es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : (es == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)cols * (cuuint64_t)es};
     const cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows};
@@ -372,13 +373,18 @@ hq_status_t step_search_common(const void* x, int src, int64_t rows, int64_t col
     return cuda_status(cudaGetLastError());
 }
 
-hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int32_t kv, void* ws, size_t ws_bytes,
-                          void* stream)
+// dst: 0 bf16, 1 fp32, 2 int8 lattice codes with group scales g_out
+hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, float* g_out, void* ws,
+                          size_t ws_bytes, void* stream)
 {
     if (!code || !y || !aligned16(y) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
     if (code->version != HQ_FORMAT_VERSION) return HQ_ERR_ARG;
     if (kv ? code->kv != 1 : (code->kv != 0 && code->kv != 2)) return HQ_ERR_ARG;
-    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (dst < 0 || dst > 2) return HQ_ERR_ARG;
+    if (dst == 2) {
+        if (!g_out || (reinterpret_cast<uintptr_t>(g_out) & 3u)) return HQ_ERR_ARG;
+        if (code->kv != 0 || code->p.lattice == HQ_A2 || code->p.tile == 64) return HQ_ERR_UNSUPPORTED;
+    }
     const hq_params_t& prm = code->p;
     if (!valid_tile(prm.tile) || prm.lattice < HQ_Z || prm.lattice > HQ_E8) return HQ_ERR_ARG;
     if (!(prm.step >= 0.00390625f && prm.step <= 64.0f)) return HQ_ERR_ARG;
@@ -387,12 +393,13 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
     if (!code->scale || !code->meta || !code->chunk_word || !code->bits || !aligned16(code->bits)) return HQ_ERR_ARG;
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
     if (!use_device_of(y)) return HQ_ERR_ARG;
-    const int es = dtype == HQ_BF16 ? 2 : 4;
+    const int es = dst == 0 ? 2 : (dst == 1 ? 4 : 1);
     CUtensorMap map;
     if (!make_map(&map, y, code->rows, code->cols, es, g.TI)) return HQ_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
     DecodeArgs a{};
+    a.g_out = g_out;
     a.rows = code->rows;
     a.cols = code->cols;
     a.beta = prm.step;
@@ -409,10 +416,18 @@ hq_status_t decode_common(const hq_code_t* code, void* y, hq_dtype_t dtype, int3
     a.bits = code->bits;
     a.cap_words = code->cap_words;
     a.ws = static_cast<WsHeader*>(ws);
-    return cuda_status(run_decode(prm.lattice, prm.tile, code->kv != 0, es == 2 ? 0 : 1, a, map, st));
+    return cuda_status(run_decode(prm.lattice, prm.tile, code->kv != 0, dst, a, map, st));
 }
 
 }  // namespace
+
+// shared with the other translation units of the library (hq_launch.h)
+bool tensor_map_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int es, int box_rows)
+{
+    return make_map(m, base, rows, cols, es, box_rows);
+}
+bool device_of(const void* p) { return use_device_of(p); }
+
 }  // namespace hq
 
 using namespace hq;
@@ -476,7 +491,13 @@ hq_status_t hq_encode_dither(const void* x, hq_dtype_t dtype, int64_t rows, int6
 
 hq_status_t hq_decode(const hq_code_t* code, void* y, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream)
 {
-    return decode_common(code, y, dtype, 0, ws, ws_bytes, stream);
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    return decode_common(code, y, dtype == HQ_BF16 ? 0 : 1, 0, nullptr, ws, ws_bytes, stream);
+}
+
+hq_status_t hq_decode_int8(const hq_code_t* code, int8_t* v_out, float* g_out, void* ws, size_t ws_bytes, void* stream)
+{
+    return decode_common(code, v_out, 2, 0, g_out, ws, ws_bytes, stream);
 }
 
 hq_status_t hq_kv_encode(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D,
@@ -491,7 +512,8 @@ hq_status_t hq_kv_encode(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H,
 
 hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream)
 {
-    return decode_common(code, kv, dtype, 1, ws, ws_bytes, stream);
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    return decode_common(code, kv, dtype == HQ_BF16 ? 0 : 1, 1, nullptr, ws, ws_bytes, stream);
 }
 
 hq_status_t hq_quantize_coeffs(const float* u, int64_t tiles, const hq_params_t* p, int32_t kv, int64_t kv_S,

@@ -27,16 +27,17 @@ struct DecodeArgs {
     int64_t cap_words;
     WsHeader* ws;
     uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
+    float* g_out;     // int8-code output: group scale of tile (r, jt) at g_out[jt rows + r]
 };
 
-template <int N, int DST>  // DST: 0 bf16, 1 fp32
+template <int N, int DST>  // DST: 0 bf16, 1 fp32, 2 int8 lattice codes (RHT domain, no transform)
 struct DecGeom {
     static constexpr int TPT = dec_tpt(N);
     static constexpr int V = N / TPT;
     static constexpr int H = V / 2;
     static constexpr int TI = kThreads / TPT;
     static constexpr int CH = TI / kChunkTiles;
-    static constexpr int ES = DST == 0 ? 2 : 4;
+    static constexpr int ES = DST == 0 ? 2 : (DST == 1 ? 4 : 1);
     static constexpr int ROWB = N * ES;
     static constexpr int NB = ROWB / 128;
     static constexpr int OUT = NB * TI * 128;
@@ -47,7 +48,7 @@ struct DecGeom {
     static constexpr int LMAX = N / 8 + 12 * N + 2 * N;
     static constexpr int GUARD = 4;  // words before and after the copied range
     static constexpr int IN_WORDS = (TI * ((LMAX + 31) / 32) + CH + 8 + 2 * GUARD + 3) / 4 * 4;
-    static constexpr int MASKS = DST == 0 ? N / 2 : N;
+    static constexpr int MASKS = DST == 0 ? N / 2 : (DST == 1 ? N : 4);
     static constexpr int LOG2N = N == 64 ? 6 : (N == 128 ? 7 : 8);
     // input stages: one (the next item is fetched once this one is parsed) or two (fetched a
     // whole item ahead, at the cost of shared memory)
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
         const bool valid = row_l < rows_valid;
         const bool stage_ok = sm.ok_ring[st] != 0;
 
-        if (sm.mask_jt != jt) {
+        if (DST != 2 && sm.mask_jt != jt) {
             build_masks_out<N, DST>(sm.mask, jt, a.seed);
             __syncthreads();
             if (tid == 0) sm.mask_jt = jt;
@@ -279,6 +280,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
 
         // ---------------- codes -> lattice point (float pairs) ----------------
         float2 P[H];
+        uint32_t out_of_int8 = 0u;  // int8-code output: some code of the tile is outside [-127, 127]
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -295,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                     unstrip_block<LAT>(sym + b * D, (cosbits >> (pos / 8)) & 1u, v);
 #pragma unroll
                     for (int i = 0; i < D; ++i) {
+                        if constexpr (DST == 2) out_of_int8 |= (uint32_t)(v[i] + 127) > 254u ? 1u : 0u;
                         float f = __int_as_float(v[i] + __float_as_int(kMagic)) - kMagic;  // exact, |v| < 2^22
                         // A2: (P, Q) -> u after the dither is taken off (in P, Q coordinates)
                         if constexpr (LAT == HQ_A2 && !KV) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
@@ -304,122 +307,159 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 }
             }
         }
-        if constexpr (KV) {
-            // the dither of this tile, taken off in the quantizer's coordinates: doubled u for E8
-            // (minus 2U), (P, Q) for A2 (then scaled to u), u for Z and D4
-            const int64_t r = r0 + row_l;
-            const uint64_t Sv = (uint64_t)a.kv_S;
-            const uint64_t dc = Sv ? (uint64_t)r % Sv : (uint64_t)r;
-            const uint32_t dc1 = Sv ? (uint32_t)((uint64_t)r / Sv) : (uint32_t)jt;
-            if constexpr (LAT == HQ_E8) {
-#pragma unroll
-                for (int g8 = 0; g8 < H / 8; ++g8) {
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float U[8];
-                        dither_e8(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8), U);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float2& q = P[8 * g8 + i];
-                            if (half) q.y = __fadd_rn(q.y, -__fmul_rn(2.0f, U[i]));
-                            else q.x = __fadd_rn(q.x, -__fmul_rn(2.0f, U[i]));
-                        }
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int b = 0; b < H / 4; ++b) {
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float U[4];
-                        dither_group<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + b), U);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            float2& q = P[4 * b + i];
-                            float f = __fadd_rn(half ? q.y : q.x, -U[i]);
-                            if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
-                            if (half) q.y = f;
-                            else q.x = f;
-                        }
-                    }
-                }
+        if constexpr (DST == 2) {
+            // ---------------- int8 lattice codes + group scale (no transform) ----------------
+            if constexpr (TPT == 2) out_of_int8 |= __shfl_xor_sync(0xffffffffu, out_of_int8, 1);
+            const bool keep = ok && out_of_int8 == 0u;
+            if (valid && ok && out_of_int8 && tau == 0) status_set(a.ws, kStRange);
+            if (valid && tau == 0) {
+                const float sh = __uint_as_float((uint32_t)sbits << 16);
+                const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
+                float gs = __fmul_rn(__fmul_rn(sh, a.beta), cn);
+                if constexpr (LAT == HQ_E8) gs = __fmul_rn(gs, 0.5f);
+                a.g_out[jt * a.rows + r0 + row_l] = gs;
             }
-        }
-        if (__any_sync(0xffffffffu, !ok)) {
+            __syncthreads();  // every thread has read its scratch: the box may be overwritten
+            // 16 codes per 16-byte chunk; chunk c of this thread's half-row holds elements 16 c ..
 #pragma unroll
-            for (int m = 0; m < H; ++m) P[m] = ok ? P[m] : make_float2(0.0f, 0.0f);
-        }
-
-        // ---------------- inverse transform: H_n p, exact for integer points ----------------
-        // in-thread strides (H within pairs, then H/2 .. 1); with two threads per tile the
-        // stride n/2 butterfly between the pair comes last
-#pragma unroll
-        for (int m = 0; m < H; ++m) P[m] = make_float2(__fadd_rn(P[m].x, P[m].y), __fadd_rn(P[m].x, -P[m].y));
-#pragma unroll
-        for (int h = H / 2; h >= 1; h /= 2)
-#pragma unroll
-            for (int m = 0; m < H; ++m)
-                if ((m & h) == 0) {
-                    const float2 x = P[m], y = P[m + h];
-                    P[m] = f2add(x, y);
-                    P[m + h] = f2sub(x, y);
-                }
-        if constexpr (TPT == 2) {
-#pragma unroll
-            for (int m = 0; m < H; ++m) {
-                const float ox = __shfl_xor_sync(0xffffffffu, P[m].x, 1);
-                const float oy = __shfl_xor_sync(0xffffffffu, P[m].y, 1);
-                // tau 0 holds a (positions < n/2), tau 1 holds b: a + b -> tau 0, a - b -> tau 1
-                P[m] = tau ? make_float2(__fadd_rn(ox, -P[m].x), __fadd_rn(oy, -P[m].y))
-                           : make_float2(__fadd_rn(P[m].x, ox), __fadd_rn(P[m].y, oy));
-            }
-        }
-
-        // ---------------- scale, sign, store into the staging box ----------------
-        const float sh = __uint_as_float((uint32_t)sbits << 16);
-        const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
-        float ht = __fmul_rn(__fmul_rn(sh, a.beta), cn);
-        if constexpr (LAT == HQ_E8) ht = __fmul_rn(ht, 0.5f);
-        const float2 h2 = make_float2(ht, ht);
-#pragma unroll
-        for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], h2);
-
-        __syncthreads();  // every thread has read its scratch: the box may be overwritten
-        if constexpr (DST == 0) {
-            // bf16: 8 elements per 16-byte chunk; chunk c holds elements 8c .. 8c+7
-#pragma unroll
-            for (int c = 0; c < H / 8; ++c) {
+            for (int c = 0; c < H / 16; ++c) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    const int e0 = tau * V + half * H + 8 * c;  // first element of the chunk
+                    const int e0 = tau * V + half * H + 16 * c;
                     uint32_t w[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float lo = half ? P[8 * c + 2 * q].y : P[8 * c + 2 * q].x;
-                        const float hi = half ? P[8 * c + 2 * q + 1].y : P[8 * c + 2 * q + 1].x;
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);  // one packed RNE conversion
-                        w[q] = *reinterpret_cast<const uint32_t*>(&b2) ^ sm.mask[e0 / 2 + q];
+                        uint32_t b4 = 0u;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float f = half ? P[16 * c + 4 * q + e].y : P[16 * c + 4 * q + e].x;
+                            b4 |= ((uint32_t)__float2int_rn(f) & 0xFFu) << (8 * e);
+                        }
+                        w[q] = keep ? b4 : 0u;
                     }
-                    const int cg = e0 / 8;
+                    const int cg = e0 / 16;
                     *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
         } else {
-#pragma unroll
-            for (int c = 0; c < H / 4; ++c) {
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int e0 = tau * V + half * H + 4 * c;
-                    uint32_t w[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float f = half ? P[4 * c + q].y : P[4 * c + q].x;
-                        w[q] = __float_as_uint(f) ^ sm.mask[e0 + q];
+            if constexpr (KV) {
+                // the dither of this tile, taken off in the quantizer's coordinates: doubled u for E8
+                // (minus 2U), (P, Q) for A2 (then scaled to u), u for Z and D4
+                const int64_t r = r0 + row_l;
+                const uint64_t Sv = (uint64_t)a.kv_S;
+                const uint64_t dc = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+                const uint32_t dc1 = Sv ? (uint32_t)((uint64_t)r / Sv) : (uint32_t)jt;
+                if constexpr (LAT == HQ_E8) {
+    #pragma unroll
+                    for (int g8 = 0; g8 < H / 8; ++g8) {
+    #pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            float U[8];
+                            dither_e8(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8), U);
+    #pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                float2& q = P[8 * g8 + i];
+                                if (half) q.y = __fadd_rn(q.y, -__fmul_rn(2.0f, U[i]));
+                                else q.x = __fadd_rn(q.x, -__fmul_rn(2.0f, U[i]));
+                            }
+                        }
                     }
-                    const int cg = e0 / 4;
-                    *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
+                } else {
+    #pragma unroll
+                    for (int b = 0; b < H / 4; ++b) {
+    #pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            float U[4];
+                            dither_group<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + b), U);
+    #pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                float2& q = P[4 * b + i];
+                                float f = __fadd_rn(half ? q.y : q.x, -U[i]);
+                                if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
+                                if (half) q.y = f;
+                                else q.x = f;
+                            }
+                        }
+                    }
+                }
+            }
+            if (__any_sync(0xffffffffu, !ok)) {
+    #pragma unroll
+                for (int m = 0; m < H; ++m) P[m] = ok ? P[m] : make_float2(0.0f, 0.0f);
+            }
+
+            // ---------------- inverse transform: H_n p, exact for integer points ----------------
+            // in-thread strides (H within pairs, then H/2 .. 1); with two threads per tile the
+            // stride n/2 butterfly between the pair comes last
+    #pragma unroll
+            for (int m = 0; m < H; ++m) P[m] = make_float2(__fadd_rn(P[m].x, P[m].y), __fadd_rn(P[m].x, -P[m].y));
+    #pragma unroll
+            for (int h = H / 2; h >= 1; h /= 2)
+    #pragma unroll
+                for (int m = 0; m < H; ++m)
+                    if ((m & h) == 0) {
+                        const float2 x = P[m], y = P[m + h];
+                        P[m] = f2add(x, y);
+                        P[m + h] = f2sub(x, y);
+                    }
+            if constexpr (TPT == 2) {
+    #pragma unroll
+                for (int m = 0; m < H; ++m) {
+                    const float ox = __shfl_xor_sync(0xffffffffu, P[m].x, 1);
+                    const float oy = __shfl_xor_sync(0xffffffffu, P[m].y, 1);
+                    // tau 0 holds a (positions < n/2), tau 1 holds b: a + b -> tau 0, a - b -> tau 1
+                    P[m] = tau ? make_float2(__fadd_rn(ox, -P[m].x), __fadd_rn(oy, -P[m].y))
+                               : make_float2(__fadd_rn(P[m].x, ox), __fadd_rn(P[m].y, oy));
+                }
+            }
+
+            // ---------------- scale, sign, store into the staging box ----------------
+            const float sh = __uint_as_float((uint32_t)sbits << 16);
+            const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
+            float ht = __fmul_rn(__fmul_rn(sh, a.beta), cn);
+            if constexpr (LAT == HQ_E8) ht = __fmul_rn(ht, 0.5f);
+            const float2 h2 = make_float2(ht, ht);
+    #pragma unroll
+            for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], h2);
+
+            __syncthreads();  // every thread has read its scratch: the box may be overwritten
+            if constexpr (DST == 0) {
+                // bf16: 8 elements per 16-byte chunk; chunk c holds elements 8c .. 8c+7
+    #pragma unroll
+                for (int c = 0; c < H / 8; ++c) {
+    #pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int e0 = tau * V + half * H + 8 * c;  // first element of the chunk
+                        uint32_t w[4];
+    #pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float lo = half ? P[8 * c + 2 * q].y : P[8 * c + 2 * q].x;
+                            const float hi = half ? P[8 * c + 2 * q + 1].y : P[8 * c + 2 * q + 1].x;
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(lo, hi);  // one packed RNE conversion
+                            w[q] = *reinterpret_cast<const uint32_t*>(&b2) ^ sm.mask[e0 / 2 + q];
+                        }
+                        const int cg = e0 / 8;
+                        *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            } else {
+    #pragma unroll
+                for (int c = 0; c < H / 4; ++c) {
+    #pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int e0 = tau * V + half * H + 4 * c;
+                        uint32_t w[4];
+    #pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float f = half ? P[4 * c + q].y : P[4 * c + q].x;
+                            w[q] = __float_as_uint(f) ^ sm.mask[e0 + q];
+                        }
+                        const int cg = e0 / 4;
+                        *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                    }
                 }
             }
         }

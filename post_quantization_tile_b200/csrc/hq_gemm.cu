@@ -1,0 +1,293 @@
+// hq_gemm.cu -- int8 tensor-core GEMM over the weight's lattice codes with one binary32 scale per
+// tile (tcgen05 MMA, TMEM accumulators, TMA operand loads).
+//
+// Y[m, r] = sa_m * sum_t g[t, r] S_{m,r,t},  S_{m,r,t} = sum_{j in group t} A[m, j] V[r, j]
+// with A int8 [M, K] (activations after the same RHT as the weight), V int8 [N, K] (the weight's
+// integer codes in the RHT domain) and g [K / 128, N] the per-tile scales.  The group sums are
+// exact int32 MMA results; the scales are applied in binary32 as acc = fma(S, g, acc) over the
+// groups in order, then y = acc * sa_m.  This is the int8 MMA path of the method (abstract: 8-bit
+// tensor-core MMA paths, int8 ahead of fp8 on the post-RHT lattice output), with the group scale
+// the decoder would otherwise apply.
+//
+// One CTA computes a 128 x 128 tile of Y: warp 0 streams 128 x 128-byte boxes of A and V into a
+// 4-stage ring with TMA (128-byte swizzle, the canonical K-major layout of the MMA); warp 1 issues
+// four tcgen05.mma.kind::i8 (M 128, N 128, K 32) per group into one of four TMEM accumulator slots
+// (4 x 128 columns); warps 2-5 drain each finished slot (tcgen05.ld), convert the int32 sums,
+// apply the group scales with paired binary32 fma and release the slot, so MMA and scaling overlap.
+// Every wait is bounded: on a timeout the kernel records HQ_ERR_TIMEOUT and winds down.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/hq.h"
+#include "hq_common.cuh"
+#include "hq_launch.h"
+
+namespace hq {
+namespace {
+
+constexpr float kMagicGemm = 12582912.0f;  // 1.5 * 2^23
+constexpr int kMagicBits = 0x4B400000;
+
+constexpr int GM = 128, GN = 128, GK = 128;  // CTA tile (M, N) and K group
+constexpr int GSTAGES = 4;                   // operand ring
+constexpr int GACC = 4;                      // TMEM accumulator slots of GN columns
+constexpr int GTHREADS = 192;
+constexpr int GKMAX = 8192;                  // scales of every group stay in shared memory
+
+struct GemmSmem {
+    alignas(1024) int8_t a[GSTAGES][GM * GK];
+    alignas(1024) int8_t b[GSTAGES][GN * GK];
+    alignas(16) float g[GKMAX / GK][GN];
+    alignas(8) uint64_t full[GSTAGES];
+    uint64_t empty[GSTAGES];
+    uint64_t acc_full[GACC];
+    uint64_t acc_empty[GACC];
+    uint32_t tmem_base;
+};
+
+struct GemmArgs {
+    int64_t M, N, K;
+    const float* sa;
+    const float* g;
+    WsHeader* ws;
+};
+
+// ---------------- tcgen05 wrappers ----------------
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms 1024 bytes apart
+__device__ __forceinline__ uint64_t sw128_desc(const void* p)
+{
+    const uint64_t addr = (uint64_t)((smem_u32(p) >> 4) & 0x3FFFu);
+    return addr | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// instruction descriptor: s8 x s8 -> s32, both K-major, M = GM, N = GN
+constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(GN >> 3) << 17) | ((uint32_t)(GM >> 4) << 24);
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
+{
+    const uint32_t z = 0u;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z)
+        : "memory");
+}
+
+// arrive on `bar` once every MMA issued so far by this thread has completed
+__device__ __forceinline__ void mma_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 consecutive columns of this warp's 32 TMEM lanes (one lane per thread)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+          "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__global__ void __launch_bounds__(GTHREADS, 1)
+    gemm_i8_grouped_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
+                           const __grid_constant__ CUtensorMap tY)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * GN, m0 = blockIdx.y * GM;
+    const int KB = (int)(a.K / GK);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < GSTAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int s = 0; s < GACC; ++s) {
+            mbar_init(&sm.acc_full[s], 1);
+            mbar_init(&sm.acc_empty[s], 4);  // one arrival per epilogue warp
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem_base, GACC * GN);
+    if (warp >= 2) {
+        const int c = threadIdx.x - 64;
+        for (int kb = 0; kb < KB; ++kb) sm.g[kb][c] = a.g[(int64_t)kb * a.N + n0 + c];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sm.tmem_base;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % GSTAGES;
+                if (kb >= GSTAGES && !mbar_wait(&sm.empty[s], (uint32_t)((kb / GSTAGES - 1) & 1))) {
+                    status_set(a.ws, kStTimeout);
+                    break;
+                }
+                mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(GM * GK + GN * GK));
+                tma_load_2d(sm.a[s], &tA, kb * GK, m0, &sm.full[s]);
+                tma_load_2d(sm.b[s], &tB, kb * GK, n0, &sm.full[s]);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % GSTAGES, slot = kb % GACC;
+                if (kb >= GACC && !mbar_wait(&sm.acc_empty[slot], (uint32_t)((kb / GACC - 1) & 1))) {
+                    status_set(a.ws, kStTimeout);
+                    break;
+                }
+                if (!mbar_wait(&sm.full[s], (uint32_t)((kb / GSTAGES) & 1))) {
+                    status_set(a.ws, kStTimeout);
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = sw128_desc(sm.a[s]), bd = sw128_desc(sm.b[s]);
+#pragma unroll
+                for (int kk = 0; kk < GK / 32; ++kk)  // K 32 per MMA: the start address moves 32 bytes
+                    mma_i8(tbase + (uint32_t)(slot * GN), ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), kIdescI8,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(&sm.empty[s]);
+                mma_commit(&sm.acc_full[slot]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------- epilogue: scale and accumulate each group ----------------
+        const int q = warp & 3;  // this warp's TMEM lane quarter
+        const int row = q * 32 + lane;
+        float2 acc[GN / 2];
+#pragma unroll
+        for (int c = 0; c < GN / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
+        const float2 nm = make_float2(-kMagicGemm, -kMagicGemm);
+        bool alive = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int slot = kb % GACC;
+            const bool got = mbar_wait(&sm.acc_full[slot], (uint32_t)((kb / GACC) & 1));
+            __syncwarp();  // the warp-wide TMEM loads below need the whole warp converged
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0) status_set(a.ws, kStTimeout);
+                alive = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < GN / 32; ++ch) {
+                uint32_t S[32];
+                tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + ch * 32), S);
+                const float4* gp = reinterpret_cast<const float4*>(&sm.g[kb][ch * 32]);
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const float4 g4 = gp[c4];
+                    // |S| < 2^22: adding 1.5 * 2^23 in the integer domain gives an exact float
+                    const float2 f0 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4] + kMagicBits),
+                                                             __int_as_float((int)S[4 * c4 + 1] + kMagicBits)), nm);
+                    const float2 f1 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4 + 2] + kMagicBits),
+                                                             __int_as_float((int)S[4 * c4 + 3] + kMagicBits)), nm);
+                    acc[ch * 16 + 2 * c4] = __ffma2_rn(f0, make_float2(g4.x, g4.y), acc[ch * 16 + 2 * c4]);
+                    acc[ch * 16 + 2 * c4 + 1] = __ffma2_rn(f1, make_float2(g4.z, g4.w), acc[ch * 16 + 2 * c4 + 1]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty[slot]);
+        }
+        // ---------------- output: y = acc * sa, through a swizzled staging box, TMA store ----------------
+        const float sa = a.sa[m0 + row];
+        unsigned char* stage = reinterpret_cast<unsigned char*>(&sm.a[0][0]);  // operand ring is idle now
+        if (alive) {
+#pragma unroll
+            for (int b = 0; b < GN / 32; ++b)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float2 p0 = acc[b * 16 + 2 * j], p1 = acc[b * 16 + 2 * j + 1];
+                    *reinterpret_cast<float4*>(stage + b * (GM * 128) + swz(row, j)) =
+                        make_float4(__fmul_rn(p0.x, sa), __fmul_rn(p0.y, sa), __fmul_rn(p1.x, sa), __fmul_rn(p1.y, sa));
+                }
+        }
+        fence_proxy_async();
+        named_sync(1, 128);
+        if (alive && threadIdx.x == 64) {
+#pragma unroll
+            for (int b = 0; b < GN / 32; ++b) tma_store_2d(&tY, n0 + b * 32, m0, stage + b * (GM * 128));
+            bulk_commit();
+            bulk_wait0();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tbase, GACC * GN);
+}
+
+}  // namespace
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8_t* V, const float* g,
+                                    int64_t N, int64_t K, int32_t group, float* Y, void* ws, size_t ws_bytes,
+                                    void* stream)
+{
+    if (!A || !sa || !V || !g || !Y || !ws) return HQ_ERR_ARG;
+    if (group != GK) return HQ_ERR_UNSUPPORTED;
+    if (M < GM || N < GN || K < GK || M % GM || N % GN || K % GK) return HQ_ERR_ARG;
+    if (K > GKMAX || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return HQ_ERR_UNSUPPORTED;
+    if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(V) |
+                         reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(ws) |
+                         reinterpret_cast<uintptr_t>(g) | reinterpret_cast<uintptr_t>(sa);
+    if (al & 15u) return HQ_ERR_ARG;
+    if (!device_of(A)) return HQ_ERR_ARG;
+    CUtensorMap ta, tb, ty;
+    if (!tensor_map_2d(&ta, A, M, K, 1, GM) || !tensor_map_2d(&tb, V, N, K, 1, GN) || !tensor_map_2d(&ty, Y, M, N, 4, GM))
+        return HQ_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
+    const size_t smem = sizeof(GemmSmem) + 1024;
+    static bool attr_set = false;  // per process; the attribute is per function and device-independent
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(gemm_i8_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return HQ_ERR_CUDA;
+        attr_set = true;
+    }
+    GemmArgs a{M, N, K, sa, g, static_cast<WsHeader*>(ws)};
+    const dim3 grid((unsigned)(N / GN), (unsigned)(M / GM));
+    gemm_i8_grouped_kernel<<<grid, GTHREADS, smem, st>>>(a, ta, tb, ty);
+    return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}

@@ -77,6 +77,10 @@ static cudaError_t dec_one(const DecodeArgs& a, const CUtensorMap& m, cudaStream
 template <int N, int LAT, bool KV>
 static cudaError_t dec_dst(int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st)
 {
+    if (dst == 2) {  // int8 lattice codes: integer-valued lattices without dither, 128-byte tile rows
+        if constexpr (!KV && LAT != HQ_A2 && N != 64) return dec_one<N, LAT, KV, 2>(a, m, st);
+        return cudaErrorInvalidValue;
+    }
     return dst == 0 ? dec_one<N, LAT, KV, 0>(a, m, st) : dec_one<N, LAT, KV, 1>(a, m, st);
 }
 

@@ -23,4 +23,10 @@ cudaError_t launch_decode_e8(int n, bool kv, int dst, const DecodeArgs& a, const
 
 int num_sms();
 
+// 2-D tensor map of a row-major [rows, cols] tensor of es-byte elements: box [box_rows][128 bytes],
+// 128-byte swizzle (hq_api.cu)
+bool tensor_map_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int es, int box_rows);
+// make the device that owns p current (hq_api.cu)
+bool device_of(const void* p);
+
 }  // namespace hq
