@@ -42,6 +42,14 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+def load_bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 def make_inputs():
     from post_quantization_tile_b200 import workloads as W
     return [W.llama_weight(r, c, seed=SEED + i) for i, (r, c) in enumerate(SHAPES)]
@@ -317,6 +325,7 @@ def run_gpu(args):
     value = weak_scaling_value(bf16_bytes, world, ms)
 
     kv = None if args.no_kv else run_kv(hq, dev, stream, peak)
+    gemm = None if args.no_gemm else run_gemm(hq, dev, load_bf16_peak())
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -349,6 +358,7 @@ def run_gpu(args):
                     "h2d_bytes_per_step": bf16_bytes, "d2h_bytes_per_step": bf16_bytes},
             "gpu_launches": 4 * args.steps,
             "kv_cache": kv,
+            "gemm_int8": gemm,
             "clocks": clk.summary(),
             "status": st,
         }
@@ -407,13 +417,77 @@ def run_kv(hq, dev, stream, peak):
             "bytes_per_call": moved, "status": st}
 
 
+def run_gemm(hq, dev, peak_bf16):
+    """Int8 tensor-core GEMM over lattice codes: the 4096 x 4096 E8 weight's int8 codes (decoded
+    once) times 4096 int8 activations in the RHT domain (N(0, 32^2) clipped to +-127), group
+    scales per tile.  Per-call times of hq_gemm_int8 and hq_decode_int8, outside the timed step."""
+    import torch
+
+    from post_quantization_tile_b200 import workloads as W
+    M = N = K = 4096
+    w = torch.from_numpy(W.llama_weight(N, K, seed=1).view(np.int16)).view(torch.bfloat16).to(dev)
+    code = hq.encode(w, 128, hq.E8, 0.29, seed=SEED)
+    V, g = hq.decode_int8(code)
+    rng = np.random.default_rng(6)
+    a = torch.from_numpy(np.clip(np.round(rng.standard_normal((M, K)) * 32.0), -127, 127).astype(np.int8)).to(dev)
+    sa = torch.full((M,), 0.02, dtype=torch.float32, device=dev)
+    Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+    calls = 20
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(calls)]
+    for _ in range(3):
+        hq.gemm_int8(a, sa, V, g, out=Y)
+        hq.decode_int8(code)
+    for k in range(calls):
+        ev[k][0].record()
+        hq.gemm_int8(a, sa, V, g, out=Y)
+        ev[k][1].record()
+        ev[k][2].record()
+        hq.decode_int8(code)
+        ev[k][3].record()
+    torch.cuda.synchronize()
+    st = hq.status(hq.workspace(4096))[0]
+    gm = [e[0].elapsed_time(e[1]) for e in ev]
+    dm = [e[2].elapsed_time(e[3]) for e in ev]
+    tops = 2.0 * M * N * K / (statistics.median(gm) * 1e-3) / 1e12
+    peak = 2.0 * peak_bf16  # int8 dense = 2x bf16 dense (nominal ratio)
+    return {"workload": "int8 A[4096,4096] x E8 codes of llama7b 4096x4096 (n=128 groups) -> fp32",
+            "gemm_ms_p10_p50_p90": percentiles(gm), "decode_int8_ms_p10_p50_p90": percentiles(dm),
+            "roofline": {"bound": "tensor", "achieved": tops, "peak": peak,
+                         "peak_kind": "2 x measured bf16 burst", "unit": "TOP/s", "frac": tops / peak},
+            "status": st}
+
+
 def run_profile(args):
     """One kernel on a 16384x4096 bf16 weight (134 MB, larger than L2), fixed step, three
-    launches after one set-up encode: a short, self-contained command for ncu captures."""
+    launches after one set-up encode (gemm: the int8 GEMM on 4096^3): a short, self-contained
+    command for ncu captures."""
     import torch
 
     import post_quantization_tile_b200 as hq
     from post_quantization_tile_b200 import workloads as W
+    if args.profile == "gemm":
+        # int8 GEMM over the E8 codes of a 4096 x 4096 weight and 4096 int8 activation rows
+        w = torch.from_numpy(W.llama_weight(4096, 4096, seed=1).view(np.int16)).view(torch.bfloat16).cuda()
+        code = hq.encode(w, TILE, hq.E8, 0.29, seed=SEED)
+        V, g = hq.decode_int8(code)
+        rng = np.random.default_rng(6)
+        act = np.clip(np.round(rng.standard_normal((4096, 4096)) * 32.0), -127, 127).astype(np.int8)
+        A = torch.from_numpy(act).cuda()
+        sa = torch.full((4096,), 0.02, dtype=torch.float32, device="cuda")
+        Y = torch.empty(4096, 4096, dtype=torch.float32, device="cuda")
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        torch.cuda.synchronize()
+        for i in range(3):
+            ev[i].record()
+            hq.gemm_int8(A, sa, V, g, out=Y)
+        ev[3].record()
+        torch.cuda.synchronize()
+        st = hq.status(hq.workspace(4096))[0]
+        print(json.dumps({"profile": "gemm", "ms": [ev[i].elapsed_time(ev[i + 1]) for i in range(3)], "status": st}),
+              flush=True)
+        if st != 0:
+            raise SystemExit(1)
+        return
     x = torch.from_numpy(W.llama_weight(16384, 4096, seed=9).view(np.int16)).view(torch.bfloat16).cuda()
     beta = 0.29
     code = hq.encode(x, TILE, hq.E8, beta, seed=SEED)
@@ -439,13 +513,14 @@ def run_profile(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile", choices=["encode", "decode", "count"], default=None)
+    ap.add_argument("--profile", choices=["encode", "decode", "count", "gemm"], default=None)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kv", action="store_true", help="skip the KV-cache codec fields")
+    ap.add_argument("--no-gemm", action="store_true", help="skip the int8 GEMM fields")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)

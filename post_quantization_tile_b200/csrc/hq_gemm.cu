@@ -12,8 +12,9 @@
 // One CTA computes a 128 x 128 tile of Y: warp 0 streams 128 x 128-byte boxes of A and V into a
 // 4-stage ring with TMA (128-byte swizzle, the canonical K-major layout of the MMA); warp 1 issues
 // four tcgen05.mma.kind::i8 (M 128, N 128, K 32) per group into one of four TMEM accumulator slots
-// (4 x 128 columns); warps 2-5 drain each finished slot (tcgen05.ld), convert the int32 sums,
-// apply the group scales with paired binary32 fma and release the slot, so MMA and scaling overlap.
+// (4 x 128 columns); warps 2-9 (two warpgroups, 64 columns each) read each finished slot
+// (tcgen05.ld), release it, convert the int32 sums and apply the group scales with paired binary32
+// fma, so MMA and scaling overlap.
 // Every wait is bounded: on a timeout the kernel records HQ_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -31,7 +32,8 @@ constexpr int kMagicBits = 0x4B400000;
 constexpr int GM = 128, GN = 128, GK = 128;  // CTA tile (M, N) and K group
 constexpr int GSTAGES = 4;                   // operand ring
 constexpr int GACC = 4;                      // TMEM accumulator slots of GN columns
-constexpr int GTHREADS = 192;
+constexpr int GEPI = 8;                      // epilogue warps: two warpgroups, 64 columns each
+constexpr int GTHREADS = 64 + 32 * GEPI;
 constexpr int GKMAX = 8192;                  // scales of every group stay in shared memory
 
 struct GemmSmem {
@@ -96,8 +98,9 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar)
                  : "memory");
 }
 
-// 32 consecutive columns of this warp's 32 TMEM lanes (one lane per thread)
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+// 32 consecutive columns of this warp's 32 TMEM lanes (one lane per thread); complete after
+// tmem_wait_ld()
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[32])
 {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
@@ -108,8 +111,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
           "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
         : "r"(taddr)
         : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void named_sync(int id, int threads)
 {
@@ -133,15 +137,13 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         }
         for (int s = 0; s < GACC; ++s) {
             mbar_init(&sm.acc_full[s], 1);
-            mbar_init(&sm.acc_empty[s], 4);  // one arrival per epilogue warp
+            mbar_init(&sm.acc_empty[s], GEPI);  // one arrival per epilogue warp
         }
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(&sm.tmem_base, GACC * GN);
-    if (warp >= 2) {
-        const int c = threadIdx.x - 64;
-        for (int kb = 0; kb < KB; ++kb) sm.g[kb][c] = a.g[(int64_t)kb * a.N + n0 + c];
-    }
+    for (int i = (int)threadIdx.x - 64; i >= 0 && i < KB * GN; i += 32 * GEPI)
+        sm.g[i / GN][i % GN] = a.g[(int64_t)(i / GN) * a.N + n0 + i % GN];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -188,11 +190,15 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         __syncwarp();
     } else {
         // ---------------- epilogue: scale and accumulate each group ----------------
-        const int q = warp & 3;  // this warp's TMEM lane quarter
+        // warpgroup h (warps 2-5: h = 0, warps 6-9: h = 1) takes columns 64 h .. 64 h + 63 of each
+        // slot; a warp reads the TMEM lane quarter warp % 4, one accumulator row per thread
+        const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
         const int row = q * 32 + lane;
-        float2 acc[GN / 2];
+        constexpr int HC = GN / 2;  // columns per warpgroup
+        float2 acc[HC / 2];
 #pragma unroll
-        for (int c = 0; c < GN / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
+        for (int c = 0; c < HC / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
         const float2 nm = make_float2(-kMagicGemm, -kMagicGemm);
         bool alive = true;
         for (int kb = 0; kb < KB; ++kb) {
@@ -205,42 +211,44 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 break;
             }
             tc_fence_after();
-#pragma unroll
-            for (int ch = 0; ch < GN / 32; ++ch) {
-                uint32_t S[32];
-                tmem_ld32(tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + ch * 32), S);
-                const float4* gp = reinterpret_cast<const float4*>(&sm.g[kb][ch * 32]);
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    const float4 g4 = gp[c4];
-                    // |S| < 2^22: adding 1.5 * 2^23 in the integer domain gives an exact float
-                    const float2 f0 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4] + kMagicBits),
-                                                             __int_as_float((int)S[4 * c4 + 1] + kMagicBits)), nm);
-                    const float2 f1 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4 + 2] + kMagicBits),
-                                                             __int_as_float((int)S[4 * c4 + 3] + kMagicBits)), nm);
-                    acc[ch * 16 + 2 * c4] = __ffma2_rn(f0, make_float2(g4.x, g4.y), acc[ch * 16 + 2 * c4]);
-                    acc[ch * 16 + 2 * c4 + 1] = __ffma2_rn(f1, make_float2(g4.z, g4.w), acc[ch * 16 + 2 * c4 + 1]);
-                }
-            }
+            uint32_t S[HC];
+            const uint32_t ta = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + h * HC);
+            tmem_ld32_nowait(ta, *reinterpret_cast<uint32_t(*)[32]>(&S[0]));
+            tmem_ld32_nowait(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&S[32]));
+            tmem_wait_ld();
+            // the slot is read: release it to the MMA before the arithmetic
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.acc_empty[slot]);
+            const float4* gp = reinterpret_cast<const float4*>(&sm.g[kb][h * HC]);
+#pragma unroll
+            for (int c4 = 0; c4 < HC / 4; ++c4) {
+                const float4 g4 = gp[c4];
+                // |S| < 2^22: adding 1.5 * 2^23 in the integer domain gives an exact float
+                const float2 f0 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4] + kMagicBits),
+                                                         __int_as_float((int)S[4 * c4 + 1] + kMagicBits)), nm);
+                const float2 f1 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4 + 2] + kMagicBits),
+                                                         __int_as_float((int)S[4 * c4 + 3] + kMagicBits)), nm);
+                acc[2 * c4] = __ffma2_rn(f0, make_float2(g4.x, g4.y), acc[2 * c4]);
+                acc[2 * c4 + 1] = __ffma2_rn(f1, make_float2(g4.z, g4.w), acc[2 * c4 + 1]);
+            }
         }
         // ---------------- output: y = acc * sa, through a swizzled staging box, TMA store ----------------
         const float sa = a.sa[m0 + row];
         unsigned char* stage = reinterpret_cast<unsigned char*>(&sm.a[0][0]);  // operand ring is idle now
         if (alive) {
 #pragma unroll
-            for (int b = 0; b < GN / 32; ++b)
+            for (int bb = 0; bb < HC / 32; ++bb)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const float2 p0 = acc[b * 16 + 2 * j], p1 = acc[b * 16 + 2 * j + 1];
+                    const int b = h * (HC / 32) + bb;  // 32-column box
+                    const float2 p0 = acc[bb * 16 + 2 * j], p1 = acc[bb * 16 + 2 * j + 1];
                     *reinterpret_cast<float4*>(stage + b * (GM * 128) + swz(row, j)) =
                         make_float4(__fmul_rn(p0.x, sa), __fmul_rn(p0.y, sa), __fmul_rn(p1.x, sa), __fmul_rn(p1.y, sa));
                 }
         }
         fence_proxy_async();
-        named_sync(1, 128);
+        named_sync(1, 32 * GEPI);
         if (alive && threadIdx.x == 64) {
 #pragma unroll
             for (int b = 0; b < GN / 32; ++b) tma_store_2d(&tY, n0 + b * 32, m0, stage + b * (GM * 128));
