@@ -12,7 +12,7 @@
 // One CTA computes a 128 x 128 tile of Y: warp 0 streams 128 x 128-byte boxes of A and V into a
 // 4-stage ring with TMA (128-byte swizzle, the canonical K-major layout of the MMA); warp 1 issues
 // four tcgen05.mma.kind::i8 (M 128, N 128, K 32) per group into one of four TMEM accumulator slots
-// (4 x 128 columns); warps 2-9 (two warpgroups, 64 columns each) read each finished slot
+// (4 x 128 columns); the epilogue warps (warpgroups of 32 columns each) read each finished slot
 // (tcgen05.ld), release it, convert the int32 sums and apply the group scales with paired binary32
 // fma, so MMA and scaling overlap.
 // Every wait is bounded: on a timeout the kernel records HQ_ERR_TIMEOUT and winds down.
@@ -23,6 +23,10 @@
 #include "hq_common.cuh"
 #include "hq_launch.h"
 
+#ifndef HQ_GEMM_EPI_WARPS
+#define HQ_GEMM_EPI_WARPS 16
+#endif
+
 namespace hq {
 namespace {
 
@@ -32,7 +36,7 @@ constexpr int kMagicBits = 0x4B400000;
 constexpr int GM = 128, GN = 128, GK = 128;  // CTA tile (M, N) and K group
 constexpr int GSTAGES = 4;                   // operand ring
 constexpr int GACC = 4;                      // TMEM accumulator slots of GN columns
-constexpr int GEPI = 8;                      // epilogue warps: two warpgroups, 64 columns each
+constexpr int GEPI = HQ_GEMM_EPI_WARPS;      // epilogue warps: GEPI / 4 warpgroups, GN / (GEPI / 4) columns each
 constexpr int GTHREADS = 64 + 32 * GEPI;
 constexpr int GKMAX = 8192;                  // scales of every group stay in shared memory
 
@@ -190,12 +194,13 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         __syncwarp();
     } else {
         // ---------------- epilogue: scale and accumulate each group ----------------
-        // warpgroup h (warps 2-5: h = 0, warps 6-9: h = 1) takes columns 64 h .. 64 h + 63 of each
-        // slot; a warp reads the TMEM lane quarter warp % 4, one accumulator row per thread
+        // warpgroup h (warps 2 + 4h .. 5 + 4h) takes columns HC h .. HC h + HC - 1 of each slot; a
+        // warp reads the TMEM lane quarter warp % 4, one accumulator row per thread
         const int q = warp & 3;
         const int h = (warp - 2) >> 2;
         const int row = q * 32 + lane;
-        constexpr int HC = GN / 2;  // columns per warpgroup
+        constexpr int HC = GN / (GEPI / 4);  // columns per warpgroup
+        static_assert(HC % 32 == 0, "TMEM loads take 32 columns");
         float2 acc[HC / 2];
 #pragma unroll
         for (int c = 0; c < HC / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
@@ -213,8 +218,9 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             tc_fence_after();
             uint32_t S[HC];
             const uint32_t ta = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + h * HC);
-            tmem_ld32_nowait(ta, *reinterpret_cast<uint32_t(*)[32]>(&S[0]));
-            tmem_ld32_nowait(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&S[32]));
+#pragma unroll
+            for (int c = 0; c < HC / 32; ++c)
+                tmem_ld32_nowait(ta + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&S[32 * c]));
             tmem_wait_ld();
             // the slot is read: release it to the MMA before the arithmetic
             tc_fence_before();
