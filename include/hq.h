@@ -210,7 +210,7 @@ hq_status_t hq_decode_int8(const hq_code_t* code, int8_t* v_out, float* g_out, v
  * [N, K] and g fp32 [K / 128, N] as written by hq_decode_int8, Y fp32 [M, N]; all device,
  * row-major, 16-byte aligned.  The group sums are exact; the scales are applied in binary32 as
  * acc = fma(S, g, acc) over t = 0, 1, ... from acc = 0, then Y = acc * sa[m].  group must be 128;
- * M and N multiples of 128, K a multiple of 128 up to 8192 (HQ_ERR_UNSUPPORTED / HQ_ERR_ARG
+ * M and N multiples of 128, K a multiple of 128 up to 2^20 (HQ_ERR_UNSUPPORTED / HQ_ERR_ARG
  * otherwise).  ws: at least 64 bytes; a bounded wait that ran out reports HQ_ERR_TIMEOUT there.
  */
 hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8_t* V, const float* g, int64_t N,

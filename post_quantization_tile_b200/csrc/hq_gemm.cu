@@ -9,13 +9,14 @@
 // tensor-core MMA paths, int8 ahead of fp8 on the post-RHT lattice output), with the group scale
 // the decoder would otherwise apply.
 //
-// One CTA computes a 128 x 128 tile of Y: warp 0 streams 128 x 128-byte boxes of A and V into a
-// 4-stage ring with TMA (128-byte swizzle, the canonical K-major layout of the MMA); warp 1 issues
+// Persistent CTAs (one per SM) walk the 128 x 128 tiles of Y: warp 0 streams 128 x 128-byte boxes
+// of A and V and the group's 128 scales into a 4-stage ring with TMA (128-byte swizzle, the
+// canonical K-major layout of the MMA); warp 1 issues
 // four tcgen05.mma.kind::i8 (M 128, N 128, K 32) per group into one of four TMEM accumulator slots
 // (4 x 128 columns); the epilogue warps (warpgroups of 32 columns each) read each finished slot
 // (tcgen05.ld), release it, convert the int32 sums and apply the group scales with paired binary32
-// fma, so MMA and scaling overlap.
-// Every wait is bounded: on a timeout the kernel records HQ_ERR_TIMEOUT and winds down.
+// fma, so MMA and scaling overlap; a tile's result leaves through a staging buffer and TMA stores
+// while the next tile's MMAs run.  Every wait is bounded: on a timeout the kernel records HQ_ERR_TIMEOUT and winds down.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -38,12 +39,12 @@ constexpr int GSTAGES = 4;                   // operand ring
 constexpr int GACC = 4;                      // TMEM accumulator slots of GN columns
 constexpr int GEPI = HQ_GEMM_EPI_WARPS;      // epilogue warps: GEPI / 4 warpgroups, GN / (GEPI / 4) columns each
 constexpr int GTHREADS = 64 + 32 * GEPI;
-constexpr int GKMAX = 8192;                  // scales of every group stay in shared memory
 
 struct GemmSmem {
     alignas(1024) int8_t a[GSTAGES][GM * GK];
     alignas(1024) int8_t b[GSTAGES][GN * GK];
-    alignas(16) float g[GKMAX / GK][GN];
+    alignas(1024) unsigned char out[GN / 32][GM * 128];  // output staging: 32-column boxes
+    alignas(16) float g[GSTAGES][GN];                     // the group's scales, loaded with the operands
     alignas(8) uint64_t full[GSTAGES];
     uint64_t empty[GSTAGES];
     uint64_t acc_full[GACC];
@@ -131,13 +132,14 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * GN, m0 = blockIdx.y * GM;
     const int KB = (int)(a.K / GK);
+    const int NT = (int)(a.N / GN);
+    const int tiles = (int)(a.M / GM) * NT;  // persistent: tiles blockIdx.x, + gridDim.x, ...
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < GSTAGES; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.empty[s], 1 + GEPI);  // the MMAs' commit and every epilogue warp's read of g
         }
         for (int s = 0; s < GACC; ++s) {
             mbar_init(&sm.acc_full[s], 1);
@@ -146,54 +148,65 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(&sm.tmem_base, GACC * GN);
-    for (int i = (int)threadIdx.x - 64; i >= 0 && i < KB * GN; i += 32 * GEPI)
-        sm.g[i / GN][i % GN] = a.g[(int64_t)(i / GN) * a.N + n0 + i % GN];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer: A, V boxes and the group's scales ----------------
         if (lane == 0) {
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % GSTAGES;
-                if (kb >= GSTAGES && !mbar_wait(&sm.empty[s], (uint32_t)((kb / GSTAGES - 1) & 1))) {
-                    status_set(a.ws, kStTimeout);
-                    break;
+            int it = 0;
+            bool alive = true;
+            for (int tile = blockIdx.x; alive && tile < tiles; tile += gridDim.x) {
+                const int m0 = (tile / NT) * GM, n0 = (tile % NT) * GN;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % GSTAGES;
+                    if (it >= GSTAGES && !mbar_wait(&sm.empty[s], (uint32_t)((it / GSTAGES - 1) & 1))) {
+                        status_set(a.ws, kStTimeout);
+                        alive = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(GM * GK + GN * GK + GN * 4));
+                    tma_load_2d(sm.a[s], &tA, kb * GK, m0, &sm.full[s]);
+                    tma_load_2d(sm.b[s], &tB, kb * GK, n0, &sm.full[s]);
+                    bulk_load_1d(sm.g[s], a.g + (int64_t)kb * a.N + n0, GN * 4, &sm.full[s]);
                 }
-                mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(GM * GK + GN * GK));
-                tma_load_2d(sm.a[s], &tA, kb * GK, m0, &sm.full[s]);
-                tma_load_2d(sm.b[s], &tB, kb * GK, n0, &sm.full[s]);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % GSTAGES, slot = kb % GACC;
-                if (kb >= GACC && !mbar_wait(&sm.acc_empty[slot], (uint32_t)((kb / GACC - 1) & 1))) {
-                    status_set(a.ws, kStTimeout);
-                    break;
-                }
-                if (!mbar_wait(&sm.full[s], (uint32_t)((kb / GSTAGES) & 1))) {
-                    status_set(a.ws, kStTimeout);
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t ad = sw128_desc(sm.a[s]), bd = sw128_desc(sm.b[s]);
+            int it = 0;
+            bool alive = true;
+            for (int tile = blockIdx.x; alive && tile < tiles; tile += gridDim.x) {
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % GSTAGES, slot = it % GACC;
+                    if (it >= GACC && !mbar_wait(&sm.acc_empty[slot], (uint32_t)((it / GACC - 1) & 1))) {
+                        status_set(a.ws, kStTimeout);
+                        alive = false;
+                        break;
+                    }
+                    if (!mbar_wait(&sm.full[s], (uint32_t)((it / GSTAGES) & 1))) {
+                        status_set(a.ws, kStTimeout);
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(sm.a[s]), bd = sw128_desc(sm.b[s]);
 #pragma unroll
-                for (int kk = 0; kk < GK / 32; ++kk)  // K 32 per MMA: the start address moves 32 bytes
-                    mma_i8(tbase + (uint32_t)(slot * GN), ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), kIdescI8,
-                           kk > 0 ? 1u : 0u);
-                mma_commit(&sm.empty[s]);
-                mma_commit(&sm.acc_full[slot]);
+                    for (int kk = 0; kk < GK / 32; ++kk)  // K 32 per MMA: the start address moves 32 bytes
+                        mma_i8(tbase + (uint32_t)(slot * GN), ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
+                               kIdescI8, kk > 0 ? 1u : 0u);
+                    mma_commit(&sm.empty[s]);
+                    mma_commit(&sm.acc_full[slot]);
+                }
             }
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue: scale and accumulate each group ----------------
+        // ---------------- epilogue: scale and accumulate each group, store each tile ----------------
         // warpgroup h (warps 2 + 4h .. 5 + 4h) takes columns HC h .. HC h + HC - 1 of each slot; a
         // warp reads the TMEM lane quarter warp % 4, one accumulator row per thread
         const int q = warp & 3;
@@ -201,66 +214,79 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         const int row = q * 32 + lane;
         constexpr int HC = GN / (GEPI / 4);  // columns per warpgroup
         static_assert(HC % 32 == 0, "TMEM loads take 32 columns");
-        float2 acc[HC / 2];
-#pragma unroll
-        for (int c = 0; c < HC / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
         const float2 nm = make_float2(-kMagicGemm, -kMagicGemm);
+        int it = 0;
         bool alive = true;
-        for (int kb = 0; kb < KB; ++kb) {
-            const int slot = kb % GACC;
-            const bool got = mbar_wait(&sm.acc_full[slot], (uint32_t)((kb / GACC) & 1));
-            __syncwarp();  // the warp-wide TMEM loads below need the whole warp converged
-            if (!__all_sync(0xffffffffu, got)) {
-                if (lane == 0) status_set(a.ws, kStTimeout);
-                alive = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t S[HC];
-            const uint32_t ta = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + h * HC);
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            const int m0 = (tile / NT) * GM, n0 = (tile % NT) * GN;
+            float2 acc[HC / 2];
 #pragma unroll
-            for (int c = 0; c < HC / 32; ++c)
-                tmem_ld32_nowait(ta + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&S[32 * c]));
-            tmem_wait_ld();
-            // the slot is read: release it to the MMA before the arithmetic
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.acc_empty[slot]);
-            const float4* gp = reinterpret_cast<const float4*>(&sm.g[kb][h * HC]);
+            for (int c = 0; c < HC / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
+            // after a timeout a warp keeps walking the loops without waiting, so that every
+            // epilogue warp still reaches each named barrier below
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+                if (!alive) continue;
+                const int slot = it % GACC, s = it % GSTAGES;
+                const bool got = mbar_wait(&sm.acc_full[slot], (uint32_t)((it / GACC) & 1));
+                __syncwarp();  // the warp-wide TMEM loads below need the whole warp converged
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) status_set(a.ws, kStTimeout);
+                    alive = false;
+                    continue;
+                }
+                tc_fence_after();
+                uint32_t S[HC];
+                const uint32_t ta = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + h * HC);
 #pragma unroll
-            for (int c4 = 0; c4 < HC / 4; ++c4) {
-                const float4 g4 = gp[c4];
-                // |S| < 2^22: adding 1.5 * 2^23 in the integer domain gives an exact float
-                const float2 f0 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4] + kMagicBits),
-                                                         __int_as_float((int)S[4 * c4 + 1] + kMagicBits)), nm);
-                const float2 f1 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4 + 2] + kMagicBits),
-                                                         __int_as_float((int)S[4 * c4 + 3] + kMagicBits)), nm);
-                acc[2 * c4] = __ffma2_rn(f0, make_float2(g4.x, g4.y), acc[2 * c4]);
-                acc[2 * c4 + 1] = __ffma2_rn(f1, make_float2(g4.z, g4.w), acc[2 * c4 + 1]);
+                for (int c = 0; c < HC / 32; ++c)
+                    tmem_ld32_nowait(ta + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&S[32 * c]));
+                float gv[HC];
+#pragma unroll
+                for (int c4 = 0; c4 < HC / 4; ++c4) {
+                    const float4 g4 = reinterpret_cast<const float4*>(&sm.g[s][h * HC])[c4];
+                    gv[4 * c4] = g4.x;
+                    gv[4 * c4 + 1] = g4.y;
+                    gv[4 * c4 + 2] = g4.z;
+                    gv[4 * c4 + 3] = g4.w;
+                }
+                tmem_wait_ld();
+                // slot and scales are read: release both before the arithmetic
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&sm.acc_empty[slot]);
+                    mbar_arrive(&sm.empty[s]);
+                }
+#pragma unroll
+                for (int c2 = 0; c2 < HC / 2; ++c2) {
+                    // |S| < 2^22: adding 1.5 * 2^23 in the integer domain gives an exact float
+                    const float2 f = __fadd2_rn(make_float2(__int_as_float((int)S[2 * c2] + kMagicBits),
+                                                            __int_as_float((int)S[2 * c2 + 1] + kMagicBits)), nm);
+                    acc[c2] = __ffma2_rn(f, make_float2(gv[2 * c2], gv[2 * c2 + 1]), acc[c2]);
+                }
             }
-        }
-        // ---------------- output: y = acc * sa, through a swizzled staging box, TMA store ----------------
-        const float sa = a.sa[m0 + row];
-        unsigned char* stage = reinterpret_cast<unsigned char*>(&sm.a[0][0]);  // operand ring is idle now
-        if (alive) {
+            // ---------------- output: y = acc * sa through the swizzled staging boxes, TMA store ----------------
+            if (threadIdx.x == 64) bulk_wait_read0();  // the previous tile's store has read the staging
+            named_sync(1, 32 * GEPI);
+            const float sa = a.sa[m0 + row];
 #pragma unroll
             for (int bb = 0; bb < HC / 32; ++bb)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int b = h * (HC / 32) + bb;  // 32-column box
                     const float2 p0 = acc[bb * 16 + 2 * j], p1 = acc[bb * 16 + 2 * j + 1];
-                    *reinterpret_cast<float4*>(stage + b * (GM * 128) + swz(row, j)) =
+                    *reinterpret_cast<float4*>(&sm.out[b][swz(row, j)]) =
                         make_float4(__fmul_rn(p0.x, sa), __fmul_rn(p0.y, sa), __fmul_rn(p1.x, sa), __fmul_rn(p1.y, sa));
                 }
-        }
-        fence_proxy_async();
-        named_sync(1, 32 * GEPI);
-        if (alive && threadIdx.x == 64) {
+            fence_proxy_async();
+            named_sync(1, 32 * GEPI);
+            if (threadIdx.x == 64 && alive) {
 #pragma unroll
-            for (int b = 0; b < GN / 32; ++b) tma_store_2d(&tY, n0 + b * 32, m0, stage + b * (GM * 128));
-            bulk_commit();
-            bulk_wait0();
+                for (int b = 0; b < GN / 32; ++b) tma_store_2d(&tY, n0 + b * 32, m0, &sm.out[b][0]);
+                bulk_commit();
+            }
         }
+        if (threadIdx.x == 64) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
@@ -280,7 +306,8 @@ extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M,
     if (!A || !sa || !V || !g || !Y || !ws) return HQ_ERR_ARG;
     if (group != GK) return HQ_ERR_UNSUPPORTED;
     if (M < GM || N < GN || K < GK || M % GM || N % GN || K % GK) return HQ_ERR_ARG;
-    if (K > GKMAX || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return HQ_ERR_UNSUPPORTED;
+    if (K > ((int64_t)1 << 20) || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return HQ_ERR_UNSUPPORTED;
+    if ((M / GM) * (N / GN) > ((int64_t)1 << 30)) return HQ_ERR_UNSUPPORTED;
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
     const uintptr_t al = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(V) |
                          reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(ws) |
@@ -301,7 +328,8 @@ extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M,
         attr_set = true;
     }
     GemmArgs a{M, N, K, sa, g, static_cast<WsHeader*>(ws)};
-    const dim3 grid((unsigned)(N / GN), (unsigned)(M / GM));
+    const int64_t tiles = (M / GM) * (N / GN);
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());  // persistent: one CTA per SM
     gemm_i8_grouped_kernel<<<grid, GTHREADS, smem, st>>>(a, ta, tb, ty);
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }

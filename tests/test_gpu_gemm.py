@@ -1,6 +1,7 @@
 """The int8 tensor-core GEMM over lattice codes (tcgen05) and the decode to int8 codes, on the
 GPU: bit-exact against the oracle's decode_int8 and grouped GEMM (exact group sums, binary32 fma
-over groups), at small shapes over several CTA tiles and, sampled, at 4096 x 4096 x 4096."""
+over groups), at small shapes over several CTA tiles, with more tiles than SMs (the persistent
+CTAs take several tiles each) and, sampled, at 4096 x 4096 x 4096."""
 import numpy as np
 import pytest
 import torch
@@ -52,7 +53,7 @@ def test_decode_int8_flags_codes_outside_int8(hq):
     assert torch.all(v[5] == 0) and torch.any(v[4] != 0)
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (256, 384, 1024), (384, 256, 2048)])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (256, 384, 1024), (384, 256, 2048), (2048, 1280, 256)])
 def test_gemm_int8_bit_exact(hq, M, N, K):
     w = W.llama_weight(N, K, seed=K + N)
     code = hq.encode(t_bf16(w), 128, hq.E8, 0.3, seed=5)
