@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define HQ_FORMAT_VERSION 1
+#define HQ_FORMAT_VERSION 2
 
 /* Lattices of Methodology step 2. */
 typedef enum { HQ_Z = 0, HQ_A2 = 1, HQ_D4 = 2, HQ_E8 = 3 } hq_lattice_t;
@@ -99,6 +99,8 @@ typedef struct {
  *   chunk_word  [C + 1] word offset of each chunk, [C] = total words
  *   bits        [cap_words] the bitstream; cap_words >= hq_encode_bound_words(...) always
  *               suffices, a smaller buffer yields HQ_ERR_CAPACITY with the needed size
+ *   kv_s0       KV: the position of the code's first token in every sequence (0 unless the
+ *               tokens were appended with hq_kv_encode_at)
  */
 typedef struct {
     int64_t rows, cols;
@@ -111,6 +113,7 @@ typedef struct {
     uint32_t* chunk_word;
     uint32_t* bits;
     int64_t cap_words;
+    int64_t kv_s0;
 } hq_code_t;
 
 /* Number of tiles T and chunks C of a rows x cols tensor with tile length n; -1 if invalid. */
@@ -166,6 +169,16 @@ hq_status_t hq_decode(const hq_code_t* code, void* y, hq_dtype_t dtype, void* ws
  */
 hq_status_t hq_kv_encode(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D,
                          const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Token append: encode kv[B, H, S, D] as the tokens s0 .. s0 + S - 1 of every (b, h) sequence, so
+ * the dither of token (b, h, s0 + s) is the one a whole-sequence encode would draw (for a decode
+ * step, S = 1: one head vector per (b, h)).  Each tile is coded on its own, so the tiles equal
+ * those of the whole-sequence code; the chunks (32 consecutive rows) follow this call's rows.
+ * out->kv_s0 = s0 >= 0.
+ */
+hq_status_t hq_kv_encode_at(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D, int64_t s0,
+                            const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Decode a KV tensor: the dither is regenerated and subtracted before the inverse transform. */
 hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void* ws, size_t ws_bytes,

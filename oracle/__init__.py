@@ -73,13 +73,13 @@ def lib():
         L.hqo_rice_tile.restype = i64
         L.hqo_parse_tile.argtypes = [P, i64, i32, i32, ctypes.c_uint16, P, P]
         L.hqo_parse_tile.restype = i32
-        L.hqo_encode.argtypes = [P, i32, i64, i64, i32, i32, f32, u64, i32, i64, P, P, P, P, i64, P, P, i64]
+        L.hqo_encode.argtypes = [P, i32, i64, i64, i32, i32, f32, u64, i32, i64, P, P, P, P, i64, P, P, i64, i64]
         L.hqo_encode.restype = ctypes.c_uint32
         L.hqo_quantize_coeffs.argtypes = [P, i64, i32, i32, i32, i64, u64, P, P, P, P, i64]
         L.hqo_quantize_coeffs.restype = ctypes.c_uint32
         L.hqo_parse.argtypes = [P, P, P, i64, i64, i32, i32, P]
         L.hqo_parse.restype = ctypes.c_uint32
-        L.hqo_decode.argtypes = [P, P, P, P, i64, i64, i32, i32, f32, u64, i32, i64, P, i64]
+        L.hqo_decode.argtypes = [P, P, P, P, i64, i64, i32, i32, f32, u64, i32, i64, P, i64, i64]
         L.hqo_decode.restype = ctypes.c_uint32
         _lib = L
     return _lib
@@ -239,9 +239,10 @@ class Code:
 
 
 def encode(x: np.ndarray, n: int, lattice: int, beta: float, seed: int, kv: bool = False, kv_S: int = 0,
-           want_codes: bool = False, row0: int = 0) -> Code:
+           want_codes: bool = False, row0: int = 0, kv_s0: int = 0) -> Code:
     """x: 2-D numpy array, dtype uint16 (bf16 bits) or float32.  row0: for KV, the global row of
-    x's first row when x is a slice of a larger [B*H*S, D] tensor."""
+    x's first row when x is a slice of a larger [B*H*S, D] tensor.  kv_s0: for KV, the position of
+    x's first token in every sequence (tokens appended at s0 .. s0 + kv_S - 1)."""
     assert x.ndim == 2
     if x.dtype == np.uint16:
         dtype = 0
@@ -262,12 +263,13 @@ def encode(x: np.ndarray, n: int, lattice: int, beta: float, seed: int, kv: bool
     u = np.zeros((T, n), dtype=np.float32) if want_codes else None
     st = lib().hqo_encode(_p(x), dtype, rows, cols, n, lattice, ctypes.c_float(beta), seed, int(kv), kv_S,
                           _p(scale), _p(meta), _p(cw), _p(bits), cap,
-                          _p(v) if v is not None else None, _p(u) if u is not None else None, row0)
+                          _p(v) if v is not None else None, _p(u) if u is not None else None, row0, kv_s0)
     if st & 2:
         raise ValueError("oracle rejected the arguments")
     c = Code(rows, cols, n, lattice, float(np.float32(beta)), seed, int(kv), kv_S, scale, meta, cw,
              bits[: int(cw[-1])].copy(), int(st), v, u)
     c.row0 = row0
+    c.kv_s0 = kv_s0
     return c
 
 
@@ -306,7 +308,7 @@ def decode(code: Code) -> tuple[np.ndarray, int]:
         bits = np.zeros(1, dtype=np.uint32)
     st = lib().hqo_decode(_p(code.scale), _p(code.meta), _p(code.chunk_word), _p(bits), code.rows, code.cols,
                           code.n, code.lattice, ctypes.c_float(code.beta), code.seed, code.kv, code.kv_S, _p(out),
-                          getattr(code, "row0", 0))
+                          getattr(code, "row0", 0), getattr(code, "kv_s0", 0))
     return out, int(st)
 
 

@@ -602,11 +602,13 @@ static int valid_common(int n, int lattice)
 /* kv: 0 no dither; 1 KV rows (b H + h, s) with the dither; 2 weights with the dither (option) */
 static int valid_kv(int kv, int lattice) { return (kv >= 0 && kv <= 2) && lattice >= 0 && lattice <= 3; }
 
-/* dither counter words of tile (row r of the call, tile column jt) */
-static void dither_words(int kv, int64_t r, int64_t kv_S, int64_t jt, int64_t* c1, int64_t* c)
+/* dither counter words of tile (row r of the call, tile column jt); KV rows of a call that
+ * starts at token s0 of every sequence (token append) are tokens s0 + r % kv_S */
+static void dither_words(int kv, int64_t r, int64_t kv_S, int64_t kv_s0, int64_t jt, int64_t* c1, int64_t* c)
 {
     if (kv == 1) {
         kv_row(r, kv_S, c1, c);
+        *c += kv_s0;
     } else {
         *c1 = jt;
         *c = r;
@@ -628,7 +630,7 @@ static void dither_words(int kv, int64_t r, int64_t kv_S, int64_t jt, int64_t* c
 uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n, int lattice, float beta,
                     uint64_t seed, int kv, int64_t kv_S, uint16_t* scale, uint16_t* meta,
                     uint32_t* chunk_word, uint32_t* bits, int64_t cap_words, int32_t* v_out,
-                    float* u_out, int64_t row0)
+                    float* u_out, int64_t row0, int64_t kv_s0)
 {
     if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || rows <= 0 || cols <= 0 || cols % n) return 1u << 1;
     uint32_t status = 0;
@@ -673,7 +675,7 @@ uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n,
                     for (int j = 0; j < n; ++j) u[j] = xt[j] * g;
                 }
                 int64_t c1 = 0, cw = 0;
-                if (kv) dither_words(kv, row0 + r, kv_S, jt, &c1, &cw);
+                if (kv) dither_words(kv, row0 + r, kv_S, kv_s0, jt, &c1, &cw);
                 int32_t v[HQO_MAXN];
                 quantize_tile(u, n, lattice, kv != 0, seed, c1, cw, v);
                 int k, sumq;
@@ -710,7 +712,7 @@ uint32_t hqo_quantize_coeffs(const float* u, int64_t tiles, int n, int lattice, 
         int64_t t_end = (c + 1) * 32 < tiles ? (c + 1) * 32 : tiles;
         for (int64_t t = c * 32; t < t_end; ++t) {
             int64_t c1 = 0, cw = 0;
-            if (kv) dither_words(kv, t, kv_S, 0, &c1, &cw);
+            if (kv) dither_words(kv, t, kv_S, 0, 0, &c1, &cw);
             int32_t v[HQO_MAXN];
             quantize_tile(u + t * n, n, lattice, kv != 0, seed, c1, cw, v);
             int k, sumq;
@@ -816,7 +818,7 @@ static void reconstruct_tile(const int32_t* v, int n, int lattice, int dither, u
 /* Full decode to binary64 out[rows, cols].  Returns status bits. */
 uint32_t hqo_decode(const uint16_t* scale, const uint16_t* meta, const uint32_t* chunk_word, const uint32_t* bits,
                     int64_t rows, int64_t cols, int n, int lattice, float beta, uint64_t seed, int kv,
-                    int64_t kv_S, double* out, int64_t row0)
+                    int64_t kv_S, double* out, int64_t row0, int64_t kv_s0)
 {
     if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || rows <= 0 || cols % n) return 1u << 1;
     const int64_t NT = cols / n;
@@ -827,7 +829,7 @@ uint32_t hqo_decode(const uint16_t* scale, const uint16_t* meta, const uint32_t*
         for (int64_t r = 0; r < rows; ++r) {
             int64_t t = jt * rows + r;
             int64_t c1 = 0, cw = 0;
-            if (kv) dither_words(kv, row0 + r, kv_S, jt, &c1, &cw);
+            if (kv) dither_words(kv, row0 + r, kv_S, kv_s0, jt, &c1, &cw);
             double tile[HQO_MAXN];
             reconstruct_tile(v + t * n, n, lattice, kv != 0, seed, c1, cw, scale[t], beta, jt * n, tile);
             memcpy(out + r * cols + jt * n, tile, sizeof(double) * (size_t)n);

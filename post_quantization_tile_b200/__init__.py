@@ -40,7 +40,7 @@ class CodeStruct(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("kv_S", ctypes.c_int64), ("p", Params),
                 ("kv", ctypes.c_int32), ("version", ctypes.c_int32), ("scale", ctypes.c_void_p),
                 ("meta", ctypes.c_void_p), ("chunk_word", ctypes.c_void_p), ("bits", ctypes.c_void_p),
-                ("cap_words", ctypes.c_int64)]
+                ("cap_words", ctypes.c_int64), ("kv_s0", ctypes.c_int64)]
 
 
 _lib = None
@@ -72,6 +72,8 @@ def lib():
         L.hq_kv_encode.argtypes = [P, i32, i64, i64, i64, i64, ctypes.POINTER(Params), ctypes.POINTER(CodeStruct), P,
                                    ctypes.c_size_t, P]
         L.hq_kv_decode.argtypes = [ctypes.POINTER(CodeStruct), P, i32, P, ctypes.c_size_t, P]
+        L.hq_kv_encode_at.argtypes = [P, i32, i64, i64, i64, i64, i64, ctypes.POINTER(Params),
+                                      ctypes.POINTER(CodeStruct), P, ctypes.c_size_t, P]
         L.hq_quantize_coeffs.argtypes = [P, i64, ctypes.POINTER(Params), i32, i64, P, ctypes.POINTER(CodeStruct), P,
                                          ctypes.c_size_t, P]
         L.hq_encode_count.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, P, P, ctypes.c_size_t, P]
@@ -83,7 +85,7 @@ def lib():
         L.hq_status_str.argtypes = [i32]
         L.hq_status_str.restype = ctypes.c_char_p
         L.hq_version.restype = i32
-        for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_decode", "hq_quantize_coeffs",
+        for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_encode_at", "hq_kv_decode", "hq_quantize_coeffs",
                   "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_status_read"]:
             getattr(L, f).restype = i32
         _lib = L
@@ -163,7 +165,7 @@ class Code:
     def struct(self) -> CodeStruct:
         return CodeStruct(self.rows, self.cols, self.kv_S, self.p, self.kv, lib().hq_version(),
                           self.scale.data_ptr(), self.meta.data_ptr(), self.chunk_word.data_ptr(),
-                          self.bits.data_ptr(), self.bits.numel())
+                          self.bits.data_ptr(), self.bits.numel(), getattr(self, "kv_s0", 0))
 
     @property
     def step(self) -> float:
@@ -204,6 +206,7 @@ def alloc_code(rows: int, cols: int, p: Params, device=None, cap_words: int | No
 
 def _fill(code: Code, cs: CodeStruct):
     code.rows, code.cols, code.kv_S, code.kv = cs.rows, cs.cols, cs.kv_S, cs.kv
+    code.kv_s0 = cs.kv_s0
     code.p = Params(cs.p.tile, cs.p.lattice, cs.p.step, cs.p.bps, cs.p.seed)
 
 
@@ -244,8 +247,9 @@ def decode(code: Code, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | 
 
 
 def kv_encode(kv: torch.Tensor, step: float = 0.0, bps: float = 4.0, seed: int = 0, lattice: int | str = D4,
-              out: Code | None = None, ws: Workspace | None = None) -> Code:
-    """Encode a KV tensor [B, H, S, D] with the dither (Methodology step 4; D4 by default, any lattice)."""
+              out: Code | None = None, ws: Workspace | None = None, s0: int = 0) -> Code:
+    """Encode a KV tensor [B, H, S, D] with the dither (Methodology step 4; D4 by default, any
+    lattice).  s0 > 0: the tokens are positions s0 .. s0 + S - 1 of every sequence (token append)."""
     _require_cuda(kv, "kv")
     if kv.dim() != 4:
         raise ValueError("kv must be [B, H, S, D]")
@@ -256,8 +260,12 @@ def kv_encode(kv: torch.Tensor, step: float = 0.0, bps: float = 4.0, seed: int =
     L = lib()
     w = ws or workspace(L.hq_workspace_bytes(rows, D, ctypes.byref(p)))
     cs = code.struct()
-    _check(L.hq_kv_encode(_ptr(kv), _dtype_code(kv), B, H, S, D, ctypes.byref(p), ctypes.byref(cs), w.ptr(), w.nbytes,
-                          _stream()), "hq_kv_encode")
+    if s0:
+        _check(L.hq_kv_encode_at(_ptr(kv), _dtype_code(kv), B, H, S, D, int(s0), ctypes.byref(p), ctypes.byref(cs),
+                                 w.ptr(), w.nbytes, _stream()), "hq_kv_encode_at")
+    else:
+        _check(L.hq_kv_encode(_ptr(kv), _dtype_code(kv), B, H, S, D, ctypes.byref(p), ctypes.byref(cs), w.ptr(),
+                              w.nbytes, _stream()), "hq_kv_encode")
     _fill(code, cs)
     code.ws = w
     return code

@@ -217,12 +217,14 @@ hq_status_t plan_encode(const void* x, int src, int64_t rows, int64_t cols, cons
 // common body of the encode entry points
 hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, const hq_params_t* p, int32_t kv,
                           int64_t kv_S, int32_t* v_out, hq_code_t* out, unsigned long long* count_out, void* ws,
-                          size_t ws_bytes, void* stream)
+                          size_t ws_bytes, void* stream, int64_t kv_s0 = 0)
 {
     const bool count = count_out != nullptr;
+    if (kv_s0 < 0 || (kv_s0 && kv != 1)) return HQ_ERR_ARG;
     EncodePlan pl;
     const hq_status_t ps = plan_encode(x, src, rows, cols, p, kv, kv_S, v_out, out, count, ws, ws_bytes, pl);
     if (ps != HQ_OK) return ps;
+    pl.a.kv_s0 = kv_s0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t clear = count ? sizeof(WsHeader) : sizeof(WsHeader) + (size_t)pl.g.items * 8u;
     cudaError_t e = cudaMemsetAsync(ws, 0, clear, st);
@@ -238,6 +240,7 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
         out->kv_S = kv == 1 ? kv_S : 0;
         out->p = pl.prm;
         out->kv = kv;
+        out->kv_s0 = kv == 1 ? kv_s0 : 0;
         out->version = HQ_FORMAT_VERSION;
     }
     return HQ_OK;
@@ -406,6 +409,8 @@ hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, f
     a.seed = prm.seed;
     hq::philox_round_keys(prm.seed, a.rk);
     a.kv_S = code->kv == 1 ? code->kv_S : 0;
+    a.kv_s0 = code->kv == 1 ? code->kv_s0 : 0;
+    if (a.kv_s0 < 0) return HQ_ERR_ARG;
     a.items = g.items;
     a.IB = g.IB;
     a.RB = g.RB;
@@ -508,6 +513,16 @@ hq_status_t hq_kv_encode(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H,
     if (B * H > ((int64_t)1 << 32)) return HQ_ERR_ARG;
     return encode_common(kv, dtype == HQ_BF16 ? 0 : 1, B * H * S, D, p, 1, S, nullptr, out, nullptr, ws, ws_bytes,
                          stream);
+}
+
+hq_status_t hq_kv_encode_at(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D, int64_t s0,
+                            const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (B < 1 || H < 1 || S < 1 || s0 < 0 || !p || D != p->tile) return HQ_ERR_ARG;
+    if (B * H > ((int64_t)1 << 32)) return HQ_ERR_ARG;
+    return encode_common(kv, dtype == HQ_BF16 ? 0 : 1, B * H * S, D, p, 1, S, nullptr, out, nullptr, ws, ws_bytes,
+                         stream, s0);
 }
 
 hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream)

@@ -28,6 +28,7 @@ struct DecodeArgs {
     WsHeader* ws;
     uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
     float* g_out;     // int8-code output: group scale of tile (r, jt) at g_out[jt rows + r]
+    int64_t kv_s0;    // KV: position of the code's first token in every sequence
 };
 
 template <int N, int DST>  // DST: 0 bf16, 1 fp32, 2 int8 lattice codes (RHT domain, no transform)
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 // (minus 2U), (P, Q) for A2 (then scaled to u), u for Z and D4
                 const int64_t r = r0 + row_l;
                 const uint64_t Sv = (uint64_t)a.kv_S;
-                const uint64_t dc = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+                const uint64_t dc = Sv ? (uint64_t)r % Sv + (uint64_t)a.kv_s0 : (uint64_t)r;
                 const uint32_t dc1 = Sv ? (uint32_t)((uint64_t)r / Sv) : (uint32_t)jt;
                 if constexpr (LAT == HQ_E8) {
     #pragma unroll

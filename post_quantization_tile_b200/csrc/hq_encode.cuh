@@ -32,6 +32,7 @@ struct EncodeArgs {
     unsigned long long* states;
     uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
     const RateSearch* search;  // count-only passes of a step search: the step comes from here
+    int64_t kv_s0;             // KV: position of the call's first token in every sequence
 };
 
 // SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
         if constexpr (KV) {
             const int64_t r = r0 + row_l;
             const uint64_t Sv = (uint64_t)a.kv_S;
-            dc = Sv ? (uint64_t)r % Sv : (uint64_t)r;
+            dc = Sv ? (uint64_t)r % Sv + (uint64_t)a.kv_s0 : (uint64_t)r;
             dc1 = Sv ? (uint32_t)((uint64_t)r / Sv) : (uint32_t)jt;
         }
 

@@ -45,7 +45,7 @@ def test_host_only_entry_points(libhq):
     b = L.hq_encode_bound_words(4096, 4096, ctypes.byref(p))
     assert b % 4 == 0 and b >= 4096 * 32 * (16 * 128 + 2 * 128) // 32
     assert L.hq_workspace_bytes(4096, 4096, ctypes.byref(p)) % 256 == 0
-    assert L.hq_version() == 1
+    assert L.hq_version() == 2
     assert L.hq_status_str(3) == b"bitstream buffer too small"
     # high-resolution step: E8 at 4 bps ~ 2^(2.047 - 4)
     assert abs(L.hq_step_for_rate(hq.E8, 128, 4.0) - 2 ** (0.5 * __import__("math").log2(2 * 3.141592653589793 * 2.718281828459045) - 4)) < 1e-6

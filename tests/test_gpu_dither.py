@@ -83,3 +83,19 @@ def test_gpu_dither_unbiased_and_cell_moment(hq, lattice):
     mse_u = (((y - x) ** 2).sum(1) / (128 * (sh * beta) ** 2)).mean().item()
     moment = {oracle.Z: 1 / 12, oracle.A2: 5 / 72, oracle.E8: 929 / 12960}[lattice]
     assert abs(mse_u / moment - 1.0) < 0.02
+
+
+@pytest.mark.parametrize("lattice", [oracle.D4, oracle.E8])
+def test_token_append_matches_whole_sequence_and_oracle(hq, lattice):
+    B, H, S, D = 2, 4, 48, 128
+    kb = W.kv_keys(B, H, S, D, seed=21)
+    full = hq.kv_encode(t_bf16(kb), step=0.8, seed=9, lattice=lattice)
+    yf = hq.kv_decode(full, (B, H, S, D), dtype=torch.float32)
+    for s0 in (1, 33, 47):
+        step = np.ascontiguousarray(kb[:, :, s0:s0 + 1, :])               # [B, H, 1, D]
+        app = hq.kv_encode(t_bf16(step), step=0.8, seed=9, lattice=lattice, s0=s0)
+        assert hq.status(app.ws)[0] == 0 and app.kv_s0 == s0
+        ya = hq.kv_decode(app, (B, H, 1, D), dtype=torch.float32)
+        assert torch.equal(ya[:, :, 0], yf[:, :, s0])
+        ref = oracle.encode(step.reshape(-1, D), D, lattice, 0.8, 9, kv=True, kv_S=1, kv_s0=s0)
+        assert_same_code(app, ref, "append")

@@ -98,3 +98,21 @@ def test_dithered_reconstruction_is_unbiased_per_vector(lattice):
 def test_d4_group_dither_is_the_kv_block_dither():
     for g in range(8):
         assert np.array_equal(oracle.dither(oracle.D4, 7, 5, 99, 32)[4 * g:4 * g + 4], oracle.dither_d4(7, 5, 99, g))
+
+
+def test_token_append_tiles_equal_the_whole_sequence_tiles():
+    # appending token s0 of every (b, h) draws the dither a whole-sequence encode draws for it:
+    # tile for tile, the codes and reconstructions agree (Methodology step 4, fresh U per vector)
+    from post_quantization_tile_b200 import workloads as W
+    B, H, S, D = 1, 3, 40, 128
+    kb = W.kv_keys(B, H, S, D, seed=12)
+    full = oracle.encode(kb.reshape(-1, D), D, oracle.D4, 0.9, 5, kv=True, kv_S=S, want_codes=True)
+    xf, _ = oracle.decode(full)
+    for s0 in (0, 7, 39):
+        step = np.ascontiguousarray(kb[:, :, s0, :].reshape(-1, D))        # [B*H, D]: one token per head
+        app = oracle.encode(step, D, oracle.D4, 0.9, 5, kv=True, kv_S=1, want_codes=True, kv_s0=s0)
+        rows = np.arange(B * H) * S + s0
+        np.testing.assert_array_equal(app.v, full.v[rows])
+        np.testing.assert_array_equal(app.meta, full.meta[rows])
+        xa, _ = oracle.decode(app)
+        np.testing.assert_array_equal(xa, xf[rows])

@@ -47,7 +47,7 @@ def test_noalloc_encode_matches_regular_encode_twice():
         assert rc == 0, f"call {call}: status {rc}"
         torch.cuda.synchronize()
         assert int(status.item()) == 0, f"call {call}: device status bits {int(status.item()):#x}"
-        assert cs.version == 1 and cs.rows == rows and cs.cols == cols and abs(cs.p.step - beta) < 1e-7
+        assert cs.version == 2 and cs.rows == rows and cs.cols == cols and abs(cs.p.step - beta) < 1e-7
         assert torch.equal(out.chunk_word, ref.chunk_word)
         assert torch.equal(out.meta, ref.meta)
         assert torch.equal(out.scale, ref.scale)
