@@ -94,7 +94,8 @@ def kernel_sources_hash() -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "post_quantization_tile_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.cu"))):
+    # the encode / decode kernels' sources (the GEMM and the host API do not change them)
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "hq_inst_*.cu"))):
         with open(f, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
