@@ -120,6 +120,22 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&v)[3
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// bounded wait that lets the hardware suspend the warp (up to about a microsecond per try)
+// instead of spinning: sixteen epilogue warps wait on the same slot barriers
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity)
+{
+    for (uint32_t i = 0; i < (1u << 20); ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(1000u)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
 __device__ __forceinline__ void named_sync(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -162,7 +178,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                 const int m0 = (tile / NT) * GM, n0 = (tile % NT) * GN;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % GSTAGES;
-                    if (it >= GSTAGES && !mbar_wait(&sm.empty[s], (uint32_t)((it / GSTAGES - 1) & 1))) {
+                    if (it >= GSTAGES && !mbar_wait_sleep(&sm.empty[s], (uint32_t)((it / GSTAGES - 1) & 1))) {
                         status_set(a.ws, kStTimeout);
                         alive = false;
                         break;
@@ -183,12 +199,12 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             for (int tile = blockIdx.x; alive && tile < tiles; tile += gridDim.x) {
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % GSTAGES, slot = it % GACC;
-                    if (it >= GACC && !mbar_wait(&sm.acc_empty[slot], (uint32_t)((it / GACC - 1) & 1))) {
+                    if (it >= GACC && !mbar_wait_sleep(&sm.acc_empty[slot], (uint32_t)((it / GACC - 1) & 1))) {
                         status_set(a.ws, kStTimeout);
                         alive = false;
                         break;
                     }
-                    if (!mbar_wait(&sm.full[s], (uint32_t)((it / GSTAGES) & 1))) {
+                    if (!mbar_wait_sleep(&sm.full[s], (uint32_t)((it / GSTAGES) & 1))) {
                         status_set(a.ws, kStTimeout);
                         alive = false;
                         break;
@@ -227,7 +243,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             for (int kb = 0; kb < KB; ++kb, ++it) {
                 if (!alive) continue;
                 const int slot = it % GACC, s = it % GSTAGES;
-                const bool got = mbar_wait(&sm.acc_full[slot], (uint32_t)((it / GACC) & 1));
+                const bool got = mbar_wait_sleep(&sm.acc_full[slot], (uint32_t)((it / GACC) & 1));
                 __syncwarp();  // the warp-wide TMEM loads below need the whole warp converged
                 if (!__all_sync(0xffffffffu, got)) {
                     if (lane == 0) status_set(a.ws, kStTimeout);
