@@ -336,13 +336,10 @@ extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
     const size_t smem = sizeof(GemmSmem) + 1024;
-    static bool attr_set = false;  // per process; the attribute is per function and device-independent
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(gemm_i8_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return HQ_ERR_CUDA;
-        attr_set = true;
-    }
+    // set on every call: the attribute belongs to the current device's context
+    if (cudaFuncSetAttribute(gemm_i8_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return HQ_ERR_CUDA;
     GemmArgs a{M, N, K, sa, g, static_cast<WsHeader*>(ws)};
     const int64_t tiles = (M / GM) * (N / GN);
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());  // persistent: one CTA per SM
