@@ -113,6 +113,27 @@ def measured_traffic(kind: str, scalars: int):
     return d[kind]["bytes_per_scalar"] * scalars
 
 
+def instruction_check():
+    """Issue slots per scalar (warp instructions x 32 / scalars) of the encode and decode kernels
+    from the committed ncu captures, if the kernels are unchanged: the secondary roof of a codec
+    that is bound by instruction issue rather than HBM."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_sources_sha256_16") != kernel_sources_hash():
+        return None
+    try:
+        return {"encode_slots_per_scalar": d["encode"]["slots_per_scalar"],
+                "decode_slots_per_scalar": d["decode"]["slots_per_scalar"],
+                "encode_issue_active": d["encode"]["issue_active"], "decode_issue_active": d["decode"]["issue_active"],
+                "slots_per_scalar_at_60pct_hbm": d["slots_per_scalar_at_60pct_hbm"],
+                "source": "profiles/roofline_traffic.json"}
+    except KeyError:
+        return None
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -360,6 +381,7 @@ def run_gpu(args):
             "gpu_launches": 4 * args.steps,
             "kv_cache": kv,
             "gemm_int8": gemm,
+            "instruction_roof": instruction_check(),
             "clocks": clk.summary(),
             "status": st,
         }
