@@ -358,7 +358,11 @@ struct BitReader {
     int avail;
     int wi;
     int lim;  // last readable word index; reads are clamped to [0, lim]
+    int c0;   // consumed() = 32 wi - avail - c0 (forward), c0 - 32 wi - avail (backward)
     const uint32_t* src;
+
+    // bits taken from the stream since begin()
+    __device__ __forceinline__ int consumed() const { return FWD ? 32 * wi - avail - c0 : c0 - 32 * wi - avail; }
 
     __device__ __forceinline__ uint32_t load()
     {
@@ -372,6 +376,7 @@ struct BitReader {
         lim = last_word;
         wi = start_or_end_bit >> 5;
         const int skip = FWD ? (start_or_end_bit & 31) : (31 - (start_or_end_bit & 31));
+        c0 = FWD ? 32 * wi + skip : 32 * wi - skip;
         const uint32_t w0 = load();
         const uint32_t w1 = load();
         W = (((unsigned long long)w0 << 32) | w1) << skip;
@@ -407,12 +412,11 @@ __device__ __forceinline__ uint32_t long_run(BitReader<FWD>& br, uint32_t limit,
     return q;
 }
 
-// one Rice code: q zeros, a one, r (k bits MSB-first); returns the zig-zag value q << k | r and
-// adds q to sq.  The caller tops the window up to at least 33 bits every four codes;
+// one Rice code: q zeros, a one, r (k bits MSB-first); returns the zig-zag value q << k | r (the
+// sum of q follows from the bits consumed: consumed() - codes (k + 1)).  The caller tops the window up to at least 33 bits every four codes;
 // a code that is longer than the bits at hand takes the slow path (refill, long runs).
 template <bool FWD>
-__device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t pow2k, uint32_t limit, bool& ok,
-                                             uint32_t& sq)
+__device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t pow2k, uint32_t limit, bool& ok)
 {
     uint32_t hi = (uint32_t)(br.W >> 32);
     int z = __clz(hi);
@@ -434,14 +438,12 @@ __device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t
         br.W <<= k;
         br.avail -= k;
         q += (uint32_t)z;
-        sq += q;
         return (q << k) | r;
     }
     // fast path: the whole code is in the top 32 bits: 0..0 1 r
     const uint32_t val = hi >> (32 - lam);      // (1 << k) | r
     br.W <<= lam;
     br.avail -= lam;
-    sq += (uint32_t)z;
     return (uint32_t)z * pow2k + (val - pow2k);  // (z << k) | r
 }
 

@@ -216,7 +216,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 BitReader<false> rb;
                 rf.begin(in, tile0 + COSB, G::IN_WORDS - 1);
                 rb.begin(in, tile0 + (int)L - 1, G::IN_WORDS - 1);
-                uint32_t sqb = 0;
 #pragma unroll 1
                 for (int g = 0; g < N / 16; ++g) {
                     uint32_t zf[8], zb[8];
@@ -226,15 +225,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                             rf.refill();
                             rb.refill();
                         }
-                        zf[j] = get_code<true>(rf, k, pow2k, sq_meta, ok, sq);
-                        zb[7 - j] = get_code<false>(rb, k, pow2k, sq_meta, ok, sqb);
+                        zf[j] = get_code<true>(rf, k, pow2k, sq_meta, ok);
+                        zb[7 - j] = get_code<false>(rb, k, pow2k, sq_meta, ok);
                     }
                     *zz_slot(sm.buf, g, tid) = make_uint4(zf[0] | (zf[1] << 16), zf[2] | (zf[3] << 16),
                                                           zf[4] | (zf[5] << 16), zf[6] | (zf[7] << 16));
                     *zz_slot(sm.buf, V / 8 - 1 - g, tid) = make_uint4(zb[0] | (zb[1] << 16), zb[2] | (zb[3] << 16),
                                                                       zb[4] | (zb[5] << 16), zb[6] | (zb[7] << 16));
                 }
-                sq += sqb;
+                // the codes' unary parts: the bits taken minus one stop bit and k remainder bits per code
+                sq = (uint32_t)(rf.consumed() + rb.consumed() - N * (k + 1));
             } else if (tau == 0) {
                 BitReader<true> br;
                 br.begin(in, tile0 + COSB, G::IN_WORDS - 1);
@@ -245,11 +245,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         if ((j & 3) == 0) br.refill();
-                        z[j] = get_code<true>(br, k, pow2k, sq_meta, ok, sq);
+                        z[j] = get_code<true>(br, k, pow2k, sq_meta, ok);
                     }
                     *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
                                                           z[4] | (z[5] << 16), z[6] | (z[7] << 16));
                 }
+                sq = (uint32_t)(br.consumed() - V * (k + 1));
             }
             else {
                 BitReader<false> br;
@@ -261,11 +262,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
 #pragma unroll
                     for (int j = 7; j >= 0; --j) {
                         if ((j & 3) == 3) br.refill();
-                        z[j] = get_code<false>(br, k, pow2k, sq_meta, ok, sq);
+                        z[j] = get_code<false>(br, k, pow2k, sq_meta, ok);
                     }
                     *zz_slot(sm.buf, g, tid) = make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16),
                                                           z[4] | (z[5] << 16), z[6] | (z[7] << 16));
                 }
+                sq = (uint32_t)(br.consumed() - V * (k + 1));
             }
             sq_part = sq;
         }
@@ -288,22 +290,44 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
             for (int g8 = 0; g8 < H / 8; ++g8) {
                 const uint4 w = *zz_slot(sm.buf, half * (H / 8) + g8, tid);
                 const uint32_t zw[4] = {w.x, w.y, w.z, w.w};
-                int32_t sym[8];
+                if constexpr (LAT == HQ_E8 && DST != 2) {
+                    // zig-zag -> doubled E8 point in one pass: 2 unzigzag(z) = z ^ -(z & 1), so
+                    // v_i = 2 w_i + c = (z_i ^ -(z_i & 1)) + c for i < 7, the parity p of w_0 .. w_6
+                    // is bit 1 of the XOR of those, and v_7 = 2 (2 h + p) + c; the binary32 value
+                    // comes from adding 1.5 * 2^23 in the integer domain (exact, |v| < 2^22)
+                    const int cm = (int)((cosbits >> (half * (H / 8) + g8)) & 1u) + __float_as_int(kMagic);
+                    int t[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) sym[j] = unzigzag((zw[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);  // !ok: zeroed below
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t z = (zw[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+                        t[j] = (int)(z ^ (0u - (z & 1u)));
+                    }
+                    const int p2 = (t[0] ^ t[1] ^ t[2] ^ t[3] ^ t[4] ^ t[5] ^ t[6]) & 2;  // 2 p
 #pragma unroll
-                for (int b = 0; b < 8 / D; ++b) {
-                    const int pos = half * H + g8 * 8 + b * D;
-                    int32_t v[D];
-                    unstrip_block<LAT>(sym + b * D, (cosbits >> (pos / 8)) & 1u, v);
+                    for (int i = 0; i < 8; ++i) {
+                        const int vb = i < 7 ? t[i] + cm : 2 * t[7] + p2 + cm;
+                        const float f = __int_as_float(vb) - kMagic;  // !ok: zeroed below
+                        if (half) P[g8 * 8 + i].y = f;
+                        else P[g8 * 8 + i].x = f;
+                    }
+                } else {
+                    int32_t sym[8];
 #pragma unroll
-                    for (int i = 0; i < D; ++i) {
-                        if constexpr (DST == 2) out_of_int8 |= (uint32_t)(v[i] + 127) > 254u ? 1u : 0u;
-                        float f = __int_as_float(v[i] + __float_as_int(kMagic)) - kMagic;  // exact, |v| < 2^22
-                        // A2: (P, Q) -> u after the dither is taken off (in P, Q coordinates)
-                        if constexpr (LAT == HQ_A2 && !KV) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
-                        if (half) P[g8 * 8 + b * D + i].y = f;
-                        else P[g8 * 8 + b * D + i].x = f;
+                    for (int j = 0; j < 8; ++j) sym[j] = unzigzag((zw[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);  // !ok: zeroed below
+#pragma unroll
+                    for (int b = 0; b < 8 / D; ++b) {
+                        const int pos = half * H + g8 * 8 + b * D;
+                        int32_t v[D];
+                        unstrip_block<LAT>(sym + b * D, (cosbits >> (pos / 8)) & 1u, v);
+#pragma unroll
+                        for (int i = 0; i < D; ++i) {
+                            if constexpr (DST == 2) out_of_int8 |= (uint32_t)(v[i] + 127) > 254u ? 1u : 0u;
+                            float f = __int_as_float(v[i] + __float_as_int(kMagic)) - kMagic;  // exact, |v| < 2^22
+                            // A2: (P, Q) -> u after the dither is taken off (in P, Q coordinates)
+                            if constexpr (LAT == HQ_A2 && !KV) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
+                            if (half) P[g8 * 8 + b * D + i].y = f;
+                            else P[g8 * 8 + b * D + i].x = f;
+                        }
                     }
                 }
             }
