@@ -27,6 +27,10 @@
 #ifndef HQ_GEMM_EPI_WARPS
 #define HQ_GEMM_EPI_WARPS 16
 #endif
+#ifndef HQ_GEMM_N
+#define HQ_GEMM_N 128  // output columns per CTA tile: 128, or 256 (measured slower: the 64 accumulators
+                       // per epilogue thread exceed the register budget of 576 threads)
+#endif
 
 namespace hq {
 namespace {
@@ -34,16 +38,17 @@ namespace {
 constexpr float kMagicGemm = 12582912.0f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
-constexpr int GM = 128, GN = 128, GK = 128;  // CTA tile (M, N) and K group
-constexpr int GSTAGES = 4;                   // operand ring
-constexpr int GACC = 4;                      // TMEM accumulator slots of GN columns
+constexpr int GM = 128, GN = HQ_GEMM_N, GK = 128;  // CTA tile (M, N) and K group
+constexpr int GSTAGES = GN == 128 ? 4 : 3;         // operand ring
+constexpr int GACC = 512 / GN;                     // TMEM accumulator slots of GN columns (all 512)
+constexpr int GOUT = 128;                          // columns staged per output store
 constexpr int GEPI = HQ_GEMM_EPI_WARPS;      // epilogue warps: GEPI / 4 warpgroups, GN / (GEPI / 4) columns each
 constexpr int GTHREADS = 64 + 32 * GEPI;
 
 struct GemmSmem {
     alignas(1024) int8_t a[GSTAGES][GM * GK];
     alignas(1024) int8_t b[GSTAGES][GN * GK];
-    alignas(1024) unsigned char out[GN / 32][GM * 128];  // output staging: 32-column boxes
+    alignas(1024) unsigned char out[GOUT / 32][GM * 128];  // output staging: 32-column boxes
     alignas(16) float g[GSTAGES][GN];                     // the group's scales, loaded with the operands
     alignas(8) uint64_t full[GSTAGES];
     uint64_t empty[GSTAGES];
@@ -149,7 +154,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = (int)(a.K / GK);
-    const int NT = (int)(a.N / GN);
+    const int NT = (int)((a.N + GN - 1) / GN);  // a last tile of 128 columns when N % GN = 128
     const int tiles = (int)(a.M / GM) * NT;  // persistent: tiles blockIdx.x, + gridDim.x, ...
 
     if (threadIdx.x == 0) {
@@ -183,10 +188,13 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                         alive = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(GM * GK + GN * GK + GN * 4));
+                    // rows of V past N read as zeros (TMA fill); the scales of those columns stay unset
+                    // and their results are clipped by the TMA store
+                    const uint32_t gbytes = (uint32_t)(a.N - n0 < GN ? a.N - n0 : GN) * 4u;
+                    mbar_arrive_expect_tx(&sm.full[s], (uint32_t)(GM * GK + GN * GK) + gbytes);
                     tma_load_2d(sm.a[s], &tA, kb * GK, m0, &sm.full[s]);
                     tma_load_2d(sm.b[s], &tB, kb * GK, n0, &sm.full[s]);
-                    bulk_load_1d(sm.g[s], a.g + (int64_t)kb * a.N + n0, GN * 4, &sm.full[s]);
+                    bulk_load_1d(sm.g[s], a.g + (int64_t)kb * a.N + n0, gbytes, &sm.full[s]);
                 }
             }
         }
@@ -251,55 +259,61 @@ __global__ void __launch_bounds__(GTHREADS, 1)
                     continue;
                 }
                 tc_fence_after();
-                uint32_t S[HC];
-                const uint32_t ta = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + h * HC);
+                // 32 columns at a time: load, then scale with the group's scales read from the stage
 #pragma unroll
-                for (int c = 0; c < HC / 32; ++c)
-                    tmem_ld32_nowait(ta + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&S[32 * c]));
-                float gv[HC];
+                for (int c = 0; c < HC / 32; ++c) {
+                    uint32_t S[32];
+                    const uint32_t ta = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * GN + h * HC + 32 * c);
+                    tmem_ld32_nowait(ta, S);
+                    tmem_wait_ld();
+                    if (c == HC / 32 - 1) {  // the slot is read: release it before the arithmetic
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.acc_empty[slot]);
+                    }
+                    const float4* gp = reinterpret_cast<const float4*>(&sm.g[s][h * HC + 32 * c]);
 #pragma unroll
-                for (int c4 = 0; c4 < HC / 4; ++c4) {
-                    const float4 g4 = reinterpret_cast<const float4*>(&sm.g[s][h * HC])[c4];
-                    gv[4 * c4] = g4.x;
-                    gv[4 * c4 + 1] = g4.y;
-                    gv[4 * c4 + 2] = g4.z;
-                    gv[4 * c4 + 3] = g4.w;
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 g4 = gp[c4];
+                        // |S| < 2^22: adding 1.5 * 2^23 in the integer domain gives an exact float
+                        const float2 f0 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4] + kMagicBits),
+                                                                 __int_as_float((int)S[4 * c4 + 1] + kMagicBits)), nm);
+                        const float2 f1 = __fadd2_rn(make_float2(__int_as_float((int)S[4 * c4 + 2] + kMagicBits),
+                                                                 __int_as_float((int)S[4 * c4 + 3] + kMagicBits)), nm);
+                        acc[16 * c + 2 * c4] = __ffma2_rn(f0, make_float2(g4.x, g4.y), acc[16 * c + 2 * c4]);
+                        acc[16 * c + 2 * c4 + 1] = __ffma2_rn(f1, make_float2(g4.z, g4.w), acc[16 * c + 2 * c4 + 1]);
+                    }
                 }
-                tmem_wait_ld();
-                // slot and scales are read: release both before the arithmetic
-                tc_fence_before();
+                // the stage's scales are read
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&sm.acc_empty[slot]);
-                    mbar_arrive(&sm.empty[s]);
-                }
-#pragma unroll
-                for (int c2 = 0; c2 < HC / 2; ++c2) {
-                    // |S| < 2^22: adding 1.5 * 2^23 in the integer domain gives an exact float
-                    const float2 f = __fadd2_rn(make_float2(__int_as_float((int)S[2 * c2] + kMagicBits),
-                                                            __int_as_float((int)S[2 * c2 + 1] + kMagicBits)), nm);
-                    acc[c2] = __ffma2_rn(f, make_float2(gv[2 * c2], gv[2 * c2 + 1]), acc[c2]);
-                }
+                if (lane == 0) mbar_arrive(&sm.empty[s]);
             }
             // ---------------- output: y = acc * sa through the swizzled staging boxes, TMA store ----------------
-            if (threadIdx.x == 64) bulk_wait_read0();  // the previous tile's store has read the staging
-            named_sync(1, 32 * GEPI);
+            // GOUT columns at a time; warpgroup h's columns HC h .. belong to part HC h / GOUT
             const float sa = a.sa[m0 + row];
 #pragma unroll
-            for (int bb = 0; bb < HC / 32; ++bb)
+            for (int part = 0; part < GN / GOUT; ++part) {
+                if (threadIdx.x == 64) bulk_wait_read0();  // the previous store has read the staging
+                named_sync(1, 32 * GEPI);
+                if ((h * HC) / GOUT == part) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int b = h * (HC / 32) + bb;  // 32-column box
-                    const float2 p0 = acc[bb * 16 + 2 * j], p1 = acc[bb * 16 + 2 * j + 1];
-                    *reinterpret_cast<float4*>(&sm.out[b][swz(row, j)]) =
-                        make_float4(__fmul_rn(p0.x, sa), __fmul_rn(p0.y, sa), __fmul_rn(p1.x, sa), __fmul_rn(p1.y, sa));
+                    for (int bb = 0; bb < HC / 32; ++bb)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int b = (h * HC - part * GOUT) / 32 + bb;  // 32-column box of this part
+                            const float2 p0 = acc[bb * 16 + 2 * j], p1 = acc[bb * 16 + 2 * j + 1];
+                            *reinterpret_cast<float4*>(&sm.out[b][swz(row, j)]) = make_float4(
+                                __fmul_rn(p0.x, sa), __fmul_rn(p0.y, sa), __fmul_rn(p1.x, sa), __fmul_rn(p1.y, sa));
+                        }
                 }
-            fence_proxy_async();
-            named_sync(1, 32 * GEPI);
-            if (threadIdx.x == 64 && alive) {
+                fence_proxy_async();
+                named_sync(1, 32 * GEPI);
+                if (threadIdx.x == 64 && alive && n0 + part * GOUT < a.N) {  // no store starts past N
 #pragma unroll
-                for (int b = 0; b < GN / 32; ++b) tma_store_2d(&tY, n0 + b * 32, m0, &sm.out[b][0]);
-                bulk_commit();
+                    for (int b = 0; b < GOUT / 32; ++b)
+                        tma_store_2d(&tY, n0 + part * GOUT + b * 32, m0, &sm.out[b][0]);
+                    bulk_commit();
+                }
             }
         }
         if (threadIdx.x == 64) bulk_wait0();
@@ -321,9 +335,9 @@ extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M,
 {
     if (!A || !sa || !V || !g || !Y || !ws) return HQ_ERR_ARG;
     if (group != GK) return HQ_ERR_UNSUPPORTED;
-    if (M < GM || N < GN || K < GK || M % GM || N % GN || K % GK) return HQ_ERR_ARG;
+    if (M < GM || N < 128 || K < GK || M % GM || N % 128 || K % GK) return HQ_ERR_ARG;
     if (K > ((int64_t)1 << 20) || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return HQ_ERR_UNSUPPORTED;
-    if ((M / GM) * (N / GN) > ((int64_t)1 << 30)) return HQ_ERR_UNSUPPORTED;
+    if ((M / GM) * ((N + GN - 1) / GN) > ((int64_t)1 << 30)) return HQ_ERR_UNSUPPORTED;
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
     const uintptr_t al = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(V) |
                          reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(ws) |
@@ -341,7 +355,7 @@ extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M,
         cudaSuccess)
         return HQ_ERR_CUDA;
     GemmArgs a{M, N, K, sa, g, static_cast<WsHeader*>(ws)};
-    const int64_t tiles = (M / GM) * (N / GN);
+    const int64_t tiles = (M / GM) * ((N + GN - 1) / GN);
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());  // persistent: one CTA per SM
     gemm_i8_grouped_kernel<<<grid, GTHREADS, smem, st>>>(a, ta, tb, ty);
     return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
