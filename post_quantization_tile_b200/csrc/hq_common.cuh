@@ -21,7 +21,10 @@ namespace hq {
 #define HQ_THREADS 128
 #endif
 constexpr int kThreads = HQ_THREADS;   // threads per block (one tile row each, two for n = 256)
-constexpr int kMinBlocks = 384 / kThreads;  // resident blocks per SM the register budget aims at
+#ifndef HQ_MIN_BLOCKS
+#define HQ_MIN_BLOCKS (384 / HQ_THREADS)
+#endif
+constexpr int kMinBlocks = HQ_MIN_BLOCKS;  // resident blocks per SM the register budget aims at
 constexpr int kChunkTiles = 32;        // tiles per chunk (one warp scan)
 constexpr int kStages = 2;             // input pipeline depth
 constexpr uint32_t kSpinLimit = 1u << 22;  // bounded waits: polls before giving up
