@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/hq.h"
+#include "../../include/hq_test.h"
 #include "hq_common.cuh"
 #include "hq_decode.cuh"
 #include "hq_encode.cuh"
@@ -209,6 +210,7 @@ hq_status_t plan_encode(const void* x, int src, int64_t rows, int64_t cols, cons
     a.ws = static_cast<WsHeader*>(ws);
     a.states = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + sizeof(WsHeader));
     a.search = nullptr;
+    a.test_silent_item = -1;
     pl.kv = kv != 0;
     pl.src = src;
     return HQ_OK;
@@ -217,7 +219,7 @@ hq_status_t plan_encode(const void* x, int src, int64_t rows, int64_t cols, cons
 // common body of the encode entry points
 hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, const hq_params_t* p, int32_t kv,
                           int64_t kv_S, int32_t* v_out, hq_code_t* out, unsigned long long* count_out, void* ws,
-                          size_t ws_bytes, void* stream, int64_t kv_s0 = 0)
+                          size_t ws_bytes, void* stream, int64_t kv_s0 = 0, int64_t test_silent_item = -1)
 {
     const bool count = count_out != nullptr;
     if (kv_s0 < 0 || (kv_s0 && kv != 1)) return HQ_ERR_ARG;
@@ -225,6 +227,7 @@ hq_status_t encode_common(const void* x, int src, int64_t rows, int64_t cols, co
     const hq_status_t ps = plan_encode(x, src, rows, cols, p, kv, kv_S, v_out, out, count, ws, ws_bytes, pl);
     if (ps != HQ_OK) return ps;
     pl.a.kv_s0 = kv_s0;
+    pl.a.test_silent_item = test_silent_item;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t clear = count ? sizeof(WsHeader) : sizeof(WsHeader) + (size_t)pl.g.items * 8u;
     cudaError_t e = cudaMemsetAsync(ws, 0, clear, st);
@@ -557,6 +560,16 @@ hq_status_t hq_step_search(const void* x, hq_dtype_t dtype, int64_t rows, int64_
     if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
     return step_search_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, kv, kv ? kv_S : 0, max_probes, tol_bps,
                               result, ws, ws_bytes, stream);
+}
+
+hq_status_t hq_test_encode_silent_item(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols,
+                                       const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes,
+                                       int64_t silent_item, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (silent_item < 1) return HQ_ERR_ARG;  // item 0 needs no look-back
+    return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, 0, 0, nullptr, out, nullptr, ws, ws_bytes, stream,
+                         0, silent_item);
 }
 
 hq_status_t hq_status_read(const void* ws, void* stream, int64_t* detail)

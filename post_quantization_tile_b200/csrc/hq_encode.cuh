@@ -33,6 +33,8 @@ struct EncodeArgs {
     uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
     const RateSearch* search;  // count-only passes of a step search: the step comes from here
     int64_t kv_s0;             // KV: position of the call's first token in every sequence
+    int64_t test_silent_item;  // test only: this item never publishes its offset (-1: none), so its
+                               // successor's bounded look-back must run out and report a timeout
 };
 
 // SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
@@ -545,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                     atomicAdd(&a.ws->count_bits, (unsigned long long)bits);
                 } else {
                     const unsigned long long st = ((item == 0 ? 2ull : 1ull) << 32) | acc_words;
-                    st_relaxed_u64(a.states + item, st);
+                    if (item != a.test_silent_item) st_relaxed_u64(a.states + item, st);
                 }
             }
         }
@@ -657,7 +659,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                 }
             }
             if (lane == 0) {
-                if (item > 0) st_relaxed_u64(a.states + item, (2ull << 32) | (unsigned long long)(excl + item_words));
+                if (item > 0 && item != a.test_silent_item)
+                    st_relaxed_u64(a.states + item, (2ull << 32) | (unsigned long long)(excl + item_words));
                 sm.base = excl;
             }
         }
