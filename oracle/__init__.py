@@ -81,6 +81,15 @@ def lib():
         L.hqo_parse.restype = ctypes.c_uint32
         L.hqo_decode.argtypes = [P, P, P, P, i64, i64, i32, i32, f32, u64, i32, i64, P, i64, i64]
         L.hqo_decode.restype = ctypes.c_uint32
+        L.hqo_rotate_normalize.argtypes = [P, i32, i64, i32, P, f32, P, P]
+        L.hqo_rotate_normalize.restype = ctypes.c_uint32
+        L.hqo_encode_dense.argtypes = [P, i32, i64, i32, P, i32, f32, u64, i64, i64, i64, P, P, P, P, i64, P, P]
+        L.hqo_encode_dense.restype = ctypes.c_uint32
+        L.hqo_decode_coeffs.argtypes = [P, P, P, i64, i32, i32, u64, i64, i64, i64, P]
+        L.hqo_decode_coeffs.restype = ctypes.c_uint32
+        L.hqo_unrotate.argtypes = [P, P, i64, i32, P, f32, P]
+        L.hqo_decode_dense.argtypes = [P, P, P, P, i64, i32, P, i32, f32, u64, i64, i64, i64, P]
+        L.hqo_decode_dense.restype = ctypes.c_uint32
         _lib = L
     return _lib
 
@@ -457,3 +466,96 @@ def gemm_grouped_sample(A, sa, V, g, n, idx_m, idx_r) -> np.ndarray:
     lib().hqo_gemm_grouped_sample(_p(A), _p(sa), _p(V), _p(g), V.shape[0], A.shape[1], n, _p(im), _p(ir), im.size,
                                   _p(out))
     return out
+
+
+# ----------------------------------------------------------------------------------------------
+# dense-rotation KV variant (a caller-given orthogonal Q in place of H_n D)
+# ----------------------------------------------------------------------------------------------
+KV_DENSE = 3   # Code.kv of a dense-rotation KV code (dither words of KV rows)
+
+
+def _dtype_code(x: np.ndarray) -> int:
+    if x.dtype == np.uint16:
+        return 0
+    if x.dtype == np.float32:
+        return 1
+    raise TypeError("x must be uint16 (bf16 bits) or float32")
+
+
+def rotate_normalize(x: np.ndarray, Q: np.ndarray, beta: float):
+    """u = (Q x) / (s_hat beta) per row in binary32 (fma chain in ascending i) and the bf16 RMS
+    bits.  Returns (u float32 [rows, n], scale uint16 [rows], status)."""
+    x = np.ascontiguousarray(x)
+    Q = np.ascontiguousarray(Q, dtype=np.float32)
+    rows, n = x.shape
+    u = np.zeros((rows, n), dtype=np.float32)
+    scale = np.zeros(rows, dtype=np.uint16)
+    st = lib().hqo_rotate_normalize(_p(x), _dtype_code(x), rows, n, _p(Q), ctypes.c_float(beta), _p(u), _p(scale))
+    if st & 2:
+        raise ValueError("oracle rejected the arguments")
+    return u, scale, int(st)
+
+
+def encode_dense(x: np.ndarray, Q: np.ndarray, lattice: int, beta: float, seed: int, kv_S: int,
+                 row0: int = 0, kv_s0: int = 0, want_codes: bool = False) -> Code:
+    """Dense-rotation KV encode of x [rows, n] (head vectors of a [B, H, S, n] tensor with S = kv_S;
+    row0 the global row of x's first row, kv_s0 the first token position)."""
+    x = np.ascontiguousarray(x)
+    Q = np.ascontiguousarray(Q, dtype=np.float32)
+    rows, n = x.shape
+    C = (rows + 31) // 32
+    cap = bound_words(rows, n, n)
+    scale = np.zeros(rows, dtype=np.uint16)
+    meta = np.zeros(rows, dtype=np.uint16)
+    cw = np.zeros(C + 1, dtype=np.uint32)
+    bits = np.zeros(cap, dtype=np.uint32)
+    v = np.zeros((rows, n), dtype=np.int32) if want_codes else None
+    u = np.zeros((rows, n), dtype=np.float32) if want_codes else None
+    st = lib().hqo_encode_dense(_p(x), _dtype_code(x), rows, n, _p(Q), lattice, ctypes.c_float(beta), seed, kv_S,
+                                row0, kv_s0, _p(scale), _p(meta), _p(cw), _p(bits), cap,
+                                _p(v) if v is not None else None, _p(u) if u is not None else None)
+    if st & 2:
+        raise ValueError("oracle rejected the arguments")
+    c = Code(rows, n, n, lattice, float(np.float32(beta)), seed, KV_DENSE, kv_S, scale, meta, cw,
+             bits[: int(cw[-1])].copy(), int(st), v, u)
+    c.row0 = row0
+    c.kv_s0 = kv_s0
+    return c
+
+
+def _bits_or_pad(code: Code) -> np.ndarray:
+    bits = np.ascontiguousarray(code.bits, dtype=np.uint32)
+    return bits if bits.size else np.zeros(1, dtype=np.uint32)
+
+
+def decode_coeffs(code: Code) -> tuple[np.ndarray, int]:
+    """Lattice points minus the KV dither, in u units, float64 [rows, n] (one tile column)."""
+    p = np.zeros((code.rows, code.n), dtype=np.float64)
+    st = lib().hqo_decode_coeffs(_p(code.meta), _p(code.chunk_word), _p(_bits_or_pad(code)), code.rows, code.n,
+                                 code.lattice, code.seed, code.kv_S, getattr(code, "row0", 0),
+                                 getattr(code, "kv_s0", 0), _p(p))
+    if st & 2:
+        raise ValueError("oracle rejected the arguments")
+    return p, int(st)
+
+
+def unrotate(p: np.ndarray, scale: np.ndarray, Q: np.ndarray, beta: float) -> np.ndarray:
+    """x_hat = Q^T p (s_hat beta) per row, float64."""
+    p = np.ascontiguousarray(p, dtype=np.float64)
+    scale = np.ascontiguousarray(scale, dtype=np.uint16)
+    Q = np.ascontiguousarray(Q, dtype=np.float32)
+    out = np.zeros_like(p)
+    lib().hqo_unrotate(_p(p), _p(scale), p.shape[0], p.shape[1], _p(Q), ctypes.c_float(beta), _p(out))
+    return out
+
+
+def decode_dense(code: Code, Q: np.ndarray) -> tuple[np.ndarray, int]:
+    """Dense-rotation KV decode to float64 [rows, n] and status bits."""
+    Q = np.ascontiguousarray(Q, dtype=np.float32)
+    out = np.zeros((code.rows, code.n), dtype=np.float64)
+    st = lib().hqo_decode_dense(_p(code.scale), _p(code.meta), _p(code.chunk_word), _p(_bits_or_pad(code)),
+                                code.rows, code.n, _p(Q), code.lattice, ctypes.c_float(code.beta), code.seed,
+                                code.kv_S, getattr(code, "row0", 0), getattr(code, "kv_s0", 0), _p(out))
+    if st & 2:
+        raise ValueError("oracle rejected the arguments")
+    return out, int(st)

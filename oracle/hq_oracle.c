@@ -699,11 +699,24 @@ uint32_t hqo_encode(const void* x, int dtype, int64_t rows, int64_t cols, int n,
  * (t / kv_S, t % kv_S) is added first; kv = 2: the dither of tile (t, 0).  Outputs as for
  * hqo_encode (no scale).
  */
+static uint32_t quantize_rows(const float* u, int64_t tiles, int n, int lattice, int kv, int64_t kv_S,
+                              int64_t row0, int64_t kv_s0, uint64_t seed, int32_t* v_out, uint16_t* meta,
+                              uint32_t* chunk_word, uint32_t* bits, int64_t cap_words);
+
 uint32_t hqo_quantize_coeffs(const float* u, int64_t tiles, int n, int lattice, int kv, int64_t kv_S,
                              uint64_t seed, int32_t* v_out, uint16_t* meta, uint32_t* chunk_word,
                              uint32_t* bits, int64_t cap_words)
 {
     if (!valid_common(n, lattice) || !valid_kv(kv, lattice) || tiles <= 0) return 1u << 1;
+    return quantize_rows(u, tiles, n, lattice, kv, kv_S, 0, 0, seed, v_out, meta, chunk_word, bits, cap_words);
+}
+
+/* rows of normalised coefficients (one tile each, chunks of 32 rows) -> codes and bitstream; the
+ * dither words of row t are those of row row0 + t of a call starting at token kv_s0 */
+static uint32_t quantize_rows(const float* u, int64_t tiles, int n, int lattice, int kv, int64_t kv_S,
+                              int64_t row0, int64_t kv_s0, uint64_t seed, int32_t* v_out, uint16_t* meta,
+                              uint32_t* chunk_word, uint32_t* bits, int64_t cap_words)
+{
     memset(bits, 0, (size_t)cap_words * 4);
     bitw_t w = {bits, cap_words, 0, 0};
     int64_t RB = (tiles + 31) / 32;
@@ -712,7 +725,7 @@ uint32_t hqo_quantize_coeffs(const float* u, int64_t tiles, int n, int lattice, 
         int64_t t_end = (c + 1) * 32 < tiles ? (c + 1) * 32 : tiles;
         for (int64_t t = c * 32; t < t_end; ++t) {
             int64_t c1 = 0, cw = 0;
-            if (kv) dither_words(kv, t, kv_S, 0, 0, &c1, &cw);
+            if (kv) dither_words(kv, row0 + t, kv_S, kv_s0, 0, &c1, &cw);
             int32_t v[HQO_MAXN];
             quantize_tile(u + t * n, n, lattice, kv != 0, seed, c1, cw, v);
             int k, sumq;
@@ -932,4 +945,126 @@ void hqo_gemm_grouped_sample(const int8_t* A, const float* sa, const int8_t* V, 
                              int n, const int64_t* idx_m, const int64_t* idx_r, int64_t count, float* out)
 {
     for (int64_t i = 0; i < count; ++i) out[i] = hqo_gemm_one(A, sa, V, g, N, K, n, idx_m[i], idx_r[i]);
+}
+
+
+/* ------------------------------------------------------------------------------------------ */
+/* Dense-rotation KV variant.  Methodology step 4 ("Bias Correction for KV Cache") allows the     */
+/* per-layer rotation of the KV path to be either the sign diagonal or a dense random          */
+/* orthogonal matrix drawn from the Haar measure (the QJL-style rotation, credited in Key       */
+/* Contributions with the gain at 1.7-2.5 bps).  The caller passes Q (n x n, row-major,         */
+/* y = Q x).  Reading: the RMS scale, lattice, dither, stripping and Rice coding are the        */
+/* codec's; there is no sign diagonal (Q is random already) and no c_n (Q is orthonormal).      */
+/* Binary32 forward: y_j = fma chain over i = 0 .. n-1 of Q[j][i] x_i from 0, then             */
+/* u_j = y_j * (1 / (s_hat beta)).  Zero and non-finite tiles as the codec.                    */
+/* ------------------------------------------------------------------------------------------ */
+uint32_t hqo_rotate_normalize(const void* x, int dtype, int64_t rows, int n, const float* Q, float beta,
+                              float* u_out, uint16_t* scale_out)
+{
+    if (!(n == 64 || n == 128) || rows <= 0) return 1u << 1;
+    uint32_t status = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        float xt[HQO_MAXN];
+        int finite = 1;
+        for (int i = 0; i < n; ++i) {
+            xt[i] = dtype == 0 ? hqo_bf16_to_f32(((const uint16_t*)x)[r * n + i]) : ((const float*)x)[r * n + i];
+            if (!isfinite(xt[i])) finite = 0;
+        }
+        float s = finite ? hqo_rms(xt, n) : 0.0f;
+        uint16_t sh = hqo_f32_to_bf16(s);
+        float shf = hqo_bf16_to_f32(sh);
+        if (!finite || !isfinite(shf)) {
+            status |= HQO_ST_NONFINITE;
+            sh = 0;
+            shf = 0.0f;
+        } else if (shf < 1.2621774483536189e-29f /* 2^-96 */) {
+            sh = 0;
+            shf = 0.0f;
+        }
+        scale_out[r] = sh;
+        if (shf == 0.0f) {
+            for (int j = 0; j < n; ++j) u_out[r * n + j] = 0.0f;
+            continue;
+        }
+        float g = 1.0f / (shf * beta);
+        for (int j = 0; j < n; ++j) {
+            float acc = 0.0f;
+            for (int i = 0; i < n; ++i) acc = fmaf(Q[j * n + i], xt[i], acc);
+            u_out[r * n + j] = acc * g;
+        }
+    }
+    return status;
+}
+
+/*
+ * Dense-rotation KV encode: x [rows, n] (rows = B*H*S head vectors of a [B, H, S, n] tensor,
+ * row0 = global row of x's first row, tokens starting at kv_s0), codes with the KV dither of
+ * row (b H + h, kv_s0 + s).  Outputs as hqo_encode with one tile column.
+ */
+uint32_t hqo_encode_dense(const void* x, int dtype, int64_t rows, int n, const float* Q, int lattice, float beta,
+                          uint64_t seed, int64_t kv_S, int64_t row0, int64_t kv_s0, uint16_t* scale, uint16_t* meta,
+                          uint32_t* chunk_word, uint32_t* bits, int64_t cap_words, int32_t* v_out, float* u_out)
+{
+    if (!valid_common(n, lattice) || n > 128 || rows <= 0 || kv_S <= 0 || kv_s0 < 0) return 1u << 1;
+    float* u = (float*)malloc(sizeof(float) * (size_t)(rows * n));
+    if (!u) return 1u << 1;
+    uint32_t status = hqo_rotate_normalize(x, dtype, rows, n, Q, beta, u, scale);
+    status |= quantize_rows(u, rows, n, lattice, 1, kv_S, row0, kv_s0, seed, v_out, meta, chunk_word, bits, cap_words);
+    if (u_out) memcpy(u_out, u, sizeof(float) * (size_t)(rows * n));
+    free(u);
+    return status;
+}
+
+/* The lattice points of a code of rows x n normalised coefficients (one tile column) in u units,
+ * minus the KV dither of row (b H + h, kv_s0 + s): E8 v/2, A2 (P/2, Q sqrt3/2), Z and D4 v, the
+ * dither taken off in the quantizer's coordinates.  Binary64. */
+uint32_t hqo_decode_coeffs(const uint16_t* meta, const uint32_t* chunk_word, const uint32_t* bits, int64_t rows, int n,
+                           int lattice, uint64_t seed, int64_t kv_S, int64_t row0, int64_t kv_s0, double* p_out)
+{
+    if (!valid_common(n, lattice) || rows <= 0 || kv_S <= 0) return 1u << 1;
+    int32_t* v = (int32_t*)malloc(sizeof(int32_t) * (size_t)(rows * n));
+    if (!v) return 1u << 1;
+    uint32_t status = hqo_parse(meta, chunk_word, bits, rows, n, n, lattice, v);
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t c1 = 0, cw = 0;
+        dither_words(1, row0 + r, kv_S, kv_s0, 0, &c1, &cw);
+        float U[HQO_MAXN];
+        hqo_dither(lattice, seed, c1, cw, n, U);
+        for (int i = 0; i < n; ++i) {
+            const double vi = (double)v[r * n + i], Ui = (double)U[i];
+            double p;
+            if (lattice == HQO_E8) p = 0.5 * vi - Ui;
+            else if (lattice == HQO_A2) p = (i & 1) ? (vi - Ui) * (sqrt(3.0) / 2.0) : 0.5 * (vi - Ui);
+            else p = vi - Ui;
+            p_out[r * n + i] = p;
+        }
+    }
+    free(v);
+    return status;
+}
+
+/* Inverse rotation: x_hat_i = (sum_j Q[j][i] p_j) (s_hat beta), i.e. Q^T p rescaled.  Binary64. */
+void hqo_unrotate(const double* p, const uint16_t* scale, int64_t rows, int n, const float* Q, float beta, double* out)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const double h = (double)hqo_bf16_to_f32(scale[r]) * (double)beta;
+        for (int i = 0; i < n; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < n; ++j) acc += (double)Q[j * n + i] * p[r * n + j];
+            out[r * n + i] = acc * h;
+        }
+    }
+}
+
+/* Dense-rotation KV decode to binary64 out[rows, n]. */
+uint32_t hqo_decode_dense(const uint16_t* scale, const uint16_t* meta, const uint32_t* chunk_word, const uint32_t* bits,
+                          int64_t rows, int n, const float* Q, int lattice, float beta, uint64_t seed, int64_t kv_S,
+                          int64_t row0, int64_t kv_s0, double* out)
+{
+    double* p = (double*)malloc(sizeof(double) * (size_t)(rows > 0 ? rows * n : 1));
+    if (!p) return 1u << 1;
+    uint32_t status = hqo_decode_coeffs(meta, chunk_word, bits, rows, n, lattice, seed, kv_S, row0, kv_s0, p);
+    if (!(status & 2u)) hqo_unrotate(p, scale, rows, n, Q, beta, out);
+    free(p);
+    return status;
 }

@@ -91,3 +91,13 @@ def queries(count: int, D: int = 128, seed: int = 3) -> np.ndarray:
 def gaussian_bf16(rows: int, cols: int, seed: int) -> np.ndarray:
     rng = np.random.default_rng(seed)
     return to_bf16_bits(rng.standard_normal(size=(rows, cols), dtype=np.float32))
+
+
+def haar_rotation(n: int = 128, seed: int = 8) -> np.ndarray:
+    """float32 [n, n] orthogonal matrix drawn from the Haar measure: the Q factor of a Gaussian
+    matrix with the signs of R's diagonal moved into Q (Mezzadri's correction)."""
+    rng = np.random.default_rng(seed)
+    g = rng.standard_normal((n, n))
+    q, r = np.linalg.qr(g)
+    q = q * np.sign(np.diag(r))[None, :]
+    return q.astype(np.float32)
