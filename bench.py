@@ -453,13 +453,49 @@ def run_kv(hq, dev, stream, peak):
     code_bytes = 4 * codes[0].total_words() + 4 * codes[0].scale.numel() + 4 * codes[0].chunk_word.numel()
     moved = 2 * n + code_bytes
     e50, d50 = statistics.median(enc), statistics.median(dec)
-    return {"workload": "kv_keys_8x32x8192x128_bf16_D4_dither_n128_2bps", "step": beta,
+    dense = run_kv_dense(hq, keys, beta, S, D, stream)
+    return {"workload": "kv_keys_8x32x8192x128_bf16_D4_dither_n128_2bps", "step": beta, "dense_rotation": dense,
             "payload_bps": codes[0].payload_bps(), "total_bps": codes[0].total_bps(),
             "encode_ms_p10_p50_p90": percentiles(enc), "decode_ms_p10_p50_p90": percentiles(dec),
             "encode_gbs_bf16": 2 * n / (e50 * 1e-3) / 1e9, "decode_gbs_bf16": 2 * n / (d50 * 1e-3) / 1e9,
             "encode_roofline_frac": moved / (e50 * 1e-3) / 1e9 / peak,
             "decode_roofline_frac": moved / (d50 * 1e-3) / 1e9 / peak,
             "bytes_per_call": moved, "status": st}
+
+
+def run_kv_dense(hq, keys, beta, S, D, stream):
+    """The same KV tensors through the dense-rotation variant (a seeded Haar-random 128 x 128 Q in
+    place of the RHT; binary32 rotation on the FP32 pipe): per-call encode and decode times and
+    the rotation's FP32 throughput (2 x 128 flops per scalar each way) over the whole call."""
+    import torch
+
+    from post_quantization_tile_b200 import workloads as W
+    Q = torch.from_numpy(W.haar_rotation(D, seed=8)).to(keys[0].device)
+    codes = [hq.kv_encode_dense(keys[i], Q, step=beta, seed=SEED) for i in range(2)]
+    out = torch.empty_like(keys[0])
+    calls = 6
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(calls)]
+    for k in range(2):
+        hq.kv_encode_dense(keys[k % 2], Q, step=beta, seed=SEED, out=codes[k % 2], ws=codes[k % 2].ws)
+        hq.kv_decode_dense(codes[(k + 1) % 2], Q, out=out.view(-1, D), ws=codes[(k + 1) % 2].ws)
+    for k in range(calls):
+        a, b = k % 2, (k + 1) % 2
+        ev[k][0].record(stream)
+        hq.kv_encode_dense(keys[a], Q, step=beta, seed=SEED, out=codes[a], ws=codes[a].ws)
+        ev[k][1].record(stream)
+        ev[k][2].record(stream)
+        hq.kv_decode_dense(codes[b], Q, out=out.view(-1, D), ws=codes[b].ws)
+        ev[k][3].record(stream)
+    torch.cuda.synchronize()
+    st, _ = hq.status(codes[0].ws)
+    enc = [e[0].elapsed_time(e[1]) for e in ev]
+    dec = [e[2].elapsed_time(e[3]) for e in ev]
+    n = keys[0].numel()
+    e50, d50 = statistics.median(enc), statistics.median(dec)
+    return {"encode_ms_p10_p50_p90": percentiles(enc), "decode_ms_p10_p50_p90": percentiles(dec),
+            "payload_bps": codes[0].payload_bps(),
+            "encode_rotation_tflops": 2.0 * D * n / (e50 * 1e-3) / 1e12,
+            "decode_rotation_tflops": 2.0 * D * n / (d50 * 1e-3) / 1e12, "status": st}
 
 
 def run_gemm(hq, dev, peak_bf16):

@@ -92,7 +92,8 @@ typedef struct {
  *   rows, cols  dense shape (KV: rows = B*H*S, cols = D)
  *   kv_S        S of the KV layout (dither counter); 0 for weights
  *   p           parameters with the step resolved (never 0 after encode)
- *   kv          0 plain; 1 KV rows with the dither; 2 weights with the dither (hq_encode_dither)
+ *   kv          0 plain; 1 KV rows with the dither; 2 weights with the dither (hq_encode_dither);
+ *               3 KV rows with the dither and the dense rotation (hq_kv_encode_dense)
  *   version     HQ_FORMAT_VERSION
  *   scale       [T] bf16 bit patterns of the per-tile RMS (0 = all-zero tile)
  *   meta        [T] k | (sum q << 4): the tile's Rice parameter and unary total
@@ -183,6 +184,37 @@ hq_status_t hq_kv_encode_at(const void* kv, hq_dtype_t dtype, int64_t B, int64_t
 /* Decode a KV tensor: the dither is regenerated and subtracted before the inverse transform. */
 hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void* ws, size_t ws_bytes,
                          void* stream);
+
+/*
+ * Dense-rotation KV variant (Methodology step 4, "Bias Correction for KV Cache": the per-layer
+ * rotation may be a dense Haar-random orthogonal matrix instead of the sign diagonal).  Each head
+ * vector x of kv[B, H, S, D] (device, contiguous, D == p->tile == 128) is coded as
+ *   u = (Q x) / (bf16(s) beta),  s the RMS of x (the codec's scale, zero and non-finite vectors as
+ *   in hq_encode),
+ * then quantized with the KV dither of token (b, h, s0 + s), bit-stripped and Rice-coded exactly
+ * like hq_kv_encode_at: one tile per head vector, chunks of 32 rows.  u_j is the binary32 fma chain
+ * over i = 0 .. 127 of Q[j][i] x_i from 0, multiplied by the binary32 1 / (bf16(s) beta).
+ *   Q    fp32 [128, 128] row-major (device, 4-byte aligned), orthogonal; the caller draws it (from
+ *        the Haar measure for the method's variant) and passes the same Q to the decode.  No sign
+ *        diagonal and no 1/sqrt(n) factor are applied: Q is the whole rotation.
+ *   ws   at least hq_kv_dense_workspace_bytes(B*H*S) bytes (holds the coefficients between the
+ *        rotation and the codec).
+ * out->kv = 3, out->kv_s0 = s0.  D other than 128: HQ_ERR_UNSUPPORTED.  Device errors as
+ * hq_kv_encode_at (HQ_ERR_NONFINITE counts the non-finite head vectors).
+ */
+size_t hq_kv_dense_workspace_bytes(int64_t rows);
+hq_status_t hq_kv_encode_dense(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D,
+                               int64_t s0, const float* Q, const hq_params_t* p, hq_code_t* out, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/*
+ * Decode a dense-rotation KV code (code->kv == 3) into kv[rows, 128] (device, bf16 or fp32,
+ * 16-byte aligned): p = lattice point minus the dither in u units, x_hat = (Q^T p) (bf16(s) beta)
+ * in binary32 (fma over j = 0 .. 127, then one product), rounded to nearest even for bf16.
+ * ws: hq_kv_dense_workspace_bytes(rows).  Device errors: HQ_ERR_CORRUPT (tile decoded as zeros).
+ */
+hq_status_t hq_kv_decode_dense(const hq_code_t* code, const float* Q, void* kv, hq_dtype_t dtype, void* ws,
+                               size_t ws_bytes, void* stream);
 
 /*
  * Lattice quantization, bit-stripping and Rice coding of caller-given normalised coefficients

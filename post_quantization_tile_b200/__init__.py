@@ -81,12 +81,18 @@ def lib():
         L.hq_gemm_int8.argtypes = [P, P, i64, P, P, i64, i64, i32, P, P, ctypes.c_size_t, P]
         L.hq_step_search.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, i32, ctypes.c_float, P, P,
                                      ctypes.c_size_t, P]
+        L.hq_kv_dense_workspace_bytes.argtypes = [i64]
+        L.hq_kv_dense_workspace_bytes.restype = ctypes.c_size_t
+        L.hq_kv_encode_dense.argtypes = [P, i32, i64, i64, i64, i64, i64, P, ctypes.POINTER(Params),
+                                         ctypes.POINTER(CodeStruct), P, ctypes.c_size_t, P]
+        L.hq_kv_decode_dense.argtypes = [ctypes.POINTER(CodeStruct), P, P, i32, P, ctypes.c_size_t, P]
         L.hq_status_read.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
         L.hq_status_str.argtypes = [i32]
         L.hq_status_str.restype = ctypes.c_char_p
         L.hq_version.restype = i32
         for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_encode_at", "hq_kv_decode", "hq_quantize_coeffs",
-                  "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_status_read"]:
+                  "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_status_read",
+                  "hq_kv_encode_dense", "hq_kv_decode_dense"]:
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -240,6 +246,8 @@ def decode(code: Code, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | 
     L = lib()
     w = ws or workspace(4096)
     cs = code.struct()
+    if code.kv == KV_DENSE:
+        raise ValueError("a dense-rotation KV code decodes with kv_decode_dense and its rotation Q")
     fn = L.hq_kv_decode if code.kv == 1 else L.hq_decode
     _check(fn(ctypes.byref(cs), _ptr(y), _dtype_code(y), w.ptr(), w.nbytes, _stream()), "hq_decode")
     code.ws = w
@@ -275,6 +283,54 @@ def kv_decode(code: Code, shape, dtype: torch.dtype = torch.bfloat16, out: torch
               ws: Workspace | None = None) -> torch.Tensor:
     y = decode(code, dtype=dtype, out=out, ws=ws)
     return y.view(*shape)
+
+
+KV_DENSE = 3  # Code.kv of a dense-rotation KV code
+
+
+def _check_rotation(Q: torch.Tensor, D: int):
+    _require_cuda(Q, "Q")
+    if Q.dtype != torch.float32 or tuple(Q.shape) != (D, D) or not Q.is_contiguous():
+        raise ValueError(f"Q must be a contiguous float32 [{D}, {D}] CUDA tensor")
+
+
+def kv_encode_dense(kv: torch.Tensor, Q: torch.Tensor, step: float = 0.0, bps: float = 4.0, seed: int = 0,
+                    lattice: int | str = D4, s0: int = 0, out: Code | None = None,
+                    ws: Workspace | None = None) -> Code:
+    """Encode a KV tensor [B, H, S, 128] with a dense orthogonal rotation Q (fp32 [128, 128], y = Q x)
+    in place of the RHT, then the codec's dither, lattice and Rice coding (the Haar-rotation variant
+    of Methodology step 4).  s0: first token position of every sequence (token append)."""
+    _require_cuda(kv, "kv")
+    if kv.dim() != 4:
+        raise ValueError("kv must be [B, H, S, D]")
+    B, H, S, D = kv.shape
+    _check_rotation(Q, D)
+    p = params(D, lattice, step, bps, seed)
+    rows = B * H * S
+    code = out if out is not None else alloc_code(rows, D, p, device=kv.device)
+    L = lib()
+    w = ws or workspace(L.hq_kv_dense_workspace_bytes(rows))
+    cs = code.struct()
+    _check(L.hq_kv_encode_dense(_ptr(kv), _dtype_code(kv), B, H, S, D, int(s0), _ptr(Q), ctypes.byref(p),
+                                ctypes.byref(cs), w.ptr(), w.nbytes, _stream()), "hq_kv_encode_dense")
+    _fill(code, cs)
+    code.ws = w
+    return code
+
+
+def kv_decode_dense(code: Code, Q: torch.Tensor, shape=None, dtype: torch.dtype = torch.bfloat16,
+                    out: torch.Tensor | None = None, ws: Workspace | None = None) -> torch.Tensor:
+    """Decode a dense-rotation KV code: x_hat = Q^T (lattice point - dither) (s_hat beta)."""
+    _check_rotation(Q, code.cols)
+    y = out if out is not None else torch.empty(code.rows, code.cols, dtype=dtype, device=code.bits.device)
+    _require_cuda(y, "out")
+    L = lib()
+    w = ws or workspace(L.hq_kv_dense_workspace_bytes(code.rows))
+    cs = code.struct()
+    _check(L.hq_kv_decode_dense(ctypes.byref(cs), _ptr(Q), _ptr(y), _dtype_code(y), w.ptr(), w.nbytes, _stream()),
+           "hq_kv_decode_dense")
+    code.ws = w
+    return y if shape is None else y.view(*shape)
 
 
 def quantize_coeffs(u: torch.Tensor, tile: int, lattice: int | str, seed: int = 0, kv: bool = False, kv_S: int = 0,

@@ -379,14 +379,16 @@ hq_status_t step_search_common(const void* x, int src, int64_t rows, int64_t col
     return cuda_status(cudaGetLastError());
 }
 
-// dst: 0 bf16, 1 fp32, 2 int8 lattice codes with group scales g_out
+// dst: 0 bf16, 1 fp32, 2 int8 lattice codes with group scales g_out, 3 fp32 lattice points minus the
+// dither in u units (KV tiles of 128, the dense inverse rotation's input)
 hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, float* g_out, void* ws,
                           size_t ws_bytes, void* stream)
 {
     if (!code || !y || !aligned16(y) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
     if (code->version != HQ_FORMAT_VERSION) return HQ_ERR_ARG;
     if (kv ? code->kv != 1 : (code->kv != 0 && code->kv != 2)) return HQ_ERR_ARG;
-    if (dst < 0 || dst > 2) return HQ_ERR_ARG;
+    if (dst < 0 || dst > 3) return HQ_ERR_ARG;
+    if (dst == 3 && (code->kv != 1 || code->p.tile != 128)) return HQ_ERR_UNSUPPORTED;
     if (dst == 2) {
         if (!g_out || (reinterpret_cast<uintptr_t>(g_out) & 3u)) return HQ_ERR_ARG;
         if (code->kv != 0 || code->p.lattice == HQ_A2 || code->p.tile == 64) return HQ_ERR_UNSUPPORTED;
@@ -399,7 +401,7 @@ hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, f
     if (!code->scale || !code->meta || !code->chunk_word || !code->bits || !aligned16(code->bits)) return HQ_ERR_ARG;
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
     if (!use_device_of(y)) return HQ_ERR_ARG;
-    const int es = dst == 0 ? 2 : (dst == 1 ? 4 : 1);
+    const int es = dst == 0 ? 2 : (dst == 2 ? 1 : 4);
     CUtensorMap map;
     if (!make_map(&map, y, code->rows, code->cols, es, g.TI)) return HQ_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -425,6 +427,21 @@ hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, f
     a.cap_words = code->cap_words;
     a.ws = static_cast<WsHeader*>(ws);
     return cuda_status(run_decode(prm.lattice, prm.tile, code->kv != 0, dst, a, map, st));
+}
+
+// dense-rotation KV variant: the codec's workspace, then a 256-byte status block (the rotation's
+// non-finite count), then the rows x 128 fp32 coefficients between the rotation and the codec
+struct DenseLayout {
+    size_t status_off, buf_off, total;
+};
+bool dense_layout(int64_t rows, DenseLayout& d)
+{
+    const size_t e = ws_bytes_for(rows, 128, 128);
+    if (e == 0) return false;
+    d.status_off = (e + 255u) & ~(size_t)255u;
+    d.buf_off = d.status_off + 256u;
+    d.total = d.buf_off + (((size_t)rows * 512u + 255u) & ~(size_t)255u);
+    return true;
 }
 
 }  // namespace
@@ -532,6 +549,70 @@ hq_status_t hq_kv_decode(const hq_code_t* code, void* kv, hq_dtype_t dtype, void
 {
     if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
     return decode_common(code, kv, dtype == HQ_BF16 ? 0 : 1, 1, nullptr, ws, ws_bytes, stream);
+}
+
+size_t hq_kv_dense_workspace_bytes(int64_t rows)
+{
+    DenseLayout d;
+    return rows >= 1 && dense_layout(rows, d) ? d.total : 0;
+}
+
+hq_status_t hq_kv_encode_dense(const void* kv, hq_dtype_t dtype, int64_t B, int64_t H, int64_t S, int64_t D,
+                               int64_t s0, const float* Q, const hq_params_t* p, hq_code_t* out, void* ws,
+                               size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (B < 1 || H < 1 || S < 1 || s0 < 0 || !p || !Q || !out || D != p->tile) return HQ_ERR_ARG;
+    if (D != 128) return HQ_ERR_UNSUPPORTED;
+    if (B * H > ((int64_t)1 << 32) || B * H * S > ((int64_t)1 << 31)) return HQ_ERR_ARG;
+    hq_params_t prm;
+    if (!resolve_params(p, prm)) return HQ_ERR_ARG;
+    const int64_t rows = B * H * S;
+    DenseLayout d;
+    if (!dense_layout(rows, d) || ws_bytes < d.total) return HQ_ERR_ARG;
+    if (!kv || !aligned16(kv) || (reinterpret_cast<uintptr_t>(Q) & 3u) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
+    if (!out->scale || !out->meta || !out->chunk_word || !out->bits || out->cap_words < 1) return HQ_ERR_ARG;
+    if (!use_device_of(kv)) return HQ_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(ws);
+    uint32_t* nonfinite = reinterpret_cast<uint32_t*>(w + d.status_off);
+    float* u = reinterpret_cast<float*>(w + d.buf_off);
+    if (cudaMemsetAsync(nonfinite, 0, sizeof(uint32_t), st) != cudaSuccess) return HQ_ERR_CUDA;
+    if (launch_rotate(kv, dtype == HQ_BF16, Q, prm.step, rows, u, out->scale, nonfinite, st) != cudaSuccess)
+        return HQ_ERR_CUDA;
+    hq_code_t body = *out;
+    body.scale = nullptr;  // the rotation wrote the scales
+    const hq_status_t s = encode_common(u, 2, rows, D, &prm, 1, S, nullptr, &body, nullptr, ws, ws_bytes, stream, s0);
+    if (s != HQ_OK) return s;
+    if (launch_merge_nonfinite(ws, nonfinite, st) != cudaSuccess) return HQ_ERR_CUDA;
+    out->rows = body.rows;
+    out->cols = body.cols;
+    out->kv_S = body.kv_S;
+    out->p = body.p;
+    out->kv = 3;
+    out->kv_s0 = body.kv_s0;
+    out->version = body.version;
+    return HQ_OK;
+}
+
+hq_status_t hq_kv_decode_dense(const hq_code_t* code, const float* Q, void* kv, hq_dtype_t dtype, void* ws,
+                               size_t ws_bytes, void* stream)
+{
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    if (!code || code->kv != 3 || !Q || (reinterpret_cast<uintptr_t>(Q) & 3u)) return HQ_ERR_ARG;
+    if (!kv || !aligned16(kv) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
+    if (code->cols != code->p.tile || code->rows < 1) return HQ_ERR_ARG;
+    if (code->p.tile != 128) return HQ_ERR_UNSUPPORTED;
+    DenseLayout d;
+    if (!dense_layout(code->rows, d) || ws_bytes < d.total) return HQ_ERR_ARG;
+    if (!use_device_of(kv)) return HQ_ERR_ARG;
+    float* pbuf = reinterpret_cast<float*>(static_cast<char*>(ws) + d.buf_off);
+    hq_code_t body = *code;
+    body.kv = 1;  // dither words of KV rows; the lattice points come back untransformed
+    const hq_status_t s = decode_common(&body, pbuf, 3, 1, nullptr, ws, ws_bytes, stream);
+    if (s != HQ_OK) return s;
+    return launch_unrotate(pbuf, Q, code->scale, code->p.step, code->rows, kv, dtype == HQ_BF16,
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
 hq_status_t hq_quantize_coeffs(const float* u, int64_t tiles, const hq_params_t* p, int32_t kv, int64_t kv_S,

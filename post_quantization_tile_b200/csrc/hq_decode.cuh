@@ -31,14 +31,16 @@ struct DecodeArgs {
     int64_t kv_s0;    // KV: position of the code's first token in every sequence
 };
 
-template <int N, int DST>  // DST: 0 bf16, 1 fp32, 2 int8 lattice codes (RHT domain, no transform)
+// DST: 0 bf16, 1 fp32, 2 int8 lattice codes (RHT domain, no transform), 3 fp32 lattice points minus
+// the dither in u units (no transform, no scale: the input of a dense inverse rotation)
+template <int N, int DST>
 struct DecGeom {
     static constexpr int TPT = dec_tpt(N);
     static constexpr int V = N / TPT;
     static constexpr int H = V / 2;
     static constexpr int TI = kThreads / TPT;
     static constexpr int CH = TI / kChunkTiles;
-    static constexpr int ES = DST == 0 ? 2 : (DST == 1 ? 4 : 1);
+    static constexpr int ES = DST == 0 ? 2 : (DST == 2 ? 1 : 4);
     static constexpr int ROWB = N * ES;
     static constexpr int NB = ROWB / 128;
     static constexpr int OUT = NB * TI * 128;
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
         const bool valid = row_l < rows_valid;
         const bool stage_ok = sm.ok_ring[st] != 0;
 
-        if (DST != 2 && sm.mask_jt != jt) {
+        if (DST < 2 && sm.mask_jt != jt) {
             build_masks_out<N, DST>(sm.mask, jt, a.seed);
             __syncthreads();
             if (tid == 0) sm.mask_jt = jt;
@@ -414,39 +416,47 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 for (int m = 0; m < H; ++m) P[m] = ok ? P[m] : make_float2(0.0f, 0.0f);
             }
 
-            // ---------------- inverse transform: H_n p, exact for integer points ----------------
-            // in-thread strides (H within pairs, then H/2 .. 1); with two threads per tile the
-            // stride n/2 butterfly between the pair comes last
+            if constexpr (DST == 3) {
+                // the E8 codes are doubled points: halve (exact)
+                if constexpr (LAT == HQ_E8) {
     #pragma unroll
-            for (int m = 0; m < H; ++m) P[m] = make_float2(__fadd_rn(P[m].x, P[m].y), __fadd_rn(P[m].x, -P[m].y));
-    #pragma unroll
-            for (int h = H / 2; h >= 1; h /= 2)
-    #pragma unroll
-                for (int m = 0; m < H; ++m)
-                    if ((m & h) == 0) {
-                        const float2 x = P[m], y = P[m + h];
-                        P[m] = f2add(x, y);
-                        P[m + h] = f2sub(x, y);
-                    }
-            if constexpr (TPT == 2) {
-    #pragma unroll
-                for (int m = 0; m < H; ++m) {
-                    const float ox = __shfl_xor_sync(0xffffffffu, P[m].x, 1);
-                    const float oy = __shfl_xor_sync(0xffffffffu, P[m].y, 1);
-                    // tau 0 holds a (positions < n/2), tau 1 holds b: a + b -> tau 0, a - b -> tau 1
-                    P[m] = tau ? make_float2(__fadd_rn(ox, -P[m].x), __fadd_rn(oy, -P[m].y))
-                               : make_float2(__fadd_rn(P[m].x, ox), __fadd_rn(P[m].y, oy));
+                    for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], make_float2(0.5f, 0.5f));
                 }
-            }
+            } else {
+                // ---------------- inverse transform: H_n p, exact for integer points ----------------
+                // in-thread strides (H within pairs, then H/2 .. 1); with two threads per tile the
+                // stride n/2 butterfly between the pair comes last
+        #pragma unroll
+                for (int m = 0; m < H; ++m) P[m] = make_float2(__fadd_rn(P[m].x, P[m].y), __fadd_rn(P[m].x, -P[m].y));
+        #pragma unroll
+                for (int h = H / 2; h >= 1; h /= 2)
+        #pragma unroll
+                    for (int m = 0; m < H; ++m)
+                        if ((m & h) == 0) {
+                            const float2 x = P[m], y = P[m + h];
+                            P[m] = f2add(x, y);
+                            P[m + h] = f2sub(x, y);
+                        }
+                if constexpr (TPT == 2) {
+        #pragma unroll
+                    for (int m = 0; m < H; ++m) {
+                        const float ox = __shfl_xor_sync(0xffffffffu, P[m].x, 1);
+                        const float oy = __shfl_xor_sync(0xffffffffu, P[m].y, 1);
+                        // tau 0 holds a (positions < n/2), tau 1 holds b: a + b -> tau 0, a - b -> tau 1
+                        P[m] = tau ? make_float2(__fadd_rn(ox, -P[m].x), __fadd_rn(oy, -P[m].y))
+                                   : make_float2(__fadd_rn(P[m].x, ox), __fadd_rn(P[m].y, oy));
+                    }
+                }
 
-            // ---------------- scale, sign, store into the staging box ----------------
-            const float sh = __uint_as_float((uint32_t)sbits << 16);
-            const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
-            float ht = __fmul_rn(__fmul_rn(sh, a.beta), cn);
-            if constexpr (LAT == HQ_E8) ht = __fmul_rn(ht, 0.5f);
-            const float2 h2 = make_float2(ht, ht);
-    #pragma unroll
-            for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], h2);
+                // ---------------- scale, sign, store into the staging box ----------------
+                const float sh = __uint_as_float((uint32_t)sbits << 16);
+                const float cn = N == 64 ? 0.125f : (N == 128 ? __uint_as_float(0x3DB504F3u) : 0.0625f);
+                float ht = __fmul_rn(__fmul_rn(sh, a.beta), cn);
+                if constexpr (LAT == HQ_E8) ht = __fmul_rn(ht, 0.5f);
+                const float2 h2 = make_float2(ht, ht);
+        #pragma unroll
+                for (int m = 0; m < H; ++m) P[m] = f2mul(P[m], h2);
+            }
 
             __syncthreads();  // every thread has read its scratch: the box may be overwritten
             if constexpr (DST == 0) {
@@ -479,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
     #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const float f = half ? P[4 * c + q].y : P[4 * c + q].x;
-                            w[q] = __float_as_uint(f) ^ sm.mask[e0 + q];
+                            w[q] = DST == 1 ? __float_as_uint(f) ^ sm.mask[e0 + q] : __float_as_uint(f);
                         }
                         const int cg = e0 / 4;
                         *reinterpret_cast<uint4*>(sm.buf + (cg >> 3) * (TI * 128) + swz(row_l, cg & 7)) =

@@ -81,6 +81,10 @@ static cudaError_t dec_dst(int dst, const DecodeArgs& a, const CUtensorMap& m, c
         if constexpr (!KV && LAT != HQ_A2 && N != 64) return dec_one<N, LAT, KV, 2>(a, m, st);
         return cudaErrorInvalidValue;
     }
+    if (dst == 3) {  // dithered lattice points for the dense inverse rotation: KV tiles of 128
+        if constexpr (KV && N == 128) return dec_one<N, LAT, KV, 3>(a, m, st);
+        return cudaErrorInvalidValue;
+    }
     return dst == 0 ? dec_one<N, LAT, KV, 0>(a, m, st) : dec_one<N, LAT, KV, 1>(a, m, st);
 }
 

@@ -15,13 +15,21 @@ cudaError_t launch_encode_z(int n, bool kv, int src, bool count, const EncodeArg
 cudaError_t launch_encode_a2(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_encode_d4(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_encode_e8(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
-// dst: 0 bf16, 1 fp32
+// dst: 0 bf16, 1 fp32, 2 int8 codes, 3 fp32 lattice points minus the dither (u units)
 cudaError_t launch_decode_z(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_decode_a2(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_decode_d4(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_decode_e8(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 
 int num_sms();
+
+// dense-rotation KV variant (hq_dense.cu): forward rotation to normalised coefficients, inverse
+// rotation of decoded lattice points, and the forward pass's non-finite count into the status word
+cudaError_t launch_rotate(const void* x, bool bf16, const float* Q, float beta, int64_t rows, float* u,
+                          uint16_t* scale, uint32_t* nonfinite, cudaStream_t st);
+cudaError_t launch_unrotate(const float* p, const float* Q, const uint16_t* scale, float beta, int64_t rows, void* y,
+                            bool bf16, cudaStream_t st);
+cudaError_t launch_merge_nonfinite(void* ws, const uint32_t* nonfinite, cudaStream_t st);
 
 // 2-D tensor map of a row-major [rows, cols] tensor of es-byte elements: box [box_rows][128 bytes],
 // 128-byte swizzle (hq_api.cu)

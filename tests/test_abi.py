@@ -69,3 +69,27 @@ def test_calls_reject_bad_arguments_without_a_gpu(libhq):
     p = hq.params(128, hq.Z, 0.3)
     assert L.hq_quantize_coeffs(ctypes.c_void_p(16), 8, ctypes.byref(p), 3, 0, None, ctypes.byref(cs),
                                 ctypes.c_void_p(256), 1 << 20, None) == 1   # kv must be 0, 1 or 2
+
+
+def test_dense_entry_points_check_arguments_without_a_gpu(libhq):
+    import post_quantization_tile_b200 as hq
+    L = hq.lib()
+    need = L.hq_kv_dense_workspace_bytes(1000)
+    assert need % 256 == 0 and need >= 1000 * 512 + 256 + L.hq_workspace_bytes(1000, 128, ctypes.byref(hq.params(128)))
+    assert L.hq_kv_dense_workspace_bytes(0) == 0
+    cs = hq.CodeStruct()
+    q = ctypes.c_void_p(4096)
+    p = hq.params(64, hq.D4, 1.0)            # head dimension 64: not provided
+    assert L.hq_kv_encode_dense(ctypes.c_void_p(16), 0, 1, 1, 8, 64, 0, q, ctypes.byref(p), ctypes.byref(cs),
+                                ctypes.c_void_p(256), 1 << 20, None) == 2
+    p = hq.params(128, hq.D4, 1.0)
+    assert L.hq_kv_encode_dense(ctypes.c_void_p(16), 0, 1, 1, 8, 64, 0, q, ctypes.byref(p), ctypes.byref(cs),
+                                ctypes.c_void_p(256), 1 << 20, None) == 1   # D != tile
+    assert L.hq_kv_encode_dense(ctypes.c_void_p(16), 0, 1, 1, 8, 128, -1, q, ctypes.byref(p), ctypes.byref(cs),
+                                ctypes.c_void_p(256), 1 << 20, None) == 1   # negative first token
+    assert L.hq_kv_encode_dense(ctypes.c_void_p(16), 0, 1, 1, 8, 128, 0, None, ctypes.byref(p), ctypes.byref(cs),
+                                ctypes.c_void_p(256), 1 << 20, None) == 1   # no rotation
+    cs.kv = 1                                # not a dense code
+    cs.version = 2
+    assert L.hq_kv_decode_dense(ctypes.byref(cs), q, ctypes.c_void_p(256), 1, ctypes.c_void_p(256), 1 << 20,
+                                None) == 1
