@@ -11,11 +11,15 @@
 //
 // Both are one register-tiled binary32 product Y = A B over K = 128 (forward: A = x, B = Q^T;
 // inverse: A = p, B = Q): persistent blocks keep B in shared memory (64 KB), stage 64 rows of A
-// per step, and each of the 256 threads accumulates a 4 x 8 block of Y with k ascending.  Two
-// blocks share an SM, so one block's staging overlaps the other's FMAs.  The product stays on the
-// FP32 pipe: its outputs decide integer codes, and tensor-core accumulation (order and internal
-// precision unspecified) could not reproduce the reference chain.
+// per step, and each of the 256 threads accumulates a 4 x 8 block of Y with k ascending (paired
+// binary32 fma).  A warp covers 16 rows x 2 column groups, so its reads of B, two per k, are
+// broadcasts and shared-memory bandwidth stays below the FMA pipe's.  The next step's rows are loaded into registers while the
+// current step's FMAs run, and two blocks share an SM.  The product stays on the FP32 pipe: its
+// outputs decide integer codes, and tensor-core accumulation (order and internal precision
+// unspecified) could not reproduce the reference chain.
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "../../include/hq.h"
 #include "hq_common.cuh"
@@ -33,62 +37,102 @@ struct DenseSmem {
     float B[kDN][kDN];   // B[k][c]
     float A[kDBM][kDLD];  // A[r][k]
     float rs[kDBM];       // per-row factor: forward 1 / (s_hat beta), inverse s_hat beta
-    int zr[kDBM];         // forward: the row is coded as zeros (zero or non-finite vector)
 };
-
-// 4 consecutive elements of a row as binary32
-template <bool BF16>
-__device__ __forceinline__ float4 load4(const void* base, int64_t row, int col)
-{
-    if constexpr (BF16) {
-        const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + row * kDN + col);
-        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
-                           __uint_as_float(w.y & 0xFFFF0000u));
-    } else {
-        return *reinterpret_cast<const float4*>(static_cast<const float*>(base) + row * kDN + col);
-    }
-}
 
 // B into shared memory: forward B[k][c] = Q[c][k], inverse B[k][c] = Q[k][c]
 template <bool FWD>
 __device__ __forceinline__ void load_rotation(DenseSmem& sm, const float* Q)
 {
+#pragma unroll 16
     for (int idx = threadIdx.x; idx < kDN * kDN; idx += kDThreads) {
         const int k = idx / kDN, c = idx % kDN;
         sm.B[k][c] = FWD ? Q[c * kDN + k] : Q[k * kDN + c];
     }
 }
 
-// acc[i][0..3] += A[r_i][k] B[k][c0 + 0..3], acc[i][4..7] += A[r_i][k] B[k][c0 + 64 + 0..3] for
-// k = 0 .. 127 in order; rows r_i = 4 ty + i
+// acc[i][0..3] += A[r_i][k] B[k][4 tx + 0..3], acc[i][4..7] += A[r_i][k] B[k][64 + 4 tx + 0..3] for
+// k = 0 .. 127 in order; rows r_i = ty + 16 i.  Lane l of warp w: ty = l % 16, tx = 2 w + l / 16,
+// so a warp reads 16 consecutive rows of A (row pitch 132 floats: every bank once per 8 rows) and
+// only two distinct 16-byte pieces of each half of B[k] (broadcast)
+__device__ __forceinline__ void thread_tile(int tid, int& ty, int& tx)
+{
+    const int lane = tid & 31, warp = tid >> 5;
+    ty = lane & 15;
+    tx = 2 * warp + (lane >> 4);
+}
+
 __device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, float (&acc)[4][8])
 {
+    // paired binary32 fma (two independent fma, each rounded once: the same values as scalar fma)
+    float2 c[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+        for (int j = 0; j < 4; ++j) c[i][j] = make_float2(0.0f, 0.0f);
 #pragma unroll 2
     for (int k = 0; k < kDN; k += 4) {
         float4 a[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.A[4 * ty + i][k]);
+        for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.A[ty + 16 * i][k]);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             const float4 b0 = *reinterpret_cast<const float4*>(&sm.B[k + kk][4 * tx]);
             const float4 b1 = *reinterpret_cast<const float4*>(&sm.B[k + kk][64 + 4 * tx]);
+            const float2 bp[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                                  make_float2(b1.z, b1.w)};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float av = kk == 0 ? a[i].x : (kk == 1 ? a[i].y : (kk == 2 ? a[i].z : a[i].w));
-                acc[i][0] = __fmaf_rn(av, b0.x, acc[i][0]);
-                acc[i][1] = __fmaf_rn(av, b0.y, acc[i][1]);
-                acc[i][2] = __fmaf_rn(av, b0.z, acc[i][2]);
-                acc[i][3] = __fmaf_rn(av, b0.w, acc[i][3]);
-                acc[i][4] = __fmaf_rn(av, b1.x, acc[i][4]);
-                acc[i][5] = __fmaf_rn(av, b1.y, acc[i][5]);
-                acc[i][6] = __fmaf_rn(av, b1.z, acc[i][6]);
-                acc[i][7] = __fmaf_rn(av, b1.w, acc[i][7]);
+                const float2 a2 = make_float2(av, av);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) c[i][j] = __ffma2_rn(a2, bp[j], c[i][j]);
             }
         }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[i][2 * j] = c[i][j].x;
+            acc[i][2 * j + 1] = c[i][j].y;
+        }
+}
+
+// Rows of one step in registers: warp w holds rows 8 w .. 8 w + 7 of the step, lane l elements
+// 4 l .. 4 l + 3 of each (bf16 kept packed).  The next step's rows are loaded before the current
+// step's product, so the loads are in flight while the FMAs run.
+template <bool BF16>
+struct RowRegs {
+    using T = typename std::conditional<BF16, uint2, float4>::type;
+    T w[kDBM / 8];
+};
+
+template <bool BF16>
+__device__ __forceinline__ void prefetch_rows(RowRegs<BF16>& rg, const void* base, int64_t r0, int64_t rows)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int rr = 0; rr < kDBM / 8; ++rr) {
+        const int64_t gr = r0 + warp * (kDBM / 8) + rr;
+        if constexpr (BF16) {
+            rg.w[rr] = gr < rows ? *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + gr * kDN + 4 * lane)
+                                 : make_uint2(0u, 0u);
+        } else {
+            rg.w[rr] = gr < rows ? *reinterpret_cast<const float4*>(static_cast<const float*>(base) + gr * kDN + 4 * lane)
+                                 : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+    }
+}
+
+template <bool BF16>
+__device__ __forceinline__ float4 row_value(const RowRegs<BF16>& rg, int rr)
+{
+    if constexpr (BF16) {
+        const uint2 w = rg.w[rr];
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
+                           __uint_as_float(w.y & 0xFFFF0000u));
+    } else {
+        return rg.w[rr];
     }
 }
 
@@ -101,60 +145,83 @@ __global__ void __launch_bounds__(kDThreads, 2) rotate_kernel(const void* __rest
     extern __shared__ __align__(16) unsigned char smem_raw[];
     DenseSmem& sm = *reinterpret_cast<DenseSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ty = tid / 16, tx = tid % 16;
-    load_rotation<true>(sm, Q);
+    int ty, tx;
+    thread_tile(tid, ty, tx);
     const int64_t steps = (rows + kDBM - 1) / kDBM;
+    RowRegs<BF16> rg;
+    if ((int64_t)blockIdx.x < steps) prefetch_rows<BF16>(rg, x, (int64_t)blockIdx.x * kDBM, rows);
+    load_rotation<true>(sm, Q);
     for (int64_t st = blockIdx.x; st < steps; st += gridDim.x) {
         const int64_t r0 = st * kDBM;
-        // ---- stage 8 rows per warp, lane l holding elements 4l .. 4l + 3; RMS by the pairwise tree
-#pragma unroll 1
-        for (int rr = 0; rr < kDBM / 8; ++rr) {
-            const int rl = warp * (kDBM / 8) + rr;
-            const int64_t gr = r0 + rl;
-            float4 f = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (gr < rows) f = load4<BF16>(x, gr, 4 * lane);
-            *reinterpret_cast<float4*>(&sm.A[rl][4 * lane]) = f;
-            const bool fin = isfinite(f.x) && isfinite(f.y) && isfinite(f.z) && isfinite(f.w);
-            const bool all_fin = __all_sync(0xffffffffu, fin);
-            // q_i = x_i^2; q[i] += q[i + h] for h = 1, 2 in-thread, then h = 4 .. 64 across lanes
-            float q = __fadd_rn(__fadd_rn(__fmul_rn(f.x, f.x), __fmul_rn(f.y, f.y)),
-                                __fadd_rn(__fmul_rn(f.z, f.z), __fmul_rn(f.w, f.w)));
+        // ---- stage the rows; RMS of each by the pairwise tree (q_i = x_i^2; q[i] += q[i + h] for
+        // h = 1, 2 in-thread, then h = 4 .. 64 across lanes), the warp's 8 trees interleaved
+        constexpr int RW = kDBM / 8;
+        float q[RW];
+        uint32_t bad = 0u;  // bit rr: row rr holds a non-finite element
 #pragma unroll
-            for (int m = 1; m < 32; m *= 2) {
-                const float o = __shfl_down_sync(0xffffffffu, q, m);
-                if ((lane & (2 * m - 1)) == 0) q = __fadd_rn(q, o);
-            }
-            if (lane == 0) {
-                const float s = all_fin ? __fsqrt_rn(__fmul_rn(q, 1.0f / (float)kDN)) : 0.0f;
-                uint16_t sb = f32_to_bf16_bits(s);
-                const float sh = __uint_as_float((uint32_t)sb << 16);
-                int zero = 0;
-                if (!all_fin || !isfinite(sh)) {
-                    sb = 0;
-                    zero = 1;
-                    if (gr < rows) atomicAdd(nonfinite, 1u);
-                } else if (sh < 1.2621774483536189e-29f) {  // 2^-96: coded as an all-zero tile
-                    sb = 0;
-                    zero = 1;
-                }
-                sm.zr[rl] = zero;
-                sm.rs[rl] = zero ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sh, beta));
-                if (gr < rows) scale[gr] = sb;
+        for (int rr = 0; rr < RW; ++rr) {
+            const float4 f = row_value<BF16>(rg, rr);
+            q[rr] = __fadd_rn(__fadd_rn(__fmul_rn(f.x, f.x), __fmul_rn(f.y, f.y)),
+                              __fadd_rn(__fmul_rn(f.z, f.z), __fmul_rn(f.w, f.w)));
+            const bool fin = isfinite(f.x) && isfinite(f.y) && isfinite(f.z) && isfinite(f.w);
+            bad |= (__all_sync(0xffffffffu, fin) ? 0u : 1u) << rr;
+        }
+#pragma unroll
+        for (int m = 1; m < 32; m *= 2) {
+#pragma unroll
+            for (int rr = 0; rr < RW; ++rr) {
+                const float o = __shfl_down_sync(0xffffffffu, q[rr], m);
+                if ((lane & (2 * m - 1)) == 0) q[rr] = __fadd_rn(q[rr], o);
             }
         }
+        // lane rr < 8 finishes row rr: scale bits and 1 / (s_hat beta)
+        float tot = 0.0f;
+#pragma unroll
+        for (int rr = 0; rr < RW; ++rr) {
+            const float t = __shfl_sync(0xffffffffu, q[rr], 0);
+            if (lane == rr) tot = t;
+        }
+        bool zero = false, nonfin = false;
+        if (lane < RW) {
+            const int rl = warp * RW + lane;
+            const int64_t gr = r0 + rl;
+            const bool all_fin = ((bad >> lane) & 1u) == 0u;
+            const float s = all_fin ? __fsqrt_rn(__fmul_rn(tot, 1.0f / (float)kDN)) : 0.0f;
+            uint16_t sb = f32_to_bf16_bits(s);
+            const float sh = __uint_as_float((uint32_t)sb << 16);
+            if (!all_fin || !isfinite(sh)) {
+                sb = 0;
+                zero = true;
+                nonfin = gr < rows;
+            } else if (sh < 1.2621774483536189e-29f) {  // 2^-96: coded as an all-zero tile
+                sb = 0;
+                zero = true;
+            }
+            sm.rs[rl] = zero ? 0.0f : __fdiv_rn(1.0f, __fmul_rn(sh, beta));
+            if (gr < rows) scale[gr] = sb;
+        }
+        const uint32_t nf = __popc(__ballot_sync(0xffffffffu, nonfin));
+        if (lane == 0 && nf) atomicAdd(nonfinite, nf);
+        // rows coded as zeros are staged as zeros: their products are +0 exactly, and so is u
+        const uint32_t zmask = __ballot_sync(0xffffffffu, zero);
+#pragma unroll
+        for (int rr = 0; rr < RW; ++rr) {
+            const float4 f = ((zmask >> rr) & 1u) ? make_float4(0.0f, 0.0f, 0.0f, 0.0f) : row_value<BF16>(rg, rr);
+            *reinterpret_cast<float4*>(&sm.A[warp * RW + rr][4 * lane]) = f;
+        }
         __syncthreads();
+        if (st + gridDim.x < steps) prefetch_rows<BF16>(rg, x, (st + gridDim.x) * kDBM, rows);
         float acc[4][8];
         product(sm, ty, tx, acc);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int rl = 4 * ty + i;
+            const int rl = ty + 16 * i;
             const int64_t gr = r0 + rl;
             if (gr >= rows) continue;
             const float g = sm.rs[rl];
-            const bool z = sm.zr[rl] != 0;
             float v[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = z ? 0.0f : __fmul_rn(acc[i][j], g);
+            for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(acc[i][j], g);
             float* dst = u + gr * kDN;
             *reinterpret_cast<float4*>(dst + 4 * tx) = make_float4(v[0], v[1], v[2], v[3]);
             *reinterpret_cast<float4*>(dst + 64 + 4 * tx) = make_float4(v[4], v[5], v[6], v[7]);
@@ -172,26 +239,30 @@ __global__ void __launch_bounds__(kDThreads, 2) unrotate_kernel(const float* __r
     extern __shared__ __align__(16) unsigned char smem_raw[];
     DenseSmem& sm = *reinterpret_cast<DenseSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ty = tid / 16, tx = tid % 16;
-    load_rotation<false>(sm, Q);
+    int ty, tx;
+    thread_tile(tid, ty, tx);
     const int64_t steps = (rows + kDBM - 1) / kDBM;
+    RowRegs<false> rg;
+    if ((int64_t)blockIdx.x < steps) prefetch_rows<false>(rg, p, (int64_t)blockIdx.x * kDBM, rows);
+    load_rotation<false>(sm, Q);
     for (int64_t st = blockIdx.x; st < steps; st += gridDim.x) {
         const int64_t r0 = st * kDBM;
-#pragma unroll 2
+#pragma unroll
         for (int rr = 0; rr < kDBM / 8; ++rr) {
             const int rl = warp * (kDBM / 8) + rr;
-            const int64_t gr = r0 + rl;
-            float4 f = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (gr < rows) f = load4<false>(p, gr, 4 * lane);
-            *reinterpret_cast<float4*>(&sm.A[rl][4 * lane]) = f;
-            if (lane == 0) sm.rs[rl] = gr < rows ? __fmul_rn(__uint_as_float((uint32_t)scale[gr] << 16), beta) : 0.0f;
+            *reinterpret_cast<float4*>(&sm.A[rl][4 * lane]) = rg.w[rr];
+        }
+        if (tid < kDBM) {
+            const int64_t gr = r0 + tid;
+            sm.rs[tid] = gr < rows ? __fmul_rn(__uint_as_float((uint32_t)scale[gr] << 16), beta) : 0.0f;
         }
         __syncthreads();
+        if (st + gridDim.x < steps) prefetch_rows<false>(rg, p, (st + gridDim.x) * kDBM, rows);
         float acc[4][8];
         product(sm, ty, tx, acc);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int rl = 4 * ty + i;
+            const int rl = ty + 16 * i;
             const int64_t gr = r0 + rl;
             if (gr >= rows) continue;
             const float h = sm.rs[rl];
