@@ -12,11 +12,10 @@
 // Both are one register-tiled binary32 product Y = A B over K = 128 (forward: A = x, B = Q^T;
 // inverse: A = p, B = Q): persistent blocks keep B in shared memory (64 KB), stage 64 rows of A
 // per step, and each of the 256 threads accumulates a 4 x 8 block of Y with k ascending (paired
-// binary32 fma).  A warp covers 16 rows x 2 column groups, so its reads of B, two per k, are
-// broadcasts and shared-memory bandwidth stays below the FMA pipe's.  The next step's rows are loaded into registers while the
-// current step's FMAs run, and two blocks share an SM.  The product stays on the FP32 pipe: its
-// outputs decide integer codes, and tensor-core accumulation (order and internal precision
-// unspecified) could not reproduce the reference chain.
+// binary32 fma: two independent fma per instruction, each rounded once).  The next step's rows
+// are loaded into registers while the current step's FMAs run, and two blocks share an SM.  The
+// product stays on the FP32 pipe: its outputs decide integer codes, and tensor-core accumulation
+// (order and internal precision unspecified) could not reproduce the reference chain.
 #include <cuda_runtime.h>
 
 #include <type_traits>
@@ -51,14 +50,16 @@ __device__ __forceinline__ void load_rotation(DenseSmem& sm, const float* Q)
 }
 
 // acc[i][0..3] += A[r_i][k] B[k][4 tx + 0..3], acc[i][4..7] += A[r_i][k] B[k][64 + 4 tx + 0..3] for
-// k = 0 .. 127 in order; rows r_i = ty + 16 i.  Lane l of warp w: ty = l % 16, tx = 2 w + l / 16,
-// so a warp reads 16 consecutive rows of A (row pitch 132 floats: every bank once per 8 rows) and
-// only two distinct 16-byte pieces of each half of B[k] (broadcast)
+// k = 0 .. 127 in order; rows r_i = ty + 16 i.  Lane l of warp w: tx = 4 (w % 4) + l % 4,
+// ty = 8 (w / 4) + l / 4, so a warp reads 8 consecutive rows of A (row pitch 132 floats: 32
+// distinct banks) and 64 contiguous bytes of each half of B[k].  (A warp of 16 rows x 2 column
+// groups, whose reads of B are broadcasts, needs fewer shared-memory wavefronts but measured 3%
+// slower.)
 __device__ __forceinline__ void thread_tile(int tid, int& ty, int& tx)
 {
     const int lane = tid & 31, warp = tid >> 5;
-    ty = lane & 15;
-    tx = 2 * warp + (lane >> 4);
+    tx = 4 * (warp & 3) + (lane & 3);
+    ty = 8 * (warp >> 2) + (lane >> 2);
 }
 
 __device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, float (&acc)[4][8])
