@@ -155,3 +155,48 @@ def test_dense_codes_refuse_the_other_decoders_and_other_sizes(hq, Q):
     rc = L.hq_kv_encode_dense(ctypes.c_void_p(xk.data_ptr()), 0, 1, 1, 8, 128, 0, ctypes.c_void_p(Qd.data_ptr()),
                               ctypes.byref(p128), ctypes.byref(cs128), w.ptr(), need - 256, None)
     assert rc == 1   # HQ_ERR_ARG
+
+
+def test_dense_dither_unbiased_on_gpu(hq, Q):
+    """Per key vector and query, the inner-product error over fresh dithers has mean zero (the
+    dither keeps the variant unbiased whatever the rotation); 512 keys x 32 queries, 192 seeds."""
+    kb = W.kv_keys(1, 4, 128, 128, seed=2)
+    keys = t_bf16(kb)
+    x = keys.float().reshape(-1, 128).double()
+    q = torch.from_numpy(W.queries(32, 128, seed=3)).cuda()
+    Qd = torch.from_numpy(Q).cuda()
+    M = 192
+    E = torch.zeros(M, x.shape[0], 32, dtype=torch.float64, device="cuda")
+    for m in range(M):
+        code = hq.kv_encode_dense(keys, Qd, step=1.6, seed=7000 + m)
+        y = hq.kv_decode_dense(code, Qd, dtype=torch.float32).double()
+        E[m] = (y - x) @ q.T
+    assert hq.status(code.ws)[0] == 0
+    z = E.mean(0) / (E.std(0) / np.sqrt(M))
+    assert (z.abs() > 4.5).float().mean().item() <= 1e-3
+
+
+def test_dense_replay_from_a_graph(hq, Q):
+    kb = W.kv_keys(1, 2, 96, 128, seed=8)
+    keys = t_bf16(kb)
+    Qd = torch.from_numpy(Q).cuda()
+    ref = hq.kv_encode_dense(keys, Qd, step=0.8, seed=3, lattice=oracle.E8)
+    y_ref = hq.kv_decode_dense(ref, Qd, dtype=torch.float32)
+    code = hq.alloc_code(keys.numel() // 128, 128, hq.params(128, oracle.E8, 0.8, seed=3))
+    ws = hq.Workspace(hq.lib().hq_kv_dense_workspace_bytes(keys.numel() // 128))
+    y = torch.empty_like(y_ref)
+    hq.kv_encode_dense(keys, Qd, step=0.8, seed=3, lattice=oracle.E8, out=code, ws=ws)   # warm-up
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        hq.kv_encode_dense(keys, Qd, step=0.8, seed=3, lattice=oracle.E8, out=code, ws=ws)
+        hq.kv_decode_dense(code, Qd, out=y, ws=ws)
+    code.bits.zero_()
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert hq.status(ws)[0] == 0
+    assert torch.equal(code.bits[:ref.total_words()], ref.bits[:ref.total_words()])
+    assert torch.equal(code.scale, ref.scale)
+    assert torch.equal(y, y_ref)
