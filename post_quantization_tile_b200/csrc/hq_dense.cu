@@ -11,8 +11,10 @@
 //
 // Both are one register-tiled binary32 product Y = A B over K = 128 (forward: A = x, B = Q^T;
 // inverse: A = p, B = Q): persistent blocks keep B in shared memory (64 KB), stage 64 rows of A
-// per step, and each of the 256 threads accumulates a 4 x 8 block of Y with k ascending (paired
-// binary32 fma: two independent fma per instruction, each rounded once).  The next step's rows
+// per step, and each of the 128 threads accumulates an 8 x 8 block of Y with k ascending (paired
+// binary32 fma: two independent fma per instruction, each rounded once).  Eight rows per thread
+// halve the shared-memory loads per fma against four, which kept shared memory busier than the
+// FMA pipes.  The next step's rows
 // are loaded into registers while the current step's FMAs run, and two blocks share an SM.  The
 // product stays on the FP32 pipe: its outputs decide integer codes, and tensor-core accumulation
 // (order and internal precision unspecified) could not reproduce the reference chain.
@@ -29,7 +31,10 @@ namespace {
 
 constexpr int kDN = 128;       // vector length (head dimension)
 constexpr int kDBM = 64;       // rows staged per step
-constexpr int kDThreads = 256;
+constexpr int kDThreads = 128;
+constexpr int kDWarps = kDThreads / 32;
+constexpr int kRW = kDBM / kDWarps;  // rows each warp stages per step
+constexpr int kTR = kDBM / 8;        // rows per thread in the product (row groups of 8)
 constexpr int kDLD = kDN + 4;  // padded row of the staged tile (floats)
 
 struct DenseSmem {
@@ -50,31 +55,29 @@ __device__ __forceinline__ void load_rotation(DenseSmem& sm, const float* Q)
 }
 
 // acc[i][0..3] += A[r_i][k] B[k][4 tx + 0..3], acc[i][4..7] += A[r_i][k] B[k][64 + 4 tx + 0..3] for
-// k = 0 .. 127 in order; rows r_i = ty + 16 i.  Lane l of warp w: tx = 4 (w % 4) + l % 4,
-// ty = 8 (w / 4) + l / 4, so a warp reads 8 consecutive rows of A (row pitch 132 floats: 32
-// distinct banks) and 64 contiguous bytes of each half of B[k].  (A warp of 16 rows x 2 column
-// groups, whose reads of B are broadcasts, needs fewer shared-memory wavefronts but measured 3%
-// slower.)
+// k = 0 .. 127 in order; rows r_i = ty + 8 i.  Lane l of warp w: tx = 4 w + l % 4, ty = l / 4, so a
+// warp reads 8 consecutive rows of A (row pitch 132 floats: 32 distinct banks) and 64 contiguous
+// bytes of each half of B[k].
 __device__ __forceinline__ void thread_tile(int tid, int& ty, int& tx)
 {
     const int lane = tid & 31, warp = tid >> 5;
-    tx = 4 * (warp & 3) + (lane & 3);
-    ty = 8 * (warp >> 2) + (lane >> 2);
+    tx = 4 * warp + (lane & 3);
+    ty = lane >> 2;
 }
 
-__device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, float (&acc)[4][8])
+__device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, float (&acc)[kTR][8])
 {
     // paired binary32 fma (two independent fma, each rounded once: the same values as scalar fma)
-    float2 c[4][4];
+    float2 c[kTR][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kTR; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) c[i][j] = make_float2(0.0f, 0.0f);
 #pragma unroll 2
     for (int k = 0; k < kDN; k += 4) {
-        float4 a[4];
+        float4 a[kTR];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.A[ty + 16 * i][k]);
+        for (int i = 0; i < kTR; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.A[ty + 8 * i][k]);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             const float4 b0 = *reinterpret_cast<const float4*>(&sm.B[k + kk][4 * tx]);
@@ -82,7 +85,7 @@ __device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, flo
             const float2 bp[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
                                   make_float2(b1.z, b1.w)};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < kTR; ++i) {
                 const float av = kk == 0 ? a[i].x : (kk == 1 ? a[i].y : (kk == 2 ? a[i].z : a[i].w));
                 const float2 a2 = make_float2(av, av);
 #pragma unroll
@@ -91,7 +94,7 @@ __device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, flo
         }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kTR; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             acc[i][2 * j] = c[i][j].x;
@@ -99,13 +102,13 @@ __device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, flo
         }
 }
 
-// Rows of one step in registers: warp w holds rows 8 w .. 8 w + 7 of the step, lane l elements
-// 4 l .. 4 l + 3 of each (bf16 kept packed).  The next step's rows are loaded before the current
+// Rows of one step in registers: warp w holds rows kRW w .. kRW w + kRW - 1 of the step, lane l
+// elements 4 l .. 4 l + 3 of each (bf16 kept packed).  The next step's rows are loaded before the current
 // step's product, so the loads are in flight while the FMAs run.
 template <bool BF16>
 struct RowRegs {
     using T = typename std::conditional<BF16, uint2, float4>::type;
-    T w[kDBM / 8];
+    T w[kRW];
 };
 
 template <bool BF16>
@@ -113,8 +116,8 @@ __device__ __forceinline__ void prefetch_rows(RowRegs<BF16>& rg, const void* bas
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int rr = 0; rr < kDBM / 8; ++rr) {
-        const int64_t gr = r0 + warp * (kDBM / 8) + rr;
+    for (int rr = 0; rr < kRW; ++rr) {
+        const int64_t gr = r0 + warp * kRW + rr;
         if constexpr (BF16) {
             rg.w[rr] = gr < rows ? *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + gr * kDN + 4 * lane)
                                  : make_uint2(0u, 0u);
@@ -155,8 +158,8 @@ __global__ void __launch_bounds__(kDThreads, 2) rotate_kernel(const void* __rest
     for (int64_t st = blockIdx.x; st < steps; st += gridDim.x) {
         const int64_t r0 = st * kDBM;
         // ---- stage the rows; RMS of each by the pairwise tree (q_i = x_i^2; q[i] += q[i + h] for
-        // h = 1, 2 in-thread, then h = 4 .. 64 across lanes), the warp's 8 trees interleaved
-        constexpr int RW = kDBM / 8;
+        // h = 1, 2 in-thread, then h = 4 .. 64 across lanes), the warp's trees interleaved
+        constexpr int RW = kRW;
         float q[RW];
         uint32_t bad = 0u;  // bit rr: row rr holds a non-finite element
 #pragma unroll
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(kDThreads, 2) rotate_kernel(const void* __rest
                 if ((lane & (2 * m - 1)) == 0) q[rr] = __fadd_rn(q[rr], o);
             }
         }
-        // lane rr < 8 finishes row rr: scale bits and 1 / (s_hat beta)
+        // lane rr < RW finishes row rr: scale bits and 1 / (s_hat beta)
         float tot = 0.0f;
 #pragma unroll
         for (int rr = 0; rr < RW; ++rr) {
@@ -212,11 +215,11 @@ __global__ void __launch_bounds__(kDThreads, 2) rotate_kernel(const void* __rest
         }
         __syncthreads();
         if (st + gridDim.x < steps) prefetch_rows<BF16>(rg, x, (st + gridDim.x) * kDBM, rows);
-        float acc[4][8];
+        float acc[kTR][8];
         product(sm, ty, tx, acc);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int rl = ty + 16 * i;
+        for (int i = 0; i < kTR; ++i) {
+            const int rl = ty + 8 * i;
             const int64_t gr = r0 + rl;
             if (gr >= rows) continue;
             const float g = sm.rs[rl];
@@ -249,8 +252,8 @@ __global__ void __launch_bounds__(kDThreads, 2) unrotate_kernel(const float* __r
     for (int64_t st = blockIdx.x; st < steps; st += gridDim.x) {
         const int64_t r0 = st * kDBM;
 #pragma unroll
-        for (int rr = 0; rr < kDBM / 8; ++rr) {
-            const int rl = warp * (kDBM / 8) + rr;
+        for (int rr = 0; rr < kRW; ++rr) {
+            const int rl = warp * kRW + rr;
             *reinterpret_cast<float4*>(&sm.A[rl][4 * lane]) = rg.w[rr];
         }
         if (tid < kDBM) {
@@ -259,11 +262,11 @@ __global__ void __launch_bounds__(kDThreads, 2) unrotate_kernel(const float* __r
         }
         __syncthreads();
         if (st + gridDim.x < steps) prefetch_rows<false>(rg, p, (st + gridDim.x) * kDBM, rows);
-        float acc[4][8];
+        float acc[kTR][8];
         product(sm, ty, tx, acc);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int rl = ty + 16 * i;
+        for (int i = 0; i < kTR; ++i) {
+            const int rl = ty + 8 * i;
             const int64_t gr = r0 + rl;
             if (gr >= rows) continue;
             const float h = sm.rs[rl];
