@@ -96,8 +96,8 @@ int64_t bound_words(int64_t rows, int64_t cols, int32_t n)
 size_t ws_bytes_for(int64_t rows, int64_t cols, int32_t n)
 {
     Geometry g;
-    // the encoder with the most items for this tile (bf16 input shares a tile the most)
-    if (!geometry(rows, cols, n, g, n == 64 ? 1 : (n == 256 ? 2 : enc_tpt(128, 0)))) return 0;
+    // the encoder with the most items for this tile (the one that shares a tile the most)
+    if (!geometry(rows, cols, n, g, n == 64 ? 1 : (n == 256 ? 2 : enc_tpt_max(128)))) return 0;
     return sizeof(WsHeader) + (size_t)g.items * 8u;
 }
 

@@ -81,10 +81,22 @@ static_assert(sizeof(RateSearch) <= 192, "rate search state");
 #ifndef HQ_DEC_STAGES
 #define HQ_DEC_STAGES 1
 #endif
+// fp32 coefficients at n = 128: two threads per tile halve the TMA stage (64 rows of 512 bytes),
+// so three blocks fit an SM instead of two
+#ifndef HQ_ENC_TPT128_COEF
+#define HQ_ENC_TPT128_COEF 2
+#endif
 // src: 0 bf16 weight, 1 fp32 weight, 2 fp32 coefficients (fp32 weights keep one thread per tile)
 __host__ __device__ constexpr int enc_tpt(int n, int src)
 {
-    return (n == 256 || (n == 128 && src != 1 && HQ_ENC_TPT128 == 2)) ? 2 : 1;
+    return (n == 256 || (n == 128 && ((src == 0 && HQ_ENC_TPT128 == 2) || (src == 2 && HQ_ENC_TPT128_COEF == 2))))
+               ? 2
+               : 1;
+}
+// the most threads per tile any encoder source uses (the workspace holds one look-back slot per item)
+__host__ __device__ constexpr int enc_tpt_max(int n)
+{
+    return enc_tpt(n, 0) > enc_tpt(n, 2) ? enc_tpt(n, 0) : enc_tpt(n, 2);
 }
 __host__ __device__ constexpr int dec_tpt(int n) { return (n == 256 || (n == 128 && HQ_DEC_TPT128 == 2)) ? 2 : 1; }
 
