@@ -14,10 +14,10 @@
 // per step, and each of the 128 threads accumulates an 8 x 8 block of Y with k ascending (paired
 // binary32 fma: two independent fma per instruction, each rounded once).  Eight rows per thread
 // halve the shared-memory loads per fma against four, which kept shared memory busier than the
-// FMA pipes.  The next step's rows
-// are loaded into registers while the current step's FMAs run, and two blocks share an SM.  The
-// product stays on the FP32 pipe: its outputs decide integer codes, and tensor-core accumulation
-// (order and internal precision unspecified) could not reproduce the reference chain.
+// FMA pipes.  The next step's rows are loaded into registers while the current step's FMAs run,
+// and two blocks share an SM.  The product stays on the FP32 pipe: its outputs decide integer
+// codes, and tensor-core accumulation (order and internal precision unspecified) could not
+// reproduce the reference chain.
 #include <cuda_runtime.h>
 
 #include <type_traits>
@@ -29,13 +29,13 @@
 namespace hq {
 namespace {
 
-constexpr int kDN = 128;       // vector length (head dimension)
-constexpr int kDBM = 64;       // rows staged per step
+constexpr int kDN = 128;             // vector length (head dimension)
+constexpr int kDBM = 64;             // rows staged per step
 constexpr int kDThreads = 128;
 constexpr int kDWarps = kDThreads / 32;
 constexpr int kRW = kDBM / kDWarps;  // rows each warp stages per step
 constexpr int kTR = kDBM / 8;        // rows per thread in the product (row groups of 8)
-constexpr int kDLD = kDN + 4;  // padded row of the staged tile (floats)
+constexpr int kDLD = kDN + 4;        // padded row of the staged tile (floats)
 
 struct DenseSmem {
     float B[kDN][kDN];   // B[k][c]
@@ -103,8 +103,8 @@ __device__ __forceinline__ void product(const DenseSmem& sm, int ty, int tx, flo
 }
 
 // Rows of one step in registers: warp w holds rows kRW w .. kRW w + kRW - 1 of the step, lane l
-// elements 4 l .. 4 l + 3 of each (bf16 kept packed).  The next step's rows are loaded before the current
-// step's product, so the loads are in flight while the FMAs run.
+// elements 4 l .. 4 l + 3 of each (bf16 kept packed).  The next step's rows are loaded before the
+// current step's product, so the loads are in flight while the FMAs run.
 template <bool BF16>
 struct RowRegs {
     using T = typename std::conditional<BF16, uint2, float4>::type;
