@@ -93,6 +93,14 @@ int64_t bound_words(int64_t rows, int64_t cols, int32_t n)
     return (words + 3) & ~(int64_t)3;
 }
 
+// workspace of one encoder source: the header and one look-back slot per item
+size_t ws_bytes_for_src(int64_t rows, int64_t cols, int32_t n, int src)
+{
+    Geometry g;
+    if (!geometry(rows, cols, n, g, n == 64 ? 1 : (n == 256 ? 2 : enc_tpt(128, src)))) return 0;
+    return sizeof(WsHeader) + (size_t)g.items * 8u;
+}
+
 size_t ws_bytes_for(int64_t rows, int64_t cols, int32_t n)
 {
     Geometry g;
@@ -176,7 +184,7 @@ hq_status_t plan_encode(const void* x, int src, int64_t rows, int64_t cols, cons
     if (src == 1 && prm.tile == 256) return HQ_ERR_UNSUPPORTED;
     if (src == 2 && cols != prm.tile) return HQ_ERR_ARG;
     if (!x || !aligned16(x) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
-    if (ws_bytes < ws_bytes_for(rows, cols, prm.tile)) return HQ_ERR_ARG;
+    if (ws_bytes < sizeof(WsHeader) + (size_t)g.items * 8u) return HQ_ERR_ARG;  // this source's items
     if (!count) {
         if (!out || !out->meta || !out->chunk_word || !out->bits || out->cap_words < 1) return HQ_ERR_ARG;
         if (src != 2 && !out->scale) return HQ_ERR_ARG;
@@ -452,6 +460,10 @@ bool tensor_map_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
     return make_map(m, base, rows, cols, es, box_rows);
 }
 bool device_of(const void* p) { return use_device_of(p); }
+size_t encode_workspace_bytes(int64_t rows, int64_t cols, int32_t n, int src)
+{
+    return valid_tile(n) ? ws_bytes_for_src(rows, cols, n, src) : 0;
+}
 
 }  // namespace hq
 

@@ -36,5 +36,8 @@ cudaError_t launch_merge_nonfinite(void* ws, const uint32_t* nonfinite, cudaStre
 bool tensor_map_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int es, int box_rows);
 // make the device that owns p current (hq_api.cu)
 bool device_of(const void* p);
+// workspace bytes of the encoder for one source (0 bf16, 1 fp32 weights, 2 coefficients); 0 if
+// the shape is invalid (hq_api.cu)
+size_t encode_workspace_bytes(int64_t rows, int64_t cols, int32_t n, int src);
 
 }  // namespace hq

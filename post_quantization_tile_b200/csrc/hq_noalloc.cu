@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "../../include/hq.h"
+#include "hq_launch.h"
 
 namespace {
 
@@ -43,8 +44,9 @@ extern "C" hq_status_t hq_encode_noalloc(const void* x, hq_dtype_t dtype, int64_
                                          const hq_params_t* p, hq_code_t* out, uint32_t* status_out, void* stream)
 {
     if (!p || !x) return HQ_ERR_ARG;
-    // the scratch holds a 64-byte header and 8 bytes per block of tiles
-    const size_t need = hq_workspace_bytes(rows, cols, p);
+    if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
+    // the scratch holds a 64-byte header and 8 bytes per block of tiles of this weight encoder
+    const size_t need = hq::encode_workspace_bytes(rows, cols, p->tile, dtype == HQ_BF16 ? 0 : 1);
     if (need == 0) return HQ_ERR_ARG;
     if (need > kNoallocScratchBytes) return HQ_ERR_RANGE;
     // make the device that holds x current, then find the scratch on that device
