@@ -58,19 +58,56 @@ def make_inputs():
 # ------------------------------------------------------------------------------------------------
 # CPU oracle arm (bounded sample)
 # ------------------------------------------------------------------------------------------------
-def oracle_sample(inputs, rows_per_matrix: int, steps: int):
+def oracle_sample(inputs, rows_per_matrix: int, steps: int, betas=None):
+    """The oracle's encode + decode of the first rows of each matrix, `steps` passes, timed on one
+    host thread.  Returns GB/s of bf16 input, seconds, scalars and the last pass's (code, x_hat)
+    per matrix."""
     import oracle
     t_total, elems = 0.0, 0
+    last = []
     for _ in range(steps):
-        for x in inputs:
+        last = []
+        for i, x in enumerate(inputs):
             xs = np.ascontiguousarray(x[:rows_per_matrix])
+            beta = betas[i] if betas is not None else 0.28
             t0 = time.perf_counter()
-            code = oracle.encode(xs, TILE, oracle.E8, 0.28, SEED)
-            oracle.decode(code)
+            code = oracle.encode(xs, TILE, oracle.E8, beta, SEED)
+            xo, _ = oracle.decode(code)
             t_total += time.perf_counter() - t0
             elems += xs.size
+            last.append((code, xo))
     gbs = elems * 2 / t_total / 1e9
-    return gbs, t_total, elems
+    return gbs, t_total, elems, last
+
+
+def parity_vs_oracle(codes, host, mse, last):
+    """The GPU codes of the whole matrices against the oracle's, both at the same step: tiles whose
+    scale or Rice header differ, whether the bitstreams are identical, rates and distortions."""
+    out = {"scope": "whole matrices, oracle encode at the GPU's step", "tiles": [], "tile_mismatches": [],
+           "bitstream_identical": [], "payload_bps_gpu": [], "payload_bps_oracle": [], "nmse_gpu": mse,
+           "nmse_oracle": [], "nmse_rel_diff": []}
+    for i, (ref, xo) in enumerate(last):
+        c = codes[i]
+        scale = c.scale.cpu().numpy().view(np.uint16)
+        meta = c.meta.cpu().numpy().view(np.uint16)
+        words = ref.total_words
+        bits = c.bits[:words].cpu().numpy().view(np.uint32)
+        same_cw = np.array_equal(c.chunk_word.cpu().numpy().view(np.uint32), ref.chunk_word)
+        out["tiles"].append(int(ref.tiles))
+        out["tile_mismatches"].append(int(np.count_nonzero((scale != ref.scale) | (meta != ref.meta))))
+        out["bitstream_identical"].append(bool(same_cw and np.array_equal(bits, ref.bits)))
+        out["payload_bps_gpu"].append(c.payload_bps())
+        out["payload_bps_oracle"].append(ref.payload_bits() / float(ref.rows * ref.cols))
+        xf = bf16_bits_to_f64(host[i])
+        nm = float(np.mean((xo - xf) ** 2) / np.mean(xf ** 2))
+        out["nmse_oracle"].append(nm)
+        out["nmse_rel_diff"].append(abs(mse[i] - nm) / nm)
+    return out
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    from post_quantization_tile_b200 import workloads as W
+    return W.bf16_bits_to_f32(bits).astype(np.float64)
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -141,7 +178,7 @@ def run_reference(args):
     inputs = make_inputs()
     rows = 512
     oracle_sample(inputs, rows, max(1, args.warmup // 3))
-    gbs, secs, elems = oracle_sample(inputs, rows, args.steps)
+    gbs, secs, elems, _ = oracle_sample(inputs, rows, args.steps)
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
@@ -374,9 +411,10 @@ def run_gpu(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = max(r for r, _ in SHAPES)
-        gbs, secs, elems = oracle_sample(host, rows, 2)
+        gbs, secs, elems, last = oracle_sample(host, rows, 2, betas=steps_beta)
         cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"encode+decode of both whole matrices, 2 passes ({elems} scalars, {secs:.1f} s, one thread)"}
+               "sample": f"encode+decode of both whole matrices, 2 passes ({elems} scalars, {secs:.1f} s, one thread)",
+               "parity": parity_vs_oracle(codes[0], host, mse, last)}
 
     if rank == 0:
         line = {
