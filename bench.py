@@ -578,8 +578,8 @@ def run_gemm(hq, dev, peak_bf16):
 
 def run_profile(args):
     """One kernel on a 16384x4096 bf16 weight (134 MB, larger than L2), fixed step, three
-    launches after one set-up encode (gemm: the int8 GEMM on 4096^3; kv_dense: the dense-rotation
-    KV variant): a short, self-contained command for ncu captures."""
+    launches after one set-up encode (gemm: the int8 GEMM on 4096^3; kv: the dithered D4 KV codec;
+    kv_dense: the dense-rotation KV variant): a short, self-contained command for ncu captures."""
     import torch
 
     import post_quantization_tile_b200 as hq
@@ -604,6 +604,28 @@ def run_profile(args):
         st = hq.status(hq.workspace(4096))[0]
         print(json.dumps({"profile": "gemm", "ms": [ev[i].elapsed_time(ev[i + 1]) for i in range(3)], "status": st}),
               flush=True)
+        if st != 0:
+            raise SystemExit(1)
+        return
+    if args.profile == "kv":
+        # dithered D4 KV codec on keys [8, 32, 2048, 128] bf16 (67 M scalars, 134 MB, larger than L2)
+        # at the 2-bps step: a set-up encode, then three rounds of encode + decode
+        keys = torch.from_numpy(W.kv_keys(8, 32, 2048, 128, seed=2).view(np.int16)).view(torch.bfloat16).cuda()
+        code = hq.kv_encode(keys, step=1.125, seed=SEED)
+        y = torch.empty_like(keys)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+        torch.cuda.synchronize()
+        for i in range(3):
+            ev[2 * i].record()
+            hq.kv_encode(keys, step=1.125, seed=SEED, out=code, ws=code.ws)
+            ev[2 * i + 1].record()
+            hq.decode(code, out=y.view(-1, 128), ws=code.ws)
+        ev[6].record()
+        torch.cuda.synchronize()
+        st, _ = hq.status(code.ws)
+        print(json.dumps({"profile": "kv", "encode_ms": [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(3)],
+                          "decode_ms": [ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(3)],
+                          "payload_bps": code.payload_bps(), "status": st}), flush=True)
         if st != 0:
             raise SystemExit(1)
         return
@@ -656,7 +678,7 @@ def run_profile(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile", choices=["encode", "decode", "count", "gemm", "kv_dense"], default=None)
+    ap.add_argument("--profile", choices=["encode", "decode", "count", "gemm", "kv", "kv_dense"], default=None)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
