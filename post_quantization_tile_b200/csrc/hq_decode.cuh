@@ -380,8 +380,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 if constexpr (LAT == HQ_E8) {
     #pragma unroll
                     for (int g8 = 0; g8 < H / 8; ++g8) {
-    #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
+    #pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {  // rolled: half the Philox code
                             float U[8];
                             dither_e8(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8), U);
     #pragma unroll
@@ -395,8 +395,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 } else {
     #pragma unroll
                     for (int b = 0; b < H / 4; ++b) {
-    #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
+    #pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {  // rolled: half the Philox code
                             float U[4];
                             dither_group<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + b), U);
     #pragma unroll

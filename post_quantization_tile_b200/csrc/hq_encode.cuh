@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
             *zz_slot(zzs, group, tid) =
                 make_uint4(z[0] | (z[1] << 16), z[2] | (z[3] << 16), z[4] | (z[5] << 16), z[6] | (z[7] << 16));
         };
-        constexpr int ROT = (H >= 16 && !KV) ? HQ_QUANT_ROT : 1;
+        constexpr int ROT = H >= 16 ? HQ_QUANT_ROT : 1;
         constexpr int PB = H / 8 / ROT;  // pair-blocks per round
 #pragma unroll 1
         for (int rr = 0; rr < ROT; ++rr) {
