@@ -15,3 +15,8 @@ GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "oracle_
 @pytest.mark.parametrize("case", make_golden.CASES, ids=[c[0] for c in make_golden.CASES])
 def test_oracle_matches_frozen_digest(case):
     assert make_golden.digest(case) == GOLD[case[0]]
+
+
+@pytest.mark.parametrize("case", make_golden.DENSE_CASES, ids=[c[0] for c in make_golden.DENSE_CASES])
+def test_dense_oracle_matches_frozen_digest(case):
+    assert make_golden.digest_dense(case) == GOLD[case[0]]
