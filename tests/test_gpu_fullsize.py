@@ -8,8 +8,8 @@ oracle's within the binary32 / bf16 tolerance, with the same MSE.  The rate sear
 target within 0.01 bps (Methodology step 3) on the full tensor.
 
 Workloads: LLaMA-7B-shaped 4096x4096 and 11008x4096 (E8, 3/4/5 bps), 70B-shaped 8192x28672 with
-A2/D4/E8/Z and 28672x8192 (E8), the KV keys [8, 32, 8192, 128] with the dithered D4 at 1.7/2/4 bps,
-and two DiT blocks (E8, 4 bps).
+A2/D4/E8/Z and 28672x8192 (E8), the KV keys [8, 32, 8192, 128] with the dithered D4 at 1.7/2/4 bps
+and the KV values at 2 bps, and two DiT blocks (E8, 4 bps).
 """
 import numpy as np
 import pytest
@@ -111,6 +111,12 @@ def test_kv_cache_keys_dithered_d4(hq):
     kt = _t(k)
     for target in (1.7, 2.0, 4.0):
         _check(hq, k, kt, D, hq.D4, target, seed=2, kv=True, kv_S=S, rng_seed=int(10 * target))
+
+
+def test_kv_cache_values_dithered_d4(hq):
+    B, H, S, D = 8, 32, 8192, 128
+    v = W.kv_values(B, H, S, D, seed=2).reshape(-1, D)
+    _check(hq, v, _t(v), D, hq.D4, 2.0, seed=3, kv=True, kv_S=S, rng_seed=21)
 
 
 def test_dit_two_blocks_e8(hq):
