@@ -15,7 +15,7 @@ namespace hq {
 // Kernel configuration
 // ------------------------------------------------------------------------------------------------
 #ifndef HQ_QUANT_ROT
-#define HQ_QUANT_ROT 2  // rounds of the quantizer body per tile (encode_kernel)
+#define HQ_QUANT_ROT 4  // rounds of the quantizer body per tile (encode_kernel); 2 and 8 measured slower
 #endif
 #ifndef HQ_THREADS
 #define HQ_THREADS 128
