@@ -200,3 +200,21 @@ def test_dense_replay_from_a_graph(hq, Q):
     assert torch.equal(code.bits[:ref.total_words()], ref.bits[:ref.total_words()])
     assert torch.equal(code.scale, ref.scale)
     assert torch.equal(y, y_ref)
+
+
+def test_dense_damaged_stream_and_canaries(hq, Q):
+    """A truncated dense-rotation stream decodes to HQ_ERR_CORRUPT with finite output, and nothing
+    is written past the output buffer."""
+    from test_gpu_faults import _guarded, _intact
+    kb = W.kv_keys(1, 2, 64, 128, seed=5)
+    Qd = torch.from_numpy(Q).cuda()
+    code = hq.kv_encode_dense(t_bf16(kb), Qd, step=0.9, seed=4, lattice=oracle.E8)
+    assert hq.status(code.ws)[0] == 0
+    words = code.total_words()
+    code.bits[words // 2:words] = 0                      # the second half of the stream is lost
+    rows = 128
+    yfull, y = _guarded(rows * 128, torch.float32)
+    hq.kv_decode_dense(code, Qd, out=y.view(rows, 128))
+    assert hq.status(code.ws)[0] == 5                    # HQ_ERR_CORRUPT
+    assert _intact(yfull, rows * 128)
+    assert bool(torch.isfinite(y).all().item())
