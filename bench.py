@@ -176,16 +176,21 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import oracle
     inputs = make_inputs()
     rows = 512
-    oracle_sample(inputs, rows, max(1, args.warmup // 3))
-    gbs, secs, elems, _ = oracle_sample(inputs, rows, args.steps)
+    # the step of each sample for the target rate, by the oracle's own search (untimed)
+    betas = [oracle.step_search(np.ascontiguousarray(x[:rows]), TILE, oracle.E8, BPS, seed=SEED, step0=0.28)[0]
+             for x in inputs]
+    oracle_sample(inputs, rows, max(1, args.warmup // 3), betas=betas)
+    gbs, secs, elems, last = oracle_sample(inputs, rows, args.steps, betas=betas)
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "llama7b_linear_4096x4096+11008x4096_bf16_E8_n128_4bps",
-                   "sample": f"first {rows} rows of each matrix per step"},
+                   "sample": f"first {rows} rows of each matrix per step", "step": betas,
+                   "payload_bps": [c.payload_bits() / float(c.rows * c.cols) for c, _ in last]},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"{rows} rows x 4096 of each matrix per step, {args.steps} steps"},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
