@@ -59,6 +59,7 @@ def lib():
         L.hqo_fwht_f32.argtypes = [P, i32]
         L.hqo_fwht_f64.argtypes = [P, i32]
         L.hqo_quantize_block.argtypes = [i32, P, P]
+        L.hqo_quantize_blocks.argtypes = [i32, P, i64, P]
         L.hqo_strip_block.argtypes = [i32, P, P, P]
         L.hqo_unstrip_block.argtypes = [i32, P, i32, P]
         L.hqo_dither_d4.argtypes = [u64, i64, i64, i32, P]
@@ -143,9 +144,7 @@ def quantize_blocks(lattice: int, u: np.ndarray) -> np.ndarray:
     d = LATTICE_DIM[lattice]
     u = np.ascontiguousarray(u, dtype=np.float32).reshape(-1, d)
     v = np.zeros(u.shape, dtype=np.int32)
-    L = lib()
-    for i in range(u.shape[0]):
-        L.hqo_quantize_block(lattice, _p(u[i]), _p(v[i]))
+    lib().hqo_quantize_blocks(lattice, _p(u), u.shape[0], _p(v))
     return v
 
 

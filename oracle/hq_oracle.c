@@ -171,19 +171,22 @@ void hqo_fwht_f64(double* x, int n)
 /* "Fast quantizing and decoding algorithms for lattice quantizers and codes" (IEEE T-IT 1982).*/
 /* Shared pieces:                                                                              */
 /*   a = rint(u) (ties to even), e = a - u (exact in binary32, and never -0);                  */
-/*   "toward u" for a coordinate is +1 when e < 0, else -1;                                     */
-/*   argmax / argmin of |e| compare max(|e|, 2^-31) and break ties to the lowest index.        */
+/*   "toward u" for a coordinate is +1 when e < 0, else -1 (so an exact integer u, e = 0,      */
+/*   re-rounds downward);                                                                      */
+/*   argmax / argmin of |e| compare the exact binary32 values and break ties to the lowest     */
+/*   index.                                                                                    */
+/* Where two cosets compete (E8, A2) both candidate points are formed and their squared        */
+/* Euclidean distances to the input are computed plainly in binary32 (coordinate differences,  */
+/* squares and a sum in coordinate order, each rounded once); the first coset wins ties.       */
 /* ------------------------------------------------------------------------------------------ */
-static const float TINY = 4.6566128730773926e-10f; /* 2^-31 */
-
-static float clamp_tiny(float v) { return v < TINY ? TINY : v; }
+static int toward(float e) { return (e < 0.0f) ? 1 : -1; }
 
 static int argmax_abs(const float* e, int d)
 {
     int j = 0;
-    float best = clamp_tiny(fabsf(e[0]));
+    float best = fabsf(e[0]);
     for (int i = 1; i < d; ++i) {
-        float v = clamp_tiny(fabsf(e[i]));
+        float v = fabsf(e[i]);
         if (v > best) { best = v; j = i; }
     }
     return j;
@@ -192,9 +195,9 @@ static int argmax_abs(const float* e, int d)
 static int argmin_abs(const float* e, int d)
 {
     int j = 0;
-    float best = clamp_tiny(fabsf(e[0]));
+    float best = fabsf(e[0]);
     for (int i = 1; i < d; ++i) {
-        float v = clamp_tiny(fabsf(e[i]));
+        float v = fabsf(e[i]);
         if (v < best) { best = v; j = i; }
     }
     return j;
@@ -218,80 +221,88 @@ void hqo_q_d4(const float* u, int32_t* v)
     }
     if (sum & 1) {
         int j = argmax_abs(e, 4);
-        a[j] += (e[j] < 0.0f) ? 1 : -1;
+        a[j] += toward(e[j]);
     }
     for (int i = 0; i < 4; ++i) v[i] = a[i];
 }
 
-/* E8 = D8 u (D8 + 1/2), min norm sqrt(2).  Output in doubled coordinates v = 2p (all v_i of
- * one parity, sum v = 0 mod 4).
- *   Coset A (D8): a = rint(u); if sum a is odd, move the coordinate with max |e| toward u.
- *   Coset B (D8 + 1/2): b_i = a_i + 1/2 if e_i < 0 else a_i - 1/2 (nearest half-integer);
- *     if sum (b_i - 1/2) is odd, move the coordinate farthest from its half-integer, i.e.
- *     the one with min |e|, to its other half-integer neighbour.
- *   Choice: |u - A|^2 - |u - B|^2 = sum_i (|e_i| - 1/4) + [A fixed](1 - 2 max|e|)
- *           - [B fixed](2 min|e|)  (exact algebra, from |u_i - b_i| = 1/2 - |e_i|).
- *   It is evaluated in binary32 as D = ((S - 2) + cA) - cB with S = pairwise sum of |e_i|;
- *   B is taken only when D > 0 (ties go to A). */
+/* squared distance from z to the integer point p, binary32, summed in coordinate order */
+static float dist2_int(const float* z, const int32_t* p, int d)
+{
+    float s = 0.0f;
+    for (int i = 0; i < d; ++i) {
+        float t = z[i] - (float)p[i];
+        s = s + t * t;
+    }
+    return s;
+}
+
+/* E8 = D8 u (D8 + 1/2), min norm sqrt(2), in doubled coordinates z = 2u, where its points are
+ * the integer vectors with all coordinates of one parity and sum = 0 mod 4.
+ *   Coset A (2 D8, even integers): p_i = 2 rint(u_i); if sum p = 2 mod 4, the coordinate with
+ *     the largest |e| moves by 2 toward z.
+ *   Coset B (2 D8 + 1, odd integers): p_i = the odd integer nearest z_i, 2 a_i + toward(e_i);
+ *     if sum p = 2 mod 4, the coordinate farthest from its odd integer -- the one with the
+ *     smallest |e|, since |z_i - p_i| = 1 - 2|e_i| -- moves by 2 to its other odd neighbour.
+ *   The output is the candidate with the smaller squared distance to z (A on ties). */
 void hqo_q_e8(const float* u, int32_t* v)
 {
-    float e[8], ae[8];
-    int32_t a[8];
-    int sumA = 0, nonneg = 0;
+    float z[8], e[8];
+    int32_t a[8], pA[8], pB[8];
+    int32_t sumA = 0, sumB = 0;
     for (int i = 0; i < 8; ++i) {
         float r = rintf(u[i]);
+        z[i] = 2.0f * u[i];
         e[i] = r - u[i];
-        ae[i] = fabsf(e[i]);
         a[i] = (int32_t)r;
-        sumA += a[i];
-        if (!(e[i] < 0.0f)) nonneg += 1;
     }
-    int parA = sumA & 1;
-    int parB = (sumA - nonneg) & 1; /* sum of (b_i - 1/2) = sum a_i - #{e_i >= 0} */
-    float S = ((ae[0] + ae[1]) + (ae[2] + ae[3])) + ((ae[4] + ae[5]) + (ae[6] + ae[7]));
-    int jA = argmax_abs(e, 8);
-    int mB = argmin_abs(e, 8);
-    float emax = clamp_tiny(ae[jA]);
-    float emin = clamp_tiny(ae[mB]);
-    float cA = parA ? (1.0f - 2.0f * emax) : 0.0f;
-    float cB = parB ? (2.0f * emin) : 0.0f;
-    float D = ((S - 2.0f) + cA) - cB;
-    if (!(D > 0.0f)) {
-        /* coset A: v = 2a */
-        if (parA) a[jA] += (e[jA] < 0.0f) ? 1 : -1;
-        for (int i = 0; i < 8; ++i) v[i] = 2 * a[i];
-    } else {
-        /* coset B: v = 2b, odd integers */
-        for (int i = 0; i < 8; ++i) v[i] = 2 * a[i] + ((e[i] < 0.0f) ? 1 : -1);
-        if (parB) {
-            int m = mB;
-            int toward = (e[m] < 0.0f) ? 1 : -1;
-            v[m] -= 2 * toward; /* the other neighbouring half-integer */
-        }
+    for (int i = 0; i < 8; ++i) {
+        pA[i] = 2 * a[i];
+        sumA += pA[i];
+        pB[i] = 2 * a[i] + toward(e[i]);
+        sumB += pB[i];
     }
+    if ((sumA & 3) == 2) {
+        int j = argmax_abs(e, 8);
+        pA[j] += 2 * toward(e[j]);
+    }
+    if ((sumB & 3) == 2) {
+        int m = argmin_abs(e, 8);
+        pB[m] -= 2 * toward(e[m]);
+    }
+    float dA = dist2_int(z, pA, 8);
+    float dB = dist2_int(z, pB, 8);
+    const int32_t* p = (dA <= dB) ? pA : pB;
+    for (int i = 0; i < 8; ++i) v[i] = p[i];
 }
 
 /* A2, minimum distance 1: points (P/2, Q*sqrt(3)/2) with P = Q mod 2.  Work in (P, Q) =
- * (2 u0, u1 * K), K = RN(2/sqrt 3).  The lattice is the union of the even and the odd
- * rectangular cosets of 2Z x 2Z; per coordinate X, h = X/2, a = rint(h), e = a - h.  Squared
- * distances in (P, Q) units weigh dQ three times; |even|^2 - |odd|^2 is proportional to
- * |eP| + 3|eQ| - 1, so the even point is taken when RN(|eP| + RN(3|eQ|)) <= 1. */
+ * (2 u0, u1 * K), K = RN(2/sqrt 3), where A2 is the union of the even coset 2Z x 2Z and the
+ * odd coset (2Z+1) x (2Z+1) and squared distances weigh dQ three times.  Per coordinate X the
+ * nearest even integer is 2 rint(X/2) and the nearest odd one 2 rint(X/2) + toward(rint(X/2) -
+ * X/2).  The output is the candidate with the smaller dP^2 + 3 dQ^2 (the even one on ties). */
 static const float A2_K = 1.15470053837925153f; /* RN(2/sqrt(3)) */
+
+static float a2_dist2(float P, float Q, const int32_t* p)
+{
+    float dP = P - (float)p[0], dQ = Q - (float)p[1];
+    return dP * dP + 3.0f * (dQ * dQ);
+}
 
 /* A2 nearest point given (P, Q) directly (the dither is added in these coordinates). */
 void hqo_q_a2_pq(float P, float Q, int32_t* v)
 {
     float hP = P * 0.5f, hQ = Q * 0.5f;
     float rP = rintf(hP), rQ = rintf(hQ);
-    float eP = rP - hP, eQ = rQ - hQ;
     int32_t aP = (int32_t)rP, aQ = (int32_t)rQ;
-    float E = fabsf(eP) + 3.0f * fabsf(eQ);
-    if (E <= 1.0f) {
-        v[0] = 2 * aP;
-        v[1] = 2 * aQ;
+    int32_t even[2] = {2 * aP, 2 * aQ};
+    int32_t odd[2] = {2 * aP + toward(rP - hP), 2 * aQ + toward(rQ - hQ)};
+    if (a2_dist2(P, Q, even) <= a2_dist2(P, Q, odd)) {
+        v[0] = even[0];
+        v[1] = even[1];
     } else {
-        v[0] = 2 * aP + ((eP < 0.0f) ? 1 : -1);
-        v[1] = 2 * aQ + ((eQ < 0.0f) ? 1 : -1);
+        v[0] = odd[0];
+        v[1] = odd[1];
     }
 }
 
@@ -853,6 +864,13 @@ uint32_t hqo_decode(const uint16_t* scale, const uint16_t* meta, const uint32_t*
 
 /* Small helpers exposed for the pins. */
 void hqo_quantize_block(int lattice, const float* u, int32_t* v) { quantize_block(lattice, u, v); }
+
+/* m consecutive blocks of d = dim(lattice) coordinates each */
+void hqo_quantize_blocks(int lattice, const float* u, int64_t m, int32_t* v)
+{
+    int d = lattice_dim(lattice);
+    for (int64_t b = 0; b < m; ++b) quantize_block(lattice, u + b * d, v + b * d);
+}
 
 void hqo_strip_block(int lattice, const int32_t* v, int32_t* sym, int* coset) { strip_block(lattice, v, sym, coset); }
 

@@ -79,6 +79,55 @@ def test_rms_matches_float64(n):
         assert abs(oracle.rms(x) - ref) <= 2e-6 * ref
 
 
+def _rn32_sqrt(r):
+    """binary32 nearest (ties to even) to sqrt(r) for a positive Fraction r, decided exactly:
+    f is the answer when the squares of the midpoints to its neighbours bracket r."""
+    from fractions import Fraction
+    f = np.float32(np.sqrt(float(r)))
+    for _ in range(4):
+        lo = np.nextafter(f, np.float32(0)); hi = np.nextafter(f, np.float32(np.inf))
+        mlo = (Fraction(float(lo)) + Fraction(float(f))) / 2
+        mhi = (Fraction(float(f)) + Fraction(float(hi))) / 2
+        if r < mlo * mlo:
+            f = lo
+        elif r > mhi * mhi:
+            f = hi
+        else:
+            assert r != mlo * mlo and r != mhi * mhi   # no tie for these inputs
+            return f
+    raise AssertionError("no convergence")
+
+
+# One large square in the first half of the tile and n/2 equal small squares in the second half:
+# the ascending pairwise tree adds the small squares among themselves first, so every partial sum
+# and the total are exact, while a running (sequential) sum rounds at every step.  Found by a
+# search over bf16 values for which the two sums give different bf16 scales.
+RMS_ORDER_CASES = [(64, 5.15625, 0.2373046875), (64, 6.15625, 0.2060546875), (128, 5.5625, 0.1904296875),
+                   (128, 5.625, 0.1591796875), (256, 7.90625, 0.2177734375), (256, 10.3125, 0.2373046875)]
+
+
+@pytest.mark.parametrize("n,big,small", RMS_ORDER_CASES)
+def test_rms_sums_the_squares_in_the_ascending_tree(n, big, small):
+    """The scale is sqrt(mean of squares) with the squares summed by the ascending pairwise tree
+    (the per-tile scaling of Methodology step 2 with the RMS statistic; the summation order is the
+    reading that fixes the binary32 result).  On these inputs the tree is exact, so its result is
+    the correctly rounded square root of the exact mean square, and a sequential sum is not."""
+    from fractions import Fraction
+    x = np.zeros(n, dtype=np.float32)
+    x[0] = big
+    x[n // 2:] = small
+    exact = sum(Fraction(float(v)) ** 2 for v in x) / n
+    want = _rn32_sqrt(exact)
+    got = np.float32(oracle.rms(x))
+    assert got == want, (got, want)
+    # the sequential order rounds differently, down to the stored bf16 scale
+    seq = np.float32(0.0)
+    for v in x:
+        seq = np.float32(seq + np.float32(v) * np.float32(v))
+    seq_s = np.float32(np.sqrt(np.float32(seq * np.float32(1.0 / n))))
+    assert oracle.f32_to_bf16_bits(np.array([seq_s]))[0] != oracle.f32_to_bf16_bits(np.array([got]))[0]
+
+
 @pytest.mark.parametrize("n", [64, 128, 256])
 def test_fwht_is_the_sylvester_hadamard_product(n):
     H = scipy.linalg.hadamard(n).astype(np.float64)   # natural (Sylvester) order
