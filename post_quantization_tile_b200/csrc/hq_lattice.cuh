@@ -5,10 +5,14 @@
 // quantizers and codes" (IEEE T-IT 28(2), 1982), in binary32 without contraction:
 //   a = rint(u) via the 1.5*2^23 addition (exact for |u| < 2^22, which the per-tile RMS scaling
 //   and the step range guarantee), e = a - u (exact, never -0), "toward u" = +1 when e < 0;
-//   argmax / argmin of |e| compare max(|e|, 2^-31), ties to the lowest index.  The comparison
-//   runs on 32-bit keys (clamped |e| bits << 4 | index << 1 | sign of e): the clamped bits of
-//   |e| in [2^-31, 1/2] all start with 0011, so the shift drops nothing that orders them, and one
-//   integer max / min returns the value, the lowest tied index and the sign together.
+//   argmax / argmin of |e| with ties to the lowest index.  The fast comparison runs on 32-bit keys
+//   (max(|e|, 2^-31) bits << 4 | index << 1 | sign of e): the bits of |e| in [2^-31, 1/2] all
+//   start with 0011, so the shift drops nothing that orders them, and one integer max / min returns
+//   the value, the lowest tied index and the sign together.  Where the 2^-31 floor could change the
+//   outcome (a fix-up among rounding errors below 2^-31), and where two cosets (E8, A2) come within
+//   a band of a tie that covers the rounding of the shortcut formula, the plain rule runs instead:
+//   exact argmax / argmin and both candidates' squared distances in binary32, summed in coordinate
+//   order.  Both paths therefore return the point the plain definition returns.
 #pragma once
 
 #include "hq_common.cuh"
@@ -18,6 +22,11 @@ namespace hq {
 constexpr float kMagic = 12582912.0f;         // 1.5 * 2^23
 constexpr uint32_t kTinyBits = 0x30000000u;   // 2^-31
 constexpr float kA2K = 1.15470053837925153f;  // RN(2/sqrt(3))
+// Width of the band around a coset tie in which the plain distance comparison decides.  The
+// shortcut value of |u-A|^2 - |u-B|^2 (E8) is within 1.4e-6 of the exact one and the plain
+// binary32 distance difference within 3.4e-6 (u^2 units); outside 2^-16 both have the exact sign.
+// For A2 the shortcut |eP| + 3|eQ| - 1 and the plain (dE - dO)/4 are both within 1e-6.
+constexpr float kTieBand = 1.52587890625e-05f;  // 2^-16
 
 template <int LAT>
 struct Lat;
@@ -53,24 +62,84 @@ __device__ __forceinline__ void q_d4(const float (&u)[4], int32_t (&v)[4])
 {
     int32_t sum = 0;
     uint32_t kmax = 0;
+    float e[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float r = rint_magic(u[i], v[i]);
         sum += v[i];
-        kmax = max(kmax, max_key(__fadd_rn(r, -u[i]), i, 4));
+        e[i] = __fadd_rn(r, -u[i]);
+        kmax = max(kmax, max_key(e[i], i, 4));
     }
-    const int j = 3 - (int)((kmax >> 1) & 7u);
-    const int32_t delta = (sum & 1) ? ((kmax & 1u) ? 1 : -1) : 0;
+    int j = 3 - (int)((kmax >> 1) & 7u);
+    int32_t delta = (sum & 1) ? ((kmax & 1u) ? 1 : -1) : 0;
+    if ((sum & 1) && kmax < 16u) {
+        // every |e| is below the 2^-31 floor of the keys: the exact argmax (lowest index on ties)
+        j = 0;
+        float best = fabsf(e[0]);
+#pragma unroll
+        for (int i = 1; i < 4; ++i)
+            if (fabsf(e[i]) > best) {
+                best = fabsf(e[i]);
+                j = i;
+            }
+        delta = e[j] < 0.0f ? 1 : -1;
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         if (i == j) v[i] += delta;
+}
+
+// The plain E8 coset choice from the rounding errors e (doubled coordinates z = 2u, where a coset A
+// point is 2a (+2 toward z at the fixed coordinate) and a coset B point 2a + toward (-2 toward at
+// the fixed coordinate), so z - p = -2e - c exactly): exact argmax / argmin of |e| with the lowest
+// index on ties, squared distances summed in coordinate order in binary32, A on ties.  Returns
+// isB | fix << 1 | (delta + 1) << 4, delta the move of the fixed coordinate of w.  Rarely taken:
+// kept out of line.
+struct E8Err {
+    float e[8];
+};
+static __device__ __noinline__ uint32_t e8_plain_choice(const E8Err E, const uint32_t parA, const uint32_t parB)
+{
+    int j = 0, m = 0;
+    float bmax = fabsf(E.e[0]), bmin = bmax;
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        const float a = fabsf(E.e[i]);
+        if (a > bmax) {
+            bmax = a;
+            j = i;
+        }
+        if (a < bmin) {
+            bmin = a;
+            m = i;
+        }
+    }
+    float dA = 0.0f, dB = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float t = E.e[i] < 0.0f ? 1.0f : -1.0f;
+        const float cA = (parA && i == j) ? 2.0f * t : 0.0f;
+        const float cB = (parB && i == m) ? -t : t;
+        const float xA = __fadd_rn(__fmul_rn(-2.0f, E.e[i]), -cA);
+        const float xB = __fadd_rn(__fmul_rn(-2.0f, E.e[i]), -cB);
+        dA = __fadd_rn(dA, __fmul_rn(xA, xA));
+        dB = __fadd_rn(dB, __fmul_rn(xB, xB));
+    }
+    const uint32_t isB = dA <= dB ? 0u : 1u;
+    const int fix = isB ? m : j;
+    const uint32_t dofix = isB ? parB : parA;
+    // A moves toward u (+1 when e < 0), B away from its first half-integer (-1 when e < 0)
+    const int ef = E.e[fix] < 0.0f ? 1 : -1;
+    const int delta = dofix ? (isB ? -ef : ef) : 0;
+    return isB | ((uint32_t)fix << 1) | ((uint32_t)(delta + 1) << 4);
 }
 
 // E8 = D8 u (D8 + 1/2), fused with bit-stripping.  Returns the coset bit c and writes the 8
 // symbols (w0 .. w6, (w7 - p)/2) of the nearest point v/2 (v doubled coordinates, w = (v - c)/2);
 // v itself when WANT_V.  The coset choice compares
 // |u-A|^2 - |u-B|^2 = sum(|e| - 1/4) + [A fixed](1 - 2 max|e|) - [B fixed](2 min|e|) in binary32
-// as D = ((S - 2) + cA) - cB, S the pairwise sum of |e|; B only when D > 0.
+// as D = ((S - 2) + cA) - cB, S the pairwise sum of |e|; B only when D > 0.  Within 2^-16 of a tie
+// (and where a fix-up meets the 2^-31 key floor) e8_plain_choice decides instead.
 //   A: w = a; if sum a is odd the coordinate with max |e| moves toward u.
 //   B: w = a - [e >= 0] (w + 1/2 is the half-integer toward u); if sum w is odd the coordinate
 //      with min |e| moves to its other half-integer neighbour.
@@ -102,12 +171,22 @@ __device__ __forceinline__ uint32_t e8_from_te(const float (&tv)[8], const float
     const float cA = parA ? __fadd_rn(1.0f, -__fmul_rn(2.0f, key_value(kmax))) : 0.0f;
     const float cB = parB ? __fmul_rn(2.0f, key_value(kmin)) : 0.0f;
     const float D = __fadd_rn(__fadd_rn(__fadd_rn(S, -2.0f), cA), -cB);
-    const bool isB = D > 0.0f;
+    bool isB = D > 0.0f;
     // the coordinate to fix and its direction: A moves toward u (+1 when e < 0), B away from it
     const uint32_t kf = isB ? kmin : kmax;
-    const int fix = isB ? (int)((kmin >> 1) & 7u) : 7 - (int)((kmax >> 1) & 7u);
+    int fix = isB ? (int)((kmin >> 1) & 7u) : 7 - (int)((kmax >> 1) & 7u);
     const uint32_t dofix = isB ? parB : parA;
-    const int32_t delta = dofix ? ((((kf & 1u) != 0u) != isB) ? 1 : -1) : 0;
+    int32_t delta = dofix ? ((((kf & 1u) != 0u) != isB) ? 1 : -1) : 0;
+    // near a coset tie, or where a fix-up meets the 2^-31 floor of the keys: the plain rule
+    if (fabsf(D) <= kTieBand || (parA && kmax < 16u) || (parB && kmin < 16u)) {
+        E8Err E;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) E.e[i] = ev[i];
+        const uint32_t r = e8_plain_choice(E, parA, parB);
+        isB = (r & 1u) != 0u;
+        fix = (int)((r >> 1) & 7u);
+        delta = (int32_t)(r >> 4) - 1;
+    }
     const uint32_t bmask = isB ? 0xFFFFFFFFu : 0u;
     int32_t w[8];
 #pragma unroll
@@ -161,7 +240,8 @@ __device__ __forceinline__ void e8_pair_symbols(const float2 (&p)[8], int32_t (&
     cy = e8_from_te<WANT_V>(ty, ey, sy, vy);
 }
 
-// A2 with minimum distance 1 in (P, Q) = (2 u0, u1 K); the even point when |eP| + 3|eQ| <= 1.
+// A2 with minimum distance 1 in (P, Q) = (2 u0, u1 K): the even point when |eP| + 3|eQ| <= 1, which is
+// |even|^2 <= |odd|^2 up to a factor of 4; near the tie the two distances themselves decide.
 __device__ __forceinline__ void q_a2_pq(const float P, const float Q, int32_t (&v)[2])
 {
     const float hP = __fmul_rn(P, 0.5f), hQ = __fmul_rn(Q, 0.5f);
@@ -169,7 +249,17 @@ __device__ __forceinline__ void q_a2_pq(const float P, const float Q, int32_t (&
     const float rP = rint_magic(hP, aP), rQ = rint_magic(hQ, aQ);
     const float eP = __fadd_rn(rP, -hP), eQ = __fadd_rn(rQ, -hQ);
     const float E = __fadd_rn(fabsf(eP), __fmul_rn(3.0f, fabsf(eQ)));
-    if (E <= 1.0f) {
+    bool even = E <= 1.0f;
+    if (fabsf(__fadd_rn(E, -1.0f)) <= kTieBand) {
+        // near the tie of the two cosets: both candidates' dP^2 + 3 dQ^2 in binary32
+        const float oP = (float)(2 * aP + ((eP < 0.0f) ? 1 : -1)), oQ = (float)(2 * aQ + ((eQ < 0.0f) ? 1 : -1));
+        const float dPe = __fadd_rn(P, -(float)(2 * aP)), dQe = __fadd_rn(Q, -(float)(2 * aQ));
+        const float dPo = __fadd_rn(P, -oP), dQo = __fadd_rn(Q, -oQ);
+        const float de = __fadd_rn(__fmul_rn(dPe, dPe), __fmul_rn(3.0f, __fmul_rn(dQe, dQe)));
+        const float dO = __fadd_rn(__fmul_rn(dPo, dPo), __fmul_rn(3.0f, __fmul_rn(dQo, dQo)));
+        even = de <= dO;
+    }
+    if (even) {
         v[0] = 2 * aP;
         v[1] = 2 * aQ;
     } else {

@@ -3,8 +3,10 @@
 The oracle cannot encode a 235 M-scalar matrix in test time, but tiles and chunks are
 independent: the oracle encodes whole 32-row chunks taken out of the full tensor (first, a
 random and the last chunk of every tile column), and the GPU's words for those chunks, their
-meta and scales must be bit-identical; the GPU reconstruction of those rows must match the
-oracle's within the binary32 / bf16 tolerance, with the same MSE.  The rate search hits the
+meta and scales must be bit-identical (an index may differ only within 1e-6 of a Voronoi
+boundary, counted, at most a 1e-6 fraction of the blocks); the GPU reconstruction of those rows,
+decoded both to binary32 and to bf16, must match the oracle's within the tolerance, with the
+same MSE.  The rate search hits the
 target within 0.01 bps (Methodology step 3) on the full tensor.
 
 Workloads: LLaMA-7B-shaped 4096x4096 and 11008x4096 (E8, 3/4/5 bps), 70B-shaped 8192x28672 with
@@ -38,7 +40,27 @@ def _sample_chunks(rows, rng):
     return picks
 
 
+def _chunk_subcode(scale, meta, cw, bits, rows, n, NT, rb):
+    """The device code of rows [32 rb, 32 rb + 32) as a code of its own (one chunk per tile column)."""
+    RB = (rows + 31) // 32
+    r0, r1 = 32 * rb, min(32 * rb + 32, rows)
+    h = r1 - r0
+    sub_scale = np.concatenate([scale[jt * rows + r0: jt * rows + r1] for jt in range(NT)])
+    sub_meta = np.concatenate([meta[jt * rows + r0: jt * rows + r1] for jt in range(NT)])
+    pieces = [bits[cw[jt * RB + rb]: cw[jt * RB + rb + 1]] for jt in range(NT)]
+    sub_cw = np.zeros(NT + 1, dtype=np.uint32)
+    sub_cw[1:] = np.cumsum([p.size for p in pieces])
+    sub_bits = np.concatenate(pieces + [np.zeros(1, np.uint32)])
+    assert sub_meta.size == NT * h
+    return sub_scale, sub_meta, sub_cw, sub_bits
+
+
 def _check(hq, x_host, xt, n, lattice, target, seed, kv=False, kv_S=0, rng_seed=0):
+    """Sampled chunks of the full-size code against the oracle's code of the same rows: boundary-aware
+    comparison (oracle/parity.py: bit-exact except counted near-boundary disagreements, fraction of
+    blocks <= 1e-6), reconstructions within 1e-5 max(|x_hat|, s_hat) in binary32 and within half a
+    bf16 ulp more in bf16, MSE within 0.1%."""
+    from oracle import parity
     rows, cols = x_host.shape
     beta = hq.calibrate_step(xt, n, lattice, target, seed=seed, kv=kv, kv_S=kv_S)
     if kv:
@@ -50,36 +72,37 @@ def _check(hq, x_host, xt, n, lattice, target, seed, kv=False, kv_S=0, rng_seed=
     assert st == 0
     assert abs(code.payload_bps() - target) <= 0.01
     y = hq.decode(code, dtype=torch.bfloat16)
+    y32 = hq.decode(code, dtype=torch.float32)
     assert hq.status(code.ws)[0] == 0
     cw = code.chunk_word.cpu().numpy().view(np.uint32).astype(np.int64)
     bits = code.bits.cpu().numpy().view(np.uint32)
     meta = code.meta.cpu().numpy().view(np.uint16)
     scale = code.scale.cpu().numpy().view(np.uint16)
-    RB = (rows + 31) // 32
     NT = cols // n
     rng = np.random.default_rng(rng_seed)
     err_gpu = err_ref = 0.0
+    blocks = disagreements = 0
     for rb in _sample_chunks(rows, rng):
         r0, r1 = 32 * rb, min(32 * rb + 32, rows)
         xs = np.ascontiguousarray(x_host[r0:r1])
-        ref = oracle.encode(xs, n, lattice, beta, seed, kv, kv_S, row0=r0)
-        for jt in range(NT):
-            c = jt * RB + rb
-            np.testing.assert_array_equal(bits[cw[c]:cw[c + 1]], ref.bits[ref.chunk_word[jt]:ref.chunk_word[jt + 1]],
-                                          err_msg=f"chunk words rb {rb} jt {jt}")
-            t0 = jt * rows + r0
-            np.testing.assert_array_equal(meta[t0:t0 + (r1 - r0)], ref.meta[jt * (r1 - r0):(jt + 1) * (r1 - r0)])
-            np.testing.assert_array_equal(scale[t0:t0 + (r1 - r0)], ref.scale[jt * (r1 - r0):(jt + 1) * (r1 - r0)])
+        ref = oracle.encode(xs, n, lattice, beta, seed, kv, kv_S, row0=r0, want_codes=True)
+        rep = parity.compare(*_chunk_subcode(scale, meta, cw, bits, rows, n, NT, rb), ref)
+        assert not rep.failures, f"rows {r0}..{r1}: {rep.failures[:3]}"
+        blocks += rep.blocks
+        disagreements += rep.disagreements
         xo, rst = oracle.decode(ref)
         assert rst == 0
-        yb = y[r0:r1].float().cpu().numpy().astype(np.float64)
         sh = W.bf16_bits_to_f32(ref.scale).astype(np.float64)
         scale_map = np.repeat(sh.reshape(NT, r1 - r0).T, n, axis=1)
+        y32s = y32[r0:r1].cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(y32s - xo) <= 1e-5 * np.maximum(np.abs(xo), scale_map)), "binary32 reconstruction"
+        yb = y[r0:r1].float().cpu().numpy().astype(np.float64)
         tol = 2.0 ** -8 * np.abs(xo) + 1e-5 * np.maximum(np.abs(xo), scale_map)
         assert np.all(np.abs(yb - xo) <= tol)
         xf = W.bf16_bits_to_f32(xs).astype(np.float64)
         err_gpu += np.sum((yb - xf) ** 2)
         err_ref += np.sum((W.bf16_bits_to_f32(W.to_bf16_bits(xo.astype(np.float32))).astype(np.float64) - xf) ** 2)
+    assert disagreements <= 1e-6 * blocks, f"{disagreements} boundary disagreements in {blocks} blocks"
     assert abs(err_gpu / err_ref - 1.0) < 1e-3
     return code
 

@@ -40,12 +40,16 @@ def u16(t: torch.Tensor) -> np.ndarray:
 
 
 def assert_same_code(code, ref, what=""):
-    words = ref.total_words
-    np.testing.assert_array_equal(u32(code.chunk_word), ref.chunk_word, err_msg=f"chunk_word {what}")
-    np.testing.assert_array_equal(u16(code.meta), ref.meta, err_msg=f"meta {what}")
-    if ref.scale is not None and code.scale is not None:
-        np.testing.assert_array_equal(u16(code.scale), ref.scale, err_msg=f"scale {what}")
-    np.testing.assert_array_equal(u32(code.bits)[:words], ref.bits, err_msg=f"bits {what}")
+    """Device code against the oracle's: bit-exact, except that an index may differ for an input
+    within 1e-6 of a Voronoi boundary (counted; the fraction of blocks must stay <= 1e-6, and every
+    chunk without such a block must be word-identical) -- see oracle/parity.py."""
+    from oracle import parity
+    words = int(u32(code.chunk_word)[-1])
+    scale = u16(code.scale) if (ref.scale is not None and code.scale is not None) else None
+    rep = parity.compare(scale, u16(code.meta), u32(code.chunk_word), u32(code.bits)[:max(words, 1)], ref)
+    assert not rep.failures, f"{what}: {rep.failures[:3]}"
+    assert rep.fraction <= 1e-6, f"{what}: {rep.disagreements} boundary disagreements in {rep.blocks} blocks"
+    return rep
 
 
 def _coeffs(n, tiles, seed, lattice):
@@ -74,6 +78,28 @@ def test_quantize_coeffs_bit_exact(hq, lattice, n):
     st, _ = hq.status(code.ws)
     assert st == 0
     rv, rmeta, rcw, rbits, rst = oracle.quantize_coeffs(u, n, lattice)
+    np.testing.assert_array_equal(v.cpu().numpy(), rv)
+    np.testing.assert_array_equal(u16(code.meta), rmeta)
+    np.testing.assert_array_equal(u32(code.chunk_word), rcw)
+    np.testing.assert_array_equal(u32(code.bits)[: int(rcw[-1])], rbits)
+
+
+@pytest.mark.parametrize("lattice", [oracle.E8, oracle.D4, oracle.A2])
+@pytest.mark.parametrize("n", [64, 128, 256])
+def test_quantize_coeffs_near_ties_bit_exact(hq, lattice, n):
+    """Coefficients on and within a few 1e-6 of Voronoi facets (coset ties of E8 and A2,
+    neighbour ties of D4), and blocks whose fix-up chooses among rounding errors below 2^-31:
+    the device's shortcut decisions hand these to the plain rule, so codes stay bit-exact."""
+    from lattice_inputs import facet_ties, small_error_blocks
+    d = oracle.LATTICE_DIM[lattice]
+    parts = [facet_ties(lattice, 40 * n // d, 70 + n + lattice)]
+    if lattice != oracle.A2:
+        parts.append(small_error_blocks(lattice, 16 * n // d, 90 + n + lattice))
+    u = np.ascontiguousarray(np.concatenate(parts).reshape(-1, n))
+    v, code = hq.quantize_coeffs(torch.from_numpy(u).cuda(), n, lattice)
+    assert hq.status(code.ws)[0] == 0
+    rv, rmeta, rcw, rbits, rst = oracle.quantize_coeffs(u, n, lattice)
+    assert rst == 0
     np.testing.assert_array_equal(v.cpu().numpy(), rv)
     np.testing.assert_array_equal(u16(code.meta), rmeta)
     np.testing.assert_array_equal(u32(code.chunk_word), rcw)
@@ -128,7 +154,7 @@ def test_encode_decode_match_oracle(hq, case, lattice):
     code = hq.encode(xt, tile=n, lattice=lattice, step=beta, seed=seed)
     st, _ = hq.status(code.ws)
     assert st == 0, st
-    ref = oracle.encode(x, n, lattice, beta, seed)
+    ref = oracle.encode(x, n, lattice, beta, seed, want_codes=True)
     assert_same_code(code, ref, name)
     xo, rst = oracle.decode(ref)
     assert rst == 0
@@ -165,7 +191,7 @@ def test_kv_encode_decode_match_oracle(hq, bps_beta):
     kb = W.kv_keys(B, H, S, D, seed=2)
     code = hq.kv_encode(t_bf16(kb), step=bps_beta, seed=31)
     assert hq.status(code.ws)[0] == 0
-    ref = oracle.encode(kb.reshape(-1, D), D, oracle.D4, bps_beta, 31, kv=True, kv_S=S)
+    ref = oracle.encode(kb.reshape(-1, D), D, oracle.D4, bps_beta, 31, kv=True, kv_S=S, want_codes=True)
     assert_same_code(code, ref, "kv")
     y = hq.kv_decode(code, (B, H, S, D), dtype=torch.float32)
     xo, _ = oracle.decode(ref)
