@@ -314,11 +314,14 @@ int32_t hq_version(void);
  * that loads it until the process exits.  It covers tensors with
  *     64 + 8 * (cols / tile) * ceil(rows / (tile == 256 ? 64 : 128)) <= HQ_NOALLOC_SCRATCH_BYTES
  * (e.g. 8192 x 28672 at tile 256, 16384 x 8192 at tile 128); larger tensors get HQ_ERR_RANGE
- * and nothing is enqueued.  The first call on a device looks the array's device address up
- * (cudaGetSymbolAddress) for that device; make that first call before capturing the stream
- * into a graph.  All calls share the one array and each call clears it on `stream` before its
- * kernel runs, so calls whose work overlaps on the GPU (different streams without ordering)
- * race and must not be issued.  Device errors (capacity, non-finite input, timeout) are copied
+ * and nothing is enqueued.  Like the other entry points it makes the device that holds x (device
+ * or managed memory) the calling thread's current device.  The first call on a device looks the
+ * array's device address up (cudaGetSymbolAddress) for that device, and so does the first call
+ * after that device's primary context was replaced (cudaDeviceReset destroys the array's
+ * contents and may move it); make such a call before capturing the stream into a graph.  All
+ * calls share the one array and each call clears it on `stream` before its kernel runs, so calls
+ * whose work overlaps on the GPU (different streams without ordering) race and must not be
+ * issued.  Device errors (capacity, non-finite input, timeout) are copied
  * as the status bit word (1 << hq_status_t) to *status_out (device uint32) when it is not
  * NULL.  No allocation, no synchronisation.
  */

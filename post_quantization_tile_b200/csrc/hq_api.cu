@@ -655,15 +655,19 @@ hq_status_t hq_step_search(const void* x, hq_dtype_t dtype, int64_t rows, int64_
                               result, ws, ws_bytes, stream);
 }
 
+#ifdef HQ_TEST_HOOKS
+// only in the test library (libhq_test.so): the product library does not export it
 hq_status_t hq_test_encode_silent_item(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols,
                                        const hq_params_t* p, hq_code_t* out, void* ws, size_t ws_bytes,
                                        int64_t silent_item, void* stream)
 {
     if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
     if (silent_item < 1) return HQ_ERR_ARG;  // item 0 needs no look-back
+    if (!p || p->lattice != HQ_E8) return HQ_ERR_UNSUPPORTED;  // the E8 kernels carry the hook
     return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, 0, 0, nullptr, out, nullptr, ws, ws_bytes, stream,
                          0, silent_item);
 }
+#endif
 
 hq_status_t hq_status_read(const void* ws, void* stream, int64_t* detail)
 {

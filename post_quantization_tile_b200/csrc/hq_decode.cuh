@@ -190,8 +190,19 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 sm.rowoff[ch * 32 + lane] = incl - v;
             }
         }
-        if (!mbar_wait(&sm.bar[st], parity)) status_set(a.ws, kStTimeout);
-        __syncthreads();
+        const bool arrived = mbar_wait(&sm.bar[st], parity);
+        if (!arrived) status_set(a.ws, kStTimeout);
+        if (__syncthreads_or(!arrived)) {
+            // a copy did not complete in time: issue nothing more, give every copy still in flight
+            // one more bounded wait (no copy may outlive the block), and leave
+            if (tid == 0) {
+                for (int k = 0; k < G::STAGES; ++k) {
+                    const int sk = (iter + k) % G::STAGES;
+                    if (sm.item_ring[sk] < a.items) mbar_wait(&sm.bar[sk], (uint32_t)(((iter + k) / G::STAGES) & 1));
+                }
+            }
+            break;
+        }
 
         // ---------------- parse: Rice codes -> zig-zag scratch ----------------
         uint32_t cosbits = 0;

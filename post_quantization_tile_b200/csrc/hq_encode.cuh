@@ -33,8 +33,9 @@ struct EncodeArgs {
     uint32_t rk[20];  // Philox round keys of `seed` (key words 0, 1 of rounds 0 .. 9), for the dither
     const RateSearch* search;  // count-only passes of a step search: the step comes from here
     int64_t kv_s0;             // KV: position of the call's first token in every sequence
-    int64_t test_silent_item;  // test only: this item never publishes its offset (-1: none), so its
-                               // successor's bounded look-back must run out and report a timeout
+    int64_t test_silent_item;  // read only by the test build (HQ_TEST_HOOKS): this item never publishes
+                               // its offset (-1: none), so its successor's bounded look-back must run
+                               // out and report a timeout
 };
 
 // SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
@@ -321,7 +322,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                 if (tid == 0) sm.mask_jt = jt;
             }
         }
-        if (!mbar_wait(&sm.bar, (uint32_t)(iter & 1))) status_set(a.ws, kStTimeout);
+        const bool arrived = mbar_wait(&sm.bar, (uint32_t)(iter & 1));
+        if (!arrived) status_set(a.ws, kStTimeout);
+        if (__syncthreads_or(!arrived)) {
+            // the input copy did not complete in time: one more bounded wait (the copy may not
+            // outlive the block), then leave; items after this one time out in their look-back
+            if (tid == 0) mbar_wait(&sm.bar, (uint32_t)(iter & 1));
+            break;
+        }
 
         float2 P[H];
         float sumsq;
@@ -547,7 +555,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                     atomicAdd(&a.ws->count_bits, (unsigned long long)bits);
                 } else {
                     const unsigned long long st = ((item == 0 ? 2ull : 1ull) << 32) | acc_words;
-                    if (item != a.test_silent_item) st_relaxed_u64(a.states + item, st);
+#ifdef HQ_TEST_HOOKS
+                    if (item != a.test_silent_item)
+#endif
+                        st_relaxed_u64(a.states + item, st);
                 }
             }
         }
@@ -659,7 +670,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                 }
             }
             if (lane == 0) {
+#ifdef HQ_TEST_HOOKS
                 if (item > 0 && item != a.test_silent_item)
+#else
+                if (item > 0)
+#endif
                     st_relaxed_u64(a.states + item, (2ull << 32) | (unsigned long long)(excl + item_words));
                 sm.base = excl;
             }

@@ -10,10 +10,13 @@ HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.j
            if h.endswith(".h")]
 
 
-def declared_functions():
-    text = "".join(open(h).read() for h in HEADERS)
+def declared_functions(headers=None):
+    text = "".join(open(h).read() for h in (headers or [h for h in HEADERS if not h.endswith("hq_test.h")]))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(hq_[a-z_0-9]+)\s*\(", text)))
+
+
+TEST_HEADER = os.path.join(ROOT, "include", "hq_test.h")
 
 
 @pytest.fixture(scope="module")
@@ -33,6 +36,17 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(libhq):
     missing = [f for f in declared_functions() if not hasattr(libhq, f)]
     assert not missing, missing
+
+
+def test_test_entry_points_live_only_in_the_test_library(libhq):
+    """hq_test.h's entry points are exported by libhq_test.so (built with the test hooks) and not
+    by the product library; the test library also exports every product entry point."""
+    from post_quantization_tile_b200 import build
+    test_only = declared_functions([TEST_HEADER])
+    assert test_only
+    assert not [f for f in test_only if hasattr(libhq, f)]
+    T = ctypes.CDLL(build.TEST_LIB)
+    assert not [f for f in test_only + declared_functions() if not hasattr(T, f)]
 
 
 def test_host_only_entry_points(libhq):

@@ -19,20 +19,30 @@ CANARY = 0x5A5A5A5A
 @pytest.fixture(scope="module")
 def hq():
     import post_quantization_tile_b200 as m
-    L = m.lib()
-    L.hq_test_encode_silent_item.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64,
-                                             ctypes.POINTER(m.Params), ctypes.POINTER(m.CodeStruct), ctypes.c_void_p,
-                                             ctypes.c_size_t, ctypes.c_int64, ctypes.c_void_p]
-    L.hq_test_encode_silent_item.restype = ctypes.c_int32
+    m.lib()
     return m
 
 
-def test_silent_item_times_out_and_the_context_survives(hq):
+@pytest.fixture(scope="module")
+def test_lib(hq):
+    """libhq_test.so: the library built with the test hooks (the product library has none)."""
+    from post_quantization_tile_b200 import build
+    T = ctypes.CDLL(build.TEST_LIB)
+    T.hq_test_encode_silent_item.argtypes = [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.POINTER(hq.Params), ctypes.POINTER(hq.CodeStruct), ctypes.c_void_p,
+                                             ctypes.c_size_t, ctypes.c_int64, ctypes.c_void_p]
+    T.hq_test_encode_silent_item.restype = ctypes.c_int32
+    T.hq_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(hq.Params)]
+    T.hq_workspace_bytes.restype = ctypes.c_size_t
+    return T
+
+
+def test_silent_item_times_out_and_the_context_survives(hq, test_lib):
     xb = W.llama_weight(1024, 512, seed=2)
     x = t_bf16(xb)
     p = hq.params(128, hq.E8, 0.3, 4.0, 3)
     code = hq.alloc_code(1024, 512, p)
-    L = hq.lib()
+    L = test_lib
     ws = hq.Workspace(L.hq_workspace_bytes(1024, 512, ctypes.byref(p)))
     cs = code.struct()
     rc = L.hq_test_encode_silent_item(ctypes.c_void_p(x.data_ptr()), 0, 1024, 512, ctypes.byref(p), ctypes.byref(cs),
