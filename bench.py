@@ -59,7 +59,7 @@ def make_inputs():
 # ------------------------------------------------------------------------------------------------
 # CPU oracle arm (bounded sample)
 # ------------------------------------------------------------------------------------------------
-def oracle_sample(inputs, rows_per_matrix: int, steps: int, betas=None):
+def oracle_sample(inputs, rows_per_matrix: int, steps: int, betas=None, want_codes=False):
     """The oracle's encode + decode of the first rows of each matrix, `steps` passes, timed on one
     host thread.  Returns GB/s of bf16 input, seconds, scalars and the last pass's (code, x_hat)
     per matrix."""
@@ -72,7 +72,7 @@ def oracle_sample(inputs, rows_per_matrix: int, steps: int, betas=None):
             xs = np.ascontiguousarray(x[:rows_per_matrix])
             beta = betas[i] if betas is not None else 0.28
             t0 = time.perf_counter()
-            code = oracle.encode(xs, TILE, oracle.E8, beta, SEED)
+            code = oracle.encode(xs, TILE, oracle.E8, beta, SEED, want_codes=want_codes)
             xo, _ = oracle.decode(code)
             t_total += time.perf_counter() - t0
             elems += xs.size
@@ -81,12 +81,67 @@ def oracle_sample(inputs, rows_per_matrix: int, steps: int, betas=None):
     return gbs, t_total, elems, last
 
 
+def oracle_threads(jobs, workers):
+    """Run oracle (encode, decode) jobs -- (x, n, lattice, beta, seed, kv, kv_S, row0) row ranges of
+    whole 32-row chunks -- on `workers` host threads (the oracle's C code runs with the Python lock
+    released) and return the wall-clock seconds.  Each job runs the same single-threaded code."""
+    import concurrent.futures as cf
+
+    import oracle
+
+    def one(j):
+        x, n, lat, beta, seed, kv, kv_S, row0 = j
+        code = oracle.encode(x, n, lat, beta, seed, kv, kv_S, row0=row0)
+        oracle.decode(code)
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(one, jobs))
+    return time.perf_counter() - t0
+
+
+def row_jobs(x, parts, n, lat, beta, seed, kv=False, kv_S=0):
+    rows = x.shape[0]
+    step = max(32, ((rows + parts - 1) // parts + 31) // 32 * 32)
+    return [(np.ascontiguousarray(x[r:r + step]), n, lat, beta, seed, kv, kv_S, r) for r in range(0, rows, step)]
+
+
+def cpu_baselines(host, betas, kv_keys_bits, kv_beta4):
+    """The oracle on the host cores: one thread and all threads (std::thread-style row ranges
+    through a thread pool) on the tiny fp32 weight, both LLaMA-7B matrices whole, and a sample of
+    the KV key tensor at 4 bps.  GB/s of input per entry; cores = threads used."""
+    import oracle
+
+    from post_quantization_tile_b200 import workloads as W
+    cores = os.cpu_count() or 1
+    out = {}
+    tiny = W.tiny_weight(0)
+    cases = [("tiny_fp32_256x256_E8_n64_4bps", [(tiny, 64, oracle.E8, 0.27, 0, False, 0)], 4),
+             ("llama7b_4096x4096+11008x4096_bf16_E8_n128_4bps",
+              [(x, TILE, oracle.E8, betas[i], SEED, False, 0) for i, x in enumerate(host)], 2)]
+    if kv_keys_bits is not None:
+        cases.append(("kv_keys_1x32x8192x128_bf16_D4_dither_n128_4bps (one batch entry of the key workload)",
+                      [(kv_keys_bits, 128, oracle.D4, kv_beta4, SEED, True, 8192)], 2))
+    for name, mats, es in cases:
+        scalars = sum(m[0].size for m in mats)
+        one = [j for (x, n, lat, beta, seed, kv, kvS) in mats for j in row_jobs(x, 1, n, lat, beta, seed, kv, kvS)]
+        allj = [j for (x, n, lat, beta, seed, kv, kvS) in mats for j in row_jobs(x, 4 * cores, n, lat, beta, seed, kv, kvS)]
+        t1 = oracle_threads(one, 1)
+        ta = oracle_threads(allj, cores)
+        out[name] = {"scalars": scalars, "gbs_1_thread": es * scalars / t1 / 1e9, "seconds_1_thread": t1,
+                     "gbs_all_threads": es * scalars / ta / 1e9, "seconds_all_threads": ta, "threads": cores}
+    return out
+
+
 def parity_vs_oracle(codes, host, mse, last):
     """The GPU codes of the whole matrices against the oracle's, both at the same step: tiles whose
-    scale or Rice header differ, whether the bitstreams are identical, rates and distortions."""
+    scale or Rice header differ, whether the bitstreams are identical, index disagreements within
+    1e-6 of a Voronoi boundary (oracle/parity.py: counted, fraction of lattice blocks), rates and
+    distortions."""
+    from oracle import parity
     out = {"scope": "whole matrices, oracle encode at the GPU's step", "tiles": [], "tile_mismatches": [],
-           "bitstream_identical": [], "payload_bps_gpu": [], "payload_bps_oracle": [], "nmse_gpu": mse,
-           "nmse_oracle": [], "nmse_rel_diff": []}
+           "bitstream_identical": [], "boundary_disagreements": [], "lattice_blocks": [],
+           "disagreement_fraction": [], "comparator_ok": [], "payload_bps_gpu": [], "payload_bps_oracle": [],
+           "nmse_gpu": mse, "nmse_oracle": [], "nmse_rel_diff": []}
     for i, (ref, xo) in enumerate(last):
         c = codes[i]
         scale = c.scale.cpu().numpy().view(np.uint16)
@@ -97,6 +152,12 @@ def parity_vs_oracle(codes, host, mse, last):
         out["tiles"].append(int(ref.tiles))
         out["tile_mismatches"].append(int(np.count_nonzero((scale != ref.scale) | (meta != ref.meta))))
         out["bitstream_identical"].append(bool(same_cw and np.array_equal(bits, ref.bits)))
+        cw = c.chunk_word.cpu().numpy().view(np.uint32)
+        rep = parity.compare(scale, meta, cw, c.bits[:max(int(cw[-1]), 1)].cpu().numpy().view(np.uint32), ref)
+        out["boundary_disagreements"].append(rep.disagreements)
+        out["lattice_blocks"].append(rep.blocks)
+        out["disagreement_fraction"].append(rep.fraction)
+        out["comparator_ok"].append(rep.ok)
         out["payload_bps_gpu"].append(c.payload_bps())
         out["payload_bps_oracle"].append(ref.payload_bits() / float(ref.rows * ref.cols))
         xf = bf16_bits_to_f64(host[i])
@@ -173,17 +234,28 @@ def instruction_check():
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle (the plain restatement of the method) on all host cores,
+    each step the encode + decode of the first 512 rows of both LLaMA-7B matrices at the step the
+    oracle's own search finds for 4.00 payload bps on that sample; rows go to the threads in whole
+    32-row chunks."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
     inputs = make_inputs()
     rows = 512
+    cores = os.cpu_count() or 1
     # the step of each sample for the target rate, by the oracle's own search (untimed)
     betas = [oracle.step_search(np.ascontiguousarray(x[:rows]), TILE, oracle.E8, BPS, seed=SEED, step0=0.28)[0]
              for x in inputs]
-    oracle_sample(inputs, rows, max(1, args.warmup // 3), betas=betas)
-    gbs, secs, elems, last = oracle_sample(inputs, rows, args.steps, betas=betas)
+    jobs = [j for i, x in enumerate(inputs) for j in row_jobs(np.ascontiguousarray(x[:rows]), cores, TILE, oracle.E8,
+                                                             betas[i], SEED)]
+    for _ in range(max(1, args.warmup // 3)):
+        oracle_threads(jobs, cores)
+    secs = sum(oracle_threads(jobs, cores) for _ in range(args.steps))
+    elems = args.steps * sum(rows * x.shape[1] for x in inputs)
+    gbs = elems * 2 / secs / 1e9
+    _, _, _, last = oracle_sample(inputs, rows, 1, betas=betas)
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
@@ -191,8 +263,9 @@ def run_reference(args):
         "config": {"workload": "llama7b_linear_4096x4096+11008x4096_bf16_E8_n128_4bps",
                    "sample": f"first {rows} rows of each matrix per step", "step": betas,
                    "payload_bps": [c.payload_bits() / float(c.rows * c.cols) for c, _ in last]},
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{rows} rows x 4096 of each matrix per step, {args.steps} steps"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} rows x 4096 of each matrix per step, {args.steps} steps, "
+                                   f"{cores} threads over 32-row chunks"},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -414,12 +487,21 @@ def run_gpu(args):
     kv = None if args.no_kv else run_kv(hq, dev, stream, peak)
     gemm = None if args.no_gemm else run_gemm(hq, dev, load_bf16_peak())
 
+    work = None if args.no_workloads else run_workloads(hq, dev, stream, peak, xs)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = max(r for r, _ in SHAPES)
-        gbs, secs, elems, last = oracle_sample(host, rows, 2, betas=steps_beta)
+        gbs, secs, elems, last = oracle_sample(host, rows, 1, betas=steps_beta, want_codes=True)
+        from post_quantization_tile_b200 import workloads as W
+        # one batch entry (32 heads x 8192 tokens) of the key workload's distribution
+        kvb = W.kv_keys(1, 32, 8192, 128, seed=2).reshape(-1, 128) if kv is not None else None
+        per = cpu_baselines(host, steps_beta, kvb, kv["rates"][2]["step"] if kv is not None else None)
+        main = per["llama7b_4096x4096+11008x4096_bf16_E8_n128_4bps"]
         cpu = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"encode+decode of both whole matrices, 2 passes ({elems} scalars, {secs:.1f} s, one thread)",
+               "sample": f"encode+decode of both whole matrices, 1 pass ({elems} scalars, {secs:.1f} s, one thread)",
+               "cores_all": main["threads"], "value_all_cores": main["gbs_all_threads"],
+               "per_workload": per,
                "parity": parity_vs_oracle(codes[0], host, mse, last)}
 
     if rank == 0:
@@ -446,6 +528,7 @@ def run_gpu(args):
                     "h2d_bytes_per_step": bf16_bytes, "d2h_bytes_per_step": bf16_bytes},
             "gpu_launches": 4 * args.steps,
             "kv_cache": kv,
+            "workloads": work,
             "gemm_int8": gemm,
             "instruction_roof": instruction_check(),
             "clocks": clk.summary(),
@@ -463,48 +546,193 @@ def percentiles(calls):
     return [float(v) for v in q]
 
 
+def code_bytes_of(code) -> int:
+    """Bytes of a code: the bitstream words, scale + meta (4 bytes per tile) and the chunk offsets."""
+    return 4 * code.total_words() + 4 * code.scale.numel() + 4 * code.chunk_word.numel()
+
+
+def time_pairs(stream, enc_fns, dec_fns, calls):
+    """Per-call encode and decode times (ms), round-robin over the given calls (alternating inputs
+    keep every call's data out of L2)."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(calls)]
+    for k in range(calls):
+        ev[k][0].record(stream)
+        enc_fns[k % len(enc_fns)]()
+        ev[k][1].record(stream)
+        ev[k][2].record(stream)
+        dec_fns[k % len(dec_fns)]()
+        ev[k][3].record(stream)
+    torch.cuda.synchronize()
+    return [e[0].elapsed_time(e[1]) for e in ev], [e[2].elapsed_time(e[3]) for e in ev]
+
+
+def codec_entry(name, scalars, in_bytes_per_scalar, code, enc, dec, peak, **extra):
+    """One workload's line: per-call p10/p50/p90, GB/s of input, and the roofline fraction of
+    encode and decode (algorithmic bytes = input + code, against the measured copy bandwidth)."""
+    moved = in_bytes_per_scalar * scalars + code_bytes_of(code)
+    e50, d50 = statistics.median(enc), statistics.median(dec)
+    return {"workload": name, "scalars": scalars, "payload_bps": code.payload_bps(), "total_bps": code.total_bps(),
+            "encode_ms_p10_p50_p90": percentiles(enc), "decode_ms_p10_p50_p90": percentiles(dec),
+            "encode_gbs_in": in_bytes_per_scalar * scalars / (e50 * 1e-3) / 1e9,
+            "decode_gbs_out": in_bytes_per_scalar * scalars / (d50 * 1e-3) / 1e9,
+            "encode_roofline_frac": moved / (e50 * 1e-3) / 1e9 / peak,
+            "decode_roofline_frac": moved / (d50 * 1e-3) / 1e9 / peak,
+            "bytes_per_call": moved, **extra}
+
+
 def run_kv(hq, dev, stream, peak):
-    """Dithered D4 KV-cache codec on one K tensor [8, 32, 8192, 128] bf16 (268 M scalars, 537 MB)
-    at 2 bps payload: per-call encode and decode times, outside the timed step.  Calls alternate
-    between two tensors (and two codes), 1.07 GB in all, so no call finds its input in L2."""
+    """Dithered D4 KV-cache codec on [8, 32, 8192, 128] bf16 tensors (268 M scalars, 537 MB each):
+    keys at 1.7, 2 and 4 bps payload and values at 2 bps, per-call encode and decode times outside
+    the timed step.  Calls alternate between two tensors (and two codes), 1.07 GB in all, so no
+    call finds its input in L2.  The 2-bps keys also go through the dense-rotation variant."""
     import torch
 
     from post_quantization_tile_b200 import workloads as W
     B, H, S, D = 8, 32, 8192, 128
+    n = B * H * S * D
     keys = [torch.from_numpy(W.kv_keys(B, H, S, D, seed=2 + i).view(np.int16)).view(torch.bfloat16).to(dev)
             for i in range(2)]
-    beta = hq.calibrate_step(keys[0], D, hq.D4, 2.0, seed=SEED, kv=True, kv_S=S)
-    codes = [hq.kv_encode(keys[i], step=beta, seed=SEED) for i in range(2)]
+    vals = [torch.from_numpy(W.kv_values(B, H, S, D, seed=2 + 10 * i).view(np.int16)).view(torch.bfloat16).to(dev)
+            for i in range(2)]
     out = torch.empty_like(keys[0])
-    calls = 10
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(calls)]
-    for k in range(3):
-        hq.kv_encode(keys[k % 2], step=beta, seed=SEED, out=codes[k % 2], ws=codes[k % 2].ws)
-        hq.decode(codes[(k + 1) % 2], out=out.view(-1, D), ws=codes[(k + 1) % 2].ws)
-    for k in range(calls):
-        a, b = k % 2, (k + 1) % 2
-        ev[k][0].record(stream)
-        hq.kv_encode(keys[a], step=beta, seed=SEED, out=codes[a], ws=codes[a].ws)
-        ev[k][1].record(stream)
-        ev[k][2].record(stream)
-        hq.decode(codes[b], out=out.view(-1, D), ws=codes[b].ws)
-        ev[k][3].record(stream)
+    entries = []
+    beta2 = None
+    for kind, tens, rate in (("keys", keys, 1.7), ("keys", keys, 2.0), ("keys", keys, 4.0), ("values", vals, 2.0)):
+        beta = hq.calibrate_step(tens[0], D, hq.D4, rate, seed=SEED, kv=True, kv_S=S)
+        if kind == "keys" and rate == 2.0:
+            beta2 = beta
+        codes = [hq.kv_encode(tens[i], step=beta, seed=SEED) for i in range(2)]
+        enc_fns = [lambda i=i: hq.kv_encode(tens[i], step=beta, seed=SEED, out=codes[i], ws=codes[i].ws) for i in range(2)]
+        dec_fns = [lambda i=i: hq.decode(codes[i], out=out.view(-1, D), ws=codes[i].ws) for i in (1, 0)]
+        time_pairs(stream, enc_fns, dec_fns, 3)
+        enc, dec = time_pairs(stream, enc_fns, dec_fns, 10)
+        st, _ = hq.status(codes[0].ws)
+        entries.append(codec_entry(f"kv_{kind}_8x32x8192x128_bf16_D4_dither_n128_{rate:g}bps", n, 2, codes[0], enc,
+                                   dec, peak, target_bps=rate, step=beta, status=st))
+    k2 = entries[1]
+    dense = run_kv_dense(hq, keys, beta2, S, D, stream)
+    return {"workload": "kv_keys_8x32x8192x128_bf16_D4_dither_n128_2bps", "step": k2["step"],
+            "dense_rotation": dense, "payload_bps": k2["payload_bps"], "total_bps": k2["total_bps"],
+            "encode_ms_p10_p50_p90": k2["encode_ms_p10_p50_p90"], "decode_ms_p10_p50_p90": k2["decode_ms_p10_p50_p90"],
+            "encode_gbs_bf16": k2["encode_gbs_in"], "decode_gbs_bf16": k2["decode_gbs_out"],
+            "encode_roofline_frac": k2["encode_roofline_frac"], "decode_roofline_frac": k2["decode_roofline_frac"],
+            "bytes_per_call": k2["bytes_per_call"], "status": k2["status"], "rates": entries}
+
+
+def run_workloads(hq, dev, stream, peak, xs_llama):
+    """Throughput on the other synthetic workloads, outside the timed step: the tiny fp32 weight,
+    the LLaMA-7B shapes at 3 and 5 bps, one 70B-shaped matrix per lattice at 3/4/5 bps, and the
+    whole 48-block DiT stack at 4 bps.  Each line: per-call times, GB/s and roofline fractions,
+    payload / total bps, NMSE against the input."""
+    import torch
+
+    from post_quantization_tile_b200 import workloads as W
+
+    def nmse(code, x, ws):
+        y = hq.decode(code, dtype=torch.float32, ws=ws)
+        xf = x.float()
+        return float(((y - xf) ** 2).mean().item() / (xf ** 2).mean().item())
+
+    res = {}
+    # tiny fp32 weight (256 x 256, n = 64): L2-resident and launch-bound by nature
+    xt = torch.from_numpy(W.tiny_weight(0)).to(dev)
+    beta = hq.calibrate_step(xt, 64, hq.E8, 4.0, seed=0)
+    code = hq.encode(xt, 64, hq.E8, beta, seed=0)
+    yt = torch.empty_like(xt)
+    f_e = [lambda: hq.encode(xt, 64, hq.E8, beta, seed=0, out=code, ws=code.ws)]
+    f_d = [lambda: hq.decode(code, out=yt, ws=code.ws)]
+    time_pairs(stream, f_e, f_d, 5)
+    enc, dec = time_pairs(stream, f_e, f_d, 50)
+    res["tiny_fp32"] = codec_entry("tiny_fp32_256x256_E8_n64_4bps", 65536, 4, code, enc, dec, peak, step=beta,
+                                   nmse=nmse(code, xt, code.ws), note="256 KB input: L2-resident, launch-bound",
+                                   status=hq.status(code.ws)[0])
+    # LLaMA-7B shapes at 3 and 5 bps (4 bps is the timed step); inputs rotate over the replicas
+    lines = []
+    for i, (r, c) in enumerate(SHAPES):
+        for rate in (3.0, 5.0):
+            beta = hq.calibrate_step(xs_llama[0][i], TILE, hq.E8, rate, seed=SEED)
+            codes = [hq.encode(xs_llama[k][i], TILE, hq.E8, beta, seed=SEED) for k in range(REPLICAS)]
+            y = torch.empty(r, c, dtype=torch.bfloat16, device=dev)
+            f_e = [lambda k=k: hq.encode(xs_llama[k][i], TILE, hq.E8, beta, seed=SEED, out=codes[k], ws=codes[k].ws)
+                   for k in range(REPLICAS)]
+            f_d = [lambda k=k: hq.decode(codes[k], out=y, ws=codes[k].ws) for k in (1, 2, 0)]
+            time_pairs(stream, f_e, f_d, 3)
+            enc, dec = time_pairs(stream, f_e, f_d, 15)
+            lines.append(codec_entry(f"llama7b_{r}x{c}_bf16_E8_n128_{rate:g}bps", r * c, 2, codes[0], enc, dec, peak,
+                                     target_bps=rate, step=beta, nmse=nmse(codes[0], xs_llama[0][i], codes[0].ws),
+                                     status=hq.status(codes[0].ws)[0]))
+    res["llama7b_3_5bps"] = lines
+    # lattice sweep on the 70B-shaped 8192 x 28672 matrix (470 MB, far above L2), n = 256
+    x70 = torch.from_numpy(W.llama_70b_weight(8192, 28672, seed=4).view(np.int16)).view(torch.bfloat16).to(dev)
+    y70 = torch.empty_like(x70)
+    lines = []
+    for name, lat in (("A2", hq.A2), ("D4", hq.D4), ("E8", hq.E8), ("Z", hq.Z)):
+        for rate in (3.0, 4.0, 5.0):
+            beta = hq.calibrate_step(x70, 256, lat, rate, seed=4)
+            code = hq.encode(x70, 256, lat, beta, seed=4)
+            f_e = [lambda: hq.encode(x70, 256, lat, beta, seed=4, out=code, ws=code.ws)]
+            f_d = [lambda: hq.decode(code, out=y70, ws=code.ws)]
+            time_pairs(stream, f_e, f_d, 2)
+            enc, dec = time_pairs(stream, f_e, f_d, 6)
+            lines.append(codec_entry(f"llama70b_8192x28672_bf16_{name}_n256_{rate:g}bps", x70.numel(), 2, code, enc,
+                                     dec, peak, lattice=name, target_bps=rate, step=beta, nmse=nmse(code, x70, code.ws),
+                                     status=hq.status(code.ws)[0]))
+    res["lattice_sweep_70b"] = lines
+    del x70, y70
+    torch.cuda.empty_cache()
+    res["dit_stack"] = run_dit_stack(hq, dev, stream, peak)
+    return res
+
+
+def run_dit_stack(hq, dev, stream, peak):
+    """The whole DiT-shaped stack: 48 blocks of 4 x 4096x4096 and 4096x16384 + 16384x4096 bf16
+    linears (9.66 G parameters, 19.3 GB), E8 at 4 bps, n = 128.  Weights are drawn on the device
+    (the host generator would take minutes); the step is searched per matrix; one pass encodes
+    every matrix, one pass decodes every code, each timed as a whole with CUDA events."""
+    import torch
+
+    from post_quantization_tile_b200 import workloads as W
+    blocks = 48
+    mats, betas, codes = [], [], []
+    for b in range(blocks):
+        for i, (r, c) in enumerate(W.DIT_BLOCK_SHAPES):
+            x = W.dit_linear_device(r, c, 5 + 100 * b + i, dev)
+            beta = hq.calibrate_step(x, TILE, hq.E8, 4.0, seed=5 + b)
+            mats.append(x)
+            betas.append(beta)
+            codes.append(hq.encode(x, TILE, hq.E8, beta, seed=5 + b))
+    outs = {shape: torch.empty(*shape, dtype=torch.bfloat16, device=dev) for shape in set(W.DIT_BLOCK_SHAPES)}
+    ws = codes[0].ws
+    params = sum(x.numel() for x in mats)
+
+    def enc_all():
+        for j, x in enumerate(mats):
+            hq.encode(x, TILE, hq.E8, betas[j], seed=5 + j // 6, out=codes[j], ws=ws)
+
+    def dec_all():
+        for j, cd in enumerate(codes):
+            hq.decode(cd, out=outs[tuple(mats[j].shape)], ws=ws)
+    enc_all()
+    dec_all()
     torch.cuda.synchronize()
-    st, _ = hq.status(codes[0].ws)
-    enc = [e[0].elapsed_time(e[1]) for e in ev]
-    dec = [e[2].elapsed_time(e[3]) for e in ev]
-    n = B * H * S * D
-    code_bytes = 4 * codes[0].total_words() + 4 * codes[0].scale.numel() + 4 * codes[0].chunk_word.numel()
-    moved = 2 * n + code_bytes
+    enc, dec = time_pairs(stream, [enc_all], [dec_all], 3)
+    st, _ = hq.status(ws)
+    cbytes = sum(code_bytes_of(cd) for cd in codes)
     e50, d50 = statistics.median(enc), statistics.median(dec)
-    dense = run_kv_dense(hq, keys, beta, S, D, stream)
-    return {"workload": "kv_keys_8x32x8192x128_bf16_D4_dither_n128_2bps", "step": beta, "dense_rotation": dense,
-            "payload_bps": codes[0].payload_bps(), "total_bps": codes[0].total_bps(),
-            "encode_ms_p10_p50_p90": percentiles(enc), "decode_ms_p10_p50_p90": percentiles(dec),
-            "encode_gbs_bf16": 2 * n / (e50 * 1e-3) / 1e9, "decode_gbs_bf16": 2 * n / (d50 * 1e-3) / 1e9,
-            "encode_roofline_frac": moved / (e50 * 1e-3) / 1e9 / peak,
-            "decode_roofline_frac": moved / (d50 * 1e-3) / 1e9 / peak,
-            "bytes_per_call": moved, "status": st}
+    moved = 2 * params + cbytes
+    pbits = sum(cd.payload_bps() * cd.rows * cd.cols for cd in codes)
+    res = {"workload": "dit_stack_48x(4x4096x4096+4096x16384+16384x4096)_bf16_E8_n128_4bps",
+           "parameters": params, "matrices": len(mats), "launches_per_pass": len(mats),
+           "payload_bps": pbits / params, "encode_pass_ms_p10_p50_p90": percentiles(enc),
+           "decode_pass_ms_p10_p50_p90": percentiles(dec),
+           "encode_gbs_in": 2 * params / (e50 * 1e-3) / 1e9, "decode_gbs_out": 2 * params / (d50 * 1e-3) / 1e9,
+           "encode_roofline_frac": moved / (e50 * 1e-3) / 1e9 / peak,
+           "decode_roofline_frac": moved / (d50 * 1e-3) / 1e9 / peak, "bytes_per_pass": moved,
+           "data": "device-drawn (torch CUDA generator), same distribution as the host generator", "status": st}
+    del mats, codes, outs
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_kv_dense(hq, keys, beta, S, D, stream):
@@ -692,6 +920,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kv", action="store_true", help="skip the KV-cache codec fields")
     ap.add_argument("--no-gemm", action="store_true", help="skip the int8 GEMM fields")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other workloads' throughput fields")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)

@@ -409,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
         constexpr int PB = H / 8 / ROT;  // pair-blocks per round
 #pragma unroll 1
         for (int rr = 0; rr < ROT; ++rr) {
+            uint32_t rare = 0;  // E8: blocks of this round to redo with the plain rule (bit 2 gb + lane)
 #pragma unroll
             for (int gb = 0; gb < PB; ++gb) {
                 const int g8 = rr * PB + gb;
@@ -426,8 +427,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                         for (int i = 0; i < 8; ++i) p8[i] = make_float2(__fadd_rn(p8[i].x, Ux[i]), __fadd_rn(p8[i].y, Uy[i]));
                     }
                     int32_t sx[8], sy[8], vx[8], vy[8];
-                    uint32_t cx, cy;
-                    e8_pair_symbols<SRC == 2>(p8, sx, sy, cx, cy, vx, vy);
+                    uint32_t cx, cy, rare2;
+                    e8_pair_symbols<SRC == 2>(p8, sx, sy, cx, cy, vx, vy, rare2);
+                    rare |= rare2 << (2 * gb);
                     if constexpr (SRC == 2) {
                         if (valid && a.v_out) {
                             int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V;
@@ -487,6 +489,45 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                             }
                         }
                         store_group(half * (H / 8) + g8, sym);
+                    }
+                }
+            }
+            if constexpr (LAT == HQ_E8) {
+                // blocks within 2^-16 of a coset tie, or whose fix-up meets the key floor: redo
+                // them with the plain rule and replace their symbols, coset bit and codes
+                if (rare) {
+#pragma unroll
+                    for (int gb = 0; gb < PB; ++gb) {
+#pragma unroll
+                        for (int ln = 0; ln < 2; ++ln) {
+                            if (!((rare >> (2 * gb + ln)) & 1u)) continue;
+                            const int g8 = rr * PB + gb;
+                            float u8[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) u8[i] = ln ? P[gb * 8 + i].y : P[gb * 8 + i].x;
+                            if constexpr (KV) {
+                                float U[8];
+                                dither_e8(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + ln * (H / 4) + 2 * g8), U);
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) u8[i] = __fadd_rn(u8[i], U[i]);
+                            }
+                            int32_t s8[8], v8[8];
+                            const uint32_t c = e8_symbols<SRC == 2>(u8, s8, v8);
+                            const int slot = ln * (H / 8) + g8;
+                            const uint4 old = *zz_slot(zzs, slot, tid);
+                            A -= (old.x & 0xFFFFu) + (old.x >> 16) + (old.y & 0xFFFFu) + (old.y >> 16) +
+                                 (old.z & 0xFFFFu) + (old.z >> 16) + (old.w & 0xFFFFu) + (old.w >> 16);
+                            store_group(slot, s8);
+                            const int cb = ln * (H / 8) + g8;
+                            cosbits = (cosbits & ~(1u << cb)) | (c << cb);
+                            if constexpr (SRC == 2) {
+                                if (valid && a.v_out) {
+                                    int32_t* vo = a.v_out + (r0 + row_l) * (int64_t)N + tau * V + ln * H + g8 * 8;
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i) vo[i] = v8[i];
+                                }
+                            }
+                        }
                     }
                 }
             }

@@ -5,10 +5,11 @@
 // quantizers and codes" (IEEE T-IT 28(2), 1982), in binary32 without contraction:
 //   a = rint(u) via the 1.5*2^23 addition (exact for |u| < 2^22, which the per-tile RMS scaling
 //   and the step range guarantee), e = a - u (exact, never -0), "toward u" = +1 when e < 0;
-//   argmax / argmin of |e| with ties to the lowest index.  The fast comparison runs on 32-bit keys
-//   (max(|e|, 2^-31) bits << 4 | index << 1 | sign of e): the bits of |e| in [2^-31, 1/2] all
-//   start with 0011, so the shift drops nothing that orders them, and one integer max / min returns
-//   the value, the lowest tied index and the sign together.  Where the 2^-31 floor could change the
+//   argmax / argmin of |e| with ties to the lowest index.  D4 compares exact 32-bit keys (bits of
+//   |e| << 2 | index).  E8's eight coordinates need three index bits, so its keys are
+//   max(|e|, 2^-31) bits << 4 | index << 1 | sign of e: the bits of |e| in [2^-31, 1/2] all start
+//   with 0011, so the shift drops nothing that orders them, and one integer max / min returns the
+//   value, the lowest tied index and the sign together.  Where the 2^-31 floor could change the
 //   outcome (a fix-up among rounding errors below 2^-31), and where two cosets (E8, A2) come within
 //   a band of a tie that covers the rounding of the shortcut formula, the plain rule runs instead:
 //   exact argmax / argmin and both candidates' squared distances in binary32, summed in coordinate
@@ -57,7 +58,10 @@ __device__ __forceinline__ uint32_t max_key(float e, int i, int d)
 __device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float((key >> 4) | kTinyBits); }
 
 // D4 = {v in Z^4, sum even}; v = the nearest point: round, and if the sum is odd move the
-// coordinate with the largest rounding error one step toward u.
+// coordinate with the largest rounding error one step toward u.  |e| <= 1/2, so the bits of |e|
+// fit in 30 bits and bits(e) << 2 is |e|'s bits << 2 (the sign shifts out): with the index in
+// the two low bits one integer max is the exact argmax with the lowest index on ties, for every
+// |e| down to 0.  The sign of the chosen coordinate's e is picked out afterwards.
 __device__ __forceinline__ void q_d4(const float (&u)[4], int32_t (&v)[4])
 {
     int32_t sum = 0;
@@ -68,22 +72,11 @@ __device__ __forceinline__ void q_d4(const float (&u)[4], int32_t (&v)[4])
         const float r = rint_magic(u[i], v[i]);
         sum += v[i];
         e[i] = __fadd_rn(r, -u[i]);
-        kmax = max(kmax, max_key(e[i], i, 4));
+        kmax = max(kmax, (__float_as_uint(e[i]) << 2) | (uint32_t)(3 - i));
     }
-    int j = 3 - (int)((kmax >> 1) & 7u);
-    int32_t delta = (sum & 1) ? ((kmax & 1u) ? 1 : -1) : 0;
-    if ((sum & 1) && kmax < 16u) {
-        // every |e| is below the 2^-31 floor of the keys: the exact argmax (lowest index on ties)
-        j = 0;
-        float best = fabsf(e[0]);
-#pragma unroll
-        for (int i = 1; i < 4; ++i)
-            if (fabsf(e[i]) > best) {
-                best = fabsf(e[i]);
-                j = i;
-            }
-        delta = e[j] < 0.0f ? 1 : -1;
-    }
+    const int j = 3 - (int)(kmax & 3u);
+    const float ej = j == 0 ? e[0] : (j == 1 ? e[1] : (j == 2 ? e[2] : e[3]));
+    const int32_t delta = (sum & 1) ? (ej < 0.0f ? 1 : -1) : 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         if (i == j) v[i] += delta;
@@ -93,35 +86,37 @@ __device__ __forceinline__ void q_d4(const float (&u)[4], int32_t (&v)[4])
 // point is 2a (+2 toward z at the fixed coordinate) and a coset B point 2a + toward (-2 toward at
 // the fixed coordinate), so z - p = -2e - c exactly): exact argmax / argmin of |e| with the lowest
 // index on ties, squared distances summed in coordinate order in binary32, A on ties.  Returns
-// isB | fix << 1 | (delta + 1) << 4, delta the move of the fixed coordinate of w.  Rarely taken:
-// kept out of line.
-struct E8Err {
-    float e[8];
-};
-static __device__ __noinline__ uint32_t e8_plain_choice(const E8Err E, const uint32_t parA, const uint32_t parB)
+// isB | fix << 1 | (delta + 1) << 4, delta the move of the fixed coordinate of w.  Rarely taken.
+static __device__ __forceinline__ uint32_t e8_plain_choice(const float e0, const float e1, const float e2, const float e3,
+                                                        const float e4, const float e5, const float e6, const float e7,
+                                                        const uint32_t parA, const uint32_t parB)
 {
+    const float e[8] = {e0, e1, e2, e3, e4, e5, e6, e7};
     int j = 0, m = 0;
-    float bmax = fabsf(E.e[0]), bmin = bmax;
+    float bmax = fabsf(e[0]), bmin = bmax;
+    float ej = e[0], em = e[0];
 #pragma unroll
     for (int i = 1; i < 8; ++i) {
-        const float a = fabsf(E.e[i]);
+        const float a = fabsf(e[i]);
         if (a > bmax) {
             bmax = a;
             j = i;
+            ej = e[i];
         }
         if (a < bmin) {
             bmin = a;
             m = i;
+            em = e[i];
         }
     }
     float dA = 0.0f, dB = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float t = E.e[i] < 0.0f ? 1.0f : -1.0f;
+        const float t = e[i] < 0.0f ? 1.0f : -1.0f;
         const float cA = (parA && i == j) ? 2.0f * t : 0.0f;
         const float cB = (parB && i == m) ? -t : t;
-        const float xA = __fadd_rn(__fmul_rn(-2.0f, E.e[i]), -cA);
-        const float xB = __fadd_rn(__fmul_rn(-2.0f, E.e[i]), -cB);
+        const float xA = __fadd_rn(__fmul_rn(-2.0f, e[i]), -cA);
+        const float xB = __fadd_rn(__fmul_rn(-2.0f, e[i]), -cB);
         dA = __fadd_rn(dA, __fmul_rn(xA, xA));
         dB = __fadd_rn(dB, __fmul_rn(xB, xB));
     }
@@ -129,7 +124,7 @@ static __device__ __noinline__ uint32_t e8_plain_choice(const E8Err E, const uin
     const int fix = isB ? m : j;
     const uint32_t dofix = isB ? parB : parA;
     // A moves toward u (+1 when e < 0), B away from its first half-integer (-1 when e < 0)
-    const int ef = E.e[fix] < 0.0f ? 1 : -1;
+    const int ef = (isB ? em : ej) < 0.0f ? 1 : -1;
     const int delta = dofix ? (isB ? -ef : ef) : 0;
     return isB | ((uint32_t)fix << 1) | ((uint32_t)(delta + 1) << 4);
 }
@@ -144,8 +139,12 @@ static __device__ __noinline__ uint32_t e8_plain_choice(const E8Err E, const uin
 //   B: w = a - [e >= 0] (w + 1/2 is the half-integer toward u); if sum w is odd the coordinate
 //      with min |e| moves to its other half-integer neighbour.
 // E8 decision from t = u + 1.5*2^23 and e = (t - 1.5*2^23) - u (computed by the caller)
-template <bool WANT_V>
-__device__ __forceinline__ uint32_t e8_from_te(const float (&tv)[8], const float (&ev)[8], int32_t (&s)[8], int32_t* v)
+// DEFER: instead of running the plain rule here, set `rare` and return the shortcut's point; the
+// caller then redoes the block with e8_symbols (which never defers).  Kept out of the unrolled
+// quantizer body, the rare branch does not split its straight-line code.
+template <bool WANT_V, bool DEFER = false>
+__device__ __forceinline__ uint32_t e8_from_te(const float (&tv)[8], const float (&ev)[8], int32_t (&s)[8], int32_t* v,
+                                               uint32_t* rare = nullptr)
 {
     int32_t a[8];
     float ae[8];
@@ -178,14 +177,16 @@ __device__ __forceinline__ uint32_t e8_from_te(const float (&tv)[8], const float
     const uint32_t dofix = isB ? parB : parA;
     int32_t delta = dofix ? ((((kf & 1u) != 0u) != isB) ? 1 : -1) : 0;
     // near a coset tie, or where a fix-up meets the 2^-31 floor of the keys: the plain rule
-    if (fabsf(D) <= kTieBand || (parA && kmax < 16u) || (parB && kmin < 16u)) {
-        E8Err E;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) E.e[i] = ev[i];
-        const uint32_t r = e8_plain_choice(E, parA, parB);
-        isB = (r & 1u) != 0u;
-        fix = (int)((r >> 1) & 7u);
-        delta = (int32_t)(r >> 4) - 1;
+    const bool plain = fabsf(D) <= kTieBand || (parA && kmax < 16u) || (parB && kmin < 16u);
+    if constexpr (DEFER) {
+        *rare = plain ? 1u : 0u;
+    } else {
+        if (plain) {
+            const uint32_t r = e8_plain_choice(ev[0], ev[1], ev[2], ev[3], ev[4], ev[5], ev[6], ev[7], parA, parB);
+            isB = (r & 1u) != 0u;
+            fix = (int)((r >> 1) & 7u);
+            delta = (int32_t)(r >> 4) - 1;
+        }
     }
     const uint32_t bmask = isB ? 0xFFFFFFFFu : 0u;
     int32_t w[8];
@@ -219,10 +220,11 @@ __device__ __forceinline__ uint32_t e8_symbols(const float (&u)[8], int32_t (&s)
 }
 
 // two E8 blocks at once, one in each lane of eight float2 pairs: the rounding arithmetic runs on
-// paired binary32 operations (the same roundings as e8_symbols), the decisions per lane
+// paired binary32 operations (the same roundings as e8_symbols), the decisions per lane.  rare:
+// bit 0 (lane x) / bit 1 (lane y) set where the block must be redone with e8_symbols.
 template <bool WANT_V>
 __device__ __forceinline__ void e8_pair_symbols(const float2 (&p)[8], int32_t (&sx)[8], int32_t (&sy)[8],
-                                                uint32_t& cx, uint32_t& cy, int32_t* vx, int32_t* vy)
+                                                uint32_t& cx, uint32_t& cy, int32_t* vx, int32_t* vy, uint32_t& rare)
 {
     float tx[8], ty[8], ex[8], ey[8];
     const float2 m2 = make_float2(kMagic, kMagic);
@@ -236,8 +238,10 @@ __device__ __forceinline__ void e8_pair_symbols(const float2 (&p)[8], int32_t (&
         tx[i] = t.x; ty[i] = t.y;
         ex[i] = e.x; ey[i] = e.y;
     }
-    cx = e8_from_te<WANT_V>(tx, ex, sx, vx);
-    cy = e8_from_te<WANT_V>(ty, ey, sy, vy);
+    uint32_t rx, ry;
+    cx = e8_from_te<WANT_V, true>(tx, ex, sx, vx, &rx);
+    cy = e8_from_te<WANT_V, true>(ty, ey, sy, vy, &ry);
+    rare = rx | (ry << 1);
 }
 
 // A2 with minimum distance 1 in (P, Q) = (2 u0, u1 K): the even point when |eP| + 3|eQ| <= 1, which is

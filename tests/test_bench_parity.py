@@ -39,8 +39,11 @@ def test_parity_report_on_identical_and_planted_codes():
     assert rep["bitstream_identical"] == [True, True]
     assert rep["payload_bps_gpu"] == rep["payload_bps_oracle"]
     assert max(rep["nmse_rel_diff"]) < 1e-12
+    assert rep["comparator_ok"] == [True, True] and rep["boundary_disagreements"] == [0, 0]
     codes[1].meta[5] ^= 1          # one Rice parameter changed
     codes[1].bits[3] ^= 1 << 7      # one bit flipped
     rep = bench.parity_vs_oracle(codes, host, mse, last)
     assert rep["tile_mismatches"] == [0, 1]
     assert rep["bitstream_identical"] == [True, False]
+    assert rep["comparator_ok"][0] and not rep["comparator_ok"][1]
+    assert rep["boundary_disagreements"][0] == 0
