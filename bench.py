@@ -803,11 +803,54 @@ def run_gemm(hq, dev, peak_bf16):
     dm = [e[2].elapsed_time(e[3]) for e in ev]
     tops = 2.0 * M * N * K / (statistics.median(gm) * 1e-3) / 1e12
     peak = 2.0 * peak_bf16  # int8 dense = 2x bf16 dense (nominal ratio)
+    fused = run_gemm_fused(hq, dev, code, V, g, peak)
     return {"workload": "int8 A[4096,4096] x E8 codes of llama7b 4096x4096 (n=128 groups) -> fp32",
             "gemm_ms_p10_p50_p90": percentiles(gm), "decode_int8_ms_p10_p50_p90": percentiles(dm),
             "roofline": {"bound": "tensor", "achieved": tops, "peak": peak,
                          "peak_kind": "2 x measured bf16 burst", "unit": "TOP/s", "frac": tops / peak},
-            "status": st}
+            "fused": fused, "status": st}
+
+
+def run_gemm_fused(hq, dev, code, V, g, peak):
+    """The decode fused into the GEMM's producer warps (hq_gemm_code) against the two calls
+    (hq_decode_int8, then hq_gemm_int8 on the L2-resident int8 codes) for activation row counts
+    M = 16, 128, 1024, 4096 on the 4096 x 4096 E8 code; the two-call GEMM needs M in multiples of
+    128, so M = 16 runs it on a 128-row activation tile.  Per-call p50 of each arm; both results
+    are compared bit for bit."""
+    import torch
+    N, K = code.rows, code.cols
+    rng = np.random.default_rng(7)
+    out = []
+    for M in (16, 128, 1024, 4096):
+        Mp = max(M, 128)
+        a = torch.from_numpy(np.clip(np.round(rng.standard_normal((Mp, K)) * 32.0), -127, 127).astype(np.int8)).to(dev)
+        sa = torch.full((Mp,), 0.02, dtype=torch.float32, device=dev)
+        Yf = torch.empty(M, N, dtype=torch.float32, device=dev)
+        Y2 = torch.empty(Mp, N, dtype=torch.float32, device=dev)
+        ws = hq.workspace(hq.lib().hq_gemm_code_workspace_bytes(M, N, K))
+        V2, g2 = torch.empty_like(V), torch.empty_like(g)
+        calls = 10
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(calls)]
+        for k in range(calls + 2):
+            e = ev[k - 2] if k >= 2 else None
+            if e:
+                e[0].record()
+            hq.gemm_code(a[:M], sa[:M], code, out=Yf, ws=ws)
+            if e:
+                e[1].record()
+                e[2].record()
+            V2, g2 = hq.decode_int8(code)
+            hq.gemm_int8(a, sa, V2, g2, out=Y2)
+            if e:
+                e[3].record()
+        torch.cuda.synchronize()
+        fm = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+        tm = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
+        same = bool(torch.equal(Yf, Y2[:M]))
+        st = hq.status(ws)[0]
+        out.append({"M": M, "fused_ms": fm, "decode_then_gemm_ms": tm, "fused_over_two_calls": fm / tm,
+                    "fused_tops": 2.0 * M * N * K / (fm * 1e-3) / 1e12, "bit_identical": same, "status": st})
+    return {"workload": "E8 code of llama7b 4096x4096 (n=128) x int8 activations [M, 4096]", "rows": out}
 
 
 def run_profile(args):

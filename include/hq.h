@@ -261,6 +261,25 @@ hq_status_t hq_decode_int8(const hq_code_t* code, int8_t* v_out, float* g_out, v
 hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8_t* V, const float* g, int64_t N,
                          int64_t K, int32_t group, float* Y, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * The same product as hq_decode_int8 followed by hq_gemm_int8, with the decode fused into the
+ * GEMM: producer warps decode the weight's code (Rice codes, unstrip) straight into the tensor
+ * cores' int8 operand stages, so the int8 codes never reach global memory.  W = the code's
+ * weight [N, K] (N = code->rows, K = code->cols, a multiple of 128 each; n = 128; Z, D4 or E8
+ * without dither, HQ_ERR_UNSUPPORTED otherwise); A int8 [M, K] row-major (M >= 1; rows past M of
+ * the last 128-row tile are zeros), sa fp32 [M], Y fp32 [M, N]; all device, 16-byte aligned.
+ *   Y[m, r] = sa[m] * sum_t g[t, r] S(m, r, t)
+ * bit for bit as the two-call path: exact int32 group sums, acc = fma(S, g, acc) over t = 0, 1, ...
+ * from 0 in binary32, then Y = acc * sa[m]; tiles with a code outside int8 are zero (HQ_ERR_RANGE),
+ * corrupt tiles too (HQ_ERR_CORRUPT).  When the output has too few 128 x 128 tiles to occupy the
+ * GPU, the K groups are split into ranges whose binary32 chains hand over through ws in order.
+ * ws: at least hq_gemm_code_workspace_bytes(M, N, K) bytes (status word, per-tile flags and, for
+ * split ranges, one 128 x 128 binary32 chain per output tile); calls sharing ws must not overlap.
+ */
+size_t hq_gemm_code_workspace_bytes(int64_t M, int64_t N, int64_t K);
+hq_status_t hq_gemm_code(const int8_t* A, const float* sa, int64_t M, const hq_code_t* code, float* Y, void* ws,
+                         size_t ws_bytes, void* stream);
+
 /* Result of a step search, written to device memory. */
 typedef struct {
     float step;            /* the chosen step beta                                          */

@@ -79,6 +79,9 @@ def lib():
         L.hq_encode_count.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, P, P, ctypes.c_size_t, P]
         L.hq_decode_int8.argtypes = [ctypes.POINTER(CodeStruct), P, P, P, ctypes.c_size_t, P]
         L.hq_gemm_int8.argtypes = [P, P, i64, P, P, i64, i64, i32, P, P, ctypes.c_size_t, P]
+        L.hq_gemm_code.argtypes = [P, P, i64, ctypes.POINTER(CodeStruct), P, P, ctypes.c_size_t, P]
+        L.hq_gemm_code_workspace_bytes.argtypes = [i64, i64, i64]
+        L.hq_gemm_code_workspace_bytes.restype = ctypes.c_size_t
         L.hq_step_search.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, i32, ctypes.c_float, P, P,
                                      ctypes.c_size_t, P]
         L.hq_kv_dense_workspace_bytes.argtypes = [i64]
@@ -91,7 +94,7 @@ def lib():
         L.hq_status_str.restype = ctypes.c_char_p
         L.hq_version.restype = i32
         for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_encode_at", "hq_kv_decode", "hq_quantize_coeffs",
-                  "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_status_read",
+                  "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_gemm_code", "hq_status_read",
                   "hq_kv_encode_dense", "hq_kv_decode_dense"]:
             getattr(L, f).restype = i32
         _lib = L
@@ -391,6 +394,23 @@ def gemm_int8(A: torch.Tensor, sa: torch.Tensor, V: torch.Tensor, g: torch.Tenso
     w = ws or workspace(4096)
     _check(lib().hq_gemm_int8(_ptr(A), _ptr(sa), M, _ptr(V), _ptr(g), N, K, 128, _ptr(Y), w.ptr(), w.nbytes,
                               _stream()), "hq_gemm_int8")
+    return Y
+
+
+def gemm_code(A: torch.Tensor, sa: torch.Tensor, code: Code, out: torch.Tensor | None = None,
+              ws: Workspace | None = None) -> torch.Tensor:
+    """The product of decode_int8 and gemm_int8 with the decode fused into the GEMM's producer
+    warps (hq_gemm_code): Y [M, code.rows] fp32."""
+    for t, name in ((A, "A"), (sa, "sa")):
+        _require_cuda(t, name)
+    M = A.shape[0]
+    Y = out if out is not None else torch.empty(M, code.rows, dtype=torch.float32, device=A.device)
+    L = lib()
+    w = ws or workspace(L.hq_gemm_code_workspace_bytes(M, code.rows, code.cols))
+    cs = code.struct()
+    _check(L.hq_gemm_code(_ptr(A), _ptr(sa), M, ctypes.byref(cs), _ptr(Y), w.ptr(), w.nbytes, _stream()),
+           "hq_gemm_code")
+    code.ws = w
     return Y
 
 

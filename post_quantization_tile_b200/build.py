@@ -23,11 +23,11 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          # no contraction: the encode chain is specified in binary32 without fused multiply-add
          "-fmad=false", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2", "--expt-relaxed-constexpr"]
-SOURCES = ["hq_api.cu", "hq_noalloc.cu", "hq_gemm.cu", "hq_dense.cu", "hq_inst_z.cu", "hq_inst_a2.cu", "hq_inst_d4.cu",
+SOURCES = ["hq_api.cu", "hq_noalloc.cu", "hq_gemm.cu", "hq_gemm_code.cu", "hq_dense.cu", "hq_inst_z.cu", "hq_inst_a2.cu", "hq_inst_d4.cu",
            "hq_inst_e8.cu"]
 # sources compiled a second time with the test hooks for libhq_test.so
 TEST_SOURCES = ["hq_api.cu", "hq_inst_e8.cu"]
-HEADERS = ["hq_common.cuh", "hq_lattice.cuh", "hq_encode.cuh", "hq_decode.cuh", "hq_instantiate.cuh", "hq_launch.h"]
+HEADERS = ["hq_common.cuh", "hq_tc.cuh", "hq_lattice.cuh", "hq_encode.cuh", "hq_decode.cuh", "hq_instantiate.cuh", "hq_launch.h"]
 
 
 def _newest_dep() -> float:
