@@ -427,6 +427,50 @@ __device__ __forceinline__ uint32_t long_run(BitReader<FWD>& br, uint32_t limit,
     return q;
 }
 
+// the slow path of get_code (a code longer than the bits at hand, long unary runs), out of line:
+// reader state in and out by value
+struct RdOut {
+    unsigned long long W;
+    int avail, wi;
+    uint32_t z;
+    int ok;
+};
+template <bool FWD>
+static __device__ __noinline__ RdOut get_code_slow(unsigned long long W, int avail, int wi, int lim, const uint32_t* src,
+                                                   int k, uint32_t limit)
+{
+    BitReader<FWD> br;
+    br.W = W;
+    br.avail = avail;
+    br.wi = wi;
+    br.lim = lim;
+    br.src = src;
+    br.c0 = 0;
+    bool ok = true;
+    br.refill();
+    uint32_t hi = (uint32_t)(br.W >> 32);
+    uint32_t q = 0;
+    RdOut o;
+    if (hi == 0u) {
+        q = long_run<FWD>(br, limit, ok);
+        hi = (uint32_t)(br.W >> 32);
+        if (!ok) {
+            o.W = br.W; o.avail = br.avail; o.wi = br.wi; o.z = 0u; o.ok = 0;
+            return o;
+        }
+    }
+    const int z = __clz(hi);
+    br.W <<= (z + 1);
+    br.avail -= z + 1;
+    if (br.avail < k) br.refill();
+    const uint32_t r = k ? (uint32_t)(br.W >> (64 - k)) : 0u;
+    br.W <<= k;
+    br.avail -= k;
+    q += (uint32_t)z;
+    o.W = br.W; o.avail = br.avail; o.wi = br.wi; o.z = (q << k) | r; o.ok = 1;
+    return o;
+}
+
 // one Rice code: q zeros, a one, r (k bits MSB-first); returns the zig-zag value q << k | r (the
 // sum of q follows from the bits consumed: consumed() - codes (k + 1)).  The caller tops the window up to at least 33 bits every four codes;
 // a code that is longer than the bits at hand takes the slow path (refill, long runs).
@@ -437,23 +481,12 @@ __device__ __forceinline__ uint32_t get_code(BitReader<FWD>& br, int k, uint32_t
     int z = __clz(hi);
     int lam = z + k + 1;
     if (hi == 0u || lam > br.avail) {
-        br.refill();
-        hi = (uint32_t)(br.W >> 32);
-        uint32_t q = 0;
-        if (hi == 0u) {
-            q = long_run<FWD>(br, limit, ok);
-            hi = (uint32_t)(br.W >> 32);
-            if (!ok) return 0u;
-        }
-        z = __clz(hi);
-        br.W <<= (z + 1);
-        br.avail -= z + 1;
-        if (br.avail < k) br.refill();
-        const uint32_t r = k ? (uint32_t)(br.W >> (64 - k)) : 0u;
-        br.W <<= k;
-        br.avail -= k;
-        q += (uint32_t)z;
-        return (q << k) | r;
+        const RdOut o = get_code_slow<FWD>(br.W, br.avail, br.wi, br.lim, br.src, k, limit);
+        br.W = o.W;
+        br.avail = o.avail;
+        br.wi = o.wi;
+        if (!o.ok) ok = false;
+        return o.z;
     }
     // fast path: the whole code is in the top 32 bits: 0..0 1 r
     const uint32_t val = hi >> (32 - lam);      // (1 << k) | r

@@ -230,21 +230,19 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                 rf.begin(in, tile0 + COSB, G::IN_WORDS - 1);
                 rb.begin(in, tile0 + (int)L - 1, G::IN_WORDS - 1);
 #pragma unroll 1
-                for (int g = 0; g < N / 16; ++g) {
-                    uint32_t zf[8], zb[8];
+                for (int g = 0; g < N / 8; ++g) {
+                    uint32_t zf[4], zb[4];
+                    rf.refill();
+                    rb.refill();
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if ((j & 3) == 0) {
-                            rf.refill();
-                            rb.refill();
-                        }
+                    for (int j = 0; j < 4; ++j) {
                         zf[j] = get_code<true>(rf, k, pow2k, sq_meta, ok);
-                        zb[7 - j] = get_code<false>(rb, k, pow2k, sq_meta, ok);
+                        zb[3 - j] = get_code<false>(rb, k, pow2k, sq_meta, ok);
                     }
-                    *zz_slot(sm.buf, g, tid) = make_uint4(zf[0] | (zf[1] << 16), zf[2] | (zf[3] << 16),
-                                                          zf[4] | (zf[5] << 16), zf[6] | (zf[7] << 16));
-                    *zz_slot(sm.buf, V / 8 - 1 - g, tid) = make_uint4(zb[0] | (zb[1] << 16), zb[2] | (zb[3] << 16),
-                                                                      zb[4] | (zb[5] << 16), zb[6] | (zb[7] << 16));
+                    uint2* pf = reinterpret_cast<uint2*>(zz_slot(sm.buf, g >> 1, tid)) + (g & 1);
+                    uint2* pb = reinterpret_cast<uint2*>(zz_slot(sm.buf, V / 8 - 1 - (g >> 1), tid)) + (1 - (g & 1));
+                    *pf = make_uint2(zf[0] | (zf[1] << 16), zf[2] | (zf[3] << 16));
+                    *pb = make_uint2(zb[0] | (zb[1] << 16), zb[2] | (zb[3] << 16));
                 }
                 // the codes' unary parts: the bits taken minus one stop bit and k remainder bits per code
                 sq = (uint32_t)(rf.consumed() + rb.consumed() - N * (k + 1));
