@@ -468,21 +468,27 @@ static int get_code(bitr_t* rd, int64_t* pos, int step, int k, uint32_t limit, u
 /* ------------------------------------------------------------------------------------------ */
 /* Subtractive dither (Methodology step 4): U uniform on the Voronoi cell of the lattice, in   */
 /* the coordinates its quantizer works in (u for Z, D4, E8; (P, Q) = (2 u0, u1 K) for A2).     */
-/* Group g of four consecutive coefficients of a tile draws one Philox block: key = seed,      */
-/* counter (c_lo, c1, 0x80000000 | g, c_hi) with c = s for the KV row (b H + h, s), c1 = b H + h */
-/* (the weight-path option uses c = row, c1 = tile column).  The words w_i give                */
-/* r_i = box (w_i >> 8) 2^-24, uniform on [0, box)^d: box 1 for Z, 2 for the others.  Each box */
-/* is a union of fundamental domains (Z^1; 2Z^4 in D4; 2Z^8 in E8, which holds D8; 2Z^2 in the */
-/* (P, Q) lattice P = Q mod 2), so U = r - Q(r) is uniform on the Voronoi cell.  E8 blocks     */
-/* take groups 2b and 2b+1.                                                                    */
+/* Groups 2b and 2b + 1 of four consecutive coefficients of a tile share one Philox block: key  */
+/* = seed, counter (c_lo, c1, 0x80000000 | b, c_hi) with c = s for the KV row (b H + h, s),     */
+/* c1 = b H + h (the weight-path option uses c = row, c1 = tile column).  Its 128 bits are      */
+/* eight 16-bit halves h_0 .. h_7 (h_2i the low half of word i): group 2b takes h_0 .. h_3,      */
+/* group 2b + 1 h_4 .. h_7, and r = box (h + 1/2) 2^-16, the midpoints of 2^16 equal bins of      */
+/* [0, box) (mean exactly box / 2): box 1 for Z, 2 for the others.  Each box is a union of      */
+/* fundamental domains (Z^1; 2Z^4 in D4; 2Z^8 in E8, which holds D8; 2Z^2 in the (P, Q) lattice  */
+/* P = Q mod 2), so U = r - Q(r) is uniform on the Voronoi cell up to the 2^-16 bins.  E8       */
+/* blocks take groups 2b and 2b + 1, one Philox block each.                                      */
 /* ------------------------------------------------------------------------------------------ */
 static void dither_group(uint64_t seed, int64_t c1, int64_t c, int g, float box, float r[4])
 {
-    uint32_t ctr[4] = {(uint32_t)(uint64_t)c, (uint32_t)(uint64_t)c1, 0x80000000u | (uint32_t)g,
+    uint32_t ctr[4] = {(uint32_t)(uint64_t)c, (uint32_t)(uint64_t)c1, 0x80000000u | (uint32_t)(g >> 1),
                        (uint32_t)((uint64_t)c >> 32)};
     uint32_t w[4];
     hqo_philox4x32_10(ctr, (uint32_t)seed, (uint32_t)(seed >> 32), w);
-    for (int i = 0; i < 4; ++i) r[i] = box * ((float)(w[i] >> 8) * 5.9604644775390625e-08f);
+    for (int i = 0; i < 4; ++i) {
+        int j = 4 * (g & 1) + i; /* half index within the block */
+        uint32_t h = (w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+        r[i] = box * ((float)(2u * h + 1u) * 7.62939453125e-06f); /* box (h + 1/2) 2^-16 = box (2h + 1) 2^-17, exact */
+    }
 }
 
 /* U for all n coefficients of one tile */

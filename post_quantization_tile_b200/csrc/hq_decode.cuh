@@ -403,14 +403,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
                     }
                 } else {
     #pragma unroll
-                    for (int b = 0; b < H / 4; ++b) {
+                    for (int b2 = 0; b2 < H / 8; ++b2) {
     #pragma unroll 1
                         for (int half = 0; half < 2; ++half) {  // rolled: half the Philox code
-                            float U[4];
-                            dither_group<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + b), U);
+                            // groups 2 b2, 2 b2 + 1 of this half: one Philox block
+                            float U[8];
+                            dither_pair<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * b2) >> 1, U);
     #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                float2& q = P[4 * b + i];
+                            for (int i = 0; i < 8; ++i) {
+                                float2& q = P[8 * b2 + i];
                                 float f = __fadd_rn(half ? q.y : q.x, -U[i]);
                                 if constexpr (LAT == HQ_A2) f = (i & 1) ? __fmul_rn(f, 0.866025403784438647f) : __fmul_rn(f, 0.5f);
                                 if (half) q.y = f;

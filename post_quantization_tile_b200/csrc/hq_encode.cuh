@@ -453,13 +453,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
                         // or for A2 to (P, Q) = (2 u0, u1 K), the coordinates of its quantizer
                         float U8[8];
                         if constexpr (KV) {
-#pragma unroll
-                            for (int bb = 0; bb < 2; ++bb) {
-                                float U4[4];
-                                dither_group<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8 + bb), U4);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) U8[4 * bb + i] = U4[i];
-                            }
+                            // groups 2 (g8 + ...) and the next one: one Philox block
+                            dither_pair<LAT>(a.rk, dc1, dc, (uint32_t)(tau * (V / 4) + half * (H / 4) + 2 * g8) >> 1, U8);
                             if constexpr (LAT != HQ_A2) {
 #pragma unroll
                                 for (int i = 0; i < 8; ++i) u8[i] = __fadd_rn(u8[i], U8[i]);

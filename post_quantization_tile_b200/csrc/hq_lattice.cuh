@@ -367,65 +367,67 @@ __device__ __forceinline__ void unstrip_block(const int32_t* s, uint32_t c, int3
 }
 
 // Subtractive dither ("Subtractive Dither", Methodology step 4): U uniform on the Voronoi cell,
-// in the coordinates the quantizer works in (u for Z, D4, E8; (P, Q) for A2).  Group g of four
-// consecutive coefficients of a tile draws one Philox block with counter (c_lo, c1, 0x80000000 | g,
-// c_hi) under the seed's round keys rk: c = s and c1 = b H + h for KV row (b H + h, s); c = row and
-// c1 = tile column for the weight-path option.  r_i = box (w_i >> 8) 2^-24 is uniform on
-// [0, box)^4 (box 1 for Z, 2 otherwise), a union of fundamental domains (2Z^d lies in D4, in E8
-// and in the (P, Q) lattice), so U = r - Q(r) is uniform on the cell.  E8 blocks take two groups.
-__device__ __forceinline__ void dither_r(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t g, float box,
-                                         float (&r)[4])
+// in the coordinates the quantizer works in (u for Z, D4, E8; (P, Q) for A2).  Groups 2b and 2b + 1
+// of four consecutive coefficients of a tile share one Philox block with counter (c_lo, c1,
+// 0x80000000 | b, c_hi) under the seed's round keys rk: c = s and c1 = b H + h for KV row
+// (b H + h, s); c = row and c1 = tile column for the weight-path option.  Its eight 16-bit halves
+// (low half of word i first) give r = box (h + 1/2) 2^-16, the midpoints of 2^16 bins of
+// [0, box) (box 1 for Z, 2 otherwise), a union of fundamental domains (2Z^d lies in D4, in E8 and
+// in the (P, Q) lattice), so U = r - Q(r) is uniform on the cell up to the bins.  E8 blocks take
+// one Philox block (two groups).
+__device__ __forceinline__ void dither_r8(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t b, float box,
+                                          float (&r)[8])
 {
-    const uint4 w = philox4x32_10_rk(make_uint4((uint32_t)c, c1, 0x80000000u | g, (uint32_t)(c >> 32)), rk);
-    // box (w >> 8) 2^-24: every step is exact (24-bit integers, power-of-two scales)
-    const float sc = box == 1.0f ? 5.9604644775390625e-08f : 1.1920928955078125e-07f;
-    r[0] = __fmul_rn((float)(w.x >> 8), sc);
-    r[1] = __fmul_rn((float)(w.y >> 8), sc);
-    r[2] = __fmul_rn((float)(w.z >> 8), sc);
-    r[3] = __fmul_rn((float)(w.w >> 8), sc);
+    const uint4 w = philox4x32_10_rk(make_uint4((uint32_t)c, c1, 0x80000000u | b, (uint32_t)(c >> 32)), rk);
+    // (2h + 1) 2^-16 box: a 17-bit odd integer times a power of two, exact
+    const float sc = box == 1.0f ? 7.62939453125e-06f : 1.52587890625e-05f;
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        r[2 * i] = __fmul_rn((float)(((ws[i] & 0xFFFFu) << 1) | 1u), sc);
+        r[2 * i + 1] = __fmul_rn((float)(((ws[i] >> 15) & 0x1FFFEu) | 1u), sc);
+    }
 }
 
-// U for the four coefficients of group g (Z, A2: two blocks, D4: one block)
+// U for the eight coefficients of groups 2b, 2b + 1 (Z: eight blocks, A2: four, D4: two)
 template <int LAT>
-__device__ __forceinline__ void dither_group(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t g,
-                                             float (&U)[4])
+__device__ __forceinline__ void dither_pair(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t b,
+                                            float (&U)[8])
 {
-    static_assert(LAT != HQ_E8, "E8 blocks span two groups: dither_e8");
-    float r[4];
-    dither_r(rk, c1, c, g, LAT == HQ_Z ? 1.0f : 2.0f, r);
+    static_assert(LAT != HQ_E8, "E8: dither_e8");
+    float r[8];
+    dither_r8(rk, c1, c, b, LAT == HQ_Z ? 1.0f : 2.0f, r);
     if constexpr (LAT == HQ_Z) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 8; ++i) {
             int32_t a;
             U[i] = __fadd_rn(r[i], -rint_magic(r[i], a));
         }
     } else if constexpr (LAT == HQ_A2) {
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+        for (int bb = 0; bb < 4; ++bb) {
             int32_t v[2];
-            q_a2_pq(r[2 * b], r[2 * b + 1], v);
-            U[2 * b] = __fadd_rn(r[2 * b], -(float)v[0]);
-            U[2 * b + 1] = __fadd_rn(r[2 * b + 1], -(float)v[1]);
+            q_a2_pq(r[2 * bb], r[2 * bb + 1], v);
+            U[2 * bb] = __fadd_rn(r[2 * bb], -(float)v[0]);
+            U[2 * bb + 1] = __fadd_rn(r[2 * bb + 1], -(float)v[1]);
         }
     } else {
-        int32_t q[4];
-        q_d4(r, q);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) U[i] = __fadd_rn(r[i], -(float)q[i]);
+        for (int h = 0; h < 2; ++h) {
+            const float rr[4] = {r[4 * h], r[4 * h + 1], r[4 * h + 2], r[4 * h + 3]};
+            int32_t q[4];
+            q_d4(rr, q);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) U[4 * h + i] = __fadd_rn(rr[i], -(float)q[i]);
+        }
     }
 }
 
-// U for the E8 block made of groups g0, g0 + 1 (u units)
+// U for the E8 block made of groups g0, g0 + 1 (g0 even; u units)
 __device__ __forceinline__ void dither_e8(const uint32_t (&rk)[20], uint32_t c1, uint64_t c, uint32_t g0, float (&U)[8])
 {
-    float r[8], r0[4], r1[4];
-    dither_r(rk, c1, c, g0, 2.0f, r0);
-    dither_r(rk, c1, c, g0 + 1, 2.0f, r1);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        r[i] = r0[i];
-        r[4 + i] = r1[i];
-    }
+    float r[8];
+    dither_r8(rk, c1, c, g0 >> 1, 2.0f, r);
     int32_t s[8], v[8];
     e8_symbols<true>(r, s, v);
 #pragma unroll

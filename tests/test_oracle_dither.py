@@ -116,3 +116,20 @@ def test_token_append_tiles_equal_the_whole_sequence_tiles():
         np.testing.assert_array_equal(app.meta, full.meta[rows])
         xa, _ = oracle.decode(app)
         np.testing.assert_array_equal(xa, xf[rows])
+
+
+def test_dither_draws_sixteen_bit_midpoints_from_one_philox_block_per_group_pair():
+    """The dither reading: groups 2b and 2b + 1 of a tile share the Philox4x32-10 block with counter
+    (c, c1, 0x80000000 | b, 0) (the generator pinned to curand's elsewhere); its eight 16-bit
+    halves, low half first, give r = box (h + 1/2) 2^-16.  On Z (box 1) U = r - rint(r), so r is U
+    taken mod 1; its 2^17 r are odd integers, the bins' midpoints."""
+    seed, c1, c, n = 0x5EED, 3, 1234, 64
+    U = oracle.dither(oracle.Z, seed, c1, c, n).astype(np.float64)
+    r = np.where(U < 0, U + 1.0, U)
+    odd = r * 2.0 ** 17
+    assert np.all(odd == np.round(odd)) and np.all(np.round(odd) % 2 == 1)
+    for g in range(n // 4):
+        w = oracle.philox([c, c1, 0x80000000 | (g >> 1), 0], seed & 0xFFFFFFFF, seed >> 32)
+        halves = [(int(w[j >> 1]) >> (16 * (j & 1))) & 0xFFFF for j in range(8)]
+        want = [(2 * h + 1) * 2.0 ** -17 for h in halves[4 * (g & 1):4 * (g & 1) + 4]]
+        np.testing.assert_array_equal(r[4 * g:4 * g + 4], want)
