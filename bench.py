@@ -523,6 +523,13 @@ def run_gpu(args):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "bytes_per_launch": kbytes,
                          "traffic": measured_traffic(kname, SHAPES[i_big][0] * SHAPES[i_big][1])},
+            # the 4096 x 4096 weight, the shape the throughput target names
+            "roofline_4096x4096": {
+                "encode": {"achieved": (SHAPES[0][0] * SHAPES[0][1] * 2 + code_bytes[0]) / (enc_ms[0] * 1e-3) / 1e9,
+                           "frac": (SHAPES[0][0] * SHAPES[0][1] * 2 + code_bytes[0]) / (enc_ms[0] * 1e-3) / 1e9 / peak},
+                "decode": {"achieved": (SHAPES[0][0] * SHAPES[0][1] * 2 + code_bytes[0]) / (dec_ms[0] * 1e-3) / 1e9,
+                           "frac": (SHAPES[0][0] * SHAPES[0][1] * 2 + code_bytes[0]) / (dec_ms[0] * 1e-3) / 1e9 / peak},
+                "peak": peak, "unit": "GB/s", "bytes_per_launch": SHAPES[0][0] * SHAPES[0][1] * 2 + code_bytes[0]},
             "cpu_baseline": cpu,
             "e2e": {"value": weak_scaling_value(bf16_bytes, world, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": bf16_bytes, "d2h_bytes_per_step": bf16_bytes},
@@ -884,6 +891,28 @@ def run_profile(args):
         if st != 0:
             raise SystemExit(1)
         return
+    if args.profile == "gemm_fused":
+        # decode fused into the int8 GEMM: the 4096 x 4096 E8 code against 128 activation rows
+        w = torch.from_numpy(W.llama_weight(4096, 4096, seed=1).view(np.int16)).view(torch.bfloat16).cuda()
+        code = hq.encode(w, TILE, hq.E8, 0.29, seed=SEED)
+        rng = np.random.default_rng(6)
+        A = torch.from_numpy(np.clip(np.round(rng.standard_normal((128, 4096)) * 32.0), -127, 127).astype(np.int8)).cuda()
+        sa = torch.full((128,), 0.02, dtype=torch.float32, device="cuda")
+        Y = torch.empty(128, 4096, dtype=torch.float32, device="cuda")
+        ws = hq.workspace(hq.lib().hq_gemm_code_workspace_bytes(128, 4096, 4096))
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        torch.cuda.synchronize()
+        for i in range(3):
+            ev[i].record()
+            hq.gemm_code(A, sa, code, out=Y, ws=ws)
+        ev[3].record()
+        torch.cuda.synchronize()
+        st = hq.status(ws)[0]
+        print(json.dumps({"profile": "gemm_fused", "ms": [ev[i].elapsed_time(ev[i + 1]) for i in range(3)], "status": st}),
+              flush=True)
+        if st != 0:
+            raise SystemExit(1)
+        return
     if args.profile == "kv":
         # dithered D4 KV codec on keys [8, 32, 2048, 128] bf16 (67 M scalars, 134 MB, larger than L2)
         # at the 2-bps step: a set-up encode, then three rounds of encode + decode
@@ -955,7 +984,8 @@ def run_profile(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile", choices=["encode", "decode", "count", "gemm", "kv", "kv_dense"], default=None)
+    ap.add_argument("--profile", choices=["encode", "decode", "count", "gemm", "gemm_fused", "kv", "kv_dense"],
+                    default=None)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
