@@ -623,7 +623,7 @@ hq_status_t hq_kv_decode_dense(const hq_code_t* code, const float* Q, void* kv, 
     body.kv = 1;  // dither words of KV rows; the lattice points come back untransformed
     const hq_status_t s = decode_common(&body, pbuf, 3, 1, nullptr, ws, ws_bytes, stream);
     if (s != HQ_OK) return s;
-    return launch_unrotate(pbuf, Q, code->scale, code->p.step, code->rows, kv, dtype == HQ_BF16,
+    return launch_unrotate(pbuf, Q, code->scale, code->p.step, code->rows, kv, dtype == HQ_BF16, ws,
                            static_cast<cudaStream_t>(stream)) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 

@@ -28,7 +28,7 @@ int num_sms();
 cudaError_t launch_rotate(const void* x, bool bf16, const float* Q, float beta, int64_t rows, float* u,
                           uint16_t* scale, uint32_t* nonfinite, cudaStream_t st);
 cudaError_t launch_unrotate(const float* p, const float* Q, const uint16_t* scale, float beta, int64_t rows, void* y,
-                            bool bf16, cudaStream_t st);
+                            bool bf16, void* ws, cudaStream_t st);
 cudaError_t launch_merge_nonfinite(void* ws, const uint32_t* nonfinite, cudaStream_t st);
 
 // 2-D tensor map of a row-major [rows, cols] tensor of es-byte elements: box [box_rows][128 bytes],
