@@ -107,3 +107,26 @@ def test_dense_entry_points_check_arguments_without_a_gpu(libhq):
     cs.version = 2
     assert L.hq_kv_decode_dense(ctypes.byref(cs), q, ctypes.c_void_p(256), 1, ctypes.c_void_p(256), 1 << 20,
                                 None) == 1
+
+
+def test_fused_gemm_checks_arguments_without_a_gpu(libhq):
+    import post_quantization_tile_b200 as hq
+    L = hq.lib()
+    assert L.hq_gemm_code_workspace_bytes(128, 4096, 4096) >= 256 + 4 * 32
+    # few output tiles: the K ranges hand their chains over through the workspace (64 KB per tile)
+    assert L.hq_gemm_code_workspace_bytes(16, 4096, 4096) >= 32 * 128 * 128 * 4
+    assert L.hq_gemm_code_workspace_bytes(16, 100, 4096) == 0      # N not a multiple of 128
+    assert L.hq_gemm_code_workspace_bytes(0, 128, 128) == 0
+    cs = hq.CodeStruct()
+    cs.version, cs.kv, cs.rows, cs.cols = 2, 0, 128, 256
+    cs.p = hq.params(256, hq.E8, 0.3)                              # tile 256: not provided
+    ws = ctypes.c_void_p(256)
+    assert L.hq_gemm_code(ctypes.c_void_p(16), ctypes.c_void_p(16), 16, ctypes.byref(cs), ctypes.c_void_p(16), ws,
+                          1 << 20, None) == 2
+    cs.p = hq.params(128, hq.A2, 0.3)                              # A2 codes: not provided
+    assert L.hq_gemm_code(ctypes.c_void_p(16), ctypes.c_void_p(16), 16, ctypes.byref(cs), ctypes.c_void_p(16), ws,
+                          1 << 20, None) == 2
+    cs.p = hq.params(128, hq.E8, 0.3)
+    cs.kv = 1                                                      # a dithered KV code
+    assert L.hq_gemm_code(ctypes.c_void_p(16), ctypes.c_void_p(16), 16, ctypes.byref(cs), ctypes.c_void_p(16), ws,
+                          1 << 20, None) == 1

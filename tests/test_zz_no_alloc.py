@@ -68,3 +68,37 @@ def test_noalloc_rejects_tensors_beyond_its_scratch():
     # 65536 x 65536 at tile 128 needs 8 * 512 * 512 bytes of look-back slots, far above 128 KiB
     rc = f(ctypes.c_void_p(x.data_ptr()), 0, 65536, 65536, ctypes.byref(p), ctypes.byref(cs), None, None)
     assert rc == 7   # HQ_ERR_RANGE
+
+
+def test_noalloc_accepts_managed_memory_like_the_regular_encoder():
+    """A weight in CUDA managed memory (the caller's own pool may hand out managed buffers) is
+    accepted like device memory, as hq_encode accepts it, and gives the same code."""
+    import post_quantization_tile_b200 as hq
+    from cuda.bindings import runtime as rt
+    from post_quantization_tile_b200 import workloads as W
+    f = _noalloc_fn(hq)
+    rows, cols, tile, beta, seed = 96, 512, 128, 0.3, 5
+    xb = np.ascontiguousarray(W.llama_weight(4096, 4096, seed=2)[:rows, :cols])
+    err, ptr = rt.cudaMallocManaged(xb.nbytes, rt.cudaMemAttachGlobal)
+    assert err == rt.cudaError_t.cudaSuccess
+    try:
+        err, = rt.cudaMemcpy(ptr, xb.ctypes.data, xb.nbytes, rt.cudaMemcpyKind.cudaMemcpyHostToDevice)
+        assert err == rt.cudaError_t.cudaSuccess
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+        ref = hq.encode(x, tile, hq.E8, beta, seed=seed)
+        assert hq.status(ref.ws)[0] == 0
+        p = hq.params(tile, hq.E8, beta, seed=seed)
+        out = hq.alloc_code(rows, cols, p)
+        cs = out.struct()
+        status = torch.full((1,), 0x7FFFFFFF, dtype=torch.int32, device="cuda")
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        rc = f(ctypes.c_void_p(int(ptr)), 0, rows, cols, ctypes.byref(p), ctypes.byref(cs),
+               ctypes.c_void_p(status.data_ptr()), stream)
+        assert rc == 0
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        words = ref.total_words()
+        assert torch.equal(out.chunk_word, ref.chunk_word) and torch.equal(out.bits[:words], ref.bits[:words])
+    finally:
+        torch.cuda.synchronize()
+        rt.cudaFree(ptr)
