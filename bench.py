@@ -404,23 +404,54 @@ def run_gpu(args):
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
 
+    # The step as a CUDA graph (one per replica phase: the memset and the kernel of each of the
+    # four calls, in order on one stream), captured through the public API and replayed, so that
+    # the timed region holds the GPU work alone: no host launch gaps and no timing events between
+    # the calls.  (Running the two matrices as concurrent graph branches was measured slower: the
+    # persistent grids of concurrent kernels compete for the same SM slots.)
+    graphs = []
+    for r in range(REPLICAS):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(r)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    for k in range(max(3, args.warmup)):
+        graphs[k % REPLICAS].replay()
+    torch.cuda.synchronize()
+    st, _ = hq.status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the graph warm-up")
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    e_t0 = torch.cuda.Event(enable_timing=True)
+    e_t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         time.sleep(1.0)  # let the sampler start before the timed region
         clk.mark(True)
         t0.record(stream)
         for k in range(args.steps):
-            step(args.warmup + k, record=k)
+            graphs[(args.warmup + k) % REPLICAS].replay()
         t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        # per-call times: the same steps eagerly, each call bracketed by events on its stream
+        e_t0.record(stream)
+        for k in range(args.steps):
+            step(args.warmup + k, record=k)
+        e_t1.record(stream)
         torch.cuda.synchronize()
         clk.mark(False)
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+    eager_ms = max_over_ranks(e_t0.elapsed_time(e_t1) / args.steps, dev)
+    del graphs
     enc_calls = [[enc_ev[k * len(SHAPES) + i][0].elapsed_time(enc_ev[k * len(SHAPES) + i][1])
                   for k in range(args.steps)] for i in range(len(SHAPES))]
     dec_calls = [[dec_ev[k * len(SHAPES) + i][0].elapsed_time(dec_ev[k * len(SHAPES) + i][1])
@@ -513,7 +544,11 @@ def run_gpu(args):
                        "shapes": SHAPES, "tile": TILE, "lattice": "E8", "target_bps": BPS,
                        "step": steps_beta, "payload_bps": payload_bps, "total_bps": total_bps, "nmse": mse,
                        "l2": "inputs and codes rotate over 3 replicas (124 MB bf16 each), no L2 reuse across launches",
+                       "launch": "timed steps are replays of a CUDA graph of the four API calls in order on "
+                                 "one stream; encode_ms / decode_ms and the roofline come from the same steps "
+                                 "run eagerly with events around each call (eager_ms_per_step)",
                        "parallelism": f"replicas{world}"},
+            "eager_ms_per_step": eager_ms,
             "encode_gbs": [SHAPES[i][0] * SHAPES[i][1] * 2 / (enc_ms[i] * 1e-3) / 1e9 for i in range(len(SHAPES))],
             "decode_gbs": [SHAPES[i][0] * SHAPES[i][1] * 2 / (dec_ms[i] * 1e-3) / 1e9 for i in range(len(SHAPES))],
             "encode_ms": enc_ms, "decode_ms": dec_ms,
