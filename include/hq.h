@@ -257,6 +257,8 @@ hq_status_t hq_decode_int8(const hq_code_t* code, int8_t* v_out, float* g_out, v
  * acc = fma(S, g, acc) over t = 0, 1, ... from acc = 0, then Y = acc * sa[m].  group must be 128;
  * M and N multiples of 128, K a multiple of 128 up to 2^20 (HQ_ERR_UNSUPPORTED / HQ_ERR_ARG
  * otherwise).  ws: at least 64 bytes; a bounded wait that ran out reports HQ_ERR_TIMEOUT there.
+ * The CTA tile is 128 rows by 128, 64 or 32 columns (the widest whose tiles occupy every SM); the
+ * result does not depend on it.
  */
 hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8_t* V, const float* g, int64_t N,
                          int64_t K, int32_t group, float* Y, void* ws, size_t ws_bytes, void* stream);

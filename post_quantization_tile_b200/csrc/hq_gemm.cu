@@ -9,11 +9,12 @@
 // tensor-core MMA paths, int8 ahead of fp8 on the post-RHT lattice output), with the group scale
 // the decoder would otherwise apply.
 //
-// Persistent CTAs (one per SM) walk the 128 x 128 tiles of Y: warp 0 streams 128 x 128-byte boxes
-// of A and V and the group's 128 scales into a 4-stage ring with TMA (128-byte swizzle, the
-// canonical K-major layout of the MMA); warp 1 issues
-// four tcgen05.mma.kind::i8 (M 128, N 128, K 32) per group into one of four TMEM accumulator slots
-// (4 x 128 columns); the epilogue warps (warpgroups of 32 columns each) read each finished slot
+// Persistent CTAs (one per SM) walk the 128 x GN tiles of Y (GN = 128 columns; 64 or 32 when the
+// 128-wide tiles are too few to occupy the SMs, i.e. at small M): warp 0 streams 128 x 128-byte
+// boxes of A, GN x 128-byte boxes of V and the group's GN scales into a ring with TMA (128-byte
+// swizzle, the canonical K-major layout of the MMA); warp 1 issues four
+// tcgen05.mma.kind::i8 (M 128, N GN, K 32) per group into one of 512 / GN TMEM accumulator slots
+// of GN columns; the epilogue warps (warpgroups of 32 columns each) read each finished slot
 // (tcgen05.ld), release it, convert the int32 sums and apply the group scales with paired binary32
 // fma, so MMA and scaling overlap; a tile's result leaves through a staging buffer and TMA stores
 // while the next tile's MMAs run.  Every wait is bounded: on a timeout the kernel records HQ_ERR_TIMEOUT and winds down.
@@ -25,36 +26,38 @@
 #include "hq_launch.h"
 #include "hq_tc.cuh"
 
-#ifndef HQ_GEMM_EPI_WARPS
-#define HQ_GEMM_EPI_WARPS 16
-#endif
-#ifndef HQ_GEMM_N
-#define HQ_GEMM_N 128  // output columns per CTA tile: 128, or 256 (measured slower: the 64 accumulators
-                       // per epilogue thread exceed the register budget of 576 threads)
-#endif
-
 namespace hq {
 namespace {
 
 constexpr float kMagicGemm = 12582912.0f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
-constexpr int GM = 128, GN = HQ_GEMM_N, GK = 128;  // CTA tile (M, N) and K group
-constexpr int GSTAGES = GN == 128 ? 4 : 3;         // operand ring
-constexpr int GACC = 512 / GN;                     // TMEM accumulator slots of GN columns (all 512)
-constexpr int GOUT = 128;                          // columns staged per output store
-constexpr int GEPI = HQ_GEMM_EPI_WARPS;      // epilogue warps: GEPI / 4 warpgroups, GN / (GEPI / 4) columns each
-constexpr int GTHREADS = 64 + 32 * GEPI;
+constexpr int GM = 128, GK = 128;  // CTA tile rows and K group
 
+// Tile width GN (128, 64 or 32 output columns): one epilogue warpgroup per 32 columns (a 128-wide
+// tile has 16 epilogue warps; 256 columns were measured slower: 64 accumulators per epilogue
+// thread exceed the register budget), the TMEM's 512 columns as 512 / GN accumulator slots.
+template <int GN>
+struct GemmCfg {
+    static constexpr int STAGES = GN == 128 ? 4 : (GN == 64 ? 6 : 8);  // operand ring
+    static constexpr int ACC = 512 / GN;
+    static constexpr int OUT = GN;          // columns staged per output store
+    static constexpr int EPI = GN / 8;      // epilogue warps: GN / 32 warpgroups of 32 columns
+    static constexpr int THREADS = 64 + 32 * EPI;
+    static constexpr uint32_t IDESC = idesc_i8(GM, GN);  // s8 x s8 -> s32, both K-major, M = GM, N = GN
+};
+
+template <int GN>
 struct GemmSmem {
-    alignas(1024) int8_t a[GSTAGES][GM * GK];
-    alignas(1024) int8_t b[GSTAGES][GN * GK];
-    alignas(1024) unsigned char out[GOUT / 32][GM * 128];  // output staging: 32-column boxes
-    alignas(16) float g[GSTAGES][GN];                     // the group's scales, loaded with the operands
-    alignas(8) uint64_t full[GSTAGES];
-    uint64_t empty[GSTAGES];
-    uint64_t acc_full[GACC];
-    uint64_t acc_empty[GACC];
+    using C = GemmCfg<GN>;
+    alignas(1024) int8_t a[C::STAGES][GM * GK];
+    alignas(1024) int8_t b[C::STAGES][GN * GK];
+    alignas(1024) unsigned char out[C::OUT / 32][GM * 128];  // output staging: 32-column boxes
+    alignas(16) float g[C::STAGES][GN];                     // the group's scales, loaded with the operands
+    alignas(8) uint64_t full[C::STAGES];
+    uint64_t empty[C::STAGES];
+    uint64_t acc_full[C::ACC];
+    uint64_t acc_empty[C::ACC];
     uint32_t tmem_base;
 };
 
@@ -65,17 +68,19 @@ struct GemmArgs {
     WsHeader* ws;
 };
 
-constexpr uint32_t kIdescI8 = idesc_i8(GM, GN);  // s8 x s8 -> s32, both K-major, M = GM, N = GN
-
-__global__ void __launch_bounds__(GTHREADS, 1)
+template <int GN>
+__global__ void __launch_bounds__(GemmCfg<GN>::THREADS, 1)
     gemm_i8_grouped_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
                            const __grid_constant__ CUtensorMap tY)
 {
+    using C = GemmCfg<GN>;
+    constexpr int GSTAGES = C::STAGES, GACC = C::ACC, GOUT = C::OUT, GEPI = C::EPI;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    GemmSmem<GN>& sm =
+        *reinterpret_cast<GemmSmem<GN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = (int)(a.K / GK);
-    const int NT = (int)((a.N + GN - 1) / GN);  // a last tile of 128 columns when N % GN = 128
+    const int NT = (int)(a.N / GN);  // N is a multiple of 128, so of GN
     const int tiles = (int)(a.M / GM) * NT;  // persistent: tiles blockIdx.x, + gridDim.x, ...
 
     if (threadIdx.x == 0) {
@@ -143,7 +148,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < GK / 32; ++kk)  // K 32 per MMA: the start address moves 32 bytes
                         mma_i8(tbase + (uint32_t)(slot * GN), ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
-                               kIdescI8, kk > 0 ? 1u : 0u);
+                               C::IDESC, kk > 0 ? 1u : 0u);
                     mma_commit(&sm.empty[s]);
                     mma_commit(&sm.acc_full[slot]);
                 }
@@ -245,10 +250,35 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     if (warp == 1) tmem_dealloc(tbase, GACC * GN);
 }
 
+template <int GN>
+cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
+                        cudaStream_t st)
+{
+    const size_t smem = sizeof(GemmSmem<GN>) + 1024;
+    // set on every call: the attribute belongs to the current device's context
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_grouped_kernel<GN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (a.M / GM) * (a.N / GN);
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());  // persistent: one CTA per SM
+    gemm_i8_grouped_kernel<GN><<<grid, GemmCfg<GN>::THREADS, smem, st>>>(a, ta, tb, ty);
+    return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace hq
 
 using namespace hq;
+
+// tile width: 128 columns when the 128-wide tiles fill the SMs, else the widest of 64 / 32 whose
+// tiles do (32 when none does); N is a multiple of 128, so every width divides it
+static int gemm_tile_width(int64_t M, int64_t N)
+{
+    const int64_t sms = num_sms();
+    for (int gn = 128; gn > 32; gn /= 2)
+        if ((M / GM) * (N / gn) >= sms) return gn;
+    return 32;
+}
 
 extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8_t* V, const float* g,
                                     int64_t N, int64_t K, int32_t group, float* Y, void* ws, size_t ws_bytes,
@@ -258,26 +288,21 @@ extern "C" hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M,
     if (group != GK) return HQ_ERR_UNSUPPORTED;
     if (M < GM || N < 128 || K < GK || M % GM || N % 128 || K % GK) return HQ_ERR_ARG;
     if (K > ((int64_t)1 << 20) || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return HQ_ERR_UNSUPPORTED;
-    if ((M / GM) * ((N + GN - 1) / GN) > ((int64_t)1 << 30)) return HQ_ERR_UNSUPPORTED;
+    if ((M / GM) * (N / 32) > ((int64_t)1 << 30)) return HQ_ERR_UNSUPPORTED;
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
     const uintptr_t al = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(V) |
                          reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(ws) |
                          reinterpret_cast<uintptr_t>(g) | reinterpret_cast<uintptr_t>(sa);
     if (al & 15u) return HQ_ERR_ARG;
     if (!device_of(A)) return HQ_ERR_ARG;
+    const int gn = gemm_tile_width(M, N);
     CUtensorMap ta, tb, ty;
-    if (!tensor_map_2d(&ta, A, M, K, 1, GM) || !tensor_map_2d(&tb, V, N, K, 1, GN) || !tensor_map_2d(&ty, Y, M, N, 4, GM))
+    if (!tensor_map_2d(&ta, A, M, K, 1, GM) || !tensor_map_2d(&tb, V, N, K, 1, gn) || !tensor_map_2d(&ty, Y, M, N, 4, GM))
         return HQ_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
-    const size_t smem = sizeof(GemmSmem) + 1024;
-    // set on every call: the attribute belongs to the current device's context
-    if (cudaFuncSetAttribute(gemm_i8_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return HQ_ERR_CUDA;
-    GemmArgs a{M, N, K, sa, g, static_cast<WsHeader*>(ws)};
-    const int64_t tiles = (M / GM) * ((N + GN - 1) / GN);
-    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());  // persistent: one CTA per SM
-    gemm_i8_grouped_kernel<<<grid, GTHREADS, smem, st>>>(a, ta, tb, ty);
-    return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+    const GemmArgs a{M, N, K, sa, g, static_cast<WsHeader*>(ws)};
+    const cudaError_t e = gn == 128 ? launch_gemm<128>(a, ta, tb, ty, st)
+                                    : (gn == 64 ? launch_gemm<64>(a, ta, tb, ty, st) : launch_gemm<32>(a, ta, tb, ty, st));
+    return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }

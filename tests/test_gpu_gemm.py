@@ -53,7 +53,10 @@ def test_decode_int8_flags_codes_outside_int8(hq):
     assert torch.all(v[5] == 0) and torch.any(v[4] != 0)
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (256, 384, 1024), (384, 256, 2048), (2048, 1280, 256)])
+# tile widths: 32 columns (the first three shapes; 512 x 2048 with more tiles than SMs), 64 (1024 x
+# 2048: the 128-wide tiles would leave SMs idle, the 64-wide ones fill them) and 128 (2048 x 1280)
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (256, 384, 1024), (384, 256, 2048), (512, 2048, 256),
+                                   (1024, 2048, 256), (2048, 1280, 256)])
 def test_gemm_int8_bit_exact(hq, M, N, K):
     w = W.llama_weight(N, K, seed=K + N)
     code = hq.encode(t_bf16(w), 128, hq.E8, 0.3, seed=5)
