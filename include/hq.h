@@ -273,10 +273,10 @@ hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8
  *   Y[m, r] = sa[m] * sum_t g[t, r] S(m, r, t)
  * bit for bit as the two-call path: exact int32 group sums, acc = fma(S, g, acc) over t = 0, 1, ...
  * from 0 in binary32, then Y = acc * sa[m]; tiles with a code outside int8 are zero (HQ_ERR_RANGE),
- * corrupt tiles too (HQ_ERR_CORRUPT).  When the output has too few 128 x 128 tiles to occupy the
- * GPU, the K groups are split into ranges whose binary32 chains hand over through ws in order.
- * ws: at least hq_gemm_code_workspace_bytes(M, N, K) bytes (status word, per-tile flags and, for
- * split ranges, one 128 x 128 binary32 chain per output tile); calls sharing ws must not overlap.
+ * corrupt tiles too (HQ_ERR_CORRUPT).  A CTA takes 128 activation rows against a slab of 32
+ * weight rows (one chunk of the code per K group) over all K groups, so every output element's
+ * chain stays in one CTA.  ws: at least hq_gemm_code_workspace_bytes(M, N, K) bytes (the status
+ * word); calls sharing ws must not overlap.
  */
 size_t hq_gemm_code_workspace_bytes(int64_t M, int64_t N, int64_t K);
 hq_status_t hq_gemm_code(const int8_t* A, const float* sa, int64_t M, const hq_code_t* code, float* Y, void* ws,

@@ -1,9 +1,9 @@
 """The int8 tensor-core GEMM with the weight's decode fused into its producer warps
 (hq_gemm_code), on the GPU: bit-exact against the oracle's decode_int8 + grouped GEMM -- and so
-against the two-call path -- with activation row counts that are not multiples of 128, with the K
-groups split into ranges whose binary32 chains hand over through the workspace (few output
-tiles), with more units than SMs, for the Z, D4 and E8 codes; tiles with codes outside int8 are
-zero as in hq_decode_int8; and, sampled, the 4096 x 4096 weight at M = 16 and M = 4096."""
+against the two-call path -- with activation row counts that are not multiples of 128, with fewer
+work units (128-row activation tile x 32-row weight slab) than SMs and with more, for the Z, D4
+and E8 codes; tiles with codes outside int8 are zero as in hq_decode_int8; and, sampled, the
+4096 x 4096 weight at M = 16 and M = 4096."""
 import numpy as np
 import pytest
 import torch
@@ -30,7 +30,7 @@ def _acts(M, K, seed):
 
 
 CASES = [
-    # lattice, M, N, K, beta: K ranges (few tiles), partial activation tiles, units > SMs
+    # lattice, M, N, K, beta: few units, partial activation tiles, units > SMs
     (oracle.E8, 16, 512, 1024, 0.3),
     (oracle.E8, 128, 1024, 2048, 0.29),
     (oracle.D4, 200, 384, 512, 0.45),
