@@ -12,8 +12,9 @@
 //   warp 0       TMA loads of the activation boxes (rows past M read as zeros) into a 4-stage ring;
 //   warp 1       tcgen05.mma.kind::i8 (M 128, N 32, K 32) x 4 per group into one of 16 TMEM slots;
 //   warps 2-5    epilogue: TMEM loads, int32 -> binary32, fma with the group scales, output;
-//   warps 6-17   twelve decoder warps, K group kb on warp kb mod 12: a bulk copy of the chunk's
-//                words, a warp scan of its tile lengths, then one lane per weight row reads its
+//   warps 6-21   sixteen decoder warps, K group kb on warp kb mod 16: a bulk copy of the chunk's
+//                words (read in place when longer than 4 KB), a warp scan of its tile lengths,
+//                then one lane per weight row reads its
 //                tile's Rice codes from both ends, unstrips each lattice block and writes the int8
 //                codes straight into the MMA's K-major 128-byte-swizzled operand stage (one per
 //                decoder warp), and the tile's group scale next to it.
@@ -32,14 +33,18 @@ namespace {
 
 constexpr int FM = 128, FN = 32, FK = 128;  // activation rows, weight rows per unit (one chunk), K group
 constexpr int FSA = 4;                       // activation stages
-constexpr int FDW = 12;                      // decoder warps = weight-code stages
+#ifndef HQ_FUSED_DEC_WARPS
+#define HQ_FUSED_DEC_WARPS 16
+#endif
+constexpr int FDW = HQ_FUSED_DEC_WARPS;      // decoder warps = weight-code stages
 constexpr int FACC = 16;                     // TMEM accumulator slots of FN columns (all 512)
 constexpr int FEPI = 4;                      // epilogue warps: one warpgroup, one TMEM lane quarter each
 constexpr int FTHREADS = 32 * (2 + FEPI + FDW);
 constexpr int FDEC0 = 32 * (2 + FEPI);       // first decoder thread
-constexpr int F_LMAX = FK / 8 + 12 * FK + 2 * FK;  // bits of a tile the input buffer takes (k <= 11)
+// a decoder warp's copy of one chunk: up to 1024 words (8 bits per weight); a longer chunk is
+// read from global memory where it lies
 constexpr int F_GUARD = 4;
-constexpr int F_IN_WORDS = (FN * ((F_LMAX + 31) / 32) + 8 + 2 * F_GUARD + 3) / 4 * 4;
+constexpr int F_IN_WORDS = 1024 + 8 + 2 * F_GUARD;
 constexpr uint32_t kIdescF = idesc_i8(FM, FN);
 constexpr float kMagicF = 12582912.0f;  // 1.5 * 2^23
 constexpr int kMagicBitsF = 0x4B400000;
@@ -104,8 +109,8 @@ __device__ __forceinline__ void unstrip8(const uint32_t (&z)[8], uint32_t cbit, 
 // the copied words `in`, L bits long) from both ends into row `row` of the operand stage `vst`.
 // Returns the tile's group scale.
 template <int LAT>
-__device__ __forceinline__ float decode_row(const FusedArgs& a, const uint32_t* in, int8_t* vst, int row, int tile0,
-                                            uint32_t L, uint32_t mt, uint16_t sbits, bool ok)
+__device__ __forceinline__ float decode_row(const FusedArgs& a, const uint32_t* in, int lim, int8_t* vst, int row,
+                                            int tile0, uint32_t L, uint32_t mt, uint16_t sbits, bool ok)
 {
     constexpr int COSB = LAT == HQ_E8 ? FK / 8 : 0;
     const int k = (int)(mt & 15u);
@@ -113,15 +118,15 @@ __device__ __forceinline__ float decode_row(const FusedArgs& a, const uint32_t* 
     if (ok) {
         uint32_t cosbits = 0;
         if constexpr (LAT == HQ_E8) {
-            const int cw = min(max(tile0 >> 5, 0), F_IN_WORDS - 2);
-            const unsigned long long two = ((unsigned long long)in[cw + 1] << 32) | in[cw];
+            const int cw = min(max(tile0 >> 5, 0), lim);
+            const unsigned long long two = ((unsigned long long)in[min(cw + 1, lim)] << 32) | in[cw];
             cosbits = (uint32_t)(two >> (tile0 & 31)) & 0xFFFFu;
         }
         const uint32_t pow2k = 1u << k, sq_meta = mt >> 4;
         BitReader<true> rf;
         BitReader<false> rb;
-        rf.begin(in, tile0 + COSB, F_IN_WORDS - 1);
-        rb.begin(in, tile0 + (int)L - 1, F_IN_WORDS - 1);
+        rf.begin(in, tile0 + COSB, lim);
+        rb.begin(in, tile0 + (int)L - 1, lim);
 #pragma unroll 1
         for (int g = 0; g < FK / 16; ++g) {
             uint32_t zf[8], zb[8];
@@ -324,20 +329,21 @@ __global__ void __launch_bounds__(FTHREADS, 1)
                         continue;
                     }
                 }
-                // the chunk's words: one bulk copy of their 16-byte range
+                // the chunk's words: one bulk copy of their 16-byte range, or (a chunk too long for
+                // the copy) read in place
                 const int64_t c = (int64_t)kb * a.RB + ns;
-                uint32_t cb = 0;
-                int good = 0;
+                const int64_t w0 = a.chunk_word[c], w1 = a.chunk_word[c + 1];
+                const int64_t lo = w0 & ~(int64_t)3, hi = (w1 + 3) & ~(int64_t)3;
+                const bool good = w1 > w0 && w1 <= a.cap_words;
+                const bool copied = good && (hi - lo) <= (int64_t)(F_IN_WORDS - 2 * F_GUARD);
+                const uint32_t cb = copied ? (uint32_t)(w0 - lo + F_GUARD) : 0u;
+                const uint32_t* src = copied ? in : a.bits + (good ? w0 : 0);
+                const int lim = copied ? F_IN_WORDS - 1 : (good ? (int)(w1 - w0 - 1) : 0);
                 if (lane == 0) {
-                    const int64_t w0 = a.chunk_word[c], w1 = a.chunk_word[c + 1];
-                    const int64_t lo = w0 & ~(int64_t)3, hi = (w1 + 3) & ~(int64_t)3;
-                    good = w1 >= w0 && hi <= a.cap_words && (hi - lo) <= (int64_t)(F_IN_WORDS - 2 * F_GUARD);
-                    cb = good ? (uint32_t)(w0 - lo + F_GUARD) : 0u;
                     if (!good) status_set(a.ws, kStCorrupt);
-                    const uint32_t bytes = good ? (uint32_t)((hi - lo) * 4) : 0u;
-                    if (bytes) {
-                        mbar_arrive_expect_tx(&sm.in_bar[w], bytes);
-                        bulk_load_1d(in + F_GUARD, a.bits + lo, bytes, &sm.in_bar[w]);
+                    if (copied) {
+                        mbar_arrive_expect_tx(&sm.in_bar[w], (uint32_t)((hi - lo) * 4));
+                        bulk_load_1d(in + F_GUARD, a.bits + lo, (uint32_t)((hi - lo) * 4), &sm.in_bar[w]);
                     } else {
                         mbar_arrive(&sm.in_bar[w]);
                     }
@@ -353,15 +359,13 @@ __global__ void __launch_bounds__(FTHREADS, 1)
                     const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
                     if (lane >= o) incl += y;
                 }
-                cb = __shfl_sync(0xffffffffu, cb, 0);
-                good = __shfl_sync(0xffffffffu, good, 0);
                 bool arrived = true;
                 if (lane == 0) arrived = mbar_wait(&sm.in_bar[w], (uint32_t)(j & 1));
                 ++j;
                 arrived = __shfl_sync(0xffffffffu, arrived, 0);
                 if (!arrived && lane == 0) status_set(a.ws, kStTimeout);
                 const int tile0 = (int)(cb * 32u + (incl - L));
-                const float gs = decode_row<LAT>(a, in, sm.v[w], lane, tile0, L, mt, sbits, good && arrived);
+                const float gs = decode_row<LAT>(a, src, lim, sm.v[w], lane, tile0, L, mt, sbits, good && arrived);
                 sm.g[w][lane] = gs;
                 fence_proxy_async();  // the stage is read by the tensor cores (async proxy)
                 __syncwarp();

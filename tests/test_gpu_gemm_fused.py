@@ -2,8 +2,9 @@
 (hq_gemm_code), on the GPU: bit-exact against the oracle's decode_int8 + grouped GEMM -- and so
 against the two-call path -- with activation row counts that are not multiples of 128, with fewer
 work units (128-row activation tile x 32-row weight slab) than SMs and with more, for the Z, D4
-and E8 codes; tiles with codes outside int8 are zero as in hq_decode_int8; and, sampled, the
-4096 x 4096 weight at M = 16 and M = 4096."""
+and E8 codes; tiles with codes outside int8 are zero as in hq_decode_int8; chunks too long for a
+decoder warp's copy are read in place; and, sampled, the 4096 x 4096 weight at M = 16 and
+M = 4096."""
 import numpy as np
 import pytest
 import torch
@@ -70,6 +71,28 @@ def test_fused_gemm_equals_two_call_path_and_zeroes_out_of_range_tiles(hq):
     assert hq.status(code.ws)[0] == 7     # HQ_ERR_RANGE
     V, g = hq.decode_int8(code)
     assert hq.status(code.ws)[0] == 7
+    Y2 = hq.gemm_int8(At, sat, V, g)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+
+
+def test_fused_gemm_reads_long_chunks_in_place(hq):
+    """Chunks longer than a decoder warp's 1024-word copy (about 8.5 bits per weight here: Z codes
+    spread over [-120, 120]) are read where they lie; the result is the two-call path's."""
+    n, N, K, M = 128, 256, 512, 128
+    u = np.random.default_rng(8).uniform(-120.0, 120.0, (N * K // n, n)).astype(np.float32)
+    _, code = hq.quantize_coeffs(torch.from_numpy(u).cuda(), n, hq.Z)
+    code.rows, code.cols = N, K
+    code.scale.fill_(0x3F80)
+    code.p.step = 1.0
+    cw = code.chunk_word.cpu().numpy().astype(np.int64)
+    assert (np.diff(cw) > 1024).any()   # some chunk takes the in-place path
+    a, sa = _acts(M, K, seed=10)
+    At, sat = torch.from_numpy(a).cuda(), torch.from_numpy(sa).cuda()
+    Y = hq.gemm_code(At, sat, code)
+    assert hq.status(code.ws)[0] == 0
+    V, g = hq.decode_int8(code)
+    assert hq.status(code.ws)[0] == 0
     Y2 = hq.gemm_int8(At, sat, V, g)
     torch.cuda.synchronize()
     assert torch.equal(Y, Y2)
