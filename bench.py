@@ -856,14 +856,14 @@ def run_gemm(hq, dev, peak_bf16):
 def run_gemm_fused(hq, dev, code, V, g, peak):
     """The decode fused into the GEMM's producer warps (hq_gemm_code) against the two calls
     (hq_decode_int8, then hq_gemm_int8 on the L2-resident int8 codes) for activation row counts
-    M = 16, 128, 1024, 4096 on the 4096 x 4096 E8 code; the two-call GEMM needs M in multiples of
+    M = 16, 128, 256, 1024, 4096 on the 4096 x 4096 E8 code; the two-call GEMM needs M in multiples of
     128, so M = 16 runs it on a 128-row activation tile.  Per-call p50 of each arm; both results
     are compared bit for bit."""
     import torch
     N, K = code.rows, code.cols
     rng = np.random.default_rng(7)
     out = []
-    for M in (16, 128, 1024, 4096):
+    for M in (16, 128, 256, 1024, 4096):
         Mp = max(M, 128)
         a = torch.from_numpy(np.clip(np.round(rng.standard_normal((Mp, K)) * 32.0), -127, 127).astype(np.int8)).to(dev)
         sa = torch.full((Mp,), 0.02, dtype=torch.float32, device=dev)

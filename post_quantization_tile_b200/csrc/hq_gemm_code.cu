@@ -5,16 +5,18 @@
 // the product of hq_decode_int8 followed by hq_gemm_int8 (same codes, same zeroed tiles, same
 // binary32 order acc = fma(S, g, acc) over the groups from 0, then y = acc * sa_m).
 //
-// A work unit is one activation tile of 128 rows against one weight slab of 32 rows -- one chunk
-// of the code per K group -- over all K groups, so each output element's binary32 chain runs in
-// one CTA from start to end; the slabs give 128 units per activation tile of a 4096-row weight,
-// enough to occupy the SMs at small M without splitting K.  One CTA per SM walks units:
-//   warp 0       TMA loads of the activation boxes (rows past M read as zeros) into a 4-stage ring;
-//   warp 1       tcgen05.mma.kind::i8 (M 128, N 32, K 32) x 4 per group into one of 16 TMEM slots;
-//   warps 2-5    epilogue: TMEM loads, int32 -> binary32, fma with the group scales, output;
-//   warps 6-21   sixteen decoder warps, K group kb on warp kb mod 16: a bulk copy of the chunk's
-//                words (read in place when longer than 4 KB), a warp scan of its tile lengths,
-//                then one lane per weight row reads its
+// A work unit is R activation tiles of 128 rows (R = 1, or 2 once M > 128) against one weight
+// slab of 32 rows -- one chunk of the code per K group -- over all K groups, so each output
+// element's binary32 chain runs in one CTA from start to end and each decoded chunk feeds R
+// tiles; the slabs give 128 units per activation row block of a 4096-row weight, enough to occupy
+// the SMs at small M without splitting K.  One CTA per SM walks units:
+//   warp 0       TMA loads of the activation boxes (rows past M read as zeros) into a ring;
+//   warp 1       tcgen05.mma.kind::i8 (M 128, N 32, K 32) x 4 per group and tile into a TMEM slot;
+//   warps 2 ..   epilogue, one warpgroup per activation tile: TMEM loads, int32 -> binary32, fma
+//                with the group scales, output;
+//   the rest     decoder warps (16 when R = 1, 12 when R = 2), K group kb on warp kb mod their
+//                count: a bulk copy of the chunk's words (read in place when longer than 4 KB), a
+//                warp scan of its tile lengths, then one lane per weight row reads its
 //                tile's Rice codes from both ends, unstrips each lattice block and writes the int8
 //                codes straight into the MMA's K-major 128-byte-swizzled operand stage (one per
 //                decoder warp), and the tile's group scale next to it.
@@ -32,42 +34,48 @@ namespace hq {
 namespace {
 
 constexpr int FM = 128, FN = 32, FK = 128;  // activation rows, weight rows per unit (one chunk), K group
-constexpr int FSA = 4;                       // activation stages
-#ifndef HQ_FUSED_DEC_WARPS
-#define HQ_FUSED_DEC_WARPS 16
-#endif
-constexpr int FDW = HQ_FUSED_DEC_WARPS;      // decoder warps = weight-code stages
-constexpr int FACC = 16;                     // TMEM accumulator slots of FN columns (all 512)
-constexpr int FEPI = 4;                      // epilogue warps: one warpgroup, one TMEM lane quarter each
-constexpr int FTHREADS = 32 * (2 + FEPI + FDW);
-constexpr int FDEC0 = 32 * (2 + FEPI);       // first decoder thread
+
+// R activation tiles per unit: the ring, the decoder warps (= weight-code stages), the epilogue
+// warpgroups and the TMEM slots (R x 32 columns each, all 512) follow from it; 704 threads either way
+template <int R>
+struct FusedCfg {
+    static constexpr int SA = R == 1 ? 4 : 2;      // activation stages (R boxes each)
+    static constexpr int DW = R == 1 ? 16 : 12;    // decoder warps
+    static constexpr int EPI = 4 * R;              // epilogue warps
+    static constexpr int ACC = 512 / (FN * R);     // TMEM accumulator slots
+    static constexpr int THREADS = 32 * (2 + EPI + DW);
+    static constexpr int DEC0 = 32 * (2 + EPI);    // first decoder thread
+};
 // a decoder warp's copy of one chunk: up to 1024 words (8 bits per weight); a longer chunk is
 // read from global memory where it lies
 constexpr int F_GUARD = 4;
 constexpr int F_IN_WORDS = 1024 + 8 + 2 * F_GUARD;
-constexpr uint32_t kIdescF = idesc_i8(FM, FN);
+constexpr uint32_t kIdescF = idesc_i8(FM, FN);  // per activation tile
 constexpr float kMagicF = 12582912.0f;  // 1.5 * 2^23
 constexpr int kMagicBitsF = 0x4B400000;
 
+template <int R>
 struct FusedSmem {
-    alignas(1024) int8_t a[FSA][FM * FK];
-    alignas(1024) int8_t v[FDW][FN * FK];
-    alignas(1024) unsigned char out[FM * 128];    // output staging: one 32-column box
-    alignas(16) uint32_t in[FDW][F_IN_WORDS];      // each decoder warp's chunk words
-    alignas(16) float g[FDW][FN];
-    alignas(8) uint64_t a_full[FSA];
-    uint64_t a_empty[FSA];
-    uint64_t b_full[FDW];
-    uint64_t b_empty[FDW];
-    uint64_t acc_full[FACC];
-    uint64_t acc_empty[FACC];
-    uint64_t in_bar[FDW];
+    using C = FusedCfg<R>;
+    alignas(1024) int8_t a[C::SA][R][FM * FK];
+    alignas(1024) int8_t v[C::DW][FN * FK];
+    alignas(1024) unsigned char out[R][FM * 128];  // output staging: one 32-column box per tile
+    alignas(16) uint32_t in[C::DW][F_IN_WORDS];     // each decoder warp's chunk words
+    alignas(16) float g[C::DW][FN];
+    alignas(8) uint64_t a_full[C::SA];
+    uint64_t a_empty[C::SA];
+    uint64_t b_full[C::DW];
+    uint64_t b_empty[C::DW];
+    uint64_t acc_full[C::ACC];
+    uint64_t acc_empty[C::ACC];
+    uint64_t in_bar[C::DW];
     uint32_t tmem_base;
 };
 
 struct FusedArgs {
     int64_t M, N, K;     // activation rows, weight rows, inner dimension
     int64_t KB, MT, NS;  // K groups, activation tiles, weight slabs
+    int64_t MP;          // activation row blocks of R tiles
     int64_t units;
     float beta;
     const float* sa;
@@ -162,12 +170,15 @@ __device__ __forceinline__ float decode_row(const FusedArgs& a, const uint32_t* 
     return gs;
 }
 
-template <int LAT>
-__global__ void __launch_bounds__(FTHREADS, 1)
+template <int LAT, int R>
+__global__ void __launch_bounds__(FusedCfg<R>::THREADS, 1)
     gemm_code_kernel(const FusedArgs a, const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tY)
 {
+    using C = FusedCfg<R>;
+    constexpr int FSA = C::SA, FDW = C::DW, FEPI = C::EPI, FACC = C::ACC, FDEC0 = C::DEC0;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    FusedSmem& sm = *reinterpret_cast<FusedSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    FusedSmem<R>& sm =
+        *reinterpret_cast<FusedSmem<R>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = (int)a.KB;
 
@@ -187,7 +198,7 @@ __global__ void __launch_bounds__(FTHREADS, 1)
         }
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(&sm.tmem_base, FACC * FN);
+    if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -199,7 +210,7 @@ __global__ void __launch_bounds__(FTHREADS, 1)
             int it = 0;
             bool alive = true;
             for (int64_t u = blockIdx.x; alive && u < a.units; u += gridDim.x) {
-                const int64_t mt = u / a.NS;
+                const int64_t mp = u / a.NS;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % FSA;
                     if (it >= FSA && !mbar_wait_sleep(&sm.a_empty[s], (uint32_t)((it / FSA - 1) & 1))) {
@@ -207,8 +218,11 @@ __global__ void __launch_bounds__(FTHREADS, 1)
                         alive = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sm.a_full[s], (uint32_t)(FM * FK));
-                    tma_load_2d(sm.a[s], &tA, kb * FK, (int)(mt * FM), &sm.a_full[s]);
+                    // a box whose rows all lie past M reads as zeros and still brings its bytes
+                    mbar_arrive_expect_tx(&sm.a_full[s], (uint32_t)(R * FM * FK));
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        tma_load_2d(sm.a[s][r], &tA, kb * FK, (int)((mp * R + r) * FM), &sm.a_full[s]);
                 }
             }
         }
@@ -230,11 +244,15 @@ __global__ void __launch_bounds__(FTHREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = sw128_desc(sm.a[sa]), bd = sw128_desc(sm.v[sb]);
+                    const uint64_t bd = sw128_desc(sm.v[sb]);
 #pragma unroll
-                    for (int kk = 0; kk < FK / 32; ++kk)
-                        mma_i8(tbase + (uint32_t)(slot * FN), ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), kIdescF,
-                               kk > 0 ? 1u : 0u);
+                    for (int r = 0; r < R; ++r) {
+                        const uint64_t ad = sw128_desc(sm.a[sa][r]);
+#pragma unroll
+                        for (int kk = 0; kk < FK / 32; ++kk)
+                            mma_i8(tbase + (uint32_t)((slot * R + r) * FN), ad + (uint64_t)(2 * kk),
+                                   bd + (uint64_t)(2 * kk), kIdescF, kk > 0 ? 1u : 0u);
+                    }
                     mma_commit(&sm.a_empty[sa]);
                     mma_commit(&sm.b_empty[sb]);
                     mma_commit(&sm.acc_full[slot]);
@@ -243,14 +261,16 @@ __global__ void __launch_bounds__(FTHREADS, 1)
         }
         __syncwarp();
     } else if (threadIdx.x < FDEC0) {
-        // ---------------- epilogue: one row of the unit per thread, 32 columns ----------------
-        const int q = warp & 3;  // TMEM lane quarter of this warp
+        // ---------------- epilogue: warpgroup r takes activation tile r; one row per thread ----------------
+        const int q = warp & 3;          // TMEM lane quarter of this warp
+        const int r = (warp - 2) >> 2;   // activation tile of the unit
+        const int lead = 64 + 128 * r;   // the warpgroup's first thread: staging and stores
         const int row = q * 32 + lane;
         const float2 nm = make_float2(-kMagicF, -kMagicF);
         int it = 0;
         bool alive = true;
         for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
-            const int64_t mt = u / a.NS, ns = u % a.NS;
+            const int64_t mt = (u / a.NS) * R + r, ns = u % a.NS;
             float2 acc[FN / 2];
 #pragma unroll
             for (int c = 0; c < FN / 2; ++c) acc[c] = make_float2(0.0f, 0.0f);
@@ -268,7 +288,7 @@ __global__ void __launch_bounds__(FTHREADS, 1)
                 }
                 tc_fence_after();
                 uint32_t S[32];
-                tmem_ld32_nowait(tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(slot * FN), S);
+                tmem_ld32_nowait(tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)((slot * R + r) * FN), S);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
@@ -290,23 +310,24 @@ __global__ void __launch_bounds__(FTHREADS, 1)
             }
             // ---------------- output: y = acc * sa through the swizzled staging box ----------------
             const int64_t m0 = mt * FM, n0 = ns * FN;
+            if (m0 >= a.M) continue;  // the unit's second tile lies past M: nothing to store
             const float sa = m0 + row < a.M ? a.sa[m0 + row] : 0.0f;
-            if (threadIdx.x == 64) bulk_wait_read0();  // the previous store has read the staging
-            named_sync(1, 32 * FEPI);
+            if (threadIdx.x == lead) bulk_wait_read0();  // the previous store has read the staging
+            named_sync(1 + r, 128);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float2 p0 = acc[2 * j], p1 = acc[2 * j + 1];
-                *reinterpret_cast<float4*>(&sm.out[swz(row, j)]) =
+                *reinterpret_cast<float4*>(&sm.out[r][swz(row, j)]) =
                     make_float4(__fmul_rn(p0.x, sa), __fmul_rn(p0.y, sa), __fmul_rn(p1.x, sa), __fmul_rn(p1.y, sa));
             }
             fence_proxy_async();
-            named_sync(1, 32 * FEPI);
-            if (threadIdx.x == 64 && alive) {
-                tma_store_2d(&tY, (int)n0, (int)m0, &sm.out[0]);
+            named_sync(1 + r, 128);
+            if (threadIdx.x == lead && alive) {
+                tma_store_2d(&tY, (int)n0, (int)m0, &sm.out[r][0]);
                 bulk_commit();
             }
         }
-        if (threadIdx.x == 64) bulk_wait0();
+        if (threadIdx.x == lead) bulk_wait0();
     } else {
         // ---------------- decoder warps: the weight's codes -> int8 operand stages ----------------
         constexpr int COSB = LAT == HQ_E8 ? FK / 8 : 0;
@@ -382,7 +403,19 @@ __global__ void __launch_bounds__(FTHREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tbase, FACC * FN);
+    if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+template <int LAT, int R>
+cudaError_t launch_fused(const FusedArgs& a, const CUtensorMap& ta, const CUtensorMap& ty, cudaStream_t st)
+{
+    const size_t smem = sizeof(FusedSmem<R>) + 1024;
+    const cudaError_t e =
+        cudaFuncSetAttribute(gemm_code_kernel<LAT, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)(a.units < num_sms() ? a.units : num_sms());
+    gemm_code_kernel<LAT, R><<<grid, FusedCfg<R>::THREADS, smem, st>>>(a, ta, ty);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -423,7 +456,9 @@ extern "C" hq_status_t hq_gemm_code(const int8_t* A, const float* sa, int64_t M,
     a.KB = K / FK;
     a.MT = (M + FM - 1) / FM;
     a.NS = N / FN;
-    a.units = a.MT * a.NS;
+    const int R = a.MT > 1 ? 2 : 1;  // two activation tiles per decoded slab once there are two
+    a.MP = (a.MT + R - 1) / R;
+    a.units = a.MP * a.NS;
     a.beta = p.step;
     a.sa = sa;
     a.scale = code->scale;
@@ -435,24 +470,11 @@ extern "C" hq_status_t hq_gemm_code(const int8_t* A, const float* sa, int64_t M,
     a.ws = static_cast<WsHeader*>(ws);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
-    const size_t smem = sizeof(FusedSmem) + 1024;
-    const int64_t grid64 = a.units < num_sms() ? a.units : num_sms();
-    const int grid = (int)grid64;
     cudaError_t e;
     switch (p.lattice) {
-    case HQ_Z:
-        e = cudaFuncSetAttribute(gemm_code_kernel<HQ_Z>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) gemm_code_kernel<HQ_Z><<<grid, FTHREADS, smem, st>>>(a, ta, ty);
-        break;
-    case HQ_D4:
-        e = cudaFuncSetAttribute(gemm_code_kernel<HQ_D4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) gemm_code_kernel<HQ_D4><<<grid, FTHREADS, smem, st>>>(a, ta, ty);
-        break;
-    default:
-        e = cudaFuncSetAttribute(gemm_code_kernel<HQ_E8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) gemm_code_kernel<HQ_E8><<<grid, FTHREADS, smem, st>>>(a, ta, ty);
-        break;
+    case HQ_Z: e = R == 1 ? launch_fused<HQ_Z, 1>(a, ta, ty, st) : launch_fused<HQ_Z, 2>(a, ta, ty, st); break;
+    case HQ_D4: e = R == 1 ? launch_fused<HQ_D4, 1>(a, ta, ty, st) : launch_fused<HQ_D4, 2>(a, ta, ty, st); break;
+    default: e = R == 1 ? launch_fused<HQ_E8, 1>(a, ta, ty, st) : launch_fused<HQ_E8, 2>(a, ta, ty, st); break;
     }
-    if (e != cudaSuccess) return HQ_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+    return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }

@@ -1,8 +1,8 @@
 """The int8 tensor-core GEMM with the weight's decode fused into its producer warps
 (hq_gemm_code), on the GPU: bit-exact against the oracle's decode_int8 + grouped GEMM -- and so
 against the two-call path -- with activation row counts that are not multiples of 128, with fewer
-work units (128-row activation tile x 32-row weight slab) than SMs and with more, for the Z, D4
-and E8 codes; tiles with codes outside int8 are zero as in hq_decode_int8; chunks too long for a
+work units (one or two 128-row activation tiles x 32-row weight slab) than SMs and with more,
+with an odd number of activation tiles, for the Z, D4 and E8 codes; tiles with codes outside int8 are zero as in hq_decode_int8; chunks too long for a
 decoder warp's copy are read in place; and, sampled, the 4096 x 4096 weight at M = 16 and
 M = 4096."""
 import numpy as np
@@ -36,6 +36,7 @@ CASES = [
     (oracle.E8, 128, 1024, 2048, 0.29),
     (oracle.D4, 200, 384, 512, 0.45),
     (oracle.Z, 256, 256, 256, 0.35),
+    (oracle.E8, 300, 256, 512, 0.3),      # three activation tiles: the second pair's second tile lies past M
     (oracle.E8, 1000, 640, 512, 0.3),
     (oracle.E8, 2048, 1280, 256, 0.3),
 ]
