@@ -225,6 +225,10 @@ __global__ void __launch_bounds__(FusedCfg<R>::THREADS, 1)
                         tma_load_2d(sm.a[s][r], &tA, kb * FK, (int)((mp * R + r) * FM), &sm.a_full[s]);
                 }
             }
+            // no copy outlives the block: the last boxes of each stage have landed (at once, unless
+            // the MMA side stopped on a timeout)
+            for (int j = it > FSA ? it - FSA : 0; j < it; ++j)
+                if (!mbar_wait_sleep(&sm.a_full[j % FSA], (uint32_t)((j / FSA) & 1))) status_set(a.ws, kStTimeout);
         }
         __syncwarp();
     } else if (warp == 1) {
