@@ -275,8 +275,9 @@ hq_status_t hq_gemm_int8(const int8_t* A, const float* sa, int64_t M, const int8
  * from 0 in binary32, then Y = acc * sa[m]; tiles with a code outside int8 are zero (HQ_ERR_RANGE),
  * corrupt tiles too (HQ_ERR_CORRUPT).  A CTA takes 128 activation rows against a slab of 32
  * weight rows (one chunk of the code per K group) over all K groups, so every output element's
- * chain stays in one CTA.  ws: at least hq_gemm_code_workspace_bytes(M, N, K) bytes (the status
- * word); calls sharing ws must not overlap.
+ * chain stays in one CTA (two 128-row activation tiles per slab once M > 128).  Products with
+ * (M / 256) (N / 32) (K / 128) of 2^31 or more: HQ_ERR_UNSUPPORTED.  ws: at least
+ * hq_gemm_code_workspace_bytes(M, N, K) bytes (the status word); calls sharing ws must not overlap.
  */
 size_t hq_gemm_code_workspace_bytes(int64_t M, int64_t N, int64_t K);
 hq_status_t hq_gemm_code(const int8_t* A, const float* sa, int64_t M, const hq_code_t* code, float* Y, void* ws,

@@ -463,6 +463,8 @@ extern "C" hq_status_t hq_gemm_code(const int8_t* A, const float* sa, int64_t M,
     const int R = a.MT > 1 ? 2 : 1;  // two activation tiles per decoded slab once there are two
     a.MP = (a.MT + R - 1) / R;
     a.units = a.MP * a.NS;
+    // the roles count K groups over their units in 32-bit integers, and TMA coordinates are 32-bit
+    if (a.units * a.KB >= ((int64_t)1 << 31) || a.MP * R * FM >= ((int64_t)1 << 31)) return HQ_ERR_UNSUPPORTED;
     a.beta = p.step;
     a.sa = sa;
     a.scale = code->scale;
