@@ -37,6 +37,9 @@ CASES = [
     (oracle.D4, 200, 384, 512, 0.45),
     (oracle.Z, 256, 256, 256, 0.35),
     (oracle.E8, 300, 256, 512, 0.3),      # three activation tiles: the second pair's second tile lies past M
+    (oracle.E8, 1, 128, 128, 0.3),        # the smallest product: one row, one slab, one group
+    (oracle.Z, 129, 128, 640, 0.35),      # two tiles per slab, the second holding one row
+    (oracle.D4, 257, 384, 256, 0.45),     # three tiles: a partial third, a fourth past M
     (oracle.E8, 1000, 640, 512, 0.3),
     (oracle.E8, 2048, 1280, 256, 0.3),
 ]
