@@ -148,6 +148,27 @@ hq_status_t hq_encode(const void* x, hq_dtype_t dtype, int64_t rows, int64_t col
                       hq_code_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Several weights in one launch: the same codes, chunk offsets and bitstreams as one hq_encode per
+ * item, with the tiles of all items taken by one persistent grid, so that one tensor's last wave
+ * runs beside the next tensor's tiles instead of leaving SMs idle.
+ *   count  1 .. HQ_BATCH_MAX items; all share p.tile, p.lattice and dtype (HQ_ERR_UNSUPPORTED
+ *          otherwise); each item its own x, shape, step, seed and out (as for hq_encode)
+ *   ws     device workspace of at least hq_encode_batch_workspace_bytes(count, items) bytes (one
+ *          header and every item's look-back states); the status word reports the whole batch
+ * Returns HQ_ERR_ARG for an invalid item; nothing is launched then.
+ */
+#define HQ_BATCH_MAX 16
+typedef struct {
+    const void* x;     /* device, [rows, cols] row-major, dtype elements, 16-byte aligned        */
+    hq_dtype_t dtype;  /* HQ_BF16 or HQ_F32                                                     */
+    int64_t rows, cols;
+    hq_params_t p;
+    hq_code_t* out;    /* host struct as for hq_encode: arrays set by the caller, the rest filled */
+} hq_encode_item_t;
+size_t hq_encode_batch_workspace_bytes(int32_t count, const hq_encode_item_t* items);
+hq_status_t hq_encode_batch(int32_t count, const hq_encode_item_t* items, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Weight-path dither option: as hq_encode, with the dither of tile (row, tile column) added
  * before quantization (the method applies the dither to the KV cache; here any lattice, any
  * shape).  out->kv = 2; hq_decode takes the dither off again.
@@ -162,6 +183,19 @@ hq_status_t hq_encode_dither(const void* x, hq_dtype_t dtype, int64_t rows, int6
  * as zeros).
  */
 hq_status_t hq_decode(const hq_code_t* code, void* y, hq_dtype_t dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Several weight codes in one launch: the same output as one hq_decode per item, the tiles of all
+ * items taken by one grid.  count 1 .. HQ_BATCH_MAX; all codes share p.tile and p.lattice, are
+ * weight codes without dither (kv = 0), and all outputs one dtype (HQ_ERR_UNSUPPORTED
+ * otherwise).  ws: at least 64 bytes; the status word reports the whole batch.
+ */
+typedef struct {
+    const hq_code_t* code;
+    void* y;           /* device, [rows, cols], dtype elements, 16-byte aligned */
+    hq_dtype_t dtype;  /* HQ_BF16 or HQ_F32                                     */
+} hq_decode_item_t;
+hq_status_t hq_decode_batch(int32_t count, const hq_decode_item_t* items, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Encode a KV tensor kv[B, H, S, D] (device, contiguous) with D == p->tile and the dither

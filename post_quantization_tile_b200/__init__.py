@@ -43,6 +43,17 @@ class CodeStruct(ctypes.Structure):
                 ("cap_words", ctypes.c_int64), ("kv_s0", ctypes.c_int64)]
 
 
+class EncodeItem(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("p", Params), ("out", ctypes.POINTER(CodeStruct))]
+
+
+class DecodeItem(ctypes.Structure):
+    _fields_ = [("code", ctypes.POINTER(CodeStruct)), ("y", ctypes.c_void_p), ("dtype", ctypes.c_int32)]
+
+
+BATCH_MAX = 16
+
 _lib = None
 
 
@@ -80,6 +91,10 @@ def lib():
         L.hq_decode_int8.argtypes = [ctypes.POINTER(CodeStruct), P, P, P, ctypes.c_size_t, P]
         L.hq_gemm_int8.argtypes = [P, P, i64, P, P, i64, i64, i32, P, P, ctypes.c_size_t, P]
         L.hq_gemm_code.argtypes = [P, P, i64, ctypes.POINTER(CodeStruct), P, P, ctypes.c_size_t, P]
+        L.hq_encode_batch_workspace_bytes.argtypes = [i32, ctypes.POINTER(EncodeItem)]
+        L.hq_encode_batch_workspace_bytes.restype = ctypes.c_size_t
+        L.hq_encode_batch.argtypes = [i32, ctypes.POINTER(EncodeItem), P, ctypes.c_size_t, P]
+        L.hq_decode_batch.argtypes = [i32, ctypes.POINTER(DecodeItem), P, ctypes.c_size_t, P]
         L.hq_gemm_code_workspace_bytes.argtypes = [i64, i64, i64]
         L.hq_gemm_code_workspace_bytes.restype = ctypes.c_size_t
         L.hq_step_search.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, i32, ctypes.c_float, P, P,
@@ -95,6 +110,7 @@ def lib():
         L.hq_version.restype = i32
         for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_encode_at", "hq_kv_decode", "hq_quantize_coeffs",
                   "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_gemm_code", "hq_status_read",
+                  "hq_encode_batch", "hq_decode_batch",
                   "hq_kv_encode_dense", "hq_kv_decode_dense"]:
             getattr(L, f).restype = i32
         _lib = L
@@ -239,6 +255,66 @@ def encode(x: torch.Tensor, tile: int = 128, lattice: int | str = E8, step: floa
     _fill(code, cs)
     code.ws = w
     return code
+
+
+def encode_batch(xs, tile: int = 128, lattice: int | str = E8, steps=None, seeds=None, outs=None,
+                 ws: Workspace | None = None) -> list:
+    """Encode several 2-D CUDA tensors of one dtype in one launch (hq_encode_batch): the same codes
+    as one encode() per tensor.  steps and seeds give each tensor its step and seed."""
+    n = len(xs)
+    if not 1 <= n <= BATCH_MAX:
+        raise ValueError(f"1 .. {BATCH_MAX} tensors per batch")
+    steps = steps if steps is not None else [0.0] * n
+    seeds = seeds if seeds is not None else [0] * n
+    items = (EncodeItem * n)()
+    codes, structs = [], []
+    for i, x in enumerate(xs):
+        _require_cuda(x, "x")
+        if x.dim() != 2:
+            raise ValueError("each tensor must be 2-D [rows, cols]")
+        p = params(tile, lattice, steps[i], 4.0, seeds[i])
+        rows, cols = x.shape
+        code = outs[i] if outs is not None else alloc_code(rows, cols, p, device=x.device)
+        cs = code.struct()
+        codes.append(code)
+        structs.append(cs)
+        items[i].x = x.data_ptr()
+        items[i].dtype = _dtype_code(x)
+        items[i].rows, items[i].cols = rows, cols
+        items[i].p = p
+        items[i].out = ctypes.pointer(cs)
+    L = lib()
+    w = ws or workspace(L.hq_encode_batch_workspace_bytes(n, items))
+    _check(L.hq_encode_batch(n, items, w.ptr(), w.nbytes, _stream()), "hq_encode_batch")
+    for code, cs in zip(codes, structs):
+        _fill(code, cs)
+        code.ws = w
+    return codes
+
+
+def decode_batch(codes, dtype: torch.dtype = torch.bfloat16, outs=None, ws: Workspace | None = None) -> list:
+    """Decode several weight codes (one tile size and lattice, no dither) in one launch
+    (hq_decode_batch): the same tensors as one decode() per code."""
+    n = len(codes)
+    if not 1 <= n <= BATCH_MAX:
+        raise ValueError(f"1 .. {BATCH_MAX} codes per batch")
+    items = (DecodeItem * n)()
+    ys, structs = [], []
+    for i, code in enumerate(codes):
+        y = outs[i] if outs is not None else torch.empty(code.rows, code.cols, dtype=dtype, device=code.bits.device)
+        _require_cuda(y, "out")
+        cs = code.struct()
+        ys.append(y)
+        structs.append(cs)
+        items[i].code = ctypes.pointer(cs)
+        items[i].y = y.data_ptr()
+        items[i].dtype = _dtype_code(y)
+    L = lib()
+    w = ws or workspace(4096)
+    _check(L.hq_decode_batch(n, items, w.ptr(), w.nbytes, _stream()), "hq_decode_batch")
+    for code in codes:
+        code.ws = w
+    return ys
 
 
 def decode(code: Code, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None,

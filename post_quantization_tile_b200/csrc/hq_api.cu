@@ -389,8 +389,9 @@ hq_status_t step_search_common(const void* x, int src, int64_t rows, int64_t col
 
 // dst: 0 bf16, 1 fp32, 2 int8 lattice codes with group scales g_out, 3 fp32 lattice points minus the
 // dither in u units (KV tiles of 128, the dense inverse rotation's input)
-hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, float* g_out, void* ws,
-                          size_t ws_bytes, void* stream)
+// arguments and tensor map of one decode launch
+hq_status_t plan_decode(const hq_code_t* code, void* y, int dst, int32_t kv, float* g_out, void* ws, size_t ws_bytes,
+                        DecodeArgs& a, CUtensorMap& map)
 {
     if (!code || !y || !aligned16(y) || !ws || !aligned16(ws)) return HQ_ERR_ARG;
     if (code->version != HQ_FORMAT_VERSION) return HQ_ERR_ARG;
@@ -410,11 +411,8 @@ hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, f
     if (ws_bytes < sizeof(WsHeader)) return HQ_ERR_ARG;
     if (!use_device_of(y)) return HQ_ERR_ARG;
     const int es = dst == 0 ? 2 : (dst == 2 ? 1 : 4);
-    CUtensorMap map;
     if (!make_map(&map, y, code->rows, code->cols, es, g.TI)) return HQ_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
-    DecodeArgs a{};
+    a = DecodeArgs{};
     a.g_out = g_out;
     a.rows = code->rows;
     a.cols = code->cols;
@@ -434,7 +432,19 @@ hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, f
     a.bits = code->bits;
     a.cap_words = code->cap_words;
     a.ws = static_cast<WsHeader*>(ws);
-    return cuda_status(run_decode(prm.lattice, prm.tile, code->kv != 0, dst, a, map, st));
+    return HQ_OK;
+}
+
+hq_status_t decode_common(const hq_code_t* code, void* y, int dst, int32_t kv, float* g_out, void* ws,
+                          size_t ws_bytes, void* stream)
+{
+    DecodeArgs a;
+    CUtensorMap map;
+    const hq_status_t ps = plan_decode(code, y, dst, kv, g_out, ws, ws_bytes, a, map);
+    if (ps != HQ_OK) return ps;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
+    return cuda_status(run_decode(code->p.lattice, code->p.tile, code->kv != 0, dst, a, map, st));
 }
 
 // dense-rotation KV variant: the codec's workspace, then a 256-byte status block (the rotation's
@@ -517,6 +527,124 @@ hq_status_t hq_encode(const void* x, hq_dtype_t dtype, int64_t rows, int64_t col
 {
     if (dtype != HQ_BF16 && dtype != HQ_F32) return HQ_ERR_ARG;
     return encode_common(x, dtype == HQ_BF16 ? 0 : 1, rows, cols, p, 0, 0, nullptr, out, nullptr, ws, ws_bytes, stream);
+}
+
+// ---------------- several weights in one launch ----------------
+static_assert(HQ_BATCH_MAX == kEncodeBatchMax, "batch size of the C ABI");
+
+size_t hq_encode_batch_workspace_bytes(int32_t count, const hq_encode_item_t* items)
+{
+    if (count < 1 || count > HQ_BATCH_MAX || !items) return 0;
+    size_t n = sizeof(WsHeader);
+    for (int32_t i = 0; i < count; ++i) {
+        hq_params_t prm;
+        Geometry g;
+        const int src = items[i].dtype == HQ_BF16 ? 0 : 1;
+        if (!resolve_params(&items[i].p, prm)) return 0;
+        const int tpt = prm.tile == 64 ? 1 : (prm.tile == 256 ? 2 : enc_tpt(128, src));
+        if (!geometry(items[i].rows, items[i].cols, prm.tile, g, tpt)) return 0;
+        n += (size_t)g.items * 8u;
+    }
+    return n;
+}
+
+hq_status_t hq_encode_batch(int32_t count, const hq_encode_item_t* items, void* ws, size_t ws_bytes, void* stream)
+{
+    if (count < 1 || count > HQ_BATCH_MAX || !items || !ws) return HQ_ERR_ARG;
+    const size_t need = hq_encode_batch_workspace_bytes(count, items);
+    if (need == 0 || ws_bytes < need) return HQ_ERR_ARG;
+    static EncodeBatch<kEncodeBatchMax> b;  // large; filled and launched under the lock
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    b = EncodeBatch<kEncodeBatchMax>{};
+    int device = -1;
+    int64_t item0 = 0;
+    hq_params_t prm0{};
+    for (int32_t i = 0; i < count; ++i) {
+        const hq_encode_item_t& it = items[i];
+        if (it.dtype != HQ_BF16 && it.dtype != HQ_F32) return HQ_ERR_ARG;
+        if (it.dtype != items[0].dtype) return HQ_ERR_UNSUPPORTED;
+        EncodePlan pl;
+        const hq_status_t ps = plan_encode(it.x, it.dtype == HQ_BF16 ? 0 : 1, it.rows, it.cols, &it.p, 0, 0, nullptr,
+                                           it.out, false, ws, ws_bytes, pl);
+        if (ps != HQ_OK) return ps;
+        if (i == 0) prm0 = pl.prm;
+        if (pl.prm.tile != prm0.tile || pl.prm.lattice != prm0.lattice) return HQ_ERR_UNSUPPORTED;
+        int cur = -1;
+        if (cudaGetDevice(&cur) != cudaSuccess) return HQ_ERR_CUDA;
+        if (i > 0 && cur != device) return HQ_ERR_ARG;  // one device for the whole batch
+        device = cur;
+        pl.a.states = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + sizeof(WsHeader)) + item0;
+        b.map[i] = pl.map;
+        b.arg[i] = pl.a;
+        b.item0[i] = item0;
+        item0 += pl.g.items;
+    }
+    b.item0[count] = item0;
+    b.count = count;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, need, st) != cudaSuccess) return HQ_ERR_CUDA;
+    const int src = items[0].dtype == HQ_BF16 ? 0 : 1;
+    cudaError_t e;
+    switch (prm0.lattice) {
+    case HQ_Z: e = launch_encode_batch_z(prm0.tile, src, b, st); break;
+    case HQ_A2: e = launch_encode_batch_a2(prm0.tile, src, b, st); break;
+    case HQ_D4: e = launch_encode_batch_d4(prm0.tile, src, b, st); break;
+    default: e = launch_encode_batch_e8(prm0.tile, src, b, st); break;
+    }
+    if (e != cudaSuccess) return HQ_ERR_CUDA;
+    for (int32_t i = 0; i < count; ++i) {
+        hq_code_t* out = items[i].out;
+        out->rows = items[i].rows;
+        out->cols = items[i].cols;
+        out->kv_S = 0;
+        resolve_params(&items[i].p, out->p);
+        out->kv = 0;
+        out->kv_s0 = 0;
+        out->version = HQ_FORMAT_VERSION;
+    }
+    return HQ_OK;
+}
+
+hq_status_t hq_decode_batch(int32_t count, const hq_decode_item_t* items, void* ws, size_t ws_bytes, void* stream)
+{
+    if (count < 1 || count > HQ_BATCH_MAX || !items || !ws) return HQ_ERR_ARG;
+    static DecodeBatch<kEncodeBatchMax> b;  // large; filled and launched under the lock
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    b = DecodeBatch<kEncodeBatchMax>{};
+    int device = -1;
+    int64_t item0 = 0;
+    for (int32_t i = 0; i < count; ++i) {
+        const hq_decode_item_t& it = items[i];
+        if (!it.code) return HQ_ERR_ARG;
+        if (it.dtype != HQ_BF16 && it.dtype != HQ_F32) return HQ_ERR_ARG;
+        if (it.dtype != items[0].dtype || it.code->kv != 0 || !items[0].code ||
+            it.code->p.tile != items[0].code->p.tile || it.code->p.lattice != items[0].code->p.lattice)
+            return HQ_ERR_UNSUPPORTED;
+        const hq_status_t ps = plan_decode(it.code, it.y, it.dtype == HQ_BF16 ? 0 : 1, 0, nullptr, ws, ws_bytes,
+                                           b.arg[i], b.map[i]);
+        if (ps != HQ_OK) return ps;
+        int cur = -1;
+        if (cudaGetDevice(&cur) != cudaSuccess) return HQ_ERR_CUDA;
+        if (i > 0 && cur != device) return HQ_ERR_ARG;  // one device for the whole batch
+        device = cur;
+        b.item0[i] = item0;
+        item0 += b.arg[i].items;
+    }
+    b.item0[count] = item0;
+    b.count = count;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) != cudaSuccess) return HQ_ERR_CUDA;
+    const int n = items[0].code->p.tile, dst = items[0].dtype == HQ_BF16 ? 0 : 1;
+    cudaError_t e;
+    switch (items[0].code->p.lattice) {
+    case HQ_Z: e = launch_decode_batch_z(n, dst, b, st); break;
+    case HQ_A2: e = launch_decode_batch_a2(n, dst, b, st); break;
+    case HQ_D4: e = launch_decode_batch_d4(n, dst, b, st); break;
+    default: e = launch_decode_batch_e8(n, dst, b, st); break;
+    }
+    return cuda_status(e);
 }
 
 hq_status_t hq_encode_dither(const void* x, hq_dtype_t dtype, int64_t rows, int64_t cols, const hq_params_t* p,

@@ -31,6 +31,16 @@ struct DecodeArgs {
     int64_t kv_s0;    // KV: position of the code's first token in every sequence
 };
 
+// Several codes in one launch, as EncodeBatch: code t takes the global items item0[t] ..
+// item0[t + 1] - 1 (assigned to the blocks in turn); the header (status) is shared.
+template <int MAXB>
+struct DecodeBatch {
+    CUtensorMap map[MAXB];
+    DecodeArgs arg[MAXB];
+    int64_t item0[MAXB + 1];
+    int32_t count;
+};
+
 // DST: 0 bf16, 1 fp32, 2 int8 lattice codes (RHT domain, no transform), 3 fp32 lattice points minus
 // the dither in u units (no transform, no scale: the input of a dense inverse rotation)
 template <int N, int DST>
@@ -125,8 +135,22 @@ __device__ __forceinline__ void issue_item(DecSmem<N, DST>& sm, const DecodeArgs
     }
 }
 
-template <int N, int LAT, bool KV, int DST>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap)
+// the copy of global item g of a batch into stage s (the ring holds global item numbers)
+template <int N, int DST, int MAXB>
+__device__ __forceinline__ void issue_item_batch(DecSmem<N, DST>& sm, const DecodeBatch<MAXB>& B, int s, int64_t g)
+{
+    if (g >= B.item0[B.count]) {
+        sm.item_ring[s] = g;
+        sm.ok_ring[s] = 0;
+        return;
+    }
+    const int t = MAXB == 1 ? 0 : batch_tensor<MAXB>(B.item0, B.count, g);
+    issue_item<N, DST>(sm, B.arg[t], s, g - B.item0[t]);
+    sm.item_ring[s] = g;
+}
+
+template <int N, int LAT, bool KV, int DST, int MAXB>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const __grid_constant__ DecodeBatch<MAXB> B)
 {
     using G = DecGeom<N, DST>;
     using SM = DecSmem<N, DST>;
@@ -145,25 +169,33 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
         for (int s = 0; s < G::STAGES; ++s) mbar_init(&sm.bar[s], 1);
         fence_mbar_init();
         sm.mask_jt = -1;
-        for (int s = 0; s < G::STAGES; ++s) issue_item<N, DST>(sm, a, s, (int64_t)blockIdx.x + (int64_t)s * gridDim.x);
+        for (int s = 0; s < G::STAGES; ++s)
+            issue_item_batch<N, DST, MAXB>(sm, B, s, (int64_t)blockIdx.x + (int64_t)s * gridDim.x);
     }
     __syncthreads();
+    const int64_t total = B.item0[B.count];
 
     for (int iter = 0;; ++iter) {
         const int st = iter % G::STAGES;
         const uint32_t parity = (uint32_t)((iter / G::STAGES) & 1);
-        const int64_t item = sm.item_ring[st];
-        if (item >= a.items) break;
+        const int64_t gitem = sm.item_ring[st];
+        if (gitem >= total) break;
+        // this item's code; below, `item` is its index within that code
+        const int tb = MAXB == 1 ? 0 : batch_tensor<MAXB>(B.item0, B.count, gitem);
+        const DecodeArgs& a = B.arg[tb];
+        const CUtensorMap& tmap = B.map[tb];
+        const int64_t item = gitem - B.item0[tb];
         const int64_t jt = item / a.IB, ib = item % a.IB;
         const int64_t r0 = ib * TI;
         const int rows_valid = (int)min((int64_t)TI, a.rows - r0);
         const bool valid = row_l < rows_valid;
         const bool stage_ok = sm.ok_ring[st] != 0;
 
-        if (DST < 2 && sm.mask_jt != jt) {
+        const int64_t mkey = ((int64_t)tb << 48) | jt;  // code and tile column
+        if (DST < 2 && sm.mask_jt != mkey) {
             build_masks_out<N, DST>(sm.mask, jt, a.seed);
             __syncthreads();
-            if (tid == 0) sm.mask_jt = jt;
+            if (tid == 0) sm.mask_jt = mkey;
         }
 
         // tile lengths from meta -> bit offsets within the chunks (warp 0 scans each chunk)
@@ -198,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
             if (tid == 0) {
                 for (int k = 0; k < G::STAGES; ++k) {
                     const int sk = (iter + k) % G::STAGES;
-                    if (sm.item_ring[sk] < a.items) mbar_wait(&sm.bar[sk], (uint32_t)(((iter + k) / G::STAGES) & 1));
+                    if (sm.item_ring[sk] < total) mbar_wait(&sm.bar[sk], (uint32_t)(((iter + k) / G::STAGES) & 1));
                 }
             }
             break;
@@ -290,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) decode_kernel(const Deco
         }
         if (valid && stage_ok && !ok) status_set(a.ws, kStCorrupt);
         __syncthreads();  // the input stage is consumed: fetch the next item's words
-        if (tid == 0) issue_item<N, DST>(sm, a, st, item + (int64_t)G::STAGES * gridDim.x);
+        if (tid == 0) issue_item_batch<N, DST, MAXB>(sm, B, st, gitem + (int64_t)G::STAGES * gridDim.x);
 
         // ---------------- codes -> lattice point (float pairs) ----------------
         float2 P[H];

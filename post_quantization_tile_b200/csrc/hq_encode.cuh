@@ -38,6 +38,28 @@ struct EncodeArgs {
                                // out and report a timeout
 };
 
+// Several tensors in one launch: tensor t takes the global items item0[t] .. item0[t + 1] - 1,
+// in its own order, with its own look-back chain, outputs and tensor map; the header (work
+// counter, status) is shared.  One launch of one tensor is the batch of one.
+constexpr int kEncodeBatchMax = 16;
+template <int MAXB>
+struct EncodeBatch {
+    CUtensorMap map[MAXB];
+    EncodeArgs arg[MAXB];
+    int64_t item0[MAXB + 1];
+    int32_t count;
+};
+
+template <int MAXB>
+__device__ __forceinline__ int batch_tensor(const int64_t (&item0)[MAXB + 1], int32_t count, int64_t g)
+{
+    int t = 0;
+#pragma unroll
+    for (int i = 1; i < MAXB; ++i)
+        if (i < count && g >= item0[i]) t = i;
+    return t;
+}
+
 // SRC: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients (no RMS / RHT)
 template <int N, int SRC>
 struct EncGeom {
@@ -270,8 +292,17 @@ __device__ __forceinline__ void issue_tma(EncSmem<N, SRC>& sm, const CUtensorMap
         tma_load_2d(sm.buf + b * G::TI * 128, tmap, (int)(jt * N + b * (128 / G::ES)), (int)(ib * G::TI), &sm.bar);
 }
 
-template <int N, int LAT, bool KV, int SRC, bool COUNT>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const EncodeArgs a, const __grid_constant__ CUtensorMap tmap)
+// the TMA copy of global item g of a batch
+template <int N, int SRC, int MAXB>
+__device__ __forceinline__ void issue_tma_batch(EncSmem<N, SRC>& sm, const EncodeBatch<MAXB>& B, int64_t g)
+{
+    if (g >= B.item0[B.count]) return;
+    const int t = batch_tensor<MAXB>(B.item0, B.count, g);
+    issue_tma<N, SRC>(sm, &B.map[t], B.arg[t], g - B.item0[t]);
+}
+
+template <int N, int LAT, bool KV, int SRC, bool COUNT, int MAXB>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const __grid_constant__ EncodeBatch<MAXB> B)
 {
     using G = EncGeom<N, SRC>;
     using SM = EncSmem<N, SRC>;
@@ -287,12 +318,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
     const int tau = tid % TPT;
     unsigned char* const zzs = G::SEPARATE_ZZ ? sm.zzbuf : sm.buf;
 
+    // the header (work counter, status) and a step search are shared by the batch's tensors
+    WsHeader* const hdr = B.arg[0].ws;
+    const int64_t total = B.item0[B.count];
     // a count-only pass of a finished step search does nothing (block-uniform)
-    float beta = a.beta;
+    float beta_s = B.arg[0].beta;
     if constexpr (COUNT) {
-        if (a.search) {
-            if (*(volatile const int32_t*)&a.search->done) return;
-            beta = *(volatile const float*)&a.search->probe;
+        if (B.arg[0].search) {
+            if (*(volatile const int32_t*)&B.arg[0].search->done) return;
+            beta_s = *(volatile const float*)&B.arg[0].search->probe;
         }
     }
 
@@ -301,25 +335,31 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
         mbar_init(&sm.bar, 1);
         fence_mbar_init();
         sm.mask_jt = -1;
-        const int64_t it = (int64_t)atomicAdd(&a.ws->counter, 1u);
+        const int64_t it = (int64_t)atomicAdd(&hdr->counter, 1u);
         sm.item_cur = it;
-        issue_tma<N, SRC>(sm, &tmap, a, it);
+        issue_tma_batch<N, SRC, MAXB>(sm, B, it);
     }
     __syncthreads();
 
     for (int iter = 0;; ++iter) {
-        const int64_t item = sm.item_cur;
-        if (item >= a.items) break;
+        const int64_t gitem = sm.item_cur;
+        if (gitem >= total) break;
+        // this item's tensor; below, `item` is its index within that tensor
+        const int tb = MAXB == 1 ? 0 : batch_tensor<MAXB>(B.item0, B.count, gitem);
+        const EncodeArgs& a = B.arg[tb];
+        const int64_t item = gitem - B.item0[tb];
+        const float beta = MAXB == 1 ? beta_s : a.beta;
         const int64_t jt = item / a.IB, ib = item % a.IB;
         const int64_t r0 = ib * TI;
         const int rows_valid = (int)min((int64_t)TI, a.rows - r0);
         const bool valid = row_l < rows_valid;
 
         if constexpr (SRC != 2) {
-            if (sm.mask_jt != jt) {  // block-uniform
+            const int64_t mkey = ((int64_t)tb << 48) | jt;  // tensor and tile column
+            if (sm.mask_jt != mkey) {                       // block-uniform
                 build_masks<N, SRC>(sm.mask, jt, a.seed);
                 __syncthreads();
-                if (tid == 0) sm.mask_jt = jt;
+                if (tid == 0) sm.mask_jt = mkey;
             }
         }
         const bool arrived = mbar_wait(&sm.bar, (uint32_t)(iter & 1));
@@ -335,12 +375,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
         float sumsq;
         load_row<N, SRC>(sm.buf, sm.mask, row_l, tau, P, sumsq);
         unsigned int next_claim = 0;
-        if (tid == 0) next_claim = atomicAdd(&a.ws->counter, 1u);  // used once the stage is free
+        if (tid == 0) next_claim = atomicAdd(&hdr->counter, 1u);  // used once the stage is free
         __syncthreads();  // [A] the stage is consumed (and, aliased, becomes the zig-zag scratch)
         if constexpr (G::SEPARATE_ZZ) {
             if (tid == 0) {
                 sm.item_cur = next_claim;
-                issue_tma<N, SRC>(sm, &tmap, a, next_claim);
+                issue_tma_batch<N, SRC, MAXB>(sm, B, next_claim);
             }
         }
 
@@ -602,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
         if constexpr (COUNT) {
             if (!G::SEPARATE_ZZ && tid == 0) {
                 sm.item_cur = next_claim;
-                issue_tma<N, SRC>(sm, &tmap, a, next_claim);
+                issue_tma_batch<N, SRC, MAXB>(sm, B, next_claim);
             }
             __syncthreads();
             continue;
@@ -672,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) encode_kernel(const Enco
         __syncthreads();  // [E] scratch free: load the next item (aliased scratch)
         if (!G::SEPARATE_ZZ && tid == 0) {
             sm.item_cur = next_claim;
-            issue_tma<N, SRC>(sm, &tmap, a, next_claim);
+            issue_tma_batch<N, SRC, MAXB>(sm, B, next_claim);
         }
 
         // ---------------- look-back for the item's word offset (warp 0) ----------------

@@ -9,12 +9,27 @@ namespace hq {
 
 struct EncodeArgs;
 struct DecodeArgs;
+template <int MAXB>
+struct EncodeBatch;
+template <int MAXB>
+struct DecodeBatch;
+constexpr int kEncodeBatchMaxL = 16;  // = kEncodeBatchMax (hq_encode.cuh)
 
 // src: 0 bf16 weight, 1 fp32 weight, 2 fp32 normalised coefficients; count: count-only pass
 cudaError_t launch_encode_z(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_encode_a2(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_encode_d4(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_encode_e8(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
+// several weight tensors of one tile size, lattice and source type in one launch
+cudaError_t launch_encode_batch_z(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_encode_batch_a2(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_encode_batch_d4(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_encode_batch_e8(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+// several weight codes of one tile size and lattice to bf16 (dst 0) or fp32 (dst 1) in one launch
+cudaError_t launch_decode_batch_z(int n, int dst, const DecodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_decode_batch_a2(int n, int dst, const DecodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_decode_batch_d4(int n, int dst, const DecodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_decode_batch_e8(int n, int dst, const DecodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
 // dst: 0 bf16, 1 fp32, 2 int8 codes, 3 fp32 lattice points minus the dither (u units)
 cudaError_t launch_decode_z(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_decode_a2(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m, cudaStream_t st);
