@@ -207,7 +207,7 @@ def measured_traffic(kind: str, scalars: int):
             d = json.load(f)
     except Exception:
         return None
-    if d.get("kernel_sources_sha256_16") != kernel_sources_hash():
+    if d.get("kernel_sources_sha256_16") != kernel_sources_hash() or kind not in d:
         return None
     return d[kind]["bytes_per_scalar"] * scalars
 
@@ -404,22 +404,33 @@ def run_gpu(args):
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
 
-    # The step as a CUDA graph (one per replica phase: the memset and the kernel of each of the
-    # four calls, in order on one stream), captured through the public API and replayed, so that
-    # the timed region holds the GPU work alone: no host launch gaps and no timing events between
-    # the calls.  (Running the two matrices as concurrent graph branches was measured slower: the
-    # persistent grids of concurrent kernels compete for the same SM slots.)
+    # The timed step: both matrices through one batched encode and one batched decode
+    # (hq_encode_batch / hq_decode_batch: one persistent grid takes the tiles of both, so the
+    # smaller matrix's last wave does not leave SMs idle), as a CUDA graph (one per replica phase:
+    # a workspace memset and one kernel per call) captured through the public API and replayed,
+    # so that the timed region holds the GPU work alone: no host launch gaps and no timing events
+    # between the calls.  (Running the matrices as concurrent graph branches was measured slower:
+    # the persistent grids of concurrent kernels compete for the same SM slots.)
+    ws_batch = hq.Workspace(2 * ws.nbytes, device=dev)
+
+    def step_batched(k):
+        r, rd = k % REPLICAS, (k + 1) % REPLICAS
+        hq.encode_batch(xs[r], TILE, hq.E8, steps_beta, [SEED] * len(SHAPES), outs=codes[r], ws=ws_batch)
+        hq.decode_batch(codes[rd], outs=outs, ws=ws_batch)
+
+    for k in range(max(3, args.warmup)):
+        step_batched(k)
     graphs = []
     for r in range(REPLICAS):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step(r)
+            step_batched(r)
         graphs.append(g)
     torch.cuda.synchronize()
     for k in range(max(3, args.warmup)):
         graphs[k % REPLICAS].replay()
     torch.cuda.synchronize()
-    st, _ = hq.status(ws)
+    st, _ = hq.status(ws_batch)
     if st != 0:
         raise RuntimeError(f"device status {st} after the graph warm-up")
 
@@ -440,7 +451,16 @@ def run_gpu(args):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        # per-call times: the same steps eagerly, each call bracketed by events on its stream
+        # per-call times: the same steps eagerly, each call bracketed by events on its stream:
+        # the two batched calls of the timed step, then the four single calls
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for k in range(args.steps):
+            r, rd = (args.warmup + k) % REPLICAS, (args.warmup + k + 1) % REPLICAS
+            bev[k][0].record(stream)
+            hq.encode_batch(xs[r], TILE, hq.E8, steps_beta, [SEED] * len(SHAPES), outs=codes[r], ws=ws_batch)
+            bev[k][1].record(stream)
+            hq.decode_batch(codes[rd], outs=outs, ws=ws_batch)
+            bev[k][2].record(stream)
         e_t0.record(stream)
         for k in range(args.steps):
             step(args.warmup + k, record=k)
@@ -458,6 +478,9 @@ def run_gpu(args):
                   for k in range(args.steps)] for i in range(len(SHAPES))]
     enc_ms = [statistics.mean(c) for c in enc_calls]
     dec_ms = [statistics.mean(c) for c in dec_calls]
+    encb_calls = [e[0].elapsed_time(e[1]) for e in bev]
+    decb_calls = [e[1].elapsed_time(e[2]) for e in bev]
+    encb_ms, decb_ms = statistics.mean(encb_calls), statistics.mean(decb_calls)
 
     # e2e through the public API with host buffers: every step copies each matrix in from pinned
     # host memory, encodes and decodes it and copies the reconstruction out.  Copies in, kernels
@@ -504,15 +527,19 @@ def run_gpu(args):
     st, _ = hq.status(ws)
 
     peak, peak_kind = load_peaks()
-    # dominant kernel: the larger of encode / decode of the 11008x4096 matrix
-    i_big = 1
-    enc_bytes = SHAPES[i_big][0] * SHAPES[i_big][1] * 2 + code_bytes[i_big]
-    dec_bytes = code_bytes[i_big] + SHAPES[i_big][0] * SHAPES[i_big][1] * 2
-    if enc_ms[i_big] >= dec_ms[i_big]:
-        kname, kms, kbytes = "encode", enc_ms[i_big], enc_bytes
+    # dominant kernel of the timed step: the larger of the batched encode / decode (both matrices;
+    # algorithmic bytes: the bf16 input plus the code, 2.53 B per scalar at 4.26 total bps)
+    scalars_all = sum(r * c for r, c in SHAPES)
+    b_bytes = bf16_bytes + sum(code_bytes)
+    if encb_ms >= decb_ms:
+        kname, kms = "encode_batch", encb_ms
     else:
-        kname, kms, kbytes = "decode", dec_ms[i_big], dec_bytes
+        kname, kms = "decode_batch", decb_ms
+    kbytes = b_bytes
     achieved = kbytes / (kms * 1e-3) / 1e9
+    # the single 11008 x 4096 kernels, as before batching
+    i_big = 1
+    big_bytes = SHAPES[i_big][0] * SHAPES[i_big][1] * 2 + code_bytes[i_big]
     value = weak_scaling_value(bf16_bytes, world, ms)
 
     kv = None if args.no_kv else run_kv(hq, dev, stream, peak)
@@ -544,9 +571,10 @@ def run_gpu(args):
                        "shapes": SHAPES, "tile": TILE, "lattice": "E8", "target_bps": BPS,
                        "step": steps_beta, "payload_bps": payload_bps, "total_bps": total_bps, "nmse": mse,
                        "l2": "inputs and codes rotate over 3 replicas (124 MB bf16 each), no L2 reuse across launches",
-                       "launch": "timed steps are replays of a CUDA graph of the four API calls in order on "
-                                 "one stream; encode_ms / decode_ms and the roofline come from the same steps "
-                                 "run eagerly with events around each call (eager_ms_per_step)",
+                       "launch": "timed steps are replays of a CUDA graph of two API calls (hq_encode_batch of "
+                                 "both matrices, then hq_decode_batch); encode_ms / decode_ms and the roofline "
+                                 "come from the same work run eagerly as four single calls with events around "
+                                 "each (eager_ms_per_step)",
                        "parallelism": f"replicas{world}"},
             "eager_ms_per_step": eager_ms,
             "encode_gbs": [SHAPES[i][0] * SHAPES[i][1] * 2 / (enc_ms[i] * 1e-3) / 1e9 for i in range(len(SHAPES))],
@@ -554,10 +582,21 @@ def run_gpu(args):
             "encode_ms": enc_ms, "decode_ms": dec_ms,
             "encode_ms_p10_p50_p90": [percentiles(c) for c in enc_calls],
             "decode_ms_p10_p50_p90": [percentiles(c) for c in dec_calls],
-            "roofline": {"bound": "hbm", "kernel": f"{kname} 11008x4096", "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "bytes_per_launch": kbytes,
-                         "traffic": measured_traffic(kname, SHAPES[i_big][0] * SHAPES[i_big][1])},
+            "roofline": {"bound": "hbm", "kernel": f"{kname} 4096x4096+11008x4096", "achieved": achieved,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "bytes_per_launch": kbytes, "launch_ms": kms,
+                         "traffic": measured_traffic(kname, scalars_all)},
+            "batched_ms": {"encode": encb_ms, "decode": decb_ms,
+                           "encode_p10_p50_p90": percentiles(encb_calls), "decode_p10_p50_p90": percentiles(decb_calls)},
+            # the single kernels of the larger matrix, as the bench reported before batching
+            "roofline_11008x4096": {
+                "encode": {"achieved": big_bytes / (enc_ms[i_big] * 1e-3) / 1e9,
+                           "frac": big_bytes / (enc_ms[i_big] * 1e-3) / 1e9 / peak,
+                           "traffic": measured_traffic("encode", SHAPES[i_big][0] * SHAPES[i_big][1])},
+                "decode": {"achieved": big_bytes / (dec_ms[i_big] * 1e-3) / 1e9,
+                           "frac": big_bytes / (dec_ms[i_big] * 1e-3) / 1e9 / peak,
+                           "traffic": measured_traffic("decode", SHAPES[i_big][0] * SHAPES[i_big][1])},
+                "peak": peak, "unit": "GB/s", "bytes_per_launch": big_bytes},
             # the 4096 x 4096 weight, the shape the throughput target names
             "roofline_4096x4096": {
                 "encode": {"achieved": (SHAPES[0][0] * SHAPES[0][1] * 2 + code_bytes[0]) / (enc_ms[0] * 1e-3) / 1e9,
@@ -568,7 +607,7 @@ def run_gpu(args):
             "cpu_baseline": cpu,
             "e2e": {"value": weak_scaling_value(bf16_bytes, world, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": bf16_bytes, "d2h_bytes_per_step": bf16_bytes},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": 2 * args.steps,
             "kv_cache": kv,
             "workloads": work,
             "gemm_int8": gemm,
@@ -731,8 +770,10 @@ def run_dit_stack(hq, dev, stream, peak):
     """The whole DiT-shaped stack: 48 blocks of 4 x 4096x4096 and 4096x16384 + 16384x4096 bf16
     linears (9.66 G parameters, 19.3 GB), E8 at 4 bps, n = 128.  Weights are drawn on the device
     (the host generator would take minutes); the step is searched per matrix; one pass encodes
-    every matrix, one pass decodes every code, each replayed from a CUDA graph of its calls and
-    timed as a whole with CUDA events."""
+    every matrix, one pass decodes every code, in batches of 16 matrices per launch, each pass
+    replayed from a CUDA graph of its calls and timed as a whole with CUDA events."""
+    import ctypes
+
     import torch
 
     from post_quantization_tile_b200 import workloads as W
@@ -759,31 +800,55 @@ def run_dit_stack(hq, dev, stream, peak):
     enc_all()
     dec_all()
     torch.cuda.synchronize()
-    # each pass as one CUDA graph of its 288 calls (as the headline step), replayed
+    # the passes as batches of 16 matrices (18 encode and 18 decode launches), each pass one CUDA
+    # graph of its calls (as the headline step), replayed; the batched codes equal the single ones
+    B = hq.BATCH_MAX
+    prm = hq.params(TILE, hq.E8, 0.3)
+    need = [hq.lib().hq_workspace_bytes(x.shape[0], x.shape[1], ctypes.byref(prm)) for x in mats]
+    ws_b = hq.Workspace(max(sum(need[j:j + B]) for j in range(0, len(mats), B)), device=dev)
+    # one output per batch position and shape, so that no two items of a launch share a buffer
+    pool = {shape: [torch.empty(*shape, dtype=torch.bfloat16, device=dev) for _ in range(B)]
+            for shape in set(W.DIT_BLOCK_SHAPES)}
+
+    def enc_all_b():
+        for j in range(0, len(mats), B):
+            hq.encode_batch(mats[j:j + B], TILE, hq.E8, betas[j:j + B], [5 + i // 6 for i in range(j, j + B)],
+                            outs=codes[j:j + B], ws=ws_b)
+
+    def dec_all_b():
+        for j in range(0, len(codes), B):
+            part = codes[j:j + B]
+            hq.decode_batch(part, outs=[pool[(c.rows, c.cols)][i] for i, c in enumerate(part)], ws=ws_b)
+    first = [codes[i].bits[:codes[i].total_words()].clone() for i in (0, 5, len(codes) - 1)]
+    enc_all_b()
+    dec_all_b()
+    torch.cuda.synchronize()
+    same = all(torch.equal(codes[i].bits[:codes[i].total_words()], f) for i, f in zip((0, 5, len(codes) - 1), first))
     g_enc, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_enc):
-        enc_all()
+        enc_all_b()
     with torch.cuda.graph(g_dec):
-        dec_all()
+        dec_all_b()
     g_enc.replay()
     g_dec.replay()
     torch.cuda.synchronize()
     enc, dec = time_pairs(stream, [g_enc.replay], [g_dec.replay], 3)
-    st, _ = hq.status(ws)
+    st = hq.status(ws)[0] | hq.status(ws_b)[0]
     del g_enc, g_dec
     cbytes = sum(code_bytes_of(cd) for cd in codes)
     e50, d50 = statistics.median(enc), statistics.median(dec)
     moved = 2 * params + cbytes
     pbits = sum(cd.payload_bps() * cd.rows * cd.cols for cd in codes)
     res = {"workload": "dit_stack_48x(4x4096x4096+4096x16384+16384x4096)_bf16_E8_n128_4bps",
-           "parameters": params, "matrices": len(mats), "launches_per_pass": len(mats),
+           "parameters": params, "matrices": len(mats), "launches_per_pass": (len(mats) + B - 1) // B,
+           "batched_codes_equal_single": bool(same),
            "payload_bps": pbits / params, "encode_pass_ms_p10_p50_p90": percentiles(enc),
            "decode_pass_ms_p10_p50_p90": percentiles(dec),
            "encode_gbs_in": 2 * params / (e50 * 1e-3) / 1e9, "decode_gbs_out": 2 * params / (d50 * 1e-3) / 1e9,
            "encode_roofline_frac": moved / (e50 * 1e-3) / 1e9 / peak,
            "decode_roofline_frac": moved / (d50 * 1e-3) / 1e9 / peak, "bytes_per_pass": moved,
            "data": "device-drawn (torch CUDA generator), same distribution as the host generator", "status": st}
-    del mats, codes, outs
+    del mats, codes, outs, pool
     torch.cuda.empty_cache()
     return res
 
@@ -1005,6 +1070,29 @@ def run_profile(args):
         if st != 0:
             raise SystemExit(1)
         return
+    if args.profile in ("encode_batch", "decode_batch"):
+        # the batched kernels on a 4096 x 4096 and a 12288 x 4096 weight (134 MB together)
+        xs = [torch.from_numpy(W.llama_weight(r, 4096, seed=9 + i).view(np.int16)).view(torch.bfloat16).cuda()
+              for i, r in enumerate((4096, 12288))]
+        codes = hq.encode_batch(xs, TILE, hq.E8, [0.29, 0.29], [SEED, SEED])
+        ys = [torch.empty_like(x) for x in xs]
+        ws = codes[0].ws
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        torch.cuda.synchronize()
+        for i in range(3):
+            ev[i].record()
+            if args.profile == "encode_batch":
+                hq.encode_batch(xs, TILE, hq.E8, [0.29, 0.29], [SEED, SEED], outs=codes, ws=ws)
+            else:
+                hq.decode_batch(codes, outs=ys, ws=ws)
+        ev[3].record()
+        torch.cuda.synchronize()
+        st, _ = hq.status(ws)
+        print(json.dumps({"profile": args.profile, "ms": [ev[i].elapsed_time(ev[i + 1]) for i in range(3)],
+                          "status": st}), flush=True)
+        if st != 0:
+            raise SystemExit(1)
+        return
     x = torch.from_numpy(W.llama_weight(16384, 4096, seed=9).view(np.int16)).view(torch.bfloat16).cuda()
     beta = 0.29
     code = hq.encode(x, TILE, hq.E8, beta, seed=SEED)
@@ -1030,7 +1118,8 @@ def run_profile(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile", choices=["encode", "decode", "count", "gemm", "gemm_fused", "kv", "kv_dense"],
+    ap.add_argument("--profile", choices=["encode", "decode", "count", "encode_batch", "decode_batch", "gemm",
+                                          "gemm_fused", "kv", "kv_dense"],
                     default=None)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
