@@ -130,3 +130,28 @@ def test_fused_gemm_checks_arguments_without_a_gpu(libhq):
     cs.kv = 1                                                      # a dithered KV code
     assert L.hq_gemm_code(ctypes.c_void_p(16), ctypes.c_void_p(16), 16, ctypes.byref(cs), ctypes.c_void_p(16), ws,
                           1 << 20, None) == 1
+
+
+def test_batch_entry_points_check_arguments_without_a_gpu(libhq):
+    import post_quantization_tile_b200 as hq
+    L = hq.lib()
+    items = (hq.EncodeItem * 3)()
+    for i in range(3):
+        items[i].x = 16 * (i + 1)
+        items[i].dtype = hq.BF16
+        items[i].rows, items[i].cols = 300 + i, 512
+        items[i].p = hq.params(128, hq.E8, 0.3)
+    # one header and every item's look-back states: 3, 3 and 3 items of 128 rows x 4 tile columns
+    per = [((300 + i + 127) // 128) * 4 for i in range(3)]
+    assert L.hq_encode_batch_workspace_bytes(3, items) == 64 + 8 * sum(per)
+    assert L.hq_encode_batch_workspace_bytes(0, items) == 0
+    assert L.hq_encode_batch_workspace_bytes(17, items) == 0          # more than HQ_BATCH_MAX
+    items[2].cols = 500                                                 # not a multiple of the tile
+    assert L.hq_encode_batch_workspace_bytes(3, items) == 0
+    ws = ctypes.c_void_p(256)
+    assert L.hq_encode_batch(0, items, ws, 1 << 20, None) == 1
+    assert L.hq_encode_batch(17, items, ws, 1 << 20, None) == 1
+    assert L.hq_encode_batch(3, items, ws, 1 << 20, None) == 1         # the bad item
+    dec = (hq.DecodeItem * 2)()
+    assert L.hq_decode_batch(0, dec, ws, 4096, None) == 1
+    assert L.hq_decode_batch(2, dec, ws, 4096, None) == 1              # no codes
