@@ -543,6 +543,8 @@ def run_gpu(args):
     value = weak_scaling_value(bf16_bytes, world, ms)
 
     kv = None if args.no_kv else run_kv(hq, dev, stream, peak)
+    if kv is not None:
+        kv["append_step"] = run_kv_append(hq, dev)
     gemm = None if args.no_gemm else run_gemm(hq, dev, load_bf16_peak())
 
     work = None if args.no_workloads else run_workloads(hq, dev, stream, peak, xs)
@@ -660,6 +662,54 @@ def codec_entry(name, scalars, in_bytes_per_scalar, code, enc, dec, peak, **extr
             "encode_roofline_frac": moved / (e50 * 1e-3) / 1e9 / peak,
             "decode_roofline_frac": moved / (d50 * 1e-3) / 1e9 / peak,
             "bytes_per_call": moved, **extra}
+
+
+def run_kv_append(hq, dev):
+    """One decoding step's KV appends: 64 tensors [8, 32, 1, 128] bf16 (keys and values of 32
+    layers, one token of each of 8 x 32 sequences, at position 4096), D4 with the dither at 2 bps:
+    a CUDA graph of 64 hq_kv_encode_at calls against a graph of four hq_kv_encode_batch calls of 16
+    (the same codes), each replayed 20 times between CUDA events."""
+    import ctypes
+
+    import torch
+    g = torch.Generator(device=dev).manual_seed(11)
+    kvs = [torch.randn(8, 32, 1, 128, device=dev, generator=g).bfloat16() for _ in range(64)]
+    step, s0 = 1.125, 4096
+    codes = [hq.kv_encode(kv, step=step, seed=7, s0=s0) for kv in kvs]
+    prm = hq.params(128, hq.D4, step)
+    ws1 = hq.Workspace(hq.lib().hq_workspace_bytes(256, 128, ctypes.byref(prm)), device=dev)
+    wsb = hq.Workspace(16 * hq.lib().hq_workspace_bytes(256, 128, ctypes.byref(prm)), device=dev)
+
+    def singles():
+        for i, kv in enumerate(kvs):
+            hq.kv_encode(kv, step=step, seed=7, s0=s0, out=codes[i], ws=ws1)
+
+    def batched():
+        for j in range(0, len(kvs), 16):
+            hq.kv_encode_batch(kvs[j:j + 16], [s0] * 16, [step] * 16, [7] * 16, outs=codes[j:j + 16], ws=wsb)
+    singles()
+    torch.cuda.synchronize()
+    ref = [c.bits[:c.total_words()].clone() for c in codes[::21]]
+    out = {"workload": "kv_append_64x[8,32,1,128]_bf16_D4_dither_2bps_s0=4096", "tensors": len(kvs)}
+    for name, fn in (("single_calls", singles), ("batched_calls", batched)):
+        fn()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name + "_us_per_step"] = e0.elapsed_time(e1) / 20 * 1e3
+        del gr
+    out["codes_equal"] = all(torch.equal(c.bits[:c.total_words()], r) for c, r in zip(codes[::21], ref))
+    out["status"] = hq.status(ws1)[0] | hq.status(wsb)[0]
+    return out
 
 
 def run_kv(hq, dev, stream, peak):

@@ -169,6 +169,23 @@ size_t hq_encode_batch_workspace_bytes(int32_t count, const hq_encode_item_t* it
 hq_status_t hq_encode_batch(int32_t count, const hq_encode_item_t* items, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Several KV tensors (or token appends) in one launch, e.g. the keys and values of every layer for
+ * one decoding step: the same codes as one hq_kv_encode_at (hq_kv_encode when s0 = 0) per item.
+ * Each item: kv[B, H, S, D] (device, contiguous, 16-byte aligned), the positions s0 .. s0 + S - 1,
+ * its own step and seed.  All items share D = p.tile = 128, p.lattice and dtype
+ * (HQ_ERR_UNSUPPORTED otherwise).  ws: hq_kv_encode_batch_workspace_bytes(count, items) bytes.
+ */
+typedef struct {
+    const void* kv;
+    hq_dtype_t dtype;
+    int64_t B, H, S, D, s0;
+    hq_params_t p;
+    hq_code_t* out;
+} hq_kv_item_t;
+size_t hq_kv_encode_batch_workspace_bytes(int32_t count, const hq_kv_item_t* items);
+hq_status_t hq_kv_encode_batch(int32_t count, const hq_kv_item_t* items, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Weight-path dither option: as hq_encode, with the dither of tile (row, tile column) added
  * before quantization (the method applies the dither to the KV cache; here any lattice, any
  * shape).  out->kv = 2; hq_decode takes the dither off again.

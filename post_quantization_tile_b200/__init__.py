@@ -52,6 +52,12 @@ class DecodeItem(ctypes.Structure):
     _fields_ = [("code", ctypes.POINTER(CodeStruct)), ("y", ctypes.c_void_p), ("dtype", ctypes.c_int32)]
 
 
+class KvItem(ctypes.Structure):
+    _fields_ = [("kv", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("B", ctypes.c_int64), ("H", ctypes.c_int64),
+                ("S", ctypes.c_int64), ("D", ctypes.c_int64), ("s0", ctypes.c_int64), ("p", Params),
+                ("out", ctypes.POINTER(CodeStruct))]
+
+
 BATCH_MAX = 16
 
 _lib = None
@@ -95,6 +101,9 @@ def lib():
         L.hq_encode_batch_workspace_bytes.restype = ctypes.c_size_t
         L.hq_encode_batch.argtypes = [i32, ctypes.POINTER(EncodeItem), P, ctypes.c_size_t, P]
         L.hq_decode_batch.argtypes = [i32, ctypes.POINTER(DecodeItem), P, ctypes.c_size_t, P]
+        L.hq_kv_encode_batch_workspace_bytes.argtypes = [i32, ctypes.POINTER(KvItem)]
+        L.hq_kv_encode_batch_workspace_bytes.restype = ctypes.c_size_t
+        L.hq_kv_encode_batch.argtypes = [i32, ctypes.POINTER(KvItem), P, ctypes.c_size_t, P]
         L.hq_gemm_code_workspace_bytes.argtypes = [i64, i64, i64]
         L.hq_gemm_code_workspace_bytes.restype = ctypes.c_size_t
         L.hq_step_search.argtypes = [P, i32, i64, i64, ctypes.POINTER(Params), i32, i64, i32, ctypes.c_float, P, P,
@@ -110,7 +119,7 @@ def lib():
         L.hq_version.restype = i32
         for f in ["hq_encode", "hq_encode_dither", "hq_decode", "hq_kv_encode", "hq_kv_encode_at", "hq_kv_decode", "hq_quantize_coeffs",
                   "hq_encode_count", "hq_step_search", "hq_decode_int8", "hq_gemm_int8", "hq_gemm_code", "hq_status_read",
-                  "hq_encode_batch", "hq_decode_batch",
+                  "hq_encode_batch", "hq_decode_batch", "hq_kv_encode_batch",
                   "hq_kv_encode_dense", "hq_kv_decode_dense"]:
             getattr(L, f).restype = i32
         _lib = L
@@ -356,6 +365,43 @@ def kv_encode(kv: torch.Tensor, step: float = 0.0, bps: float = 4.0, seed: int =
     _fill(code, cs)
     code.ws = w
     return code
+
+
+def kv_encode_batch(kvs, s0s=None, steps=None, seeds=None, lattice: int | str = D4, outs=None,
+                    ws: Workspace | None = None) -> list:
+    """Encode several KV tensors [B, H, S, 128] of one dtype in one launch (hq_kv_encode_batch), item i
+    as the tokens s0s[i] .. of every sequence: the same codes as one kv_encode(..., s0=s0s[i]) each."""
+    n = len(kvs)
+    if not 1 <= n <= BATCH_MAX:
+        raise ValueError(f"1 .. {BATCH_MAX} tensors per batch")
+    s0s = s0s if s0s is not None else [0] * n
+    steps = steps if steps is not None else [0.0] * n
+    seeds = seeds if seeds is not None else [0] * n
+    items = (KvItem * n)()
+    codes, structs = [], []
+    for i, kv in enumerate(kvs):
+        _require_cuda(kv, "kv")
+        if kv.dim() != 4:
+            raise ValueError("each kv must be [B, H, S, D]")
+        B, H, S, D = kv.shape
+        p = params(D, lattice, steps[i], 4.0, seeds[i])
+        code = outs[i] if outs is not None else alloc_code(B * H * S, D, p, device=kv.device)
+        cs = code.struct()
+        codes.append(code)
+        structs.append(cs)
+        items[i].kv = kv.data_ptr()
+        items[i].dtype = _dtype_code(kv)
+        items[i].B, items[i].H, items[i].S, items[i].D = B, H, S, D
+        items[i].s0 = int(s0s[i])
+        items[i].p = p
+        items[i].out = ctypes.pointer(cs)
+    L = lib()
+    w = ws or workspace(L.hq_kv_encode_batch_workspace_bytes(n, items))
+    _check(L.hq_kv_encode_batch(n, items, w.ptr(), w.nbytes, _stream()), "hq_kv_encode_batch")
+    for code, cs in zip(codes, structs):
+        _fill(code, cs)
+        code.ws = w
+    return codes
 
 
 def kv_decode(code: Code, shape, dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None,

@@ -548,11 +548,13 @@ size_t hq_encode_batch_workspace_bytes(int32_t count, const hq_encode_item_t* it
     return n;
 }
 
-hq_status_t hq_encode_batch(int32_t count, const hq_encode_item_t* items, void* ws, size_t ws_bytes, void* stream)
+// one launch over several planned encodes: item i planned by plan(i, pl); finish(i, prm) fills
+// item i's code header afterwards
+extern "C++" {
+template <typename Plan, typename Finish>
+static hq_status_t encode_batch_common(int32_t count, bool kv, int src, size_t need, void* ws, void* stream, Plan plan,
+                                       Finish finish)
 {
-    if (count < 1 || count > HQ_BATCH_MAX || !items || !ws) return HQ_ERR_ARG;
-    const size_t need = hq_encode_batch_workspace_bytes(count, items);
-    if (need == 0 || ws_bytes < need) return HQ_ERR_ARG;
     static EncodeBatch<kEncodeBatchMax> b;  // large; filled and launched under the lock
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
@@ -561,12 +563,8 @@ hq_status_t hq_encode_batch(int32_t count, const hq_encode_item_t* items, void* 
     int64_t item0 = 0;
     hq_params_t prm0{};
     for (int32_t i = 0; i < count; ++i) {
-        const hq_encode_item_t& it = items[i];
-        if (it.dtype != HQ_BF16 && it.dtype != HQ_F32) return HQ_ERR_ARG;
-        if (it.dtype != items[0].dtype) return HQ_ERR_UNSUPPORTED;
         EncodePlan pl;
-        const hq_status_t ps = plan_encode(it.x, it.dtype == HQ_BF16 ? 0 : 1, it.rows, it.cols, &it.p, 0, 0, nullptr,
-                                           it.out, false, ws, ws_bytes, pl);
+        const hq_status_t ps = plan(i, pl);
         if (ps != HQ_OK) return ps;
         if (i == 0) prm0 = pl.prm;
         if (pl.prm.tile != prm0.tile || pl.prm.lattice != prm0.lattice) return HQ_ERR_UNSUPPORTED;
@@ -580,30 +578,100 @@ hq_status_t hq_encode_batch(int32_t count, const hq_encode_item_t* items, void* 
         b.item0[i] = item0;
         item0 += pl.g.items;
     }
+    if (kv && prm0.tile != 128) return HQ_ERR_UNSUPPORTED;
     b.item0[count] = item0;
     b.count = count;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws, 0, need, st) != cudaSuccess) return HQ_ERR_CUDA;
-    const int src = items[0].dtype == HQ_BF16 ? 0 : 1;
     cudaError_t e;
     switch (prm0.lattice) {
-    case HQ_Z: e = launch_encode_batch_z(prm0.tile, src, b, st); break;
-    case HQ_A2: e = launch_encode_batch_a2(prm0.tile, src, b, st); break;
-    case HQ_D4: e = launch_encode_batch_d4(prm0.tile, src, b, st); break;
-    default: e = launch_encode_batch_e8(prm0.tile, src, b, st); break;
+    case HQ_Z: e = launch_encode_batch_z(prm0.tile, kv, src, b, st); break;
+    case HQ_A2: e = launch_encode_batch_a2(prm0.tile, kv, src, b, st); break;
+    case HQ_D4: e = launch_encode_batch_d4(prm0.tile, kv, src, b, st); break;
+    default: e = launch_encode_batch_e8(prm0.tile, kv, src, b, st); break;
     }
     if (e != cudaSuccess) return HQ_ERR_CUDA;
-    for (int32_t i = 0; i < count; ++i) {
-        hq_code_t* out = items[i].out;
-        out->rows = items[i].rows;
-        out->cols = items[i].cols;
-        out->kv_S = 0;
-        resolve_params(&items[i].p, out->p);
-        out->kv = 0;
-        out->kv_s0 = 0;
-        out->version = HQ_FORMAT_VERSION;
-    }
+    for (int32_t i = 0; i < count; ++i) finish(i, prm0);
     return HQ_OK;
+}
+}  // extern "C++"
+
+hq_status_t hq_encode_batch(int32_t count, const hq_encode_item_t* items, void* ws, size_t ws_bytes, void* stream)
+{
+    if (count < 1 || count > HQ_BATCH_MAX || !items || !ws) return HQ_ERR_ARG;
+    const size_t need = hq_encode_batch_workspace_bytes(count, items);
+    if (need == 0 || ws_bytes < need) return HQ_ERR_ARG;
+    for (int32_t i = 0; i < count; ++i) {
+        if (items[i].dtype != HQ_BF16 && items[i].dtype != HQ_F32) return HQ_ERR_ARG;
+        if (items[i].dtype != items[0].dtype) return HQ_ERR_UNSUPPORTED;
+    }
+    const int src = items[0].dtype == HQ_BF16 ? 0 : 1;
+    return encode_batch_common(
+        count, false, src, need, ws, stream,
+        [&](int32_t i, EncodePlan& pl) {
+            const hq_encode_item_t& it = items[i];
+            return plan_encode(it.x, src, it.rows, it.cols, &it.p, 0, 0, nullptr, it.out, false, ws, ws_bytes, pl);
+        },
+        [&](int32_t i, const hq_params_t&) {
+            hq_code_t* out = items[i].out;
+            out->rows = items[i].rows;
+            out->cols = items[i].cols;
+            out->kv_S = 0;
+            resolve_params(&items[i].p, out->p);
+            out->kv = 0;
+            out->kv_s0 = 0;
+            out->version = HQ_FORMAT_VERSION;
+        });
+}
+
+size_t hq_kv_encode_batch_workspace_bytes(int32_t count, const hq_kv_item_t* items)
+{
+    if (count < 1 || count > HQ_BATCH_MAX || !items) return 0;
+    size_t n = sizeof(WsHeader);
+    for (int32_t i = 0; i < count; ++i) {
+        const hq_kv_item_t& it = items[i];
+        if (it.B < 1 || it.H < 1 || it.S < 1 || it.B * it.H > ((int64_t)1 << 32)) return 0;
+        hq_params_t prm;
+        Geometry g;
+        if (!resolve_params(&it.p, prm) || it.D != prm.tile) return 0;
+        const int tpt = prm.tile == 64 ? 1 : (prm.tile == 256 ? 2 : enc_tpt(128, it.dtype == HQ_BF16 ? 0 : 1));
+        if (!geometry(it.B * it.H * it.S, it.D, prm.tile, g, tpt)) return 0;
+        n += (size_t)g.items * 8u;
+    }
+    return n;
+}
+
+hq_status_t hq_kv_encode_batch(int32_t count, const hq_kv_item_t* items, void* ws, size_t ws_bytes, void* stream)
+{
+    if (count < 1 || count > HQ_BATCH_MAX || !items || !ws) return HQ_ERR_ARG;
+    const size_t need = hq_kv_encode_batch_workspace_bytes(count, items);
+    if (need == 0 || ws_bytes < need) return HQ_ERR_ARG;
+    for (int32_t i = 0; i < count; ++i) {
+        if (items[i].dtype != HQ_BF16 && items[i].dtype != HQ_F32) return HQ_ERR_ARG;
+        if (items[i].s0 < 0) return HQ_ERR_ARG;
+        if (items[i].dtype != items[0].dtype) return HQ_ERR_UNSUPPORTED;
+    }
+    const int src = items[0].dtype == HQ_BF16 ? 0 : 1;
+    return encode_batch_common(
+        count, true, src, need, ws, stream,
+        [&](int32_t i, EncodePlan& pl) {
+            const hq_kv_item_t& it = items[i];
+            const hq_status_t ps = plan_encode(it.kv, src, it.B * it.H * it.S, it.D, &it.p, 1, it.S, nullptr, it.out,
+                                               false, ws, ws_bytes, pl);
+            pl.a.kv_s0 = it.s0;
+            return ps;
+        },
+        [&](int32_t i, const hq_params_t&) {
+            const hq_kv_item_t& it = items[i];
+            hq_code_t* out = it.out;
+            out->rows = it.B * it.H * it.S;
+            out->cols = it.D;
+            out->kv_S = it.S;
+            resolve_params(&it.p, out->p);
+            out->kv = 1;
+            out->kv_s0 = it.s0;
+            out->version = HQ_FORMAT_VERSION;
+        });
 }
 
 hq_status_t hq_decode_batch(int32_t count, const hq_decode_item_t* items, void* ws, size_t ws_bytes, void* stream)

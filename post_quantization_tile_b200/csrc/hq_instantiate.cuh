@@ -59,10 +59,16 @@ static cudaError_t enc_one(const EncodeArgs& a, const CUtensorMap& m, cudaStream
     return enc_batch<N, LAT, KV, SRC, COUNT, 1>(b, st);
 }
 
-// several weight tensors (no dither, bf16 or fp32) in one launch
+// several weight tensors (no dither, bf16 or fp32) in one launch; KV tensors (with the dither) of
+// head dimension 128
 template <int LAT>
-static cudaError_t enc_batch_dispatch(int n, int src, const EncodeBatch<kEncodeBatchMax>& b, cudaStream_t st)
+static cudaError_t enc_batch_dispatch(int n, bool kv, int src, const EncodeBatch<kEncodeBatchMax>& b, cudaStream_t st)
 {
+    if (kv) {
+        if (n != 128) return cudaErrorInvalidValue;
+        return src == 0 ? enc_batch<128, LAT, true, 0, false, kEncodeBatchMax>(b, st)
+                        : enc_batch<128, LAT, true, 1, false, kEncodeBatchMax>(b, st);
+    }
     if (src == 0) {
         if (n == 64) return enc_batch<64, LAT, false, 0, false, kEncodeBatchMax>(b, st);
         if (n == 128) return enc_batch<128, LAT, false, 0, false, kEncodeBatchMax>(b, st);
@@ -187,10 +193,10 @@ static cudaError_t dec_dispatch(int n, bool kv, int dst, const DecodeArgs& a, co
     {                                                                                                       \
         return enc_dispatch<LAT>(n, kv, src, count, a, m, st);                                              \
     }                                                                                                       \
-    cudaError_t launch_encode_batch_##SUFFIX(int n, int src, const EncodeBatch<kEncodeBatchMax>& b,          \
+    cudaError_t launch_encode_batch_##SUFFIX(int n, bool kv, int src, const EncodeBatch<kEncodeBatchMax>& b, \
                                              cudaStream_t st)                                               \
     {                                                                                                       \
-        return enc_batch_dispatch<LAT>(n, src, b, st);                                                      \
+        return enc_batch_dispatch<LAT>(n, kv, src, b, st);                                                  \
     }                                                                                                       \
     cudaError_t launch_decode_##SUFFIX(int n, bool kv, int dst, const DecodeArgs& a, const CUtensorMap& m,  \
                                        cudaStream_t st)                                                     \

@@ -20,11 +20,12 @@ cudaError_t launch_encode_z(int n, bool kv, int src, bool count, const EncodeArg
 cudaError_t launch_encode_a2(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_encode_d4(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
 cudaError_t launch_encode_e8(int n, bool kv, int src, bool count, const EncodeArgs& a, const CUtensorMap& m, cudaStream_t st);
-// several weight tensors of one tile size, lattice and source type in one launch
-cudaError_t launch_encode_batch_z(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
-cudaError_t launch_encode_batch_a2(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
-cudaError_t launch_encode_batch_d4(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
-cudaError_t launch_encode_batch_e8(int n, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+// several weight tensors (kv false), or KV tensors of head dimension 128 with the dither (kv true),
+// of one tile size, lattice and source type in one launch
+cudaError_t launch_encode_batch_z(int n, bool kv, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_encode_batch_a2(int n, bool kv, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_encode_batch_d4(int n, bool kv, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
+cudaError_t launch_encode_batch_e8(int n, bool kv, int src, const EncodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
 // several weight codes of one tile size and lattice to bf16 (dst 0) or fp32 (dst 1) in one launch
 cudaError_t launch_decode_batch_z(int n, int dst, const DecodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);
 cudaError_t launch_decode_batch_a2(int n, int dst, const DecodeBatch<kEncodeBatchMaxL>& b, cudaStream_t st);

@@ -101,3 +101,34 @@ def test_batch_refuses_mixed_tiles_and_lattices(hq):
     with pytest.raises(hq.HQError) as e:
         hq.decode_batch([code, other])
     assert e.value.code == 2
+
+
+@pytest.mark.parametrize("lattice", [oracle.D4, oracle.E8])
+def test_kv_encode_batch_equals_single_appends(hq, lattice):
+    shapes = [(2, 4, 1, 128), (2, 4, 3, 128), (1, 8, 1, 128), (3, 2, 2, 128)]
+    s0s = [0, 5, 17, 1000]
+    kvs = [torch.from_numpy(W.kv_keys(*sh[:3], 128, seed=30 + i).view(np.int16)).view(torch.bfloat16).cuda()
+           .reshape(sh) for i, sh in enumerate(shapes)]
+    steps = [1.1, 1.2, 0.9, 1.05]
+    seeds = [7, 8, 9, 10]
+    codes = hq.kv_encode_batch(kvs, s0s, steps, seeds, lattice=lattice)
+    assert hq.status(codes[0].ws)[0] == 0
+    for kv, code, s0, beta, seed in zip(kvs, codes, s0s, steps, seeds):
+        ref = hq.kv_encode(kv, step=beta, seed=seed, lattice=lattice, s0=s0)
+        assert hq.status(ref.ws)[0] == 0
+        assert (code.kv_S, code.kv_s0) == (ref.kv_S, ref.kv_s0)
+        _same_code(code, ref)
+
+
+def test_kv_encode_batch_fp32_and_refusals(hq):
+    import ctypes
+    rng = np.random.default_rng(5)
+    kvs = [torch.from_numpy(rng.standard_normal((2, 2, 4, 128)).astype(np.float32)).cuda() for _ in range(3)]
+    codes = hq.kv_encode_batch(kvs, [0, 4, 8], [1.1] * 3, [1, 2, 3])
+    for kv, code, s0, seed in zip(kvs, codes, [0, 4, 8], [1, 2, 3]):
+        _same_code(code, hq.kv_encode(kv, step=1.1, seed=seed, s0=s0))
+    # head dimension other than 128: not provided in a batch
+    kv64 = torch.from_numpy(rng.standard_normal((2, 2, 4, 64)).astype(np.float32)).cuda()
+    with pytest.raises(hq.HQError) as e:
+        hq.kv_encode_batch([kv64, kv64], [0, 0], [1.1, 1.1], [1, 1])
+    assert e.value.code == 2
